@@ -1,0 +1,276 @@
+"""Pins of the oracle's quantize / QJL / logit / value steps and of the
+packed record layout.
+
+"TQ" is the page "TurboQuant explained" (a2a-mcp.org).  Statistical checks
+use fixed seeds and bounds of several standard errors.
+"""
+
+import math
+
+import numpy as np
+import pytest
+from scipy import stats
+
+from oracle import tq_oracle as O
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _unit_rows(rng, n, d):
+    x = rng.standard_normal((n, d))
+    return x / np.linalg.norm(x, axis=1, keepdims=True)
+
+
+@pytest.mark.parametrize("d", [16, 128])
+def test_rotated_coordinates_follow_beta_law(d):
+    # TQ §Stage 1: after the rotation each coordinate of a unit vector is
+    # Beta((d-1)/2, (d-1)/2) on [-1, 1].  Kolmogorov-Smirnov against scipy.
+    rng = np.random.default_rng(1)
+    Pi, _, _ = O.rotation(d, 0x5EED0001)
+    y = (_unit_rows(rng, 20000, d) @ Pi.T)[:, 3]
+    a = (d - 1) / 2
+    assert stats.kstest(y, stats.beta(a, a, loc=-1, scale=2).cdf).pvalue > 1e-3
+
+
+def test_indices_are_nearest_centroids_brute_force():
+    # Lloyd-Max cells in one dimension are the Voronoi cells of the centroids.
+    rng = np.random.default_rng(2)
+    codec = O.make_codec(16, 3, 16, 11, 12)
+    enc = O.encode(codec, rng.standard_normal((64, 16)))
+    c = codec.cb.centroids
+    for n in range(64):
+        for j in range(16):
+            assert enc.idx[n, j] == int(np.argmin(np.abs(enc.y[n, j] - c)))
+
+
+def test_empirical_mse_matches_codebook_distortion():
+    # E||u - Pi^T c[idx]||^2 over random unit vectors equals d * D_b.
+    d, b = 128, 3
+    rng = np.random.default_rng(3)
+    codec = O.make_codec(d, b, 0, 0x5EED0001, 0)
+    U = _unit_rows(rng, 20000, d)
+    enc = O.encode(codec, U)
+    err = np.sum((U - codec.cb.centroids[enc.idx] @ codec.Pi) ** 2, axis=1)
+    se = err.std() / math.sqrt(len(err))
+    assert abs(err.mean() - d * codec.cb.distortion) < 5 * se
+
+
+def test_three_bit_cosine_similarity_community_figure():
+    # TQ §Stage 2 quotes a reconstruction cosine of 0.983+ at 3 bits; the
+    # MSE-stage reconstruction alone gives sqrt(1 - d D_3) ~ 0.983.
+    d = 128
+    rng = np.random.default_rng(4)
+    codec = O.make_codec(d, 3, 0, 0x5EED0001, 0)
+    U = _unit_rows(rng, 5000, d)
+    enc = O.encode(codec, U)
+    V = O.dequantize(codec, enc.idx, np.ones(len(U), np.float16))
+    cos = np.sum(U * V, axis=1) / np.linalg.norm(V, axis=1)
+    assert 0.980 <= cos.mean() <= 0.986
+    assert abs(cos.mean() - math.sqrt(1 - d * codec.cb.distortion)) < 2e-3
+
+
+def test_qjl_estimator_unbiased_over_seeds_with_closed_form_variance():
+    # TQ §Stage 2: the sign sketch corrects the inner-product bias.  With Pi
+    # fixed and 1000 seeds for S, the mean error is within 3 sigma / sqrt(1000)
+    # of 0, and the variance matches the closed form
+    # ||k||^2 ||r||^2 (pi/2)/m (||q||^2 - (2/pi) <q, r/||r||>^2).
+    d, b, m = 128, 3, 128
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal(d) * 2.0
+    q = rng.standard_normal(d)
+    base = O.make_codec(d, b, m, 0x5EED0001, 0)
+    est = []
+    for seed in range(1000):
+        S = O.qjl_matrix(m, d, 1000 + seed)
+        codec = O.Codec(d, b, m, base.Pi, S, base.cb)
+        enc = O.encode(codec, k[None, :])
+        # use the un-rounded norms so only the sketch is random
+        u = k / np.linalg.norm(k)
+        r = u - codec.c16[enc.idx[0]] @ codec.Pi
+        L = O.logits_from_codes(codec, q[None, :], enc.idx, enc.qneg,
+                                np.array([np.linalg.norm(k)]), np.array([np.linalg.norm(r)]))
+        est.append(L[0, 0])
+    est = np.array(est)
+    err = est - q @ k
+    sigma = err.std(ddof=1)
+    assert abs(err.mean()) < 3 * sigma / math.sqrt(len(err))
+    rhat = r / np.linalg.norm(r)
+    var_cf = (k @ k) * (r @ r) * (math.pi / 2) / m * (q @ q - (2 / math.pi) * (q @ rhat) ** 2)
+    chi2 = (len(err) - 1) * sigma ** 2 / var_cf
+    lo, hi = stats.chi2.ppf([0.0005, 0.9995], len(err) - 1)
+    assert lo < chi2 < hi
+
+
+def test_unbiased_when_rotation_also_varies():
+    d, b, m = 64, 2, 64
+    rng = np.random.default_rng(6)
+    k = rng.standard_normal(d)
+    q = rng.standard_normal(d)
+    errs = []
+    for seed in range(400):
+        codec = O.make_codec(d, b, m, 7000 + seed, 9000 + seed)
+        enc = O.encode(codec, k[None, :])
+        u = k / np.linalg.norm(k)
+        r = u - codec.c16[enc.idx[0]] @ codec.Pi
+        L = O.logits_from_codes(codec, q[None, :], enc.idx, enc.qneg,
+                                np.array([np.linalg.norm(k)]), np.array([np.linalg.norm(r)]))
+        errs.append(L[0, 0] - q @ k)
+    errs = np.array(errs)
+    assert abs(errs.mean()) < 3 * errs.std(ddof=1) / math.sqrt(len(errs))
+
+
+def test_high_bit_width_recovers_exact_logits():
+    # The estimate converges to the exact dot product as b grows: the residual
+    # norm, and with it the error, halves with every extra bit (Lloyd-Max
+    # distortion ~ 4^-b).  At b = 8 with m = 128 the rms error is below
+    # 1e-3 ||q|| ||k||; what is left is the sketch's own standard deviation
+    # ||r|| sqrt(pi / (2 m)) plus the fp16 rounding of the norms.
+    d, m = 128, 128
+    rng = np.random.default_rng(7)
+    K = rng.standard_normal((256, d)) * 3.0
+    Qv = rng.standard_normal((8, d))
+    exact = O.exact_logits(Qv, K)
+    scale = np.linalg.norm(Qv, axis=1)[:, None] * np.linalg.norm(K, axis=1)[None, :]
+    rms = []
+    for b in range(1, 9):
+        codec = O.make_codec(d, b, m, 0x5EED0001, 0x5EED0002)
+        enc = O.encode(codec, K)
+        L = O.logits_from_codes(codec, Qv, enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+        rel = (L - exact) / scale
+        rms.append(math.sqrt(np.mean(rel ** 2)))
+        pred = math.sqrt(d * codec.cb.distortion) * math.sqrt(math.pi / (2 * m))
+        assert 0.7 * pred < rms[-1] < 1.3 * pred + 3e-4
+    assert rms[-1] < 1e-3
+    assert all(rms[i] / rms[i + 1] > 1.6 for i in range(6))
+
+
+def test_mse_only_logits_equal_inner_product_with_reconstruction():
+    # With m = 0 the logit is <q, v_hat>: rotating the query once (Pi q) and
+    # dotting with c16[idx] is the same as dequantizing the key first.
+    rng = np.random.default_rng(8)
+    codec = O.make_codec(64, 3, 0, 21, 0)
+    K = rng.standard_normal((50, 64))
+    Qv = rng.standard_normal((5, 64))
+    enc = O.encode(codec, K)
+    L = O.logits_from_codes(codec, Qv, enc.idx, None, enc.norm16, None)
+    Vh = O.dequantize(codec, enc.idx, enc.norm16)
+    assert np.allclose(L, Qv @ Vh.T, rtol=1e-12, atol=1e-12)
+    W = rng.random((5, 50))
+    assert np.allclose(O.weighted_values(codec, W, enc.idx, enc.norm16), W @ Vh, rtol=1e-12, atol=1e-12)
+
+
+def test_high_bit_width_values_reconstruct():
+    rng = np.random.default_rng(9)
+    codec = O.make_codec(128, 8, 0, 0x5EED0001, 0)
+    V = rng.standard_normal((64, 128))
+    enc = O.encode(codec, V)
+    Vh = O.dequantize(codec, enc.idx, enc.norm16)
+    rel = np.linalg.norm(Vh - V, axis=1) / np.linalg.norm(V, axis=1)
+    assert rel.max() < 2e-2 and rel.mean() < math.sqrt(128 * codec.cb.distortion) * 1.2
+
+
+def test_zero_vector():
+    codec = O.make_codec(128, 3, 128, 1, 2)
+    X = np.zeros((2, 128))
+    X[1, 5] = 1.0
+    enc = O.encode(codec, X)
+    assert np.all(enc.idx[0] == 4) and float(enc.norm16[0]) == 0.0
+    L = O.logits_from_codes(codec, np.ones((1, 128)), enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+    assert L[0, 0] == 0.0
+
+
+def test_norm_side_values_are_fp16():
+    codec = O.make_codec(64, 2, 64, 1, 2)
+    X = np.full((1, 64), 1.0 / 3.0)
+    enc = O.encode(codec, X)
+    assert enc.norm16.dtype == np.float16
+    assert float(enc.norm16[0]) == float(np.float16(math.sqrt(64) / 3.0))
+
+
+# --- packed layout -----------------------------------------------------------
+
+@pytest.mark.parametrize("d,b,m", [(128, 3, 128), (128, 2, 128), (128, 4, 128), (128, 1, 128),
+                                   (128, 3, 0), (64, 3, 64), (200, 2, 200), (200, 4, 200), (96, 3, 0)])
+def test_pack_unpack_round_trip(d, b, m):
+    rng = np.random.default_rng(10)
+    lay = O.Layout(d, b, m, 64, 2)
+    idx = rng.integers(0, 1 << b, size=(33, d))
+    qneg = rng.random((33, m)) < 0.5 if m else None
+    words = O.pack_codes(lay, idx, qneg)
+    assert words.shape == (33, 4, lay.words)
+    idx2, qneg2 = O.unpack_codes(lay, words)
+    assert np.array_equal(idx, idx2)
+    if m:
+        assert np.array_equal(qneg, qneg2)
+
+
+def test_record_sizes():
+    # d = 128, m = 128: 3-bit keys are 64 code bytes + 4 norm bytes = 68 B,
+    # 2-bit keys 52 B, 4-bit keys 84 B; 3-bit values (no QJL) 48 + 2 = 50 B.
+    sizes = {(3, 128): 68, (2, 128): 52, (4, 128): 84, (3, 0): 50}
+    for (b, m), total in sizes.items():
+        lay = O.Layout(128, b, m, 64, 8)
+        assert lay.code_bytes + lay.norm_bytes == total
+    assert O.Layout(128, 3, 128, 64, 8).head_block_bytes == 64 * 68
+
+
+def test_layout_hand_worked_bits():
+    # d = 64, b = 3, m = 64: E = F = 16, one sign, one magnitude and one QJL
+    # word per chunk.  Hand-derived from the layout rules:
+    #  coordinate 5  -> chunk 0, l = 5: sign bit (5%32)//2 + 16 = 18,
+    #                   magnitude bits at 8*(5%4) + 2*((5%16)//4) = 10
+    #  idx 1 with H = 4 is neg = 1, mu = 2: sign word 1<<18, magnitude 2<<10.
+    #  coordinate 17 -> chunk 1, l = 1: sign bit 16, magnitude bits at 8.
+    #  idx 7 is neg = 0, mu = 3 -> magnitude word 3<<8.
+    #  projection 34 -> chunk 2, l = 2: bit 1; projection 63 -> chunk 3, l = 15: bit 23.
+    lay = O.Layout(64, 3, 64, 64, 1)
+    idx = np.full((1, 64), 4)
+    idx[0, 5] = 1
+    idx[0, 17] = 7
+    qneg = np.zeros((1, 64), bool)
+    qneg[0, 34] = True
+    qneg[0, 63] = True
+    w = O.pack_codes(lay, idx, qneg)[0]
+    assert [int(v) for v in w[0]] == [1 << 18, 2 << 10, 0]
+    assert [int(v) for v in w[1]] == [0, 3 << 8, 0]
+    assert [int(v) for v in w[2]] == [0, 0, 1 << 1]
+    assert [int(v) for v in w[3]] == [0, 0, 1 << 23]
+
+
+def test_layout_hand_worked_bits_b2_b4():
+    # b = 2 (H = 2), d = 128: E = 32; coordinate 6 -> chunk 0, l = 6:
+    # sign bit 3 (l%32//2) + 0 = 3, magnitude bit 8*(6%4) + 6//4 = 17.
+    # idx 0 -> neg 1, mu 1.
+    lay = O.Layout(128, 2, 0, 64, 1)
+    idx = np.full((1, 128), 2)
+    idx[0, 6] = 0
+    w = O.pack_codes(lay, idx, None)[0]
+    assert [int(v) for v in w[0]] == [1 << 3, 1 << 17]
+    # b = 4 (H = 8), d = 128: E = 32, nibble words of 8 elements;
+    # coordinate 37 -> chunk 1, l = 5: word 0, nibble 4*((5%8)//2 + 4*(5%2)) = 4*6 = 24.
+    # idx 2 -> neg 1, mu 5 -> nibble 0b1101.
+    lay = O.Layout(128, 4, 0, 64, 1)
+    idx = np.full((1, 128), 8)
+    idx[0, 37] = 2
+    w = O.pack_codes(lay, idx, None)[0]
+    assert [int(v) for v in w[1]] == [0b1101 << 24, 0, 0, 0]
+    assert not w[0].any() and not w[2].any() and not w[3].any()
+
+
+def test_pages_round_trip_with_block_table():
+    rng = np.random.default_rng(11)
+    lay = O.Layout(128, 3, 128, 64, 2)
+    n_pages = 8
+    pages = np.zeros(n_pages * lay.page_bytes, np.uint8)
+    bt = rng.permutation(n_pages).reshape(2, 4).astype(np.int32)
+    codec = O.make_codec(128, 3, 128, 5, 6)
+    X = rng.standard_normal((150, 128))
+    enc = O.encode(codec, X)
+    pos = np.arange(30, 180)
+    O.write_pages(lay, pages, bt, 1, 1, pos, enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+    idx, qneg, n16, r16 = O.read_pages(lay, pages, bt, 1, 1, pos)
+    assert np.array_equal(idx, enc.idx) and np.array_equal(qneg, enc.qneg)
+    assert np.array_equal(n16, enc.norm16) and np.array_equal(r16, enc.rnorm16)
+    # head 0 of sequence 1 and everything of sequence 0 stay untouched
+    for p in bt[0]:
+        assert not pages[p * lay.page_bytes:(p + 1) * lay.page_bytes].any()
