@@ -1,0 +1,422 @@
+#!/usr/bin/env python
+"""Benchmark of the TurboQuant KV-cache codec on B200.
+
+Workload (decode step): batch 1, 8 KV heads / 32 query heads (GQA 4), head
+dim 128, context 32768, bf16 K/V ~ N(0,1) x per-channel log-uniform [0.1, 10]
+scales; keys coded with b = 3 Lloyd-Max bits + a 128-row QJL sketch (68-byte
+records), values with b = 3 (50-byte records), 64-token pages through a
+permuted block table.
+
+One step = the whole hot path of a decode step: quantize-and-append the new
+token's K and V, fused logits of 32 query heads over the 32768 packed keys
+(query rotated once), and the value path (weighted accumulation of the
+packed values in the rotated space, rotated back once).  Every step reads a
+different one of R cache replicas (R x 31 MB > the 126 MB L2), so the codes
+come from HBM.
+
+Headline metric: fused 3-bit logits HBM GB/s = algorithmic bytes of the
+logits call (68 B per key + 4 B per logit + the query) / its device time
+(CUDA events around each logits launch, summed over the timed steps, max
+over ranks).  Secondary: keys quantized/s of the append kernel on the
+prefill-shaped batch (16 x 8 x 4096 bf16 keys).
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+(N > 1 under torch.distributed.run: every rank runs its own replica of the
+workload; weak scaling, no collective on the data path.)
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+B, HKV, HQ, D, CTX, PT, BITS, M = 1, 8, 32, 128, 32768, 64, 3, 128
+KEY_REC, VAL_REC = 68, 50
+LOGIT_BYTES = B * HKV * CTX * KEY_REC + B * HQ * CTX * 4 + B * HQ * D * 2
+VALUE_BYTES = B * HKV * CTX * VAL_REC + B * HQ * CTX * 4 + B * HQ * D * 4
+APPEND_BYTES = 2 * B * HKV * D * 2 + B * HKV * (KEY_REC + VAL_REC)
+APPEND_CFG = dict(batch=16, heads=8, n_new=4096)
+WORKLOAD = "decode step: batch 1, 8 KV / 32 query heads, head_dim 128, context 32768, keys b=3 + QJL m=128, values b=3"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), float(j.get("bf16_tflops", 1590.0)), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples while the GPU is busy."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        self.proc.wait()
+        self.f.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _init_pg(ws, backend):
+    import datetime
+
+    import torch.distributed as dist
+    if ws > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+
+
+def _max_over_ranks(x: float, ws: int, device) -> float:
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU baseline
+
+def oracle_logits_sample(n_keys: int, seed: int = 1002):
+    """Times the oracle's logits path (unpack packed pages + estimator) on
+    n_keys keys of one KV head with its 4 query heads."""
+    from kv_cache_vector_rotate_b200 import synth
+    from oracle import tq_oracle as O
+    n_keys = max(64, (n_keys // PT) * PT)
+    data = synth.decode_step(seed, 1, 1, 4, n_keys, D)
+    codec = O.make_codec(D, BITS, M, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(D, BITS, M, PT, 1)
+    bt = synth.block_table(seed, 1, n_keys // PT)
+    enc = O.encode(codec, data["k"][1][0, 0])
+    pages = np.zeros(lay.page_bytes * (n_keys // PT), np.uint8)
+    O.write_pages(lay, pages, bt, 0, 0, np.arange(n_keys), enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+    q = data["q"][1][0]
+    t0 = time.perf_counter()
+    idx, qneg, n16, r16 = O.read_pages(lay, pages, bt, 0, 0, np.arange(n_keys))
+    O.logits_from_codes(codec, q, idx, qneg, n16, r16)
+    dt = time.perf_counter() - t0
+    nbytes = n_keys * KEY_REC + 4 * n_keys * 4 + 4 * D * 2
+    return nbytes, dt
+
+
+def _cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float = 12.0):
+    nb, dt = oracle_logits_sample(4096)
+    per_key = dt / 4096
+    n = int(min(CTX, max(4096, budget_s / max(per_key, 1e-9) / 2)))
+    nb, dt = oracle_logits_sample(n)
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": _cpu_threads(), "kind": "oracle",
+            "sample": f"oracle unpack + logits of {n} packed 3-bit keys x 4 query heads (one KV head of the workload), {dt:.1f} s"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if ws > 1:
+        _init_pg(ws, "gloo")
+        if rank != 0:
+            _barrier(ws)
+            return
+    # calibrate one step to fit the whole run in ~90 s
+    nb, dt = oracle_logits_sample(2048)
+    per_key = dt / 2048
+    n_keys = int(max(256, min(CTX, 90.0 / (args.steps + args.warmup) / max(per_key, 1e-9))))
+    for _ in range(args.warmup):
+        oracle_logits_sample(n_keys)
+    tot_b, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        b_, t_ = oracle_logits_sample(n_keys)
+        tot_b += b_
+        tot_t += t_
+    v = tot_b / tot_t / 1e9
+    line = {
+        "metric": "fused 3-bit logits HBM GB/s", "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": WORKLOAD, "sample_keys_per_step": n_keys},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _cpu_threads(), "kind": "oracle",
+                         "sample": f"{n_keys} keys of one KV head x 4 query heads per step"},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    if ws > 1:
+        _barrier(ws)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    _init_pg(ws, "nccl")
+    dev = torch.device("cuda", local)
+    tq.load_library()
+    hbm_peak, _, peak_src = _peaks()
+
+    data = synth.decode_step(1002, B, HKV, HQ, CTX, D)
+    as_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    K = as_bf16(data["k"][0])
+    V = as_bf16(data["v"][0])
+    q = as_bf16(data["q"][0])
+    kcb = tq.Codebook(D, BITS, M, synth.SEED_PI, synth.SEED_S)
+    vcb = tq.Codebook(D, BITS, 0, synth.SEED_PI, 0)
+    pps = CTX // PT
+    bt = torch.from_numpy(synth.block_table(1003, B, pps))
+    R = args.replicas
+    zero = torch.zeros(B, dtype=torch.int32, device=dev)
+    kc, vc = [], []
+    for r in range(R):
+        kc.append(tq.PagedCache.allocate(kcb, pps, PT, HKV, bt, device=dev))
+        vc.append(tq.PagedCache.allocate(vcb, pps, PT, HKV, bt, device=dev))
+        tq.quantize_append(kcb, K, zero, kc[r])
+        tq.quantize_append(vcb, V, zero, vc[r])
+    del K, V
+    ctx_t = torch.full((B,), CTX, dtype=torch.int32, device=dev)
+    last = torch.full((B,), CTX - 1, dtype=torch.int32, device=dev)
+    knew = as_bf16(data["k"][0][:, :, -1:, :])
+    vnew = as_bf16(data["v"][0][:, :, -1:, :])
+    W = torch.from_numpy(synth.softmax_like_weights(1004, B, HQ, CTX)).to(dev)
+    Lout = torch.empty(B, HQ, CTX, dtype=torch.float32, device=dev)
+    Oout = torch.empty(B, HQ, D, dtype=torch.float32, device=dev)
+    lws = torch.empty(tq.logits_workspace_bytes(kcb, B, HKV, HQ), dtype=torch.uint8, device=dev)
+    vws = torch.empty(max(16, tq.values_workspace_bytes(vcb, B, HKV, HQ, CTX)), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(r, ev=None):
+        if ev is not None:
+            ev[0].record()
+        tq.quantize_append(kcb, knew, last, kc[r])
+        tq.quantize_append(vcb, vnew, last, vc[r])
+        if ev is not None:
+            ev[1].record()
+        tq.logits(kcb, kc[r], q, ctx_t, CTX, out=Lout, workspace=lws)
+        if ev is not None:
+            ev[2].record()
+        tq.dequant_values(vcb, vc[r], ctx_t, CTX, B, weights=W, out=Oout, workspace=vws)
+        if ev is not None:
+            ev[3].record()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up (W steps) plus a short soak so the clock samples see the GPU under load
+    for i in range(args.warmup):
+        step(i % R)
+    t_end = time.time() + 1.0
+    i = 0
+    while time.time() < t_end:
+        step(i % R)
+        i += 1
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    _barrier(ws)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for s in range(args.steps):
+        step(s % R, evs[s])
+    t1.record()
+    torch.cuda.synchronize()
+    _barrier(ws)
+    total_ms = t0.elapsed_time(t1)
+    app_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    log_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    val_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    total_ms = _max_over_ranks(total_ms, ws, dev)
+    log_ms = _max_over_ranks(log_ms, ws, dev)
+    val_ms = _max_over_ranks(val_ms, ws, dev)
+    app_ms = _max_over_ranks(app_ms, ws, dev)
+
+    # e2e: the same step through host buffers (pinned), copies inside the region
+    q_h = q.cpu().pin_memory()
+    kn_h = knew.cpu().pin_memory()
+    vn_h = vnew.cpu().pin_memory()
+    L_h = torch.empty_like(Lout, device="cpu").pin_memory()
+    O_h = torch.empty_like(Oout, device="cpu").pin_memory()
+
+    def e2e_step(r):
+        q.copy_(q_h, non_blocking=True)
+        knew.copy_(kn_h, non_blocking=True)
+        vnew.copy_(vn_h, non_blocking=True)
+        step(r)
+        L_h.copy_(Lout, non_blocking=True)
+        O_h.copy_(Oout, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(i % R)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(args.steps):
+        e2e_step(s % R)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(e0.elapsed_time(e1), ws, dev)
+    clk = clocks.stop()
+
+    # keys quantized/s on the prefill-shaped batch (16 x 8 x 4096 bf16 keys)
+    kq = None
+    if not args.no_append_phase:
+        kq = append_phase(args, dev, ws)
+
+    n = ws
+    steps = args.steps
+    logits_gbs = n * LOGIT_BYTES * steps / (log_ms * 1e-3) / 1e9
+    line = {
+        "metric": "fused 3-bit logits HBM GB/s", "value": logits_gbs, "unit": "GB/s", "n_gpus": n,
+        "steps": steps, "warmup": args.warmup, "ms_per_step": total_ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B * n, "seq_len": CTX, "parallelism": f"replicas{n}",
+                   "l2": f"{R} cache replicas rotated per step ({R * 31} MB > 126 MB L2)",
+                   "logits_ms_per_step": log_ms / steps, "values_ms_per_step": val_ms / steps,
+                   "append_ms_per_step": app_ms / steps,
+                   "values_gbs": n * VALUE_BYTES * steps / (val_ms * 1e-3) / 1e9},
+        "roofline": {"bound": "hbm", "achieved": logits_gbs / n, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": logits_gbs / n / hbm_peak, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs (copy, burst)",
+                     "kernel": "tq_logits (query prep + fused logits), per launch"},
+        "e2e": {"value": n * LOGIT_BYTES * steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": q.numel() * 2 + knew.numel() * 2 + vnew.numel() * 2,
+                "d2h_bytes_per_step": Lout.numel() * 4 + Oout.numel() * 4,
+                "ms_per_step": e2e_ms / steps},
+        "gpu_launches": 6 * steps,
+        "clocks": clk,
+    }
+    if kq is not None:
+        line["keys_quantized"] = kq
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def append_phase(args, dev, ws):
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    c = APPEND_CFG
+    bits16, _ = synth.append_batch(1005, c["batch"], c["heads"], c["n_new"], D)
+    X = torch.from_numpy(bits16.view(np.int16)).view(torch.bfloat16).to(dev)
+    cb = tq.Codebook(D, BITS, M, synth.SEED_PI, synth.SEED_S)
+    pps = c["n_new"] // PT
+    bt = torch.from_numpy(synth.block_table(1006, c["batch"], pps))
+    cache = tq.PagedCache.allocate(cb, c["batch"] * pps, PT, c["heads"], bt, device=dev)
+    start = torch.zeros(c["batch"], dtype=torch.int32, device=dev)
+    n_steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        tq.quantize_append(cb, X, start, cache)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n_steps):
+        tq.quantize_append(cb, X, start, cache)
+    b.record()
+    torch.cuda.synchronize()
+    ms = _max_over_ranks(a.elapsed_time(b), ws, dev) / n_steps
+    keys = c["batch"] * c["heads"] * c["n_new"]
+    hbm_peak, bf16_peak, _ = _peaks()
+    gbs = keys * (D * 2 + KEY_REC) / (ms * 1e-3) / 1e9
+    return {"value": ws * keys / (ms * 1e-3), "unit": "keys/s", "ms_per_launch": ms, "launches": n_steps,
+            "config": "online append: 16 x 8 KV heads x 4096 new bf16 tokens (1% outliers x30), d=128, b=3 + QJL m=128, 64-token pages",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--no-append-phase", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,203 @@
+/*
+ * tq.h -- C ABI of the TurboQuant KV-cache codec for NVIDIA B200 (sm_100a).
+ *
+ * Method source ("TQ" below): the web page "TurboQuant 설명: 무엇인지와 LLM
+ * 메모리 6배 절약 구현 방법" (TurboQuant explained: what it is and how to
+ * implement 6x LLM memory savings), a2a-mcp.org:
+ *   TQ §Stage 1  random orthogonal rotation (QR of a Gaussian matrix), the
+ *                Beta((d-1)/2,(d-1)/2) coordinate law, Lloyd-Max quantizer;
+ *   TQ §Stage 2  1-bit QJL sign sketch of the residual (bias correction);
+ *   TQ §How it works / §How to implement  logits straight from the indices
+ *                with the query rotated once; quantize on every cache update.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Pointers named "device" must point to memory of the current CUDA device;
+ *    "host" pointers to ordinary host memory.  The library never allocates
+ *    cache, input, output or workspace memory: the caller owns all of it.  The
+ *    only library-owned memory is the small set of constant tables inside a
+ *    tq_codebook (freed by tq_codebook_free).
+ *  - Calls that take a stream are asynchronous on that stream (pass 0 for the
+ *    legacy default stream); they return after the launches are queued.
+ *  - Argument errors are detected on the host and returned synchronously
+ *    (TQ_EINVAL / TQ_EUNSUPPORTED) with nothing launched; tq_last_error()
+ *    then returns a message (thread-local, valid until the next call).
+ *  - Errors found by the kernels (a block-table entry outside [0, n_pages), a
+ *    norm too large for fp16, a bounded wait that gave up) are OR-ed into
+ *    *error_word of the cache (TQ_DEV_ERR_* bits) when it is not NULL.  The
+ *    kernels never trap; read the word after synchronizing the stream.  An
+ *    out-of-range page is skipped (nothing read or written through it).
+ *  - Shapes are row-major and contiguous unless a stride is given.
+ *
+ * Packed record layout (layout version 1)
+ * ---------------------------------------
+ * d_pad = 64 ceil(d/64), m_pad = 64 ceil(m/64), E = d_pad/4, F = m_pad/4.
+ * A record is 4 chunks; chunk t holds coordinates [tE, tE+E) and QJL rows
+ * [tF, tF+F) as 32-bit words: sign words, magnitude words (b = 2, 3) or
+ * nibble words (b = 4), then QJL words.  Level indices are stored as sign
+ * (1 = negative centroid) and magnitude mu (distance from the middle of the
+ * codebook); QJL bit = 1 where (S r)_i < 0.  Bit positions of the element at
+ * local position l: sign/QJL word l/32 bit (l%32)/2 + 16(l%2); 1-bit
+ * magnitude word l/32 bit 8(l%4) + (l%32)/4; 2-bit magnitude word l/16 bits
+ * 8(l%4) + 2((l%16)/4) (+1); nibble word l/8 bits 4((l%8)/2 + 4(l%2)) (..+3).
+ * Padding coordinates store zero bits.  A page holds page_tokens tokens of
+ * every KV head; a head block is page_tokens records followed by
+ * page_tokens norm slots (fp16 ||x||, then fp16 ||r|| when m > 0), padded to
+ * 16 bytes.  Token `pos` of sequence b, head h lives in page
+ * block_table[b * max_pages_per_seq + pos / page_tokens], slot
+ * pos % page_tokens.  tq_layout() reports the sizes.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_EINVAL = 1,        /* bad argument (NULL pointer, bad size, misalignment) */
+  TQ_EUNSUPPORTED = 2,  /* valid but not built (e.g. bits > 4 on the GPU path) */
+  TQ_ERANGE = 3,        /* a value outside its representable range */
+  TQ_ETIMEOUT = 4,      /* a bounded device wait gave up */
+  TQ_ECUDA = 5,         /* a CUDA runtime call failed */
+  TQ_ENOMEM = 6         /* the codebook's constant tables could not be allocated */
+} tq_status;
+
+typedef enum { TQ_BF16 = 0, TQ_F16 = 1, TQ_F32 = 2 } tq_dtype;
+
+/* Bits OR-ed into tq_cache.error_word by the kernels. */
+#define TQ_DEV_ERR_PAGE 1u     /* block-table entry outside [0, n_pages) */
+#define TQ_DEV_ERR_RANGE 2u    /* a norm >= 65520 became +inf in fp16 */
+#define TQ_DEV_ERR_TIMEOUT 4u  /* a bounded mbarrier wait gave up */
+
+/* Codec parameters.  d: head dimension, a multiple of 8 with 8 <= d <= 256.
+ * bits: Lloyd-Max bits per coordinate, 1..4 on the GPU path (TQ §Stage 1).
+ * m: QJL rows (TQ §Stage 2), 0 (MSE-only, e.g. values) or m_pad == d_pad.
+ * seed_pi / seed_s seed the Gaussian matrices of Pi and S (SplitMix64 used as
+ * a counter-based generator, Box-Muller normals, row-major fill). */
+typedef struct {
+  int32_t d;
+  int32_t bits;
+  int32_t m;
+  uint64_t seed_pi;
+  uint64_t seed_s;
+} tq_params;
+
+typedef struct tq_codebook tq_codebook;
+
+/* Sizes of the packed format for a codebook (see "Packed record layout"). */
+typedef struct {
+  int32_t d_pad;
+  int32_t m_pad;
+  int32_t words_per_chunk;   /* 32-bit words in each of the 4 chunks */
+  int32_t code_bytes;        /* bytes of one record (16 * words_per_chunk) */
+  int32_t norm_bytes;        /* bytes of one norm slot: 4 with QJL, else 2 */
+  int32_t head_block_bytes;  /* page_tokens records + norm slots, 16-aligned */
+  int64_t page_bytes;        /* n_kv_heads * head_block_bytes */
+} tq_layout_info;
+
+/* A paged cache of packed records, owned by the caller.  pages: device,
+ * n_pages * page_bytes bytes, 16-byte aligned.  block_table: device int32
+ * [batch, max_pages_per_seq].  page_tokens: a multiple of 16, 16..256.
+ * error_word: device uint32 or NULL. */
+typedef struct {
+  void* pages;
+  int64_t n_pages;
+  int32_t page_tokens;
+  int32_t n_kv_heads;
+  const int32_t* block_table;
+  int64_t max_pages_per_seq;
+  uint32_t* error_word;
+} tq_cache;
+
+/* Builds the codebook on the host in float64 and uploads its constant tables
+ * to the current device (synchronously): Pi = Q of the QR of the seeded
+ * Gaussian d x d matrix with diag(R) > 0 (TQ §Stage 1); S, the seeded
+ * Gaussian m x d matrix (TQ §Stage 2); the Lloyd-Max centroids and midpoint
+ * boundaries of the Beta((d-1)/2,(d-1)/2) law by numerical integration
+ * (TQ §Stage 1).  *out receives a handle owned by the caller. */
+tq_status tq_codebook_build(const tq_params* params, tq_codebook** out);
+
+/* Same as tq_codebook_build but builds only the float64 host tables (no
+ * device is touched).  Such a codebook can be exported and inspected, and is
+ * rejected with TQ_EINVAL by the calls that launch kernels. */
+tq_status tq_codebook_build_host(const tq_params* params, tq_codebook** out);
+
+/* Releases the handle and its device tables.  NULL is allowed. */
+void tq_codebook_free(tq_codebook* cb);
+
+/* Copies the float64 host tables of a codebook into caller arrays (each may
+ * be NULL): pi [d*d] row-major (y = Pi x), s [m*d], centroids [2^bits]
+ * ascending, boundaries [2^bits - 1]. */
+tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s,
+                             double* centroids, double* boundaries);
+
+/* Fills *info with the packed-format sizes for this codebook. */
+tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_heads,
+                    tq_layout_info* info);
+
+/* Online quantize-and-append (TQ §Stage 1 + §Stage 2; TQ §How to implement:
+ * quantization on every cache update).  x: device [batch, n_kv_heads, n_new,
+ * d] of dtype.  start_pos: device int32 [batch], position of x[b, :, 0].
+ * For every vector: ||x|| (fp32, stored fp16), y = Pi x / ||x||, indices
+ * by threshold search over the Lloyd-Max boundaries, and when m > 0 the
+ * residual r = y - c16[idx] (rotated space), ||r|| (fp16) and the m signs of
+ * S r; the packed record is written into its page slot.  Each token owns its
+ * bytes, so appends that start inside a page are safe; calls on one stream
+ * are ordered.  Returns TQ_EINVAL for bad shapes, dtype or pointers. */
+tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtype,
+                             int64_t batch, int32_t n_kv_heads, int64_t n_new,
+                             const int32_t* start_pos, const tq_cache* cache,
+                             void* stream);
+
+/* Workspace (device bytes) that tq_logits needs for these sizes. */
+size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                 int32_t n_q_heads);
+
+/* Fused logits from the packed keys (TQ §Stage 2 and §How it works): for
+ * query head hq of sequence b (KV head hq / (n_q_heads / n_kv_heads)) and
+ * every key position t < ctx_len[b],
+ *   out[(b * n_q_heads + hq) * out_stride + t] = ||k|| ( <Pi q, c16[idx]>
+ *        + sqrt(pi/2)/m ||r|| <S q, sign> )   (sign_i = -1 where the bit is 1)
+ * with the query rotated once.  No 1/sqrt(d) scale, no softmax.  Positions
+ * t >= ctx_len[b] are not written.  q: device [batch, n_q_heads, d] of dtype.
+ * ctx_len: device int32 [batch], each <= max_ctx <= out_stride.  workspace:
+ * device, at least tq_logits_workspace_bytes(), 16-byte aligned. */
+tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
+                    tq_dtype dtype, int64_t batch, int32_t n_q_heads,
+                    const int32_t* ctx_len, int64_t max_ctx, float* out,
+                    int64_t out_stride, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/* Workspace (device bytes) that tq_dequant_values needs for these sizes. */
+size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                 int32_t n_q_heads, int64_t max_ctx);
+
+/* Value path from packed records (MSE reconstruction v_hat = ||v|| Pi^T
+ * c16[idx]).  Mode A (weights == NULL): out device [batch, n_kv_heads,
+ * out_stride, d] of out_dtype receives v_hat for t < ctx_len[b].  Mode B
+ * (weights != NULL, device fp32 [batch, n_q_heads, w_stride]): out device
+ * fp32 [batch, n_q_heads, d] receives sum_{t < ctx_len[b]} weights[b,hq,t]
+ * v_hat_t, accumulated in the rotated space and rotated back once.  For mode B
+ * out_dtype must be TQ_F32 and out_stride is ignored.  workspace: device, at
+ * least tq_values_workspace_bytes() (0 is enough for mode A). */
+tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache,
+                            const float* weights, int64_t w_stride, int64_t batch,
+                            int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx,
+                            void* out, tq_dtype out_dtype, int64_t out_stride,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/* Message for the last failed call on this thread ("" if none). */
+const char* tq_last_error(void);
+
+/* Layout version of the packed records written and read by this build. */
+int32_t tq_layout_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H_ */

@@ -1,0 +1,368 @@
+// C ABI of libtq: argument checks, codebook construction / upload, dispatch.
+// The method follows "TurboQuant explained" (a2a-mcp.org), §Stage 1 and
+// §Stage 2; the entry points are documented in include/tq.h.
+
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+
+#include "codebook_host.h"
+#include "tq_internal.cuh"
+
+namespace tq {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+tq_status fail(tq_status st, const std::string& msg) {
+  g_last_error = msg;
+  return st;
+}
+
+tq_status cuda_fail(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return TQ_OK;
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return TQ_ECUDA;
+}
+
+tq_status launch_quantize_simt(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
+                               int n_kv_heads, int64_t n_new, const int32_t* start_pos,
+                               const CacheView& cv, cudaStream_t st);
+tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
+                             int n_kv_heads, int64_t n_new, const int32_t* start_pos,
+                             const CacheView& cv, cudaStream_t st, bool* handled);
+
+// IEEE binary16 bits of x, rounded to nearest-even directly from double.
+static uint16_t f64_to_f16_bits(double x) {
+  const uint16_t sign = std::signbit(x) ? 0x8000 : 0;
+  const double a = std::fabs(x);
+  if (a >= 65520.0) return sign | 0x7C00;
+  if (a == 0.0) return sign;
+  int e;
+  std::frexp(a, &e);                           // a = f 2^e, f in [0.5, 1)
+  const int E = std::max(e - 1, -14);          // exponent of the fp16 quantum
+  const double quantum = std::ldexp(1.0, E - 10);
+  const double v = std::nearbyint(a / quantum) * quantum;   // round half to even
+  if (v < std::ldexp(1.0, -14)) return sign | (uint16_t)(v / std::ldexp(1.0, -24));
+  std::frexp(v, &e);
+  const int ev = e - 1;
+  if (ev > 15) return sign | 0x7C00;
+  const uint16_t mant = (uint16_t)((v / std::ldexp(1.0, ev) - 1.0) * 1024.0);
+  return sign | (uint16_t)((ev + 15) << 10) | mant;
+}
+
+static float f16_bits_to_float(uint16_t h) {
+  __half_raw r;
+  r.x = h;
+  return __half2float(__half(r));
+}
+
+static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static tq_status check_params(const tq_params* p) {
+  if (!p) return fail(TQ_EINVAL, "params is NULL");
+  if (p->d < 8 || p->d > 256 || p->d % 8 != 0)
+    return fail(TQ_EINVAL, "d must be a multiple of 8 in [8, 256]");
+  if (p->bits < 1 || p->bits > 4) return fail(TQ_EUNSUPPORTED, "bits must be in [1, 4]");
+  if (p->m < 0) return fail(TQ_EINVAL, "m must be >= 0");
+  if (p->m > 0 && 64 * ((p->m + 63) / 64) != 64 * ((p->d + 63) / 64))
+    return fail(TQ_EUNSUPPORTED, "m must be 0 or round up to the same multiple of 64 as d");
+  return TQ_OK;
+}
+
+static void build_host_tables(tq_codebook* cb, const tq_params* p) {
+  const int d = p->d, m = p->m;
+  std::vector<double> G((size_t)d * d);
+  tqhost::gaussian_fill(p->seed_pi, G.size(), G.data());
+  cb->pi = tqhost::orthogonal_factor(G, d);
+  cb->s.assign((size_t)m * d, 0.0);
+  if (m > 0) tqhost::gaussian_fill(p->seed_s, cb->s.size(), cb->s.data());
+  tqhost::LloydMax lm = tqhost::lloyd_max(d, p->bits);
+  cb->centroids = lm.centroids;
+  cb->boundaries = lm.boundaries;
+  cb->s_row_norm_max = 0.0;
+  for (int i = 0; i < m; ++i) {
+    double s2 = 0.0;
+    for (int k = 0; k < d; ++k) s2 += cb->s[(size_t)i * d + k] * cb->s[(size_t)i * d + k];
+    cb->s_row_norm_max = std::max(cb->s_row_norm_max, std::sqrt(s2));
+  }
+  cb->qjl_scale = m > 0 ? std::sqrt(3.14159265358979323846 / 2.0) / m : 0.0;
+  const int K = 1 << p->bits, H = K / 2;
+  for (int i = 0; i < 16; ++i) cb->cent16[i] = 0;
+  for (int i = 0; i < 8; ++i) cb->mag16[i] = 0;
+  for (int i = 0; i < K; ++i) cb->cent16[i] = f64_to_f16_bits(cb->centroids[i]);
+  for (int mu = 0; mu < H; ++mu) cb->mag16[mu] = cb->cent16[H + mu];
+}
+
+static tq_status upload(tq_codebook* cb) {
+  const Layout& L = cb->lay;
+  const int d = L.d, dp = L.d_pad, mp = L.m_pad, K = 1 << L.bits;
+  auto al = [](size_t n) { return (n + 255) / 256 * 256; };
+  const size_t sz_pi = al((size_t)dp * d * 4), sz_s = al((size_t)mp * d * 4 + 4),
+               sz_srot = al((size_t)mp * dp * 4 + 4), sz_b = al(16 * 4), sz_c = al(16 * 4),
+               sz_pibf = al((size_t)2 * dp * dp * 2), sz_srbf = al((size_t)2 * mp * dp * 2 + 4);
+  const size_t total = sz_pi + sz_s + sz_srot + sz_b + sz_c + sz_pibf + sz_srbf;
+  std::vector<uint8_t> host(total, 0);
+  size_t off = 0;
+  auto take = [&](size_t n) { size_t o = off; off += n; return o; };
+  const size_t o_pi = take(sz_pi), o_s = take(sz_s), o_srot = take(sz_srot), o_b = take(sz_b),
+               o_c = take(sz_c), o_pibf = take(sz_pibf), o_srbf = take(sz_srbf);
+  float* pi32 = reinterpret_cast<float*>(host.data() + o_pi);
+  float* s32 = reinterpret_cast<float*>(host.data() + o_s);
+  float* srot32 = reinterpret_cast<float*>(host.data() + o_srot);
+  float* b32 = reinterpret_cast<float*>(host.data() + o_b);
+  float* c32 = reinterpret_cast<float*>(host.data() + o_c);
+  __nv_bfloat16* pibf = reinterpret_cast<__nv_bfloat16*>(host.data() + o_pibf);
+  __nv_bfloat16* srbf = reinterpret_cast<__nv_bfloat16*>(host.data() + o_srbf);
+  for (int j = 0; j < d; ++j)
+    for (int k = 0; k < d; ++k) pi32[(size_t)j * d + k] = (float)cb->pi[(size_t)j * d + k];
+  for (int i = 0; i < L.m; ++i)
+    for (int k = 0; k < d; ++k) s32[(size_t)i * d + k] = (float)cb->s[(size_t)i * d + k];
+  // S_rot = S Pi^T: the residual is formed in the rotated space, and
+  // S r = S Pi^T (Pi r).
+  for (int i = 0; i < L.m; ++i)
+    for (int j = 0; j < d; ++j) {
+      double acc = 0.0;
+      for (int k = 0; k < d; ++k) acc += cb->s[(size_t)i * d + k] * cb->pi[(size_t)j * d + k];
+      srot32[(size_t)i * dp + j] = (float)acc;
+      const __nv_bfloat16 hi = __double2bfloat16(acc);
+      srbf[(size_t)i * dp + j] = hi;
+      srbf[(size_t)mp * dp + (size_t)i * dp + j] = __double2bfloat16(acc - (double)__bfloat162float(hi));
+    }
+  for (int j = 0; j < d; ++j)
+    for (int k = 0; k < d; ++k) {
+      const double v = cb->pi[(size_t)j * d + k];
+      const __nv_bfloat16 hi = __double2bfloat16(v);
+      pibf[(size_t)j * dp + k] = hi;
+      pibf[(size_t)dp * dp + (size_t)j * dp + k] = __double2bfloat16(v - (double)__bfloat162float(hi));
+    }
+  for (int i = 0; i < K - 1; ++i) b32[i] = (float)cb->boundaries[i];
+  for (int i = 0; i < K; ++i) c32[i] = f16_bits_to_float(cb->cent16[i]);
+
+  void* dev = nullptr;
+  cudaError_t e = cudaMalloc(&dev, total);
+  if (e != cudaSuccess) return fail(TQ_ENOMEM, std::string("codebook tables: ") + cudaGetErrorString(e));
+  e = cudaMemcpy(dev, host.data(), total, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    cudaFree(dev);
+    return cuda_fail(e, "codebook upload");
+  }
+  uint8_t* base = reinterpret_cast<uint8_t*>(dev);
+  cb->dev_block = dev;
+  cb->pi32 = reinterpret_cast<float*>(base + o_pi);
+  cb->s32 = reinterpret_cast<float*>(base + o_s);
+  cb->srot32 = reinterpret_cast<float*>(base + o_srot);
+  cb->bound32 = reinterpret_cast<float*>(base + o_b);
+  cb->cent32 = reinterpret_cast<float*>(base + o_c);
+  cb->pi_bf = reinterpret_cast<__nv_bfloat16*>(base + o_pibf);
+  cb->srot_bf = reinterpret_cast<__nv_bfloat16*>(base + o_srbf);
+  return TQ_OK;
+}
+
+static tq_status make_view(const tq_codebook* cb, const tq_cache* c, CacheView* v) {
+  if (!c) return fail(TQ_EINVAL, "cache is NULL");
+  if (!c->pages || !c->block_table) return fail(TQ_EINVAL, "cache pages / block_table is NULL");
+  if (!aligned(c->pages, 16)) return fail(TQ_EINVAL, "cache pages must be 16-byte aligned");
+  if (c->page_tokens < 16 || c->page_tokens > 256 || c->page_tokens % 16 != 0)
+    return fail(TQ_EINVAL, "page_tokens must be a multiple of 16 in [16, 256]");
+  if (c->n_kv_heads < 1 || c->n_pages < 1 || c->max_pages_per_seq < 1)
+    return fail(TQ_EINVAL, "cache sizes must be positive");
+  v->pages = reinterpret_cast<uint8_t*>(c->pages);
+  v->n_pages = c->n_pages;
+  v->page_tokens = c->page_tokens;
+  v->n_kv_heads = c->n_kv_heads;
+  v->block_table = c->block_table;
+  v->max_pages = c->max_pages_per_seq;
+  v->err = c->error_word;
+  v->head_block_bytes = cb->lay.head_block_bytes(c->page_tokens);
+  v->page_bytes = v->head_block_bytes * c->n_kv_heads;
+  return TQ_OK;
+}
+
+static tq_status check_cb(const tq_codebook* cb) {
+  if (!cb) return fail(TQ_EINVAL, "codebook is NULL");
+  if (!cb->dev_block) return fail(TQ_EINVAL, "codebook has no device tables (host-only build)");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev != cb->device) return fail(TQ_EINVAL, "codebook was built for another device");
+  return TQ_OK;
+}
+
+static size_t dtype_size(tq_dtype dt) { return dt == TQ_F32 ? 4 : 2; }
+static bool dtype_ok(tq_dtype dt) { return dt == TQ_BF16 || dt == TQ_F16 || dt == TQ_F32; }
+
+}  // namespace tq
+
+using namespace tq;
+
+extern "C" {
+
+const char* tq_last_error(void) { return g_last_error.c_str(); }
+
+int32_t tq_layout_version(void) { return kLayoutVersion; }
+
+static tq_status build_common(const tq_params* params, tq_codebook** out, bool device) {
+  if (!out) return fail(TQ_EINVAL, "out is NULL");
+  *out = nullptr;
+  tq_status s = check_params(params);
+  if (s != TQ_OK) return s;
+  tq_codebook* cb = new (std::nothrow) tq_codebook();
+  if (!cb) return fail(TQ_ENOMEM, "out of host memory");
+  cb->lay = Layout::make(params->d, params->bits, params->m);
+  cb->seed_pi = params->seed_pi;
+  cb->seed_s = params->seed_s;
+  cb->device = -1;
+  cb->dev_block = nullptr;
+  build_host_tables(cb, params);
+  if (device) {
+    cudaError_t e = cudaGetDevice(&cb->device);
+    if (e != cudaSuccess) {
+      delete cb;
+      return cuda_fail(e, "cudaGetDevice");
+    }
+    s = upload(cb);
+    if (s != TQ_OK) {
+      delete cb;
+      return s;
+    }
+  }
+  *out = cb;
+  return TQ_OK;
+}
+
+tq_status tq_codebook_build(const tq_params* params, tq_codebook** out) {
+  return build_common(params, out, true);
+}
+
+// Host tables only (no device upload): for inspecting a codebook without a GPU.
+tq_status tq_codebook_build_host(const tq_params* params, tq_codebook** out) {
+  return build_common(params, out, false);
+}
+
+void tq_codebook_free(tq_codebook* cb) {
+  if (!cb) return;
+  if (cb->dev_block) cudaFree(cb->dev_block);
+  delete cb;
+}
+
+tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s, double* centroids,
+                             double* boundaries) {
+  if (!cb) return fail(TQ_EINVAL, "codebook is NULL");
+  if (pi) std::memcpy(pi, cb->pi.data(), cb->pi.size() * sizeof(double));
+  if (s && !cb->s.empty()) std::memcpy(s, cb->s.data(), cb->s.size() * sizeof(double));
+  if (centroids) std::memcpy(centroids, cb->centroids.data(), cb->centroids.size() * sizeof(double));
+  if (boundaries)
+    std::memcpy(boundaries, cb->boundaries.data(), cb->boundaries.size() * sizeof(double));
+  return TQ_OK;
+}
+
+tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_heads,
+                    tq_layout_info* info) {
+  if (!cb || !info) return fail(TQ_EINVAL, "codebook / info is NULL");
+  if (page_tokens < 16 || page_tokens > 256 || page_tokens % 16 != 0 || n_kv_heads < 1)
+    return fail(TQ_EINVAL, "page_tokens must be a multiple of 16 in [16, 256], n_kv_heads >= 1");
+  const Layout& L = cb->lay;
+  info->d_pad = L.d_pad;
+  info->m_pad = L.m_pad;
+  info->words_per_chunk = L.W;
+  info->code_bytes = L.code_bytes;
+  info->norm_bytes = L.norm_bytes;
+  info->head_block_bytes = (int32_t)L.head_block_bytes(page_tokens);
+  info->page_bytes = L.head_block_bytes(page_tokens) * n_kv_heads;
+  return TQ_OK;
+}
+
+tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtype, int64_t batch,
+                             int32_t n_kv_heads, int64_t n_new, const int32_t* start_pos,
+                             const tq_cache* cache, void* stream) {
+  tq_status s = check_cb(cb);
+  if (s != TQ_OK) return s;
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_quantize_append: bad dtype");
+  if (batch < 0 || n_new < 0) return fail(TQ_EINVAL, "tq_quantize_append: negative size");
+  CacheView cv;
+  s = make_view(cb, cache, &cv);
+  if (s != TQ_OK) return s;
+  if (n_kv_heads != cache->n_kv_heads)
+    return fail(TQ_EINVAL, "tq_quantize_append: n_kv_heads differs from the cache's");
+  if (batch == 0 || n_new == 0) return TQ_OK;
+  if (!x || !start_pos) return fail(TQ_EINVAL, "tq_quantize_append: x / start_pos is NULL");
+  if (!aligned(x, dtype_size(dtype))) return fail(TQ_EINVAL, "tq_quantize_append: x misaligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bool handled = false;
+  s = launch_quantize_tc(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st, &handled);
+  if (handled || s != TQ_OK) return s;
+  return launch_quantize_simt(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st);
+}
+
+size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                 int32_t n_q_heads) {
+  if (!cb || batch < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)
+    return 0;
+  return logits_workspace(cb, batch * n_kv_heads, n_q_heads / n_kv_heads);
+}
+
+tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q, tq_dtype dtype,
+                    int64_t batch, int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx,
+                    float* out, int64_t out_stride, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  tq_status s = check_cb(cb);
+  if (s != TQ_OK) return s;
+  CacheView cv;
+  s = make_view(cb, cache, &cv);
+  if (s != TQ_OK) return s;
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_logits: bad dtype");
+  if (batch < 0 || max_ctx < 0 || max_ctx > INT32_MAX) return fail(TQ_EINVAL, "tq_logits: bad size");
+  if (n_q_heads < cv.n_kv_heads || n_q_heads % cv.n_kv_heads)
+    return fail(TQ_EINVAL, "tq_logits: n_q_heads must be a multiple of the cache's n_kv_heads");
+  if (out_stride < max_ctx) return fail(TQ_EINVAL, "tq_logits: out_stride < max_ctx");
+  if (max_ctx > cv.max_pages * cv.page_tokens)
+    return fail(TQ_EINVAL, "tq_logits: max_ctx exceeds the block table");
+  if (batch == 0 || max_ctx == 0) return TQ_OK;
+  if (!q || !ctx_len || !out || !workspace) return fail(TQ_EINVAL, "tq_logits: NULL pointer");
+  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 16))
+    return fail(TQ_EINVAL, "tq_logits: misaligned pointer");
+  return launch_logits(cb, cv, q, dtype, batch, n_q_heads, ctx_len, max_ctx, out, out_stride,
+                       workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                 int32_t n_q_heads, int64_t max_ctx) {
+  if (!cb || batch < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)
+    return 0;
+  return values_workspace(cb, batch, n_kv_heads, n_q_heads, max_ctx);
+}
+
+tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache, const float* weights,
+                            int64_t w_stride, int64_t batch, int32_t n_q_heads,
+                            const int32_t* ctx_len, int64_t max_ctx, void* out, tq_dtype out_dtype,
+                            int64_t out_stride, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  tq_status s = check_cb(cb);
+  if (s != TQ_OK) return s;
+  CacheView cv;
+  s = make_view(cb, cache, &cv);
+  if (s != TQ_OK) return s;
+  if (!dtype_ok(out_dtype)) return fail(TQ_EINVAL, "tq_dequant_values: bad dtype");
+  if (batch < 0 || max_ctx < 0 || max_ctx > INT32_MAX) return fail(TQ_EINVAL, "tq_dequant_values: bad size");
+  if (max_ctx > cv.max_pages * cv.page_tokens)
+    return fail(TQ_EINVAL, "tq_dequant_values: max_ctx exceeds the block table");
+  if (weights) {
+    if (out_dtype != TQ_F32) return fail(TQ_EINVAL, "tq_dequant_values: mode B writes fp32");
+    if (n_q_heads < cv.n_kv_heads || n_q_heads % cv.n_kv_heads)
+      return fail(TQ_EINVAL, "tq_dequant_values: n_q_heads must be a multiple of n_kv_heads");
+    if (w_stride < max_ctx) return fail(TQ_EINVAL, "tq_dequant_values: w_stride < max_ctx");
+  } else if (out_stride < max_ctx) {
+    return fail(TQ_EINVAL, "tq_dequant_values: out_stride < max_ctx");
+  }
+  if (batch == 0 || max_ctx == 0) return TQ_OK;
+  if (!ctx_len || !out) return fail(TQ_EINVAL, "tq_dequant_values: NULL pointer");
+  if (weights && !workspace) return fail(TQ_EINVAL, "tq_dequant_values: mode B needs a workspace");
+  return launch_values(cb, cv, weights, w_stride, batch, n_q_heads, ctx_len, max_ctx, out,
+                       out_dtype, out_stride, workspace, workspace_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

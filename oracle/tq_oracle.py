@@ -304,16 +304,21 @@ def quantize_indices(Y: np.ndarray, boundaries: np.ndarray) -> np.ndarray:
     return np.sum(Y[..., None] >= boundaries[None, None, :], axis=-1)
 
 
+def qjl_sketch(codec: Codec, U: np.ndarray, idx: np.ndarray):
+    """TQ §Stage 2 for unit rows U coded by idx: (S r, r < 0 bits, fp16 ||r||)
+    with the residual r = u - Pi^T c16[idx] taken in the original space."""
+    R = U - codec.c16[idx] @ codec.Pi
+    proj = R @ codec.S.T
+    return proj, proj < 0.0, fp16(np.sqrt(np.sum(R * R, axis=1)))
+
+
 def encode(codec: Codec, X: np.ndarray) -> Encoded:
     U, n = unit_and_norm(X)
     Y = U @ codec.Pi.T
     idx = quantize_indices(Y, codec.cb.boundaries)
     qneg = rnorm16 = proj = None
     if codec.m > 0:
-        R = U - codec.c16[idx] @ codec.Pi          # residual in the original space
-        proj = R @ codec.S.T
-        qneg = proj < 0.0
-        rnorm16 = fp16(np.sqrt(np.sum(R * R, axis=1)))
+        proj, qneg, rnorm16 = qjl_sketch(codec, U, idx)
     return Encoded(idx, qneg, fp16(n), rnorm16, Y, proj)
 
 

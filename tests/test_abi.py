@@ -1,0 +1,78 @@
+"""The C-ABI library loads, exports every entry point of include/tq.h, and its
+host-side codebook tables agree with the oracle (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from kv_cache_vector_rotate_b200 import tq
+from oracle import tq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _header_functions():
+    text = open(os.path.join(ROOT, "include", "tq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tq.load_library()
+    names = _header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(tq.EXPORTS)
+
+
+def test_layout_version():
+    assert tq.load_library().tq_layout_version() == 1
+
+
+@pytest.mark.parametrize("d,bits,m", [(128, 3, 128), (128, 2, 128), (128, 4, 0), (64, 1, 64), (200, 4, 200)])
+def test_host_tables_match_oracle(d, bits, m):
+    cb = tq.Codebook(d, bits, m, 0x5EED0001, 0x5EED0002, device=False)
+    t = cb.export()
+    Pi, _, _ = O.rotation(d, 0x5EED0001)
+    assert np.max(np.abs(t["pi"] - Pi)) < 1e-12
+    if m:
+        S = O.qjl_matrix(m, d, 0x5EED0002)
+        assert np.max(np.abs(t["s"] - S)) < 1e-13
+    ob = O.lloyd_max(d, bits)
+    assert np.max(np.abs(t["centroids"] - ob.centroids)) < 1e-12
+    assert np.max(np.abs(t["boundaries"] - ob.boundaries)) < 1e-12
+    assert np.array_equal(O.fp16(t["centroids"]), O.fp16(ob.centroids))
+
+
+@pytest.mark.parametrize("d,bits,m,pt,h", [(128, 3, 128, 64, 8), (128, 3, 0, 64, 8), (128, 2, 128, 32, 2),
+                                           (128, 4, 128, 64, 1), (200, 2, 200, 64, 1), (64, 1, 64, 16, 3)])
+def test_layout_sizes_match_oracle(d, bits, m, pt, h):
+    cb = tq.Codebook(d, bits, m, 1, 2, device=False)
+    info = cb.layout(pt, h)
+    lay = O.Layout(d, bits, m, pt, h)
+    assert info.d_pad == lay.d_pad and info.words_per_chunk == lay.words
+    assert info.code_bytes == lay.code_bytes and info.norm_bytes == lay.norm_bytes
+    assert info.head_block_bytes == lay.head_block_bytes and info.page_bytes == lay.page_bytes
+
+
+@pytest.mark.parametrize("d,bits,m,status", [(100, 3, 128, tq.TQ_EINVAL), (128, 5, 128, tq.TQ_EUNSUPPORTED),
+                                             (128, 0, 128, tq.TQ_EUNSUPPORTED), (264, 3, 0, tq.TQ_EINVAL),
+                                             (128, 3, 64, tq.TQ_EUNSUPPORTED), (128, 3, -1, tq.TQ_EINVAL)])
+def test_bad_params_rejected_on_host(d, bits, m, status):
+    with pytest.raises(tq.TqError) as e:
+        tq.Codebook(d, bits, m, 1, 2, device=False)
+    assert e.value.status == status
+    assert tq.load_library().tq_last_error()
+
+
+def test_host_only_codebook_refuses_kernels():
+    cb = tq.Codebook(128, 3, 128, 1, 2, device=False)
+    lib = tq.load_library()
+    cs = tq.CacheStruct(None, 1, 64, 1, None, 1, None)
+    st = lib.tq_quantize_append(cb.handle, None, 0, 1, 1, 1, None, ctypes.byref(cs), None)
+    assert st == tq.TQ_EINVAL
+    assert b"host-only" in lib.tq_last_error()

@@ -1,0 +1,159 @@
+"""GPU parity of tq_logits and tq_dequant_values against the fp64 oracle.
+
+The caches are written by the ORACLE (oracle/ packs the records); the GPU
+reads them through the C ABI, so the logits and values are compared given
+identical codes.  Tolerances are those of tests/parity.py.
+"""
+
+import numpy as np
+import pytest
+
+from kv_cache_vector_rotate_b200 import synth
+from oracle import tq_oracle as O
+from parity import LOGIT_TOL, VALUE_TOL, logit_error, oracle_pages
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def tqm():
+    from kv_cache_vector_rotate_b200 import tq as tqmod
+    tqmod.load_library()
+    return tqmod
+
+
+def _oracle_cache(tqm, codec, lay, keys, ctx, pt, seed):
+    """keys [batch, heads, ctx_max, d] float64; ctx [batch] -> (cb, cache, encs, bt)."""
+    batch, heads, cmax, d = keys.shape
+    pps = (cmax + pt - 1) // pt
+    bt = synth.block_table(seed, batch, pps)
+    encs = {}
+    for b in range(batch):
+        for h in range(heads):
+            pos = np.arange(ctx[b])
+            encs[(b, h)] = (pos, O.encode(codec, keys[b, h, : ctx[b]]))
+    pages = oracle_pages(lay, batch * pps, bt, encs)
+    cb = tqm.Codebook(codec.d, codec.bits, codec.m, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, batch * pps, pt, heads, torch.from_numpy(bt))
+    cache.pages.copy_(torch.from_numpy(pages))
+    return cb, cache, encs, bt
+
+
+def _q_tensor(q_vals, dtype):
+    t = torch.from_numpy(q_vals.astype(np.float32)).cuda()
+    return t.to({"bf16": torch.bfloat16, "f16": torch.float16, "f32": torch.float32}[dtype])
+
+
+def _check_logits(codec, q, encs, L_gpu, ctx, heads, G):
+    worst = 0.0
+    for (b, h), (pos, enc) in encs.items():
+        Qg = q[b, h * G:(h + 1) * G]
+        L = O.logits_from_codes(codec, Qg, enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+        err = logit_error(L_gpu[b, h * G:(h + 1) * G, : ctx[b]], L, np.linalg.norm(Qg, axis=1),
+                          enc.norm16, codec.d)
+        worst = max(worst, err)
+    assert worst <= LOGIT_TOL, worst
+    return worst
+
+
+def test_tiny_config_logits(tqm):
+    # 4096 fp32 keys with outlier channels, 16 fp32 queries on one KV head.
+    K, Q, _ = synth.tiny_keys()
+    d, bits, m, pt = 128, 3, 128, 64
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, 1)
+    keys = K.astype(np.float64)[None, None]
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, lay, keys, [4096], pt, 21)
+    q = Q.astype(np.float64)[None]
+    ctx = torch.tensor([4096], dtype=torch.int32, device="cuda")
+    L = tqm.logits(cb, cache, _q_tensor(q, "f32"), ctx, 4096)
+    torch.cuda.synchronize()
+    _check_logits(codec, q, encs, L.cpu().numpy(), [4096], 1, 16)
+    assert cache.errors() == 0
+
+
+@pytest.mark.parametrize("d,bits,m,G,dtype", [
+    (128, 3, 128, 4, "bf16"), (128, 2, 128, 4, "bf16"), (128, 4, 128, 4, "f16"),
+    (128, 1, 128, 2, "f32"), (128, 3, 0, 4, "bf16"), (64, 3, 64, 5, "bf16"),
+    (200, 2, 200, 3, "f32"), (256, 4, 256, 8, "bf16"), (192, 3, 192, 1, "bf16"),
+])
+def test_logits_ragged_context(tqm, d, bits, m, G, dtype):
+    batch, heads, pt = 2, 2, 32
+    ctx = [1000, 333]
+    rng = np.random.default_rng(22)
+    keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-2, 2, size=(1, heads, 1, d)))
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, lay, keys, ctx, pt, 23)
+    qf = rng.standard_normal((batch, heads * G, d)).astype(np.float32)
+    if dtype == "bf16":
+        _, q = synth.to_bf16(qf)
+    elif dtype == "f16":
+        q = qf.astype(np.float16).astype(np.float64)
+    else:
+        q = qf.astype(np.float64)
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    out = torch.full((batch, heads * G, max(ctx)), float("nan"), device="cuda")
+    tqm.logits(cb, cache, _q_tensor(q, dtype), ctx_t, max(ctx), out=out)
+    torch.cuda.synchronize()
+    L = out.cpu().numpy()
+    _check_logits(codec, q, encs, L, ctx, heads, G)
+    assert np.all(np.isnan(L[1, :, ctx[1]:]))          # positions past ctx_len untouched
+    assert cache.errors() == 0
+
+
+def test_logits_decode_config_full_size(tqm):
+    # batch 1, 8 KV heads / 32 query heads, d = 128, context 32768, bf16 keys
+    # with per-channel log-uniform scales; b = 3 + QJL m = 128.
+    batch, hkv, hq, ctx, d, pt = 1, 8, 32, 32768, 128, 64
+    data = synth.decode_step(1002, batch, hkv, hq, ctx, d)
+    codec = O.make_codec(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, 3, 128, pt, hkv)
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, lay, data["k"][1], [ctx], pt, 24)
+    qbits, q = data["q"]
+    qt = torch.from_numpy(qbits.view(np.int16)).view(torch.bfloat16).cuda()
+    L = tqm.logits(cb, cache, qt, torch.tensor([ctx], dtype=torch.int32, device="cuda"), ctx)
+    torch.cuda.synchronize()
+    _check_logits(codec, q, encs, L.cpu().numpy(), [ctx], hkv, hq // hkv)
+
+
+def test_logits_empty_context(tqm):
+    cb = tqm.Codebook(128, 3, 128, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, 1, 64, 1, torch.zeros(2, 1, dtype=torch.int32))
+    q = torch.ones(2, 4, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.full((2, 4, 64), 7.0, device="cuda")
+    tqm.logits(cb, cache, q, torch.tensor([0, 0], dtype=torch.int32, device="cuda"), 64, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+@pytest.mark.parametrize("d,bits", [(128, 3), (128, 2), (200, 4), (64, 1)])
+def test_values_mode_a_and_b(tqm, d, bits):
+    batch, heads, G, pt = 2, 2, 4, 64
+    ctx = [700, 129]
+    rng = np.random.default_rng(31)
+    vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
+    codec = O.make_codec(d, bits, 0, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, 0, pt, heads)
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, lay, vals, ctx, pt, 32)
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    # mode A
+    outA = tqm.dequant_values(cb, cache, ctx_t, max(ctx), batch)
+    # mode B
+    W = synth.softmax_like_weights(33, batch, heads * G, max(ctx))
+    outB = tqm.dequant_values(cb, cache, ctx_t, max(ctx), batch, weights=torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    A = outA.cpu().numpy()
+    B = outB.cpu().numpy()
+    for (b, h), (pos, enc) in encs.items():
+        Vh = O.dequantize(codec, enc.idx, enc.norm16)
+        err = np.abs(A[b, h, : ctx[b]] - Vh)
+        assert np.all(err <= VALUE_TOL * np.max(np.abs(Vh), axis=1, keepdims=True) + 1e-30)
+        assert not A[b, h, ctx[b]:].any()
+        Wg = W[b, h * G:(h + 1) * G, : ctx[b]].astype(np.float64)
+        o = Wg @ Vh
+        scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
+        assert np.all(np.abs(B[b, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None])
+    assert cache.errors() == 0

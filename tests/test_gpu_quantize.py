@@ -1,0 +1,149 @@
+"""GPU parity of tq_quantize_append against the fp64 oracle (through the C ABI).
+
+Inputs come from kv_cache_vector_rotate_b200.synth; expected values only from
+oracle/.  Tolerances are those of tests/parity.py.
+"""
+
+import numpy as np
+import pytest
+
+from kv_cache_vector_rotate_b200 import synth
+from oracle import tq_oracle as O
+from parity import compare_codes
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _dev_tensor(bits_or_vals, dtype):
+    if dtype == "bf16":
+        return torch.from_numpy(bits_or_vals.view(np.int16)).view(torch.bfloat16).cuda()
+    if dtype == "f16":
+        return torch.from_numpy(bits_or_vals.astype(np.float16)).cuda()
+    return torch.from_numpy(bits_or_vals.astype(np.float32)).cuda()
+
+
+def _run_append(tqm, d, bits, m, x_dev, start_pos, n_pages, page_tokens, bt, cb=None):
+    cb = cb or tqm.Codebook(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, n_pages, page_tokens, x_dev.shape[1], torch.from_numpy(bt))
+    tqm.quantize_append(cb, x_dev, torch.tensor(start_pos, dtype=torch.int32, device="cuda"), cache)
+    torch.cuda.synchronize()
+    return cb, cache
+
+
+def _read_back(lay, cache, bt, b, h, pos):
+    pages = cache.pages.cpu().numpy()
+    return O.read_pages(lay, pages, bt, b, h, pos)
+
+
+@pytest.fixture(scope="module")
+def tqm():
+    from kv_cache_vector_rotate_b200 import tq as tqmod
+    tqmod.load_library()
+    return tqmod
+
+
+def test_tiny_config_fp32_with_outliers(tqm):
+    # d = 128, 4096 fp32 keys ~ N(0,1) with 4 outlier channels x20, b = 3 + QJL m = 128.
+    K, _, _ = synth.tiny_keys()
+    d, bits, m, pt = 128, 3, 128, 64
+    bt = synth.block_table(7, 1, 4096 // pt)
+    x = torch.from_numpy(K).cuda().view(1, 1, 4096, d)
+    cb, cache = _run_append(tqm, d, bits, m, x, [0], 4096 // pt, pt, bt)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, 1)
+    idx, qneg, n16, r16 = _read_back(lay, cache, bt, 0, 0, np.arange(4096))
+    ora = O.encode(codec, K.astype(np.float64))
+    stats = compare_codes(codec, K.astype(np.float64), ora, idx, qneg, n16, r16)
+    assert cache.errors() == 0
+    print(stats)
+
+
+@pytest.mark.parametrize("d,bits,m,dtype", [
+    (128, 2, 128, "bf16"), (128, 4, 128, "f16"), (128, 3, 0, "bf16"), (128, 1, 128, "f32"),
+    (64, 3, 64, "bf16"), (200, 2, 200, "bf16"), (256, 3, 256, "f32"), (96, 4, 0, "bf16"),
+    (192, 3, 192, "bf16"),
+])
+def test_shapes_bits_dtypes_ragged_midpage(tqm, d, bits, m, dtype):
+    batch, heads, n_new, pt = 2, 3, 101, 32
+    start = [5, 70]                      # appends that begin inside a page
+    pages_per_seq = (max(start) + n_new + pt - 1) // pt
+    bt = synth.block_table(11, batch, pages_per_seq)
+    rng = np.random.default_rng(12)
+    xf = rng.standard_normal((batch, heads, n_new, d)).astype(np.float32) * 3.0
+    if dtype == "bf16":
+        bits16, vals = synth.to_bf16(xf)
+        x = _dev_tensor(bits16, "bf16")
+    elif dtype == "f16":
+        vals = xf.astype(np.float16).astype(np.float64)
+        x = _dev_tensor(vals, "f16")
+    else:
+        vals = xf.astype(np.float64)
+        x = _dev_tensor(vals, "f32")
+    cb, cache = _run_append(tqm, d, bits, m, x, start, batch * pages_per_seq, pt, bt)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    for b in range(batch):
+        for h in range(heads):
+            pos = start[b] + np.arange(n_new)
+            idx, qneg, n16, r16 = _read_back(lay, cache, bt, b, h, pos)
+            X = vals[b, h]
+            compare_codes(codec, X, O.encode(codec, X), idx, qneg, n16, r16)
+    # slots before the start positions were never written
+    pages = cache.pages.cpu().numpy()
+    rec, nrm = O.token_offsets(lay, bt, 1, 0, np.arange(start[1]))
+    assert not pages[rec[:, None] + np.arange(lay.code_bytes)[None, :]].any()
+    assert cache.errors() == 0
+
+
+def test_two_appends_equal_one(tqm):
+    d, bits, m, pt = 128, 3, 128, 64
+    rng = np.random.default_rng(13)
+    bits16, vals = synth.to_bf16(rng.standard_normal((1, 2, 127, d)).astype(np.float32))
+    bt = synth.block_table(14, 1, 2)
+    x = _dev_tensor(bits16, "bf16")
+    cb, one = _run_append(tqm, d, bits, m, x, [0], 2, pt, bt)
+    two = tqm.PagedCache.allocate(cb, 2, pt, 2, torch.from_numpy(bt))
+    tqm.quantize_append(cb, x[:, :, :37].contiguous(), torch.tensor([0], dtype=torch.int32, device="cuda"), two)
+    tqm.quantize_append(cb, x[:, :, 37:].contiguous(), torch.tensor([37], dtype=torch.int32, device="cuda"), two)
+    torch.cuda.synchronize()
+    assert torch.equal(one.pages, two.pages)
+
+
+def test_zero_vectors_and_norm_overflow(tqm):
+    d, bits, m, pt = 128, 3, 128, 16
+    x = np.zeros((1, 1, 32, d), np.float32)
+    x[0, 0, 1, 3] = 1.0
+    x[0, 0, 2, :] = 7000.0        # ||x|| = 79195 > 65504: stored as +inf, error bit set
+    bt = np.arange(2, dtype=np.int32).reshape(1, 2)
+    cb, cache = _run_append(tqm, d, bits, m, torch.from_numpy(x).cuda(), [0], 2, pt, bt)
+    lay = O.Layout(d, bits, m, pt, 1)
+    idx, qneg, n16, r16 = _read_back(lay, cache, bt, 0, 0, np.arange(32))
+    assert np.all(idx[0] == 4) and float(n16[0]) == 0.0
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    ora = O.encode(codec, x[0, 0].astype(np.float64))
+    assert np.array_equal(idx[0], ora.idx[0])
+    assert np.isinf(n16[2])
+    assert cache.errors() & tqm.DEV_ERR_RANGE
+
+
+def test_out_of_range_page_is_skipped_and_reported(tqm):
+    d, bits, m, pt = 128, 3, 128, 16
+    rng = np.random.default_rng(15)
+    x = torch.from_numpy(rng.standard_normal((1, 1, 48, d)).astype(np.float32)).cuda()
+    bt = np.array([[0, 99, 1]], dtype=np.int32)   # page 99 does not exist (3 pages)
+    cb, cache = _run_append(tqm, d, bits, m, x, [0], 3, pt, bt)
+    assert cache.errors() & tqm.DEV_ERR_PAGE
+    lay = O.Layout(d, bits, m, pt, 1)
+    pages = cache.pages.cpu().numpy().reshape(3, lay.page_bytes)
+    assert pages[0].any() and pages[1].any() and not pages[2].any()
+
+
+def test_empty_append_is_a_no_op(tqm):
+    cb = tqm.Codebook(128, 3, 128, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, 1, 64, 1, torch.zeros(1, 1, dtype=torch.int32))
+    x = torch.zeros(1, 1, 0, 128, dtype=torch.bfloat16, device="cuda")
+    tqm.quantize_append(cb, x, torch.zeros(1, dtype=torch.int32, device="cuda"), cache)
+    torch.cuda.synchronize()
+    assert not cache.pages.any()
