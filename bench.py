@@ -272,7 +272,7 @@ def run_ours(args):
     # warm-up (W steps) plus a short soak so the clock samples see the GPU under load
     for i in range(args.warmup):
         step(i % R)
-    t_end = time.time() + 1.0
+    t_end = time.time() + args.soak
     i = 0
     while time.time() < t_end:
         step(i % R)
@@ -407,6 +407,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of extra warm-up steps (clock samples)")
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
