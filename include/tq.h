@@ -173,6 +173,30 @@ tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
                     int64_t out_stride, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* tq_logits for callers that cannot allocate device memory where they call
+ * it (a serving loop whose memory is an arena carved up at start-up, a host
+ * framework or plugin interface that hands an operator no workspace, code
+ * that must not call cudaMalloc/cudaFree on its hot path because those can
+ * block or synchronize the device).  The paper has no counterpart: this is an
+ * interface variant, not a step of the method.  Arguments and results are
+ * those of tq_logits; the workspace comes from a file-scope device array of
+ * tq_logits_noalloc_scratch_bytes() = 1 MiB that every device loading the
+ * library holds until exit.  A request needing more than that
+ * (tq_logits_workspace_bytes() > 1 MiB) returns TQ_EINVAL with nothing
+ * launched.  Every call on a device shares the array, so calls that overlap
+ * on the GPU race; order them on one stream (or with events).  Each call
+ * rewrites all of the scratch it reads, so nothing needs clearing.  The first
+ * call on a device looks up the array's address (cudaGetSymbolAddress, with
+ * that device current); make it before any stream capture.  Allocates
+ * nothing. */
+tq_status tq_logits_noalloc(const tq_codebook* cb, const tq_cache* cache, const void* q,
+                            tq_dtype dtype, int64_t batch, int32_t n_q_heads,
+                            const int32_t* ctx_len, int64_t max_ctx, float* out,
+                            int64_t out_stride, void* stream);
+
+/* Size in bytes of the static scratch behind tq_logits_noalloc. */
+size_t tq_logits_noalloc_scratch_bytes(void);
+
 /* Workspace (device bytes) that tq_dequant_values needs for these sizes. */
 size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
                                  int32_t n_q_heads, int64_t max_ctx);

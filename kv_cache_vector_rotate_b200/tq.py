@@ -24,6 +24,7 @@ EXPORTS = (
     "tq_codebook_build", "tq_codebook_build_host", "tq_codebook_free", "tq_codebook_export",
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
+    "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes",
 )
 
 
@@ -77,6 +78,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_values_workspace_bytes": (sz, [vp, i64, i32, i32, i64]),
         "tq_dequant_values": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i64, i64, i32, vp, i64,
                                     vp, i32, i64, vp, sz, vp]),
+        "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
+        "tq_logits_noalloc_scratch_bytes": (sz, []),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_layout_version": (i32, []),
     }
@@ -247,4 +250,19 @@ def dequant_values(cb: Codebook, cache: PagedCache, ctx_len, max_ctx: int, batch
         cb.handle, ctypes.byref(cs), _ptr(weights), w_stride, batch, hq, _ptr(ctx_len), max_ctx,
         _ptr(out), _dtype_code(out), o_stride, _ptr(ws), 0 if ws is None else ws.numel(),
         _stream(stream)))
+    return out
+
+
+def logits_noalloc(cb: Codebook, cache: PagedCache, q, ctx_len, max_ctx: int, out=None, stream=None):
+    """tq_logits_noalloc: tq_logits with its scratch taken from the library's
+    static device array (for callers that cannot allocate device memory)."""
+    import torch
+    assert q.is_cuda and q.is_contiguous() and q.dim() == 3
+    b, hq, d = q.shape
+    if out is None:
+        out = torch.empty(b, hq, max_ctx, dtype=torch.float32, device=q.device)
+    cs = cache.struct()
+    _check(load_library().tq_logits_noalloc(cb.handle, ctypes.byref(cs), _ptr(q), _dtype_code(q), b, hq,
+                                             _ptr(ctx_len), max_ctx, _ptr(out), out.stride(1),
+                                             _stream(stream)))
     return out
