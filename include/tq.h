@@ -29,18 +29,21 @@
  *    out-of-range page is skipped (nothing read or written through it).
  *  - Shapes are row-major and contiguous unless a stride is given.
  *
- * Packed record layout (layout version 1)
+ * Packed record layout (layout version 3)
  * ---------------------------------------
  * d_pad = 64 ceil(d/64), m_pad = 64 ceil(m/64), E = d_pad/4, F = m_pad/4.
  * A record is 4 chunks; chunk t holds coordinates [tE, tE+E) and QJL rows
- * [tF, tF+F) as 32-bit words: sign words, magnitude words (b = 2, 3) or
- * nibble words (b = 4), then QJL words.  Level indices are stored as sign
- * (1 = negative centroid) and magnitude mu (distance from the middle of the
- * codebook); QJL bit = 1 where (S r)_i < 0.  Bit positions of the element at
- * local position l: sign/QJL word l/32 bit (l%32)/2 + 16(l%2); 1-bit
- * magnitude word l/32 bit 8(l%4) + (l%32)/4; 2-bit magnitude word l/16 bits
- * 8(l%4) + 2((l%16)/4) (+1); nibble word l/8 bits 4((l%8)/2 + 4(l%2)) (..+3).
- * Padding coordinates store zero bits.  A page holds page_tokens tokens of
+ * [tF, tF+F) as 32-bit words: index words, then ceil(F/32) QJL words.  The
+ * stored code of a coordinate is its level index for b <= 3 and the nibble
+ * neg << 3 | mu for b = 4 (idx >= 8: neg 0, mu = idx - 8; else neg 1,
+ * mu = 7 - idx).  Bit k of the code of local element l: b = 1: word l/32, bit
+ * 4(l%8) + (l%32)/8; b = 2: word l/16, bit 4(l%8) + 2((l%16)/8) + k; b = 3:
+ * groups of 32 elements in 3 words, element l' = l%32 of group g = l/32 at
+ * word 3g + l'/8, bit 4(l'%8) + k when l' < 24, else word 3g + k, bit
+ * 4(l' - 24) + 3 (a last group of 16 uses 2 words, word 3(E/32) + l'/8, bit
+ * 4(l'%8) + k); b = 4: word l/8, bit 4((l%8)/2 + 4(l%2)) + k.  QJL row l:
+ * QJL word l/32, bit 8(l%4) + (l%32)/4, set where (S r)_i < 0.
+ * Padding coordinates store code 0.  A page holds page_tokens tokens of
  * every KV head; a head block is page_tokens records followed by
  * page_tokens norm slots (fp16 ||x||, then fp16 ||r|| when m > 0), padded to
  * 16 bytes.  Token `pos` of sequence b, head h lives in page
@@ -102,7 +105,7 @@ typedef struct {
 
 /* A paged cache of packed records, owned by the caller.  pages: device,
  * n_pages * page_bytes bytes, 16-byte aligned.  block_table: device int32
- * [batch, max_pages_per_seq].  page_tokens: a multiple of 16, 16..256.
+ * [batch, max_pages_per_seq].  page_tokens: a power of two, 16..256.
  * error_word: device uint32 or NULL. */
 typedef struct {
   void* pages;

@@ -94,6 +94,35 @@ static void build_host_tables(tq_codebook* cb, const tq_params* p) {
   for (int i = 0; i < 8; ++i) cb->mag16[i] = 0;
   for (int i = 0; i < K; ++i) cb->cent16[i] = f64_to_f16_bits(cb->centroids[i]);
   for (int mu = 0; mu < H; ++mu) cb->mag16[mu] = cb->cent16[H + mu];
+  cb->table_exp = 0;
+  cb->int8_hi[0] = cb->int8_hi[1] = cb->int8_lo[0] = cb->int8_lo[1] = 0u;
+}
+
+// b <= 3: the smallest f for which every c16 level times 2^f is an integer
+// (the finest fp16 spacing among the levels), and the int8 slices of those
+// integers.  Fails when an integer would not fit 16 bits.
+static bool make_int8_tables(tq_codebook* cb) {
+  const int K = 1 << cb->lay.bits;
+  int f = -30;
+  for (int i = 0; i < K; ++i) {
+    const float c = f16_bits_to_float(cb->cent16[i]);
+    if (c == 0.0f) continue;
+    int e;
+    std::frexp(std::fabs((double)c), &e);            // |c| in [2^(e-1), 2^e)
+    const int spacing_exp = std::max(e - 1, -14) - 10;  // fp16 spacing at |c|
+    f = std::max(f, -spacing_exp);
+  }
+  for (int i = 0; i < K; ++i) {
+    const double v = std::ldexp((double)f16_bits_to_float(cb->cent16[i]), f);
+    if (v != std::nearbyint(v) || std::fabs(v) > 32639.0) return false;
+    const int iv = (int)v;
+    const int hi = (iv + 128) >> 8;
+    const int lo = iv - 256 * hi;
+    cb->int8_hi[i / 4] |= (uint32_t)(uint8_t)(int8_t)hi << (8 * (i % 4));
+    cb->int8_lo[i / 4] |= (uint32_t)(uint8_t)(int8_t)lo << (8 * (i % 4));
+  }
+  cb->table_exp = f;
+  return true;
 }
 
 static tq_status upload(tq_codebook* cb) {
@@ -101,23 +130,32 @@ static tq_status upload(tq_codebook* cb) {
   const int d = L.d, dp = L.d_pad, mp = L.m_pad, K = 1 << L.bits;
   auto al = [](size_t n) { return (n + 255) / 256 * 256; };
   const size_t sz_pi = al((size_t)dp * d * 4), sz_s = al((size_t)mp * d * 4 + 4),
-               sz_srot = al((size_t)mp * dp * 4 + 4), sz_b = al(16 * 4), sz_c = al(16 * 4),
+               sz_srott = al((size_t)dp * mp * 4 + 4), sz_b = al(16 * 4), sz_c = al(16 * 4),
                sz_pibf = al((size_t)2 * dp * dp * 2), sz_srbf = al((size_t)2 * mp * dp * 2 + 4);
-  const size_t total = sz_pi + sz_s + sz_srot + sz_b + sz_c + sz_pibf + sz_srbf;
+  const size_t sz_pit = al((size_t)d * dp * 4), sz_st = al((size_t)d * mp * 4 + 4);
+  const size_t total = sz_pi + sz_s + sz_srott + sz_b + sz_c + sz_pibf + sz_srbf + sz_pit + sz_st;
   std::vector<uint8_t> host(total, 0);
   size_t off = 0;
   auto take = [&](size_t n) { size_t o = off; off += n; return o; };
-  const size_t o_pi = take(sz_pi), o_s = take(sz_s), o_srot = take(sz_srot), o_b = take(sz_b),
-               o_c = take(sz_c), o_pibf = take(sz_pibf), o_srbf = take(sz_srbf);
+  const size_t o_pi = take(sz_pi), o_s = take(sz_s), o_srott = take(sz_srott), o_b = take(sz_b),
+               o_c = take(sz_c), o_pibf = take(sz_pibf), o_srbf = take(sz_srbf),
+               o_pit = take(sz_pit), o_st = take(sz_st);
   float* pi32 = reinterpret_cast<float*>(host.data() + o_pi);
   float* s32 = reinterpret_cast<float*>(host.data() + o_s);
-  float* srot32 = reinterpret_cast<float*>(host.data() + o_srot);
+  float* srott32 = reinterpret_cast<float*>(host.data() + o_srott);
   float* b32 = reinterpret_cast<float*>(host.data() + o_b);
   float* c32 = reinterpret_cast<float*>(host.data() + o_c);
   __nv_bfloat16* pibf = reinterpret_cast<__nv_bfloat16*>(host.data() + o_pibf);
   __nv_bfloat16* srbf = reinterpret_cast<__nv_bfloat16*>(host.data() + o_srbf);
+  float* pit32 = reinterpret_cast<float*>(host.data() + o_pit);
+  float* st32 = reinterpret_cast<float*>(host.data() + o_st);
   for (int j = 0; j < d; ++j)
-    for (int k = 0; k < d; ++k) pi32[(size_t)j * d + k] = (float)cb->pi[(size_t)j * d + k];
+    for (int k = 0; k < d; ++k) {
+      pi32[(size_t)j * d + k] = (float)cb->pi[(size_t)j * d + k];
+      pit32[(size_t)k * dp + j] = (float)cb->pi[(size_t)j * d + k];
+    }
+  for (int i = 0; i < L.m; ++i)
+    for (int k = 0; k < d; ++k) st32[(size_t)k * mp + i] = (float)cb->s[(size_t)i * d + k];
   for (int i = 0; i < L.m; ++i)
     for (int k = 0; k < d; ++k) s32[(size_t)i * d + k] = (float)cb->s[(size_t)i * d + k];
   // S_rot = S Pi^T: the residual is formed in the rotated space, and
@@ -126,7 +164,7 @@ static tq_status upload(tq_codebook* cb) {
     for (int j = 0; j < d; ++j) {
       double acc = 0.0;
       for (int k = 0; k < d; ++k) acc += cb->s[(size_t)i * d + k] * cb->pi[(size_t)j * d + k];
-      srot32[(size_t)i * dp + j] = (float)acc;
+      srott32[(size_t)j * mp + i] = (float)acc;
       const __nv_bfloat16 hi = __double2bfloat16(acc);
       srbf[(size_t)i * dp + j] = hi;
       srbf[(size_t)mp * dp + (size_t)i * dp + j] = __double2bfloat16(acc - (double)__bfloat162float(hi));
@@ -153,11 +191,13 @@ static tq_status upload(tq_codebook* cb) {
   cb->dev_block = dev;
   cb->pi32 = reinterpret_cast<float*>(base + o_pi);
   cb->s32 = reinterpret_cast<float*>(base + o_s);
-  cb->srot32 = reinterpret_cast<float*>(base + o_srot);
+  cb->srott32 = reinterpret_cast<float*>(base + o_srott);
   cb->bound32 = reinterpret_cast<float*>(base + o_b);
   cb->cent32 = reinterpret_cast<float*>(base + o_c);
   cb->pi_bf = reinterpret_cast<__nv_bfloat16*>(base + o_pibf);
   cb->srot_bf = reinterpret_cast<__nv_bfloat16*>(base + o_srbf);
+  cb->pit32 = reinterpret_cast<float*>(base + o_pit);
+  cb->st32 = reinterpret_cast<float*>(base + o_st);
   return TQ_OK;
 }
 
@@ -165,8 +205,8 @@ static tq_status make_view(const tq_codebook* cb, const tq_cache* c, CacheView* 
   if (!c) return fail(TQ_EINVAL, "cache is NULL");
   if (!c->pages || !c->block_table) return fail(TQ_EINVAL, "cache pages / block_table is NULL");
   if (!aligned(c->pages, 16)) return fail(TQ_EINVAL, "cache pages must be 16-byte aligned");
-  if (c->page_tokens < 16 || c->page_tokens > 256 || c->page_tokens % 16 != 0)
-    return fail(TQ_EINVAL, "page_tokens must be a multiple of 16 in [16, 256]");
+  if (c->page_tokens < 16 || c->page_tokens > 256 || (c->page_tokens & (c->page_tokens - 1)) != 0)
+    return fail(TQ_EINVAL, "page_tokens must be a power of two in [16, 256]");
   if (c->n_kv_heads < 1 || c->n_pages < 1 || c->max_pages_per_seq < 1)
     return fail(TQ_EINVAL, "cache sizes must be positive");
   v->pages = reinterpret_cast<uint8_t*>(c->pages);
@@ -217,6 +257,10 @@ static tq_status build_common(const tq_params* params, tq_codebook** out, bool d
   cb->device = -1;
   cb->dev_block = nullptr;
   build_host_tables(cb, params);
+  if (params->bits <= 3 && !make_int8_tables(cb)) {
+    delete cb;
+    return fail(TQ_EUNSUPPORTED, "codebook levels do not fit the 16-bit integer tables");
+  }
   if (device) {
     cudaError_t e = cudaGetDevice(&cb->device);
     if (e != cudaSuccess) {
@@ -262,8 +306,8 @@ tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s, doubl
 tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_heads,
                     tq_layout_info* info) {
   if (!cb || !info) return fail(TQ_EINVAL, "codebook / info is NULL");
-  if (page_tokens < 16 || page_tokens > 256 || page_tokens % 16 != 0 || n_kv_heads < 1)
-    return fail(TQ_EINVAL, "page_tokens must be a multiple of 16 in [16, 256], n_kv_heads >= 1");
+  if (page_tokens < 16 || page_tokens > 256 || (page_tokens & (page_tokens - 1)) != 0 || n_kv_heads < 1)
+    return fail(TQ_EINVAL, "page_tokens must be a power of two in [16, 256], n_kv_heads >= 1");
   const Layout& L = cb->lay;
   info->d_pad = L.d_pad;
   info->m_pad = L.m_pad;

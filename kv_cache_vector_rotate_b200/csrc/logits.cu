@@ -5,113 +5,204 @@
 //   L = ||k|| ( sum_j (Pi q)_j c16[idx_j] + sqrt(pi/2)/m ||r|| sum_i (S q)_i s_i )
 // evaluated from the indices and sign bits without dequantizing the key.
 //
-// Design.  The two sums are dot products of a decoded key row with the
-// query group that shares its KV head.  A warp takes 16 keys at a time, turns
-// each key's bits into fp16 operand registers (the centroid magnitudes come
-// out of a byte-permute of the magnitude table, the signs are OR-ed into bit
-// 15), and runs m16n8k16 tensor-core MMAs against the query group held as
-// fp16 hi + lo halves (4 queries x {hi, lo} = the 8 columns).  The operand
-// never leaves registers, so HBM traffic is the 68-byte records plus the
-// logits.  The per-coordinate fragment order is fixed by the record layout:
-// thread t of a quad owns chunk t, i.e. the bits it loads are exactly the
-// bits its A fragment needs.
+// Design.  Both sums are dot products of a decoded key row with the query
+// group that shares its KV head, so a warp takes 16 keys at a time and runs
+// them through the tensor cores with the key operand built in registers:
+//  * codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer of
+//    at most 16 bits for every level, so a key element is two int8 slices;
+//    eight stored codes form one byte-permute selector after a single mask,
+//    and two permutes of 8-byte tables give the high and low slices of four
+//    elements.  (Pi q) is quantized to 16-bit integers scaled by its largest
+//    entry, also as two int8 slices; the four slice products are accumulated
+//    exactly in int32 and combined in fp32.
+//  * codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
+//    levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
+//  * sign term: m16n8k32 int8 MMAs.  The stored sign bits are spread to 0/1
+//    bytes with one shift and mask per 4 bits; S q is quantized to 16-bit
+//    integers z, and sum_i s_i z_i = sum_i z_i - 2 sum_i beta_i z_i.
+// The operands never leave registers, so HBM traffic is the 68-byte records
+// plus the logits.  Thread t of a quad owns chunk t of every record: the bits
+// it loads are exactly the bits its fragments need.
 
 #include "tq_internal.cuh"
 
 namespace tqd {
 
 // ---- query preparation ------------------------------------------------------
-// Workspace: fragments uint2 [groups][qtiles][KS0 + KS1][32 lanes], then
-// inverse scales float [batch * n_q_heads][2].
+// Workspace: codebook fragments uint2 [gq][KC][32] (KC = E/8 int8 k-steps, or
+// E/4 fp16 k-steps for b = 4), QJL fragments uint2 [gq][F/8][32]
+// (gq = group x query tile), per-query scalars float4 [batch * n_q_heads] =
+// {codebook scale, QJL step, sum z, 0}.
+
+constexpr int kSliceMax = 32639;   // |z| bound: the high int8 slice stays in [-128, 127]
+constexpr int kPrepStageFloats = 16384;   // 64 KB of the matrix staged at a time
 
 struct PrepParams {
   const void* q;
   tq_dtype dtype;
-  int d, E, F;           // E, F: coordinates / QJL rows per chunk
+  int d, d_pad, m_pad, E, F;   // E, F: coordinates / QJL rows per chunk
   int n_q_heads, n_kv_heads, G, qtiles;
-  const float* pi32;     // [d_pad][d]
-  const float* s32;      // [m_pad][d]
-  float s_row_norm_max;
+  int cb_int8;           // codebook fragments as int8 slices (b <= 3) or fp16 hi/lo (b = 4)
+  float cb_unscale;      // 2^-f: c16 * 2^f are the integer table entries
+  const float* pit32;    // Pi^T [d][d_pad]
+  const float* st32;     // S^T  [d][m_pad]
   uint2* frag;
-  float* inv_scale;
+  uint2* qfrag;
+  float4* scal;
 };
 
-// One warp per (group, query tile, k-step) writes the 32 lane fragments of
-// that k-step, zeros included (padding rows and query slots past G), so the
-// workspace needs no clearing.  Lane (g, t) holds column g = 2 * query +
-// {0: hi, 1: lo} at rows t * Ep + 4 ks + {0, 1} (first register) and
-// {2, 3} (second register) of Pi q (codebook part) or S q (QJL part).
-// grid: (groups * qtiles, KS0 + KS1); block 32.
-__global__ void __launch_bounds__(32) prep_queries_kernel(PrepParams p) {
-  const int lane = threadIdx.x;
-  const int g = lane >> 2, t = lane & 3;
+// Writes the int8 slices of z into the fragment of MMA k-step l / 8: lane
+// (2 * query + slice) * 4 + t, register (l / 4) % 2, byte l % 4.
+__device__ __forceinline__ void put_slices(uint2* base, int Ep, int row, int query, int z) {
+  const int zh = (z + 128) >> 8;            // floor((z + 128) / 256)
+  const int zl = z - 256 * zh;              // in [-128, 127]
+  const int t = row / Ep, l = row % Ep;
+  const int kk = l / 8, hreg = (l >> 2) & 1, e = l & 3;
+  int8_t* fr = reinterpret_cast<int8_t*>(base + kk * 32);
+  fr[((2 * query) * 4 + t) * 8 + hreg * 4 + e] = (int8_t)zh;
+  fr[((2 * query + 1) * 4 + t) * 8 + hreg * 4 + e] = (int8_t)zl;
+}
+
+// Rotates and sketches each query once (TQ §How it works: the query is
+// pre-rotated once and reused over the whole context).  CTA (group x query
+// tile, part): part 0 computes every row of Pi q, part 1 every row of S q;
+// warp w handles query w of the tile, lane l rows l, l + 32, ...  The matrix
+// (Pi^T or S^T) streams through shared memory in 64 KB tiles with all copies
+// in flight at once.  Every fragment slot is written (zeros for padding rows
+// and for query slots past G), so the workspace needs no clearing.
+// grid: (groups * qtiles, 1 + (m_pad > 0)); block 128; dynamic smem 64 KB.
+__global__ void __launch_bounds__(128) prep_queries_kernel(PrepParams p) {
+  asm volatile("griddepcontrol.launch_dependents;");
+  extern __shared__ float4 prep_dyn[];
+  float* mt = reinterpret_cast<float*>(prep_dyn);
+  __shared__ float qs[4][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = blockIdx.x;
   const int gi = gq / p.qtiles, qt = gq % p.qtiles;
   const int b = gi / p.n_kv_heads, kv = gi % p.n_kv_heads;
-  const int KS0 = p.E / 4;
-  const int ksg = blockIdx.y;
-  const int part = ksg < KS0 ? 0 : 1;
-  const int ks = part == 0 ? ksg : ksg - KS0;
-  const int Ep = part == 0 ? p.E : p.F;
-  const int ql = qt * 4 + (g >> 1);
-  const int hl = g & 1;
   const int d = p.d;
-  uint32_t regs[2] = {0u, 0u};
-  if (ql < p.G) {
-    const int hq = kv * p.G + ql;
-    const int64_t qrow = (int64_t)b * p.n_q_heads + hq;
-    float n2 = 0.0f;
-    for (int k = 0; k < d; ++k) {
-      const float v = load_elem(p.q, qrow * d + k, p.dtype);
-      n2 = fmaf(v, v, n2);
-    }
-    // |(Pi q)_j| <= ||q|| and |(S q)_i| <= max_i ||S_i|| ||q||: a power-of-two
-    // scale puts every entry below 2^14, so the fp16 hi part cannot overflow
-    // and hi + lo keep about 22 significant bits.
-    const float qn = sqrtf(n2);
-    const float bound = part == 0 ? qn : qn * p.s_row_norm_max;
-    int e = 0;
-    if (bound > 0.0f) frexpf(bound, &e);
-    const float scale = ldexpf(1.0f, 14 - e);
-    if (t == 0 && ks == 0 && hl == 0) p.inv_scale[qrow * 2 + part] = 1.0f / scale;
-    const float* M = part == 0 ? p.pi32 : p.s32;
-    __half vals[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int i = t * Ep + 4 * ks + r;          // row of Pi (or S), padded rows are zero
-      const float* mr = M + (size_t)i * d;
-      float v = 0.0f;
-      for (int k = 0; k < d; ++k) v = fmaf(__ldg(mr + k), load_elem(p.q, qrow * d + k, p.dtype), v);
-      const float vs = v * scale;
-      const __half hi = __float2half_rn(vs);
-      vals[r] = hl == 0 ? hi : __float2half_rn(vs - __half2float(hi));
-    }
-    regs[0] = (uint32_t)__half_as_ushort(vals[0]) | ((uint32_t)__half_as_ushort(vals[1]) << 16);
-    regs[1] = (uint32_t)__half_as_ushort(vals[2]) | ((uint32_t)__half_as_ushort(vals[3]) << 16);
+  const int ql = qt * 4 + warp;
+  const bool valid = ql < p.G;
+  const int64_t qrow = (int64_t)b * p.n_q_heads + kv * p.G + (valid ? ql : 0);
+  float n2 = 0.0f;
+  for (int k = lane; k < d; k += 32) {
+    const float v = valid ? load_elem(p.q, qrow * d + k, p.dtype) : 0.0f;
+    qs[warp][k] = v;
+    n2 = fmaf(v, v, n2);
   }
-  const int KS = KS0 + p.F / 4;
-  p.frag[((int64_t)gq * KS + ksg) * 32 + lane] = make_uint2(regs[0], regs[1]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, o);
+  const float qn = sqrtf(n2);
+  const int part = blockIdx.y;
+  const int rows = part == 0 ? p.d_pad : p.m_pad;     // multiple of 64, <= 256
+  const float* Mt = part == 0 ? p.pit32 : p.st32;     // [d][rows]
+  const int tile = min(rows, (kPrepStageFloats / d) & ~31);
+
+  float v[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) v[r] = 0.0f;
+  for (int r0 = 0; r0 < rows; r0 += tile) {
+    const int tn = min(tile, rows - r0);
+    __syncthreads();                 // previous tile consumed (and qs complete)
+    const int n4 = d * tn / 4;
+    for (int e = threadIdx.x; e < n4; e += 128) {
+      const int k = e / (tn / 4), c4 = e % (tn / 4);
+      const unsigned dst = (unsigned)__cvta_generic_to_shared(mt + k * tn + 4 * c4);
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst),
+                   "l"(Mt + (size_t)k * rows + r0 + 4 * c4) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int row = 32 * r + lane;
+      if (row >= r0 && row < r0 + tn) {
+        float acc = 0.0f;
+#pragma unroll 8
+        for (int k = 0; k < d; ++k) acc = fmaf(mt[k * tn + row - r0], qs[warp][k], acc);
+        v[r] = acc;
+      }
+    }
+  }
+  const int nr = rows / 32;
+  if (part == 0 && !p.cb_int8) {
+    // fp16 hi + lo: a power of two puts every |(Pi q)_j| <= ||q|| below 2^14
+    int e = 0;
+    if (qn > 0.0f) frexpf(qn, &e);
+    const float scale = ldexpf(1.0f, 14 - e);
+    const int KS = p.E / 4;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r >= nr) break;
+      const int row = 32 * r + lane;
+      __half hi = __float2half_rn(0.0f), lo = hi;
+      if (valid) {
+        const float vs = v[r] * scale;
+        hi = __float2half_rn(vs);
+        lo = __float2half_rn(vs - __half2float(hi));
+      }
+      const int t = row / p.E, l = row % p.E;
+      __half* fr = reinterpret_cast<__half*>(p.frag + ((int64_t)gq * KS + l / 4) * 32);
+      const int half_idx = ((l >> 1) & 1) * 2 + (l & 1);
+      fr[((2 * warp) * 4 + t) * 4 + half_idx] = hi;       // column 2 * query: hi part
+      fr[((2 * warp + 1) * 4 + t) * 4 + half_idx] = lo;   // column 2 * query + 1: lo part
+    }
+    if (valid && lane == 0) p.scal[qrow].x = 1.0f / scale;
+    return;
+  }
+  // 16-bit fixed point scaled by the largest entry, as two int8 slices
+  float mx = 0.0f;
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+    if (r < nr) mx = fmaxf(mx, fabsf(v[r]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float step = mx > 0.0f ? mx / (float)kSliceMax : 0.0f;
+  const int Ep = part == 0 ? p.E : p.F;
+  const int ksteps = Ep / 8;
+  uint2* base = (part == 0 ? p.frag : p.qfrag) + (int64_t)gq * ksteps * 32;
+  int zsum = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    if (r >= nr) break;
+    int z = 0;
+    if (valid && step > 0.0f) z = max(-kSliceMax, min(kSliceMax, __float2int_rn(v[r] / step)));
+    zsum += z;
+    put_slices(base, Ep, 32 * r + lane, warp, z);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) zsum += __shfl_xor_sync(0xffffffffu, zsum, o);
+  if (valid && lane == 0) {
+    if (part == 0) {
+      p.scal[qrow].x = step * p.cb_unscale;
+    } else {
+      p.scal[qrow].y = step;
+      p.scal[qrow].z = (float)zsum;   // exact: |sum| < 2^24
+    }
+  }
 }
 
 // ---- logits ---------------------------------------------------------------------
 
 struct LogitsParams {
   tq::CacheView cv;
+  int page_shift;            // log2(page_tokens)
   const int32_t* ctx_len;
   int n_kv_heads, n_q_heads, G, qtiles;
   int keys_per_cta;
   int max_ctx;               // ctx_len values are clamped to [0, max_ctx]
   const uint2* frag;
-  const float* inv_scale;
+  const uint2* qfrag;
+  const float4* scal;
   float* out;
   int64_t out_stride;
-  uint32_t pool0, pool1;     // fp16 magnitude table for the byte permute (b <= 3)
-  uint32_t lo0, lo1, hi0, hi1;  // low / high bytes of the 8 magnitudes (b = 4)
+  uint32_t th0, th1, tl0, tl1;  // b <= 3: high / low int8 slices of c16 * 2^f, levels 0..7
+  uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
   float qjl_scale;
 };
 
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                         uint32_t a3, uint2 b) {
+__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint2 b) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
@@ -119,45 +210,55 @@ __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
 }
 
-// The two fp16 pairs (h = 0: elements 4ks, 4ks+1; h = 1: 4ks+2, 4ks+3) of
-// k-step ks of the codebook part, decoded from one chunk's words.
+__device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint2 b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+}
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint2 b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+}
+
+// Byte-permute selector of the codes of local elements 8 kk .. 8 kk + 7 of a
+// chunk (layout version 3, b <= 3): nibble i holds the code of element 8 kk + i.
 template <int BITS, int E>
-__device__ __forceinline__ void decode_index_pair(const uint32_t* w, int ks, const LogitsParams& p,
-                                                  uint32_t& h0, uint32_t& h1) {
-  constexpr int n_sign = BITS == 4 ? 0 : (E + 31) / 32;
-  if constexpr (BITS == 4) {
-    const uint32_t x = w[ks / 2] >> (8 * (ks % 2));
-    const uint32_t sel = (x & 0x77u) | ((x >> 8) & 0x7700u);
-    const uint32_t lo = prmt(p.lo0, p.lo1, sel);
-    const uint32_t hi = prmt(p.hi0, p.hi1, sel);
-    h0 = prmt(lo, hi, 0x6240u) | ((x << 12) & 0x80008000u);
-    h1 = prmt(lo, hi, 0x7351u) | ((x << 8) & 0x80008000u);
+__device__ __forceinline__ uint32_t code_selector(const uint32_t* w, int kk) {
+  if constexpr (BITS == 1) {
+    return (w[kk / 4] >> (kk % 4)) & 0x11111111u;
+  } else if constexpr (BITS == 2) {
+    return (w[kk / 2] >> (2 * (kk % 2))) & 0x33333333u;
   } else {
-    const uint32_t sw = w[ks / 8];
-    const int pi0 = 2 * (ks % 8);
-    const uint32_t s0 = (sw << (15 - pi0)) & 0x80008000u;
-    const uint32_t s1 = (sw << (14 - pi0)) & 0x80008000u;
-    uint32_t m0, m1;
-    if constexpr (BITS == 1) {
-      m0 = m1 = p.pool0;
-    } else {
-      uint32_t v;
-      if constexpr (BITS == 2) v = (w[n_sign + ks / 8] >> (ks % 8)) & 0x01010101u;
-      else v = (w[n_sign + ks / 4] >> (2 * (ks % 4))) & 0x03030303u;
-      const uint32_t sel = v * 0x22u + 0x10101010u;
-      m0 = prmt(p.pool0, p.pool1, sel);
-      m1 = prmt(p.pool0, p.pool1, sel >> 16);
+    constexpr int full = E / 32;          // complete 32-element groups
+    const int g = kk / 4, j = kk % 4;
+    if (g < full) {
+      if (j < 3) return w[3 * g + j] & 0x77777777u;
+      return ((w[3 * g] >> 3) & 0x11111111u) | ((w[3 * g + 1] >> 2) & 0x22222222u) |
+             ((w[3 * g + 2] >> 1) & 0x44444444u);
     }
-    h0 = m0 | s0;
-    h1 = m1 | s1;
+    return w[3 * full + (kk - 4 * full)] & 0x77777777u;
   }
 }
 
-// The +-1 fp16 pairs of k-step ks of the QJL part.
-__device__ __forceinline__ void decode_sign_pair(uint32_t qw, int ks, uint32_t& h0, uint32_t& h1) {
-  const int pi0 = 2 * (ks % 8);
-  h0 = 0x3C003C00u | ((qw << (15 - pi0)) & 0x80008000u);
-  h1 = 0x3C003C00u | ((qw << (14 - pi0)) & 0x80008000u);
+// b = 4: the two fp16 pairs (elements 4ks, 4ks+1 and 4ks+2, 4ks+3) of k-step
+// ks from the sign-magnitude nibbles (magnitude bytes by permute, sign ORed
+// into bit 15 of each half).
+__device__ __forceinline__ void decode_nibble_pair(const uint32_t* w, int ks, const LogitsParams& p,
+                                                   uint32_t& h0, uint32_t& h1) {
+  const uint32_t x = w[ks / 2] >> (8 * (ks % 2));
+  const uint32_t sel = (x & 0x77u) | ((x >> 8) & 0x7700u);
+  const uint32_t lo = prmt(p.lo0, p.lo1, sel);
+  const uint32_t hi = prmt(p.hi0, p.hi1, sel);
+  h0 = prmt(lo, hi, 0x6240u) | ((x << 12) & 0x80008000u);
+  h1 = prmt(lo, hi, 0x7351u) | ((x << 8) & 0x80008000u);
 }
 
 template <int W>
@@ -180,17 +281,69 @@ __device__ __forceinline__ void load_chunk(const uint8_t* src, uint32_t (&w)[W])
   }
 }
 
-// grid: (chunks of keys, batch * n_kv_heads, query tiles of 4); block 128.
-template <int BITS, int E, int F>
-__global__ void __launch_bounds__(128) logits_kernel(LogitsParams p) {
-  constexpr int KS0 = E / 4, KS1 = F / 4;
-  constexpr int n_sign = BITS == 4 ? 0 : (E + 31) / 32;
-  constexpr int n_mag = BITS == 2 ? (E + 31) / 32 : BITS == 3 ? E / 16 : 0;
-  constexpr int n_nib = BITS == 4 ? E / 8 : 0;
-  constexpr int q0 = n_sign + n_mag + n_nib;
-  constexpr int W = q0 + (F + 31) / 32;
+constexpr int kLogitsWarps = 8;     // warps per CTA
+constexpr int kPrefetch = 3;        // 16-key tiles in flight per warp
+constexpr int kCtaPages = 64;       // block-table entries staged per CTA
+
+// One warp's share of a 16-key tile: this thread's chunk of keys g and g+8,
+// and their norm slots.
+template <int W>
+struct KeyTile {
+  uint32_t wa[W], wb[W];
+  uint32_t na, nb;
+};
+
+template <int W, int NB>
+__device__ __forceinline__ void load_tile(KeyTile<W>& kt, const uint8_t* hb, int P, int slot, int g,
+                                          int t, bool va, bool vb) {
   constexpr int CB = 16 * W;
+  if (va) {
+    load_chunk<W>(hb + (slot + g) * CB + t * 4 * W, kt.wa);
+    const uint8_t* ns = hb + P * CB + (slot + g) * NB;
+    kt.na = NB == 4 ? __ldg(reinterpret_cast<const uint32_t*>(ns))
+                    : (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(ns));
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i) kt.wa[i] = 0u;
+    kt.na = 0u;
+  }
+  if (vb) {
+    load_chunk<W>(hb + (slot + g + 8) * CB + t * 4 * W, kt.wb);
+    const uint8_t* ns = hb + P * CB + (slot + g + 8) * NB;
+    kt.nb = NB == 4 ? __ldg(reinterpret_cast<const uint32_t*>(ns))
+                    : (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(ns));
+  } else {
+#pragma unroll
+    for (int i = 0; i < W; ++i) kt.wb[i] = 0u;
+    kt.nb = 0u;
+  }
+}
+
+__device__ __forceinline__ float lo_half(uint32_t v) {
+  return __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float hi_half(uint32_t v) {
+  return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+}
+
+// grid: (chunks of keys, batch * n_kv_heads, query tiles of 4); block 256.
+// Each warp walks the CTA's 16-key tiles with stride kLogitsWarps, keeping
+// kPrefetch tiles of 128-bit loads in flight.  The CTA's block-table entries
+// are staged in shared memory first, so a tile's loads never wait on a
+// dependent page-id load; page_tokens is a power of two, so page and slot
+// are a shift and a mask.  The query fragments are read only after
+// griddepcontrol.wait: the kernel may start while the query preparation
+// kernel (programmatic dependent launch) is still running.
+template <int BITS, int E, int F>
+__global__ void __launch_bounds__(kLogitsWarps * 32, E >= 64 ? 1 : 2) logits_kernel(LogitsParams p) {
+  constexpr bool kInt8 = BITS <= 3;
+  constexpr int KC = kInt8 ? E / 8 : E / 4;   // codebook MMA k-steps
+  constexpr int KQ = F / 8;                   // sign-term MMA k-steps
+  constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
+                   : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
+  constexpr int W = q0 + (F + 31) / 32;
   constexpr int NB = F > 0 ? 4 : 2;
+  __shared__ int64_t page_base[kCtaPages];   // byte offset of this head's block, -1 if bad
 
   const int gi = blockIdx.y;
   const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
@@ -201,83 +354,118 @@ __global__ void __launch_bounds__(128) logits_kernel(LogitsParams p) {
   const int k1 = min(k0 + p.keys_per_cta, ctx);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
+  const int ps = p.page_shift;
+  const int P = 1 << ps;
+  const int first_page = k0 >> ps;
+  const int n_pages = ((k1 - 1) >> ps) - first_page + 1;
+  for (int j = threadIdx.x; j < n_pages; j += blockDim.x) {
+    const int64_t page = p.cv.block_table[(int64_t)b * p.cv.max_pages + first_page + j];
+    int64_t off = -1;
+    if (page >= 0 && page < p.cv.n_pages) off = page * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes;
+    else report(p.cv.err, TQ_DEV_ERR_PAGE);
+    page_base[j] = off;
+  }
+  __syncthreads();
 
-  // query fragments of this group / query tile, kept in registers
-  uint2 bq[KS0 + KS1];
-  const uint2* fsrc = p.frag + ((int64_t)gi * p.qtiles + qt) * (KS0 + KS1) * 32 + lane;
+  const int n_tiles = (k1 - k0 + 15) >> 4;
+  const int n_my = warp < n_tiles ? (n_tiles - warp + kLogitsWarps - 1) / kLogitsWarps : 0;
+  auto issue = [&](KeyTile<W>& kt, int i) {
+    const int base = k0 + 16 * (warp + kLogitsWarps * i);
+    const int64_t off = page_base[(base >> ps) - first_page];
+    const bool ok = off >= 0;
+    load_tile<W, NB>(kt, p.cv.pages + (ok ? off : 0), P, base & (P - 1), g, t, ok && base + g < k1,
+                     ok && base + g + 8 < k1);
+  };
+
+  KeyTile<W> buf[kPrefetch];
 #pragma unroll
-  for (int ks = 0; ks < KS0 + KS1; ++ks) bq[ks] = fsrc[ks * 32];
+  for (int s = 0; s < kPrefetch; ++s)
+    if (s < n_my) issue(buf[s], s);
+
+  // the query fragments come from the preparation kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int gq = gi * p.qtiles + qt;
+  uint2 bq[KC];
+  const uint2* fsrc = p.frag + (int64_t)gq * KC * 32 + lane;
+#pragma unroll
+  for (int kk = 0; kk < KC; ++kk) bq[kk] = fsrc[kk * 32];
+  uint2 bz[KQ > 0 ? KQ : 1];
+  if constexpr (KQ > 0) {
+    const uint2* qsrc = p.qfrag + (int64_t)gq * KQ * 32 + lane;
+#pragma unroll
+    for (int kk = 0; kk < KQ; ++kk) bz[kk] = qsrc[kk * 32];
+  }
   const int qidx = qt * 4 + t;                  // this thread's query within the group
   const bool qvalid = qidx < p.G;
   const int hq = h * p.G + (qvalid ? qidx : 0);
-  const float inv0 = p.inv_scale[((int64_t)b * p.n_q_heads + hq) * 2];
-  const float inv1 = F > 0 ? p.inv_scale[((int64_t)b * p.n_q_heads + hq) * 2 + 1] : 0.0f;
+  const float4 sc = p.scal[(int64_t)b * p.n_q_heads + hq];
+  const float c0 = sc.x;
+  const float c1 = F > 0 ? p.qjl_scale * sc.y : 0.0f;
+  const float zsum = sc.z;
   float* orow = p.out + ((int64_t)b * p.n_q_heads + hq) * p.out_stride;
 
-  const int n_tiles = (k1 - k0 + 15) >> 4;
-  for (int tile = warp; tile < n_tiles; tile += 4) {
-    const int base = k0 + tile * 16;
-    const int64_t page = p.cv.block_table[(int64_t)b * p.cv.max_pages + base / p.cv.page_tokens];
-    if (page < 0 || page >= p.cv.n_pages) {
-      if (lane == 0) report(p.cv.err, TQ_DEV_ERR_PAGE);
-      continue;
-    }
-    const uint8_t* hb = p.cv.pages + page * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes;
-    const int slot = base % p.cv.page_tokens;
-    const int ra = base + g, rb = base + g + 8;
-    uint32_t wa[W], wb[W];
-    float kna = 0.f, rna = 0.f, knb = 0.f, rnb = 0.f;
-    if (ra < k1) {
-      load_chunk<W>(hb + (int64_t)(slot + g) * CB + t * 4 * W, wa);
-      const uint8_t* ns = hb + (int64_t)p.cv.page_tokens * CB + (int64_t)(slot + g) * NB;
-      if constexpr (F > 0) {
-        const __half2 nr = __ldg(reinterpret_cast<const __half2*>(ns));
-        kna = __low2float(nr); rna = __high2float(nr);
-      } else {
-        kna = __half2float(__ldg(reinterpret_cast<const __half*>(ns)));
+  for (int i0 = 0; i0 < n_my; i0 += kPrefetch) {
+#pragma unroll
+    for (int s = 0; s < kPrefetch; ++s) {
+      const int i = i0 + s;
+      if (i < n_my) {
+        const KeyTile<W> cur = buf[s];
+        if (i + kPrefetch < n_my) issue(buf[s], i + kPrefetch);
+        const int base = k0 + 16 * (warp + kLogitsWarps * i);
+        if (page_base[(base >> ps) - first_page] < 0) continue;
+        float la, lb;
+        if constexpr (kInt8) {
+          // codebook term: int8 slices of c16 * 2^f against those of (Pi q)
+          int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int kk = 0; kk < KC; ++kk) {
+            const uint32_t sa = code_selector<BITS, E>(cur.wa, kk);
+            const uint32_t sb = code_selector<BITS, E>(cur.wb, kk);
+            const uint32_t sa2 = sa >> 16, sb2 = sb >> 16;
+            mma_s8s8(ah, prmt(p.th0, p.th1, sa), prmt(p.th0, p.th1, sb), prmt(p.th0, p.th1, sa2),
+                     prmt(p.th0, p.th1, sb2), bq[kk]);
+            mma_s8s8(al, prmt(p.tl0, p.tl1, sa), prmt(p.tl0, p.tl1, sb), prmt(p.tl0, p.tl1, sa2),
+                     prmt(p.tl0, p.tl1, sb2), bq[kk]);
+          }
+          // columns 2t / 2t+1: high / low slice of query t
+          la = c0 * fmaf(65536.0f, (float)ah[0], fmaf(256.0f, (float)(ah[1] + al[0]), (float)al[1]));
+          lb = c0 * fmaf(65536.0f, (float)ah[2], fmaf(256.0f, (float)(ah[3] + al[2]), (float)al[3]));
+        } else {
+          float acc0[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int ks = 0; ks < KC; ++ks) {
+            uint32_t a0, a2, a1, a3;
+            decode_nibble_pair(cur.wa, ks, p, a0, a2);
+            decode_nibble_pair(cur.wb, ks, p, a1, a3);
+            mma_f16(acc0, a0, a1, a2, a3, bq[ks]);
+          }
+          // columns 2t (hi) and 2t+1 (lo) belong to query t of this tile
+          la = c0 * (acc0[0] + acc0[1]);
+          lb = c0 * (acc0[2] + acc0[3]);
+        }
+        if constexpr (F > 0) {
+          // sign term: 0/1 bytes of the sign bits against the int8 slices of z
+          int acc1[4] = {0, 0, 0, 0};
+#pragma unroll
+          for (int kk = 0; kk < KQ; ++kk) {
+            const uint32_t xa = cur.wa[q0 + kk / 4] >> (2 * (kk % 4));
+            const uint32_t xb = cur.wb[q0 + kk / 4] >> (2 * (kk % 4));
+            mma_u8s8(acc1, xa & 0x01010101u, xb & 0x01010101u, (xa >> 1) & 0x01010101u,
+                     (xb >> 1) & 0x01010101u, bz[kk]);
+          }
+          const float ta = zsum - 2.0f * (float)(256 * acc1[0] + acc1[1]);
+          const float tb = zsum - 2.0f * (float)(256 * acc1[2] + acc1[3]);
+          la = fmaf(c1 * hi_half(cur.na), ta, la);
+          lb = fmaf(c1 * hi_half(cur.nb), tb, lb);
+        }
+        la *= lo_half(cur.na);
+        lb *= lo_half(cur.nb);
+        const int ra = base + g, rb = ra + 8;
+        if (qvalid) {
+          if (ra < k1) __stcs(orow + ra, la);
+          if (rb < k1) __stcs(orow + rb, lb);
+        }
       }
-    } else {
-#pragma unroll
-      for (int i = 0; i < W; ++i) wa[i] = 0u;
-    }
-    if (rb < k1) {
-      load_chunk<W>(hb + (int64_t)(slot + g + 8) * CB + t * 4 * W, wb);
-      const uint8_t* ns = hb + (int64_t)p.cv.page_tokens * CB + (int64_t)(slot + g + 8) * NB;
-      if constexpr (F > 0) {
-        const __half2 nr = __ldg(reinterpret_cast<const __half2*>(ns));
-        knb = __low2float(nr); rnb = __high2float(nr);
-      } else {
-        knb = __half2float(__ldg(reinterpret_cast<const __half*>(ns)));
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < W; ++i) wb[i] = 0u;
-    }
-
-    float acc0[4] = {0.f, 0.f, 0.f, 0.f};
-    float acc1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ks = 0; ks < KS0; ++ks) {
-      uint32_t a0, a2, a1, a3;
-      decode_index_pair<BITS, E>(wa, ks, p, a0, a2);
-      decode_index_pair<BITS, E>(wb, ks, p, a1, a3);
-      mma16816(acc0, a0, a1, a2, a3, bq[ks]);
-    }
-    if constexpr (F > 0) {
-#pragma unroll
-      for (int ks = 0; ks < KS1; ++ks) {
-        uint32_t a0, a2, a1, a3;
-        decode_sign_pair(wa[q0 + ks / 8], ks, a0, a2);
-        decode_sign_pair(wb[q0 + ks / 8], ks, a1, a3);
-        mma16816(acc1, a0, a1, a2, a3, bq[KS0 + ks]);
-      }
-    }
-    // columns 2t (hi) and 2t+1 (lo) belong to query t of this tile
-    const float la = kna * fmaf(p.qjl_scale * rna * inv1, acc1[0] + acc1[1], inv0 * (acc0[0] + acc0[1]));
-    const float lb = knb * fmaf(p.qjl_scale * rnb * inv1, acc1[2] + acc1[3], inv0 * (acc0[2] + acc0[3]));
-    if (qvalid) {
-      if (ra < k1) orow[ra] = la;
-      if (rb < k1) orow[rb] = lb;
     }
   }
 }
@@ -286,16 +474,40 @@ __global__ void __launch_bounds__(128) logits_kernel(LogitsParams p) {
 
 namespace tq {
 
-size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
+struct LogitsWs {
+  size_t frag, qfrag, scal, total;
+};
+
+static int codebook_ksteps(const Layout& L) { return L.bits <= 3 ? L.E / 8 : L.E / 4; }
+
+static LogitsWs logits_ws_layout(const tq_codebook* cb, int64_t groups, int G, int64_t batch_heads) {
+  auto al = [](size_t n) { return (n + 255) / 256 * 256; };
   const int qtiles = (G + 3) / 4;
-  const size_t frag = (size_t)groups * qtiles * (cb->lay.E / 4 + cb->lay.F / 4) * 32 * sizeof(uint2);
-  const size_t inv = (size_t)groups * G * 2 * sizeof(float);
-  return ((frag + 255) / 256) * 256 + inv;
+  LogitsWs w;
+  w.frag = al((size_t)groups * qtiles * codebook_ksteps(cb->lay) * 32 * sizeof(uint2));
+  w.qfrag = al((size_t)groups * qtiles * (cb->lay.F / 8) * 32 * sizeof(uint2));
+  w.scal = al((size_t)batch_heads * sizeof(float4));
+  w.total = w.frag + w.qfrag + w.scal;
+  return w;
+}
+
+size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
+  return logits_ws_layout(cb, groups, G, groups * G).total;
 }
 
 template <int BITS, int E, int F>
 static void run_logits(const tqd::LogitsParams& p, dim3 grid, cudaStream_t st) {
-  tqd::logits_kernel<BITS, E, F><<<grid, 128, 0, st>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
 }
 
 template <int BITS>
@@ -311,8 +523,6 @@ static bool dispatch_logits(const Layout& L, const tqd::LogitsParams& p, dim3 gr
   return false;
 }
 
-static uint32_t pack2(uint16_t lo, uint16_t hi) { return (uint32_t)lo | ((uint32_t)hi << 16); }
-
 tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* q, tq_dtype dt,
                         int64_t batch, int n_q_heads, const int32_t* ctx_len, int64_t max_ctx,
                         float* out, int64_t out_stride, void* ws, size_t ws_bytes,
@@ -321,32 +531,49 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   const int G = n_q_heads / cv.n_kv_heads;
   const int qtiles = (G + 3) / 4;
   const int64_t groups = batch * cv.n_kv_heads;
-  const size_t need = logits_workspace(cb, groups, G);
-  if (ws_bytes < need) return fail(TQ_EINVAL, "tq_logits: workspace too small");
+  const LogitsWs wl = logits_ws_layout(cb, groups, G, batch * n_q_heads);
+  if (ws_bytes < wl.total) return fail(TQ_EINVAL, "tq_logits: workspace too small");
   if (max_ctx == 0 || batch == 0) return TQ_OK;
-  const size_t frag_bytes = (size_t)groups * qtiles * (L.E / 4 + L.F / 4) * 32 * sizeof(uint2);
-  uint2* frag = reinterpret_cast<uint2*>(ws);
-  float* inv = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + ((frag_bytes + 255) / 256) * 256);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  uint2* frag = reinterpret_cast<uint2*>(wsb);
+  uint2* qfrag = reinterpret_cast<uint2*>(wsb + wl.frag);
+  float4* scal = reinterpret_cast<float4*>(wsb + wl.frag + wl.qfrag);
+
   tqd::PrepParams pp;
   pp.q = q;
   pp.dtype = dt;
   pp.d = L.d;
+  pp.d_pad = L.d_pad;
+  pp.m_pad = L.m_pad;
   pp.E = L.E;
   pp.F = L.F;
   pp.n_q_heads = n_q_heads;
   pp.n_kv_heads = cv.n_kv_heads;
   pp.G = G;
   pp.qtiles = qtiles;
-  pp.pi32 = cb->pi32;
-  pp.s32 = cb->s32;
-  pp.s_row_norm_max = (float)cb->s_row_norm_max;
+  pp.cb_int8 = L.bits <= 3 ? 1 : 0;
+  pp.cb_unscale = std::ldexp(1.0f, -cb->table_exp);
+  pp.pit32 = cb->pit32;
+  pp.st32 = cb->st32;
   pp.frag = frag;
-  pp.inv_scale = inv;
-  dim3 pgrid((unsigned)(groups * qtiles), (unsigned)(L.E / 4 + L.F / 4));
-  tqd::prep_queries_kernel<<<pgrid, 32, 0, st>>>(pp);
+  pp.qfrag = qfrag;
+  pp.scal = scal;
+  static bool prep_attr = false;
+  const int prep_smem = tqd::kPrepStageFloats * (int)sizeof(float);
+  if (!prep_attr) {
+    cudaError_t e = cudaFuncSetAttribute(tqd::prep_queries_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, prep_smem);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_logits: smem attribute");
+    prep_attr = true;
+  }
+  dim3 pgrid((unsigned)(groups * qtiles), (unsigned)(L.m_pad > 0 ? 2 : 1));
+  tqd::prep_queries_kernel<<<pgrid, 128, prep_smem, st>>>(pp);
 
   tqd::LogitsParams lp;
   lp.cv = cv;
+  int ps = 0;
+  while ((1 << ps) < cv.page_tokens) ++ps;
+  lp.page_shift = ps;
   lp.ctx_len = ctx_len;
   lp.n_kv_heads = cv.n_kv_heads;
   lp.n_q_heads = n_q_heads;
@@ -359,15 +586,22 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   int64_t kpc = (max_ctx + chunks - 1) / chunks;
   kpc = ((kpc + 63) / 64) * 64;
   if (kpc < 64) kpc = 64;
+  // a CTA stages at most kCtaPages block-table entries (its range may start
+  // inside a page, hence the 2 spare entries)
+  const int64_t kpc_cap = ((int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 64) * 64;
+  if (kpc > kpc_cap) kpc = kpc_cap;
   lp.keys_per_cta = (int)kpc;
   lp.max_ctx = (int)max_ctx;
   lp.frag = frag;
-  lp.inv_scale = inv;
+  lp.qfrag = qfrag;
+  lp.scal = scal;
   lp.out = out;
   lp.out_stride = out_stride;
+  lp.th0 = cb->int8_hi[0];
+  lp.th1 = cb->int8_hi[1];
+  lp.tl0 = cb->int8_lo[0];
+  lp.tl1 = cb->int8_lo[1];
   const uint16_t* M = cb->mag16;
-  lp.pool0 = L.bits == 1 ? pack2(M[0], M[0]) : L.bits == 2 ? pack2(M[0], M[1]) : pack2(M[0], M[1]);
-  lp.pool1 = L.bits == 3 ? pack2(M[2], M[3]) : 0u;
   lp.lo0 = lp.lo1 = lp.hi0 = lp.hi1 = 0u;
   if (L.bits == 4) {
     for (int i = 0; i < 4; ++i) {

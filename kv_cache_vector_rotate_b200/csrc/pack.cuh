@@ -1,5 +1,5 @@
-// Packing of one chunk of a record (layout version 1) and the paged-slot
-// address arithmetic, shared by the quantize kernels.
+// Record-chunk word counts (layout version 3) and the paged-slot address
+// arithmetic, shared by the quantize kernels.
 #pragma once
 
 #include "tq_internal.cuh"
@@ -9,42 +9,35 @@ namespace tqd {
 // Words of one chunk for BITS and E coordinates / F QJL rows per chunk.
 template <int BITS, int E, int F>
 struct ChunkWords {
-  static constexpr int n_sign = BITS == 4 ? 0 : (E + 31) / 32;
-  static constexpr int n_mag = BITS == 2 ? (E + 31) / 32 : BITS == 3 ? E / 16 : 0;
-  static constexpr int n_nib = BITS == 4 ? E / 8 : 0;
+  static constexpr int n_idx = BITS == 1 ? (E + 31) / 32
+                             : BITS == 2 ? E / 16
+                             : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16)
+                                         : E / 8;
   static constexpr int n_qjl = (F + 31) / 32;
-  static constexpr int W = n_sign + n_mag + n_nib + n_qjl;
-  static constexpr int q0 = n_sign + n_mag + n_nib;
+  static constexpr int W = n_idx + n_qjl;
+  static constexpr int q0 = n_idx;
 };
 
-// Adds element l with level index idx to the chunk words.  Callers unroll
-// their element loops so that l, and every shift below, is a constant.
-template <int BITS, int E, int F>
-__device__ __forceinline__ void pack_index(uint32_t* w, int l, int idx) {
-  using CW = ChunkWords<BITS, E, F>;
-  constexpr int H = 1 << (BITS - 1);
-  const uint32_t neg = idx < H ? 1u : 0u;
-  const uint32_t mu = neg ? (uint32_t)(H - 1 - idx) : (uint32_t)(idx - H);
-  if constexpr (BITS == 4) {
-    w[l / 8] |= ((neg << 3) | mu) << nib_bit(l);
-  } else {
-    w[l / 32] |= neg << sign_bit(l);
-    if constexpr (BITS == 2) w[CW::n_sign + l / 32] |= mu << mag1_bit(l);
-    if constexpr (BITS == 3) w[CW::n_sign + l / 16] |= mu << mag2_bit(l);
+// ORs the stored code of local element l (level index idx) into the chunk
+// words w (shared memory; several threads may target one word).
+template <int BITS, int E>
+__device__ __forceinline__ void or_code_bits(uint32_t* w, int l, int idx) {
+  const uint32_t code = stored_code<BITS>(idx);
+  if (BITS == 3 && l / 32 < E / 32 && l % 32 >= 24) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+      if ((code >> k) & 1u) atomicOr(w + code_word<BITS, E>(l, k), 1u << code_bit<BITS, E>(l, k));
+  } else if (code) {
+    atomicOr(w + code_word<BITS, E>(l, 0), code << code_bit<BITS, E>(l, 0));
   }
 }
 
-template <int BITS, int E, int F>
-__device__ __forceinline__ void pack_qjl(uint32_t* w, int l, bool negative) {
-  using CW = ChunkWords<BITS, E, F>;
-  w[CW::q0 + l / 32] |= (negative ? 1u : 0u) << sign_bit(l);
-}
-
 // Byte offset of the head block holding token `pos` of sequence b, head h,
-// or -1 (and an error bit) when the block-table entry is out of range.
+// or -1 (and an error bit) when the position is past the block table or the
+// block-table entry is out of range.
 __device__ __forceinline__ int64_t head_block_offset(const tq::CacheView& cv, int64_t b, int h,
                                                      int64_t pos) {
-  if (pos < 0 || pos >= cv.max_pages * cv.page_tokens) {   // past the block table
+  if (pos < 0 || pos >= cv.max_pages * cv.page_tokens) {
     report(cv.err, TQ_DEV_ERR_PAGE);
     return -1;
   }

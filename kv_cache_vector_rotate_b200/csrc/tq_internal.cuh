@@ -13,16 +13,24 @@
 
 namespace tq {
 
-constexpr int kLayoutVersion = 1;
+constexpr int kLayoutVersion = 3;
 
-// Sizes of the packed record format (layout version 1).
+// Sizes of the packed record format (layout version 3).
 struct Layout {
   int d, bits, m;
   int d_pad, m_pad;   // 64-multiples
   int E, F;           // coordinates / QJL rows per chunk
-  int n_sign, n_mag, n_nib, n_qjl, W;   // words per chunk
+  int n_idx, n_qjl, W;   // words per chunk
   int code_bytes, norm_bytes;
 
+  static int index_words(int bits, int E) {
+    switch (bits) {
+      case 1: return (E + 31) / 32;
+      case 2: return E / 16;
+      case 3: return 3 * (E / 32) + 2 * ((E % 32) / 16);
+      default: return E / 8;
+    }
+  }
   static Layout make(int d, int bits, int m) {
     Layout L{};
     L.d = d;
@@ -32,11 +40,9 @@ struct Layout {
     L.m_pad = m > 0 ? 64 * ((m + 63) / 64) : 0;
     L.E = L.d_pad / 4;
     L.F = L.m_pad / 4;
-    L.n_sign = bits == 4 ? 0 : (L.E + 31) / 32;
-    L.n_mag = bits == 2 ? (L.E + 31) / 32 : bits == 3 ? L.E / 16 : 0;
-    L.n_nib = bits == 4 ? L.E / 8 : 0;
+    L.n_idx = index_words(bits, L.E);
     L.n_qjl = (L.F + 31) / 32;
-    L.W = L.n_sign + L.n_mag + L.n_nib + L.n_qjl;
+    L.W = L.n_idx + L.n_qjl;
     L.code_bytes = 16 * L.W;
     L.norm_bytes = m > 0 ? 4 : 2;
     return L;
@@ -62,7 +68,9 @@ struct tq_codebook {
   void* dev_block;
   float* pi32;        // [d_pad][d]   Pi, rows >= d zero         (query rotation, v0 quantize)
   float* s32;         // [m_pad][d]   S, rows >= m zero           (query sketch)
-  float* srot32;      // [m_pad][d_pad] S Pi^T, zero padded        (residual sketch)
+  float* srott32;     // [d_pad][m_pad] (S Pi^T)^T, zero padded    (residual sketch, coalesced)
+  float* pit32;       // [d][d_pad]   Pi^T, columns >= d zero     (query rotation, coalesced)
+  float* st32;        // [d][m_pad]   S^T, columns >= m zero      (query sketch, coalesced)
   float* bound32;     // [2^b - 1]    boundaries (fp32)
   float* cent32;      // [2^b]        float(fp16(c))
   __nv_bfloat16* pi_bf;    // tensor-core operands: [2][d_pad][d_pad] hi, lo of Pi
@@ -70,6 +78,11 @@ struct tq_codebook {
   // fp16 bit patterns of the reconstruction magnitudes M[mu] = c16[H + mu]
   uint16_t mag16[8];
   uint16_t cent16[16];
+  // b <= 3: c16[i] * 2^table_exp is an integer v_i with |v_i| <= 32639, split
+  // into int8 slices v_i = 256 hi_i + lo_i (hi_i = floor((v_i + 128) / 256));
+  // the slices of levels 0..7 packed as bytes (int8_hi[0] = levels 0..3).
+  int table_exp;
+  uint32_t int8_hi[2], int8_lo[2];
 };
 
 namespace tq {
@@ -128,13 +141,47 @@ __device__ __forceinline__ float load_elem(const void* p, int64_t i, tq_dtype dt
   return __half2float(reinterpret_cast<const __half*>(p)[i]);
 }
 
-// Sign-word bit of local element l: word l/32, bit (l%32)/2 + 16 (l%2).
-__host__ __device__ constexpr int sign_bit(int l) { return (l % 32) / 2 + 16 * (l % 2); }
-// 1-bit magnitude (b = 2): word l/32, bit 8 (l%4) + (l%32)/4.
-__host__ __device__ constexpr int mag1_bit(int l) { return 8 * (l % 4) + (l % 32) / 4; }
-// 2-bit magnitude (b = 3): word l/16, bits p, p+1 with p = 8 (l%4) + 2 ((l%16)/4).
-__host__ __device__ constexpr int mag2_bit(int l) { return 8 * (l % 4) + 2 * ((l % 16) / 4); }
-// nibble (b = 4): word l/8, bits 4 ((l%8)/2 + 4 (l%2)).
-__host__ __device__ constexpr int nib_bit(int l) { return 4 * ((l % 8) / 2 + 4 * (l % 2)); }
+// Layout version 3.  Bit k of the stored code of local element l of a chunk
+// lives at index word code_word(l, k), bit code_bit(l, k).  The stored code is
+// the level index for b <= 3 and the sign-magnitude nibble neg << 3 | mu for
+// b = 4.  The b <= 3 positions make eight codes a byte-permute selector after
+// one mask (b = 1: >> (l%32)/8 & 0x11111111; b = 2: >> 2((l%16)/8) &
+// 0x33333333; b = 3: & 0x77777777, the last 8 of each group of 32 from the
+// top bits of the group's three words).
+template <int BITS, int E>
+__host__ __device__ constexpr int code_word(int l, int k) {
+  if (BITS == 1) return l / 32;
+  if (BITS == 2) return l / 16;
+  if (BITS == 3) {
+    const int g = l / 32, lp = l % 32;
+    if (g < E / 32) return lp < 24 ? 3 * g + lp / 8 : 3 * g + k;
+    return 3 * (E / 32) + lp / 8;
+  }
+  return l / 8;
+}
+template <int BITS, int E>
+__host__ __device__ constexpr int code_bit(int l, int k) {
+  if (BITS == 1) return 4 * (l % 8) + (l % 32) / 8;
+  if (BITS == 2) return 4 * (l % 8) + 2 * ((l % 16) / 8) + k;
+  if (BITS == 3) {
+    const int g = l / 32, lp = l % 32;
+    if (g < E / 32 && lp >= 24) return 4 * (lp - 24) + 3;
+    return 4 * (lp % 8) + k;
+  }
+  return 4 * ((l % 8) / 2 + 4 * (l % 2)) + k;
+}
+// Stored code of level index idx (b = 4: sign-magnitude nibble, H = 8).
+template <int BITS>
+__host__ __device__ constexpr uint32_t stored_code(int idx) {
+  if (BITS < 4) return (uint32_t)idx;
+  return idx < 8 ? (8u | (uint32_t)(7 - idx)) : (uint32_t)(idx - 8);
+}
+template <int BITS>
+__host__ __device__ constexpr int level_index(uint32_t code) {
+  if (BITS < 4) return (int)code;
+  return (code & 8u) ? 7 - (int)(code & 7u) : 8 + (int)(code & 7u);
+}
+// QJL-word bit of local row l: word l/32, bit 8 (l%4) + (l%32)/4.
+__host__ __device__ constexpr int qjl_bit(int l) { return 8 * (l % 4) + (l % 32) / 4; }
 
 }  // namespace tqd

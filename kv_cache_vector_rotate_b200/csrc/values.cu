@@ -32,23 +32,17 @@ struct ValuesParams {
   int max_ctx;              // ctx_len values are clamped to [0, max_ctx]
 };
 
-// Level index of local element l of a chunk.
+// Level index of local element l of a chunk (layout version 3).
 template <int BITS, int E>
 __device__ __forceinline__ int unpack_index(const uint32_t* w, int l) {
-  constexpr int H = 1 << (BITS - 1);
-  constexpr int n_sign = BITS == 4 ? 0 : (E + 31) / 32;
-  uint32_t neg, mu;
-  if constexpr (BITS == 4) {
-    const uint32_t nib = (w[l / 8] >> nib_bit(l)) & 15u;
-    neg = nib >> 3;
-    mu = nib & 7u;
+  uint32_t code = 0u;
+  if (BITS == 3 && l / 32 < E / 32 && l % 32 >= 24) {
+#pragma unroll
+    for (int k = 0; k < 3; ++k) code |= ((w[code_word<BITS, E>(l, k)] >> code_bit<BITS, E>(l, k)) & 1u) << k;
   } else {
-    neg = (w[l / 32] >> sign_bit(l)) & 1u;
-    if constexpr (BITS == 1) mu = 0u;
-    else if constexpr (BITS == 2) mu = (w[n_sign + l / 32] >> mag1_bit(l)) & 1u;
-    else mu = (w[n_sign + l / 16] >> mag2_bit(l)) & 3u;
+    code = (w[code_word<BITS, E>(l, 0)] >> code_bit<BITS, E>(l, 0)) & ((1u << BITS) - 1u);
   }
-  return neg ? (int)(H - 1 - mu) : (int)(H + mu);
+  return level_index<BITS>(code);
 }
 
 // Stages 16 tokens: cs[tok][j] = ||v|| c16[idx_j] (0 past the context or for

@@ -362,25 +362,27 @@ def exact_logits(Qv: np.ndarray, K: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Packed record layout, version 1 (the byte format the CUDA library reads and
+# Packed record layout, version 3 (the byte format the CUDA library reads and
 # writes; written here from its specification, independently of the library).
 #
 # d_pad = 64 ceil(d/64), m_pad = 64 ceil(m/64); E = d_pad/4, F = m_pad/4.
 # Coordinate j lives in chunk t = j // E at local position l = j % E;
 # projection i lives in chunk t = i // F at local position l = i % F.
-# A level index is stored sign-magnitude: with H = 2^(b-1), idx >= H gives
-# neg = 0, mu = idx - H; idx < H gives neg = 1, mu = H - 1 - idx.
-# Words of one chunk, in order (32-bit little endian):
-#   b <= 3: ceil(E/32) sign words, then magnitude words
-#           (b = 2: ceil(E/32) words of 1 bit, b = 3: E/16 words of 2 bits);
-#   b = 4 : E/8 nibble words (nibble = neg << 3 | mu);
-#   then ceil(F/32) QJL words (bit = 1 where (S r)_i < 0).
-# Bit positions of local element l:
-#   sign / QJL : word l//32, bit (l%32)//2 + 16 (l%2)
-#   mag, b = 2 : word l//32, bit 8 (l%4) + (l%32)//4
-#   mag, b = 3 : word l//16, bits p, p+1 with p = 8 (l%4) + 2 ((l%16)//4)
-#   nibble     : word l//8,  bits 4 ((l%8)//2 + 4 (l%2)) .. +3
-# Padding coordinates and projections store zero bits.
+# Words of one chunk (32-bit little endian): index words, then ceil(F/32) QJL
+# words (bit = 1 where (S r)_i < 0).  Stored code of an element: its level
+# index for b <= 3; for b = 4 the sign-magnitude nibble neg << 3 | mu (with
+# H = 8: idx >= H -> neg 0, mu = idx - H; idx < H -> neg 1, mu = H - 1 - idx).
+# Bit k of the code of local element l lives at (index word, bit):
+#   b = 1 : (l//32, 4 (l%8) + (l%32)//8)                       ceil(E/32) words
+#   b = 2 : (l//16, 4 (l%8) + 2 ((l%16)//8) + k)               E/16 words
+#   b = 3 : 32-element groups of 3 words; with g = l//32, l' = l%32:
+#           l' < 24 -> (3g + l'//8, 4 (l'%8) + k);
+#           l' >= 24 -> (3g + k, 4 (l' - 24) + 3);
+#           a last group of 16 (E % 32 == 16) takes 2 words:
+#           (3 (E//32) + l'//8, 4 (l'%8) + k)
+#   b = 4 : (l//8, 4 ((l%8)//2 + 4 (l%2)) + k)                E/8 words
+#   QJL   : row l at (l//32, 8 (l%4) + (l%32)//4) of the QJL words
+# Padding coordinates and projections store code 0 and sign bit 0.
 # A record is the 4 chunks back to back (CB = 16 W bytes).  A page holds P
 # tokens for each of n_kv_heads heads; a head block is P records followed by P
 # norm slots (fp16 ||x|| then, when m > 0, fp16 ||r||), padded to 16 bytes.
@@ -412,16 +414,9 @@ class Layout:
         return self.m_pad // 4
 
     @property
-    def n_sign(self) -> int:
-        return 0 if self.bits == 4 else (self.E + 31) // 32
-
-    @property
-    def n_mag(self) -> int:
-        return {1: 0, 2: (self.E + 31) // 32, 3: self.E // 16, 4: 0}[self.bits]
-
-    @property
-    def n_nib(self) -> int:
-        return self.E // 8 if self.bits == 4 else 0
+    def n_idx(self) -> int:
+        E = self.E
+        return {1: (E + 31) // 32, 2: E // 16, 3: 3 * (E // 32) + 2 * ((E % 32) // 16), 4: E // 8}[self.bits]
 
     @property
     def n_qjl(self) -> int:
@@ -429,7 +424,7 @@ class Layout:
 
     @property
     def words(self) -> int:
-        return self.n_sign + self.n_mag + self.n_nib + self.n_qjl
+        return self.n_idx + self.n_qjl
 
     @property
     def code_bytes(self) -> int:
@@ -449,41 +444,64 @@ class Layout:
         return self.n_kv_heads * self.head_block_bytes
 
 
-def _sign_mag(idx: np.ndarray, bits: int) -> tuple[np.ndarray, np.ndarray]:
-    H = 1 << (bits - 1)
+def code_bit_position(lay: Layout, l: int, k: int) -> tuple[int, int]:
+    """(index word, bit) of bit k of the stored code of local element l."""
+    E, b = lay.E, lay.bits
+    if b == 1:
+        return l // 32, 4 * (l % 8) + (l % 32) // 8
+    if b == 2:
+        return l // 16, 4 * (l % 8) + 2 * ((l % 16) // 8) + k
+    if b == 3:
+        g, lp = divmod(l, 32)
+        if g < E // 32:
+            if lp < 24:
+                return 3 * g + lp // 8, 4 * (lp % 8) + k
+            return 3 * g + k, 4 * (lp - 24) + 3
+        return 3 * (E // 32) + lp // 8, 4 * (lp % 8) + k
+    return l // 8, 4 * ((l % 8) // 2 + 4 * (l % 2)) + k
+
+
+def qjl_bit_position(l: int) -> tuple[int, int]:
+    """(QJL word, bit) of local projection row l."""
+    return l // 32, 8 * (l % 4) + (l % 32) // 4
+
+
+def _stored_code(idx: np.ndarray, bits: int) -> np.ndarray:
+    if bits < 4:
+        return idx.astype(np.uint64)
+    H = 8
     neg = idx < H
     mu = np.where(neg, H - 1 - idx, idx - H)
-    return neg.astype(np.uint64), mu.astype(np.uint64)
+    return ((neg.astype(np.uint64) << np.uint64(3)) | mu.astype(np.uint64))
+
+
+def _level_index(code: np.ndarray, bits: int) -> np.ndarray:
+    code = code.astype(np.int64)
+    if bits < 4:
+        return code
+    neg, mu = code >> 3, code & 7
+    return np.where(neg == 1, 7 - mu, 8 + mu)
 
 
 def pack_codes(lay: Layout, idx: np.ndarray, qneg: np.ndarray | None) -> np.ndarray:
     """[N, d] indices (+ [N, m] QJL bits) -> [N, 4, W] uint32 words."""
     N = idx.shape[0]
-    H = 1 << (lay.bits - 1)
-    full = np.full((N, lay.d_pad), H, dtype=np.int64)    # padding stores zero bits
+    full = np.zeros((N, lay.d_pad), dtype=np.int64)
     full[:, :lay.d] = idx
-    neg, mu = _sign_mag(full, lay.bits)
+    code = _stored_code(full, lay.bits)
+    code[:, lay.d:] = 0                       # padding stores code 0
     words = np.zeros((N, 4, lay.words), dtype=np.uint64)
+    one = np.uint64(1)
     for j in range(lay.d_pad):
         t, l = divmod(j, lay.E)
-        if lay.bits == 4:
-            w, p = l // 8, 4 * ((l % 8) // 2 + 4 * (l % 2))
-            words[:, t, w] |= ((neg[:, j] << np.uint64(3)) | mu[:, j]) << np.uint64(p)
-            continue
-        w, p = l // 32, (l % 32) // 2 + 16 * (l % 2)
-        words[:, t, w] |= neg[:, j] << np.uint64(p)
-        if lay.bits == 2:
-            w, p = lay.n_sign + l // 32, 8 * (l % 4) + (l % 32) // 4
-            words[:, t, w] |= mu[:, j] << np.uint64(p)
-        elif lay.bits == 3:
-            w, p = lay.n_sign + l // 16, 8 * (l % 4) + 2 * ((l % 16) // 4)
-            words[:, t, w] |= mu[:, j] << np.uint64(p)
+        for k in range(lay.bits):
+            w, p = code_bit_position(lay, l, k)
+            words[:, t, w] |= ((code[:, j] >> np.uint64(k)) & one) << np.uint64(p)
     if lay.m > 0:
-        q0 = lay.n_sign + lay.n_mag + lay.n_nib
         for i in range(lay.m):
             t, l = divmod(i, lay.F)
-            w, p = q0 + l // 32, (l % 32) // 2 + 16 * (l % 2)
-            words[:, t, w] |= qneg[:, i].astype(np.uint64) << np.uint64(p)
+            w, p = qjl_bit_position(l)
+            words[:, t, lay.n_idx + w] |= qneg[:, i].astype(np.uint64) << np.uint64(p)
     return words.astype(np.uint32)
 
 
@@ -491,37 +509,21 @@ def unpack_codes(lay: Layout, words: np.ndarray) -> tuple[np.ndarray, np.ndarray
     """Inverse of ``pack_codes``: [N, 4, W] uint32 -> ([N, d] idx, [N, m] qneg)."""
     w64 = words.astype(np.uint64)
     N = w64.shape[0]
-    H = 1 << (lay.bits - 1)
-    idx = np.zeros((N, lay.d), dtype=np.int64)
     one = np.uint64(1)
+    code = np.zeros((N, lay.d), dtype=np.uint64)
     for j in range(lay.d):
         t, l = divmod(j, lay.E)
-        if lay.bits == 4:
-            w, p = l // 8, 4 * ((l % 8) // 2 + 4 * (l % 2))
-            nib = (w64[:, t, w] >> np.uint64(p)) & np.uint64(15)
-            neg, mu = nib >> np.uint64(3), nib & np.uint64(7)
-        else:
-            w, p = l // 32, (l % 32) // 2 + 16 * (l % 2)
-            neg = (w64[:, t, w] >> np.uint64(p)) & one
-            if lay.bits == 1:
-                mu = np.zeros(N, dtype=np.uint64)
-            elif lay.bits == 2:
-                w, p = lay.n_sign + l // 32, 8 * (l % 4) + (l % 32) // 4
-                mu = (w64[:, t, w] >> np.uint64(p)) & one
-            else:
-                w, p = lay.n_sign + l // 16, 8 * (l % 4) + 2 * ((l % 16) // 4)
-                mu = (w64[:, t, w] >> np.uint64(p)) & np.uint64(3)
-        neg = neg.astype(np.int64)
-        mu = mu.astype(np.int64)
-        idx[:, j] = np.where(neg == 1, H - 1 - mu, H + mu)
+        for k in range(lay.bits):
+            w, p = code_bit_position(lay, l, k)
+            code[:, j] |= ((w64[:, t, w] >> np.uint64(p)) & one) << np.uint64(k)
+    idx = _level_index(code, lay.bits)
     qneg = None
     if lay.m > 0:
-        q0 = lay.n_sign + lay.n_mag + lay.n_nib
         qneg = np.zeros((N, lay.m), dtype=bool)
         for i in range(lay.m):
             t, l = divmod(i, lay.F)
-            w, p = q0 + l // 32, (l % 32) // 2 + 16 * (l % 2)
-            qneg[:, i] = ((w64[:, t, w] >> np.uint64(p)) & one) == one
+            w, p = qjl_bit_position(l)
+            qneg[:, i] = ((w64[:, t, lay.n_idx + w] >> np.uint64(p)) & one) == one
     return idx, qneg
 
 

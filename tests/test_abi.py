@@ -30,7 +30,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_layout_version():
-    assert tq.load_library().tq_layout_version() == 1
+    assert tq.load_library().tq_layout_version() == 3
 
 
 @pytest.mark.parametrize("d,bits,m", [(128, 3, 128), (128, 2, 128), (128, 4, 0), (64, 1, 64), (200, 4, 200)])
@@ -76,3 +76,12 @@ def test_host_only_codebook_refuses_kernels():
     st = lib.tq_quantize_append(cb.handle, None, 0, 1, 1, 1, None, ctypes.byref(cs), None)
     assert st == tq.TQ_EINVAL
     assert b"host-only" in lib.tq_last_error()
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3])
+def test_integer_codebook_tables_fit_for_every_supported_d(bits):
+    # The fused-logits kernel for b <= 3 needs every fp16 level times 2^f to be
+    # a 16-bit integer; building the codebook checks it and fails otherwise.
+    for d in range(8, 257, 8):
+        cb = tq.Codebook(d, bits, 0, 3, 4, device=False)
+        cb.close()

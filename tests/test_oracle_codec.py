@@ -215,40 +215,58 @@ def test_record_sizes():
 
 
 def test_layout_hand_worked_bits():
-    # d = 64, b = 3, m = 64: E = F = 16, one sign, one magnitude and one QJL
-    # word per chunk.  Hand-derived from the layout rules:
-    #  coordinate 5  -> chunk 0, l = 5: sign bit (5%32)//2 + 16 = 18,
-    #                   magnitude bits at 8*(5%4) + 2*((5%16)//4) = 10
-    #  idx 1 with H = 4 is neg = 1, mu = 2: sign word 1<<18, magnitude 2<<10.
-    #  coordinate 17 -> chunk 1, l = 1: sign bit 16, magnitude bits at 8.
-    #  idx 7 is neg = 0, mu = 3 -> magnitude word 3<<8.
-    #  projection 34 -> chunk 2, l = 2: bit 1; projection 63 -> chunk 3, l = 15: bit 23.
+    # d = 64, b = 3, m = 64: E = F = 16, so each chunk holds a trailing group of
+    # 16 elements in 2 index words (code bit k of element l at word l//8, bit
+    # 4 (l%8) + k) and one QJL word (row l at bit 8 (l%4) + (l%32)//4).
+    #  coordinate 5  -> chunk 0, l = 5: code 1 -> word 0 bit 20.
+    #  coordinate 17 -> chunk 1, l = 1: code 7 -> word 0 bits 4, 5, 6.
+    #  coordinate 26 -> chunk 1, l = 10: code 6 -> word 1 bits 9, 10.
+    #  projection 34 -> chunk 2, l = 2: bit 16; projection 63 -> chunk 3, l = 15: bit 27.
     lay = O.Layout(64, 3, 64, 64, 1)
-    idx = np.full((1, 64), 4)
+    assert lay.n_idx == 2 and lay.words == 3
+    idx = np.zeros((1, 64), dtype=np.int64)
     idx[0, 5] = 1
     idx[0, 17] = 7
+    idx[0, 26] = 6
     qneg = np.zeros((1, 64), bool)
     qneg[0, 34] = True
     qneg[0, 63] = True
     w = O.pack_codes(lay, idx, qneg)[0]
-    assert [int(v) for v in w[0]] == [1 << 18, 2 << 10, 0]
-    assert [int(v) for v in w[1]] == [0, 3 << 8, 0]
-    assert [int(v) for v in w[2]] == [0, 0, 1 << 1]
-    assert [int(v) for v in w[3]] == [0, 0, 1 << 23]
+    assert [int(v) for v in w[0]] == [1 << 20, 0, 0]
+    assert [int(v) for v in w[1]] == [0b111 << 4, 0b11 << 9, 0]
+    assert [int(v) for v in w[2]] == [0, 0, 1 << 16]
+    assert [int(v) for v in w[3]] == [0, 0, 1 << 27]
 
 
-def test_layout_hand_worked_bits_b2_b4():
-    # b = 2 (H = 2), d = 128: E = 32; coordinate 6 -> chunk 0, l = 6:
-    # sign bit 3 (l%32//2) + 0 = 3, magnitude bit 8*(6%4) + 6//4 = 17.
-    # idx 0 -> neg 1, mu 1.
-    lay = O.Layout(128, 2, 0, 64, 1)
-    idx = np.full((1, 128), 2)
-    idx[0, 6] = 0
+def test_layout_hand_worked_bits_dense_groups():
+    # b = 3, d = 128: E = 32, one full group of 3 words per chunk.
+    #  element 9  (l' = 9 < 24): code 5 -> word 1, bits 4 + {0, 2}.
+    #  element 26 (l' = 26 >= 24, e = 2): code 6 -> bit 1 in word 1 and bit 2
+    #  in word 2, both at bit 4 e + 3 = 11.
+    lay = O.Layout(128, 3, 0, 64, 1)
+    assert lay.n_idx == 3
+    idx = np.zeros((1, 128), dtype=np.int64)
+    idx[0, 9] = 5
+    idx[0, 26] = 6
     w = O.pack_codes(lay, idx, None)[0]
-    assert [int(v) for v in w[0]] == [1 << 3, 1 << 17]
-    # b = 4 (H = 8), d = 128: E = 32, nibble words of 8 elements;
-    # coordinate 37 -> chunk 1, l = 5: word 0, nibble 4*((5%8)//2 + 4*(5%2)) = 4*6 = 24.
-    # idx 2 -> neg 1, mu 5 -> nibble 0b1101.
+    assert [int(v) for v in w[0]] == [0, (1 << 4) | (1 << 6) | (1 << 11), 1 << 11]
+    # b = 2, d = 128: E = 32, 2 words; element 13 (l%16 = 13): code 2 ->
+    # word 0, bit 4 (13%8) + 2 (13//8) + 1 = 23.
+    lay = O.Layout(128, 2, 0, 64, 1)
+    idx = np.zeros((1, 128), dtype=np.int64)
+    idx[0, 13] = 2
+    idx[0, 32 + 20] = 3           # chunk 1, l = 20: word 1, bits 4*4 + 2*0 = 16, 17
+    w = O.pack_codes(lay, idx, None)[0]
+    assert [int(v) for v in w[0]] == [1 << 23, 0]
+    assert [int(v) for v in w[1]] == [0, 0b11 << 16]
+    # b = 1: element 11 (l%32 = 11): word 0, bit 4 (11%8) + 11//8 = 13.
+    lay = O.Layout(128, 1, 0, 64, 1)
+    idx = np.zeros((1, 128), dtype=np.int64)
+    idx[0, 11] = 1
+    assert [int(v) for v in O.pack_codes(lay, idx, None)[0, 0]] == [1 << 13]
+    # b = 4 (sign-magnitude nibbles, H = 8), d = 128: coordinate 37 -> chunk 1,
+    # l = 5: word 0, nibble at 4 ((5%8)//2 + 4 (5%2)) = 24; idx 2 -> neg 1,
+    # mu 5 -> nibble 0b1101.
     lay = O.Layout(128, 4, 0, 64, 1)
     idx = np.full((1, 128), 8)
     idx[0, 37] = 2
