@@ -15,9 +15,10 @@ different one of R cache replicas (R x 31 MB > the 126 MB L2), so the codes
 come from HBM.
 
 Headline metric: fused 3-bit logits HBM GB/s = algorithmic bytes of the
-logits call (68 B per key + 4 B per logit + the query) / its device time
-(CUDA events around each logits launch, summed over the timed steps, max
-over ranks).  Secondary: keys quantized/s of the append kernel on the
+logits call (68 B per key + 4 B per logit + the query) / its device time:
+CUDA events around a CUDA graph of K back-to-back logits calls (query
+preparation + fused logits, replicas rotated), max over ranks.  The timed
+region of the step itself is a graph of exactly K decode steps.  Secondary: keys quantized/s of the append kernel on the
 prefill-shaped batch (16 x 8 x 4096 bf16 keys).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -267,37 +268,58 @@ def run_ours(args):
         if ev is not None:
             ev[3].record()
 
-    clocks = ClockSampler(local)
-    clocks.start()
-    # warm-up (W steps) plus a short soak so the clock samples see the GPU under load
-    for i in range(args.warmup):
+    # warm-up: W eager steps (every replica is touched, kernels and attributes set up)
+    for i in range(max(args.warmup, R)):
         step(i % R)
-    t_end = time.time() + args.soak
-    i = 0
-    while time.time() < t_end:
-        step(i % R)
-        i += 1
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
-    _barrier(ws)
+    # The timed work runs as CUDA graphs: launching from Python through ctypes
+    # costs more per call than the GPU needs per call, so eager launches would
+    # time the host.  Graph `full` holds exactly K decode steps (step s reads
+    # replica s % R); the per-part graphs hold the same K calls of one part.
+    K = args.steps
+    parts = {
+        "full": lambda r: step(r),
+        "append": lambda r: (tq.quantize_append(kcb, knew, last, kc[r]), tq.quantize_append(vcb, vnew, last, vc[r])),
+        "logits": lambda r: tq.logits(kcb, kc[r], q, ctx_t, CTX, out=Lout, workspace=lws),
+        "values": lambda r: tq.dequant_values(vcb, vc[r], ctx_t, CTX, B, weights=W, out=Oout, workspace=vws),
+    }
+    graphs = {}
+    cap_stream = torch.cuda.Stream()
+    for name, fn in parts.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            for s_ in range(K):
+                fn(s_ % R)
+        graphs[name] = g
+    for g in graphs.values():
+        g.replay()
     torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for s in range(args.steps):
-        step(s % R, evs[s])
-    t1.record()
-    torch.cuda.synchronize()
-    _barrier(ws)
-    total_ms = t0.elapsed_time(t1)
-    app_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
-    log_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    val_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
-    total_ms = _max_over_ranks(total_ms, ws, dev)
-    log_ms = _max_over_ranks(log_ms, ws, dev)
-    val_ms = _max_over_ranks(val_ms, ws, dev)
-    app_ms = _max_over_ranks(app_ms, ws, dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    # soak so the clock samples see the GPU under load
+    t_end = time.time() + args.soak
+    while time.time() < t_end:
+        graphs["full"].replay()
+        torch.cuda.synchronize()
+
+    def timed(name):
+        _barrier(ws)
+        torch.cuda.synchronize()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record()
+        graphs[name].replay()
+        b_.record()
+        torch.cuda.synchronize()
+        _barrier(ws)
+        return _max_over_ranks(a_.elapsed_time(b_), ws, dev)
+
+    total_ms = timed("full")          # the timed region: exactly K steps
+    app_ms = timed("append")
+    log_ms = timed("logits")
+    val_ms = timed("values")
+    del graphs
 
     # e2e: the same step through host buffers (pinned), copies inside the region
     q_h = q.cpu().pin_memory()
@@ -327,6 +349,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(e0.elapsed_time(e1), ws, dev)
     clk = clocks.stop()
+    clk["window"] = "samples over the graph soak, the timed graphs and the e2e loop"
 
     # keys quantized/s on the prefill-shaped batch (16 x 8 x 4096 bf16 keys)
     kq = None
