@@ -169,7 +169,10 @@ size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n
  * with the query rotated once.  No 1/sqrt(d) scale, no softmax.  Positions
  * t >= ctx_len[b] are not written.  q: device [batch, n_q_heads, d] of dtype.
  * ctx_len: device int32 [batch], each <= max_ctx <= out_stride.  workspace:
- * device, at least tq_logits_workspace_bytes(), 16-byte aligned. */
+ * device, at least tq_logits_workspace_bytes(), 16-byte aligned (the rotated,
+ * sketched queries as tensor-core fragments).  Two kernel launches: the
+ * query preparation, then the logits kernel by programmatic dependent
+ * launch (it streams the cache while the queries are prepared). */
 tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
                     tq_dtype dtype, int64_t batch, int32_t n_q_heads,
                     const int32_t* ctx_len, int64_t max_ctx, float* out,
@@ -180,8 +183,8 @@ tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
  * it (a serving loop whose memory is an arena carved up at start-up, a host
  * framework or plugin interface that hands an operator no workspace, code
  * that must not call cudaMalloc/cudaFree on its hot path because those can
- * block or synchronize the device).  The paper has no counterpart: this is an
- * interface variant, not a step of the method.  Arguments and results are
+ * block or synchronize the device).  The method has no counterpart: this is
+ * an interface variant, not a step of the method.  Arguments and results are
  * those of tq_logits; the workspace comes from a file-scope device array of
  * tq_logits_noalloc_scratch_bytes() = 1 MiB that every device loading the
  * library holds until exit.  A request needing more than that

@@ -133,13 +133,15 @@ static tq_status upload(tq_codebook* cb) {
                sz_srott = al((size_t)dp * mp * 4 + 4), sz_b = al(16 * 4), sz_c = al(16 * 4),
                sz_pibf = al((size_t)2 * dp * dp * 2), sz_srbf = al((size_t)2 * mp * dp * 2 + 4);
   const size_t sz_pit = al((size_t)d * dp * 4), sz_st = al((size_t)d * mp * 4 + 4);
-  const size_t total = sz_pi + sz_s + sz_srott + sz_b + sz_c + sz_pibf + sz_srbf + sz_pit + sz_st;
+  const int R = dp + mp, d16 = (d + 15) / 16;
+  const size_t sz_qf = al((size_t)(R / 16) * d16 * 2 * 32 * 16);
+  const size_t total = sz_pi + sz_s + sz_srott + sz_b + sz_c + sz_pibf + sz_srbf + sz_pit + sz_st + sz_qf;
   std::vector<uint8_t> host(total, 0);
   size_t off = 0;
   auto take = [&](size_t n) { size_t o = off; off += n; return o; };
   const size_t o_pi = take(sz_pi), o_s = take(sz_s), o_srott = take(sz_srott), o_b = take(sz_b),
                o_c = take(sz_c), o_pibf = take(sz_pibf), o_srbf = take(sz_srbf),
-               o_pit = take(sz_pit), o_st = take(sz_st);
+               o_pit = take(sz_pit), o_st = take(sz_st), o_qf = take(sz_qf);
   float* pi32 = reinterpret_cast<float*>(host.data() + o_pi);
   float* s32 = reinterpret_cast<float*>(host.data() + o_s);
   float* srott32 = reinterpret_cast<float*>(host.data() + o_srott);
@@ -178,6 +180,37 @@ static tq_status upload(tq_codebook* cb) {
     }
   for (int i = 0; i < K - 1; ++i) b32[i] = (float)cb->boundaries[i];
   for (int i = 0; i < K; ++i) c32[i] = f16_bits_to_float(cb->cent16[i]);
+  // [Pi ; S] as bf16 hi + lo A fragments of mma.m16n8k16 (row-major A): lane
+  // (g, t) holds {A[g][2t], A[g][2t+1]}, {A[g+8][2t], ..}, {A[g][2t+8], ..},
+  // {A[g+8][2t+8], ..} of each 16 x 16 block, low half first.
+  {
+    uint32_t* qf = reinterpret_cast<uint32_t*>(host.data() + o_qf);
+    auto elem = [&](int r, int k) -> double {
+      if (k >= d) return 0.0;
+      if (r < dp) return r < d ? cb->pi[(size_t)r * d + k] : 0.0;
+      const int i = r - dp;
+      return i < L.m ? cb->s[(size_t)i * d + k] : 0.0;
+    };
+    auto bf_bits = [](double v) -> uint32_t {
+      const __nv_bfloat16 h = __double2bfloat16(v);
+      return (uint32_t)*reinterpret_cast<const uint16_t*>(&h);
+    };
+    auto part = [&](double v, int h) -> uint32_t {
+      const __nv_bfloat16 hi = __double2bfloat16(v);
+      return h == 0 ? bf_bits(v) : bf_bits(v - (double)__bfloat162float(hi));
+    };
+    for (int mt = 0; mt < R / 16; ++mt)
+      for (int j = 0; j < d16; ++j)
+        for (int h = 0; h < 2; ++h)
+          for (int lane = 0; lane < 32; ++lane) {
+            const int g = lane >> 2, t = lane & 3;
+            const int r0 = 16 * mt + g, k0 = 16 * j + 2 * t;
+            const int rr[4] = {r0, r0 + 8, r0, r0 + 8}, kk[4] = {k0, k0, k0 + 8, k0 + 8};
+            uint32_t* dst = qf + ((((size_t)mt * d16 + j) * 2 + h) * 32 + lane) * 4;
+            for (int x = 0; x < 4; ++x)
+              dst[x] = part(elem(rr[x], kk[x]), h) | (part(elem(rr[x], kk[x] + 1), h) << 16);
+          }
+  }
 
   void* dev = nullptr;
   cudaError_t e = cudaMalloc(&dev, total);
@@ -198,6 +231,7 @@ static tq_status upload(tq_codebook* cb) {
   cb->srot_bf = reinterpret_cast<__nv_bfloat16*>(base + o_srbf);
   cb->pit32 = reinterpret_cast<float*>(base + o_pit);
   cb->st32 = reinterpret_cast<float*>(base + o_st);
+  cb->qprep_frag = reinterpret_cast<uint4*>(base + o_qf);
   return TQ_OK;
 }
 

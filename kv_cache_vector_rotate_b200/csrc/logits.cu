@@ -5,274 +5,48 @@
 //   L = ||k|| ( sum_j (Pi q)_j c16[idx_j] + sqrt(pi/2)/m ||r|| sum_i (S q)_i s_i )
 // evaluated from the indices and sign bits without dequantizing the key.
 //
-// Design.  Both sums are dot products of a decoded key row with the query
-// group that shares its KV head, so a warp takes 16 keys at a time and runs
-// them through the tensor cores with the key operand built in registers:
-//  * codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer of
-//    at most 16 bits for every level, so a key element is two int8 slices;
-//    eight stored codes form one byte-permute selector after a single mask,
-//    and two permutes of 8-byte tables give the high and low slices of four
-//    elements.  (Pi q) is quantized to 16-bit integers scaled by its largest
-//    entry, also as two int8 slices; the slice products are accumulated
-//    exactly in int32 and combined at the end.
-//  * codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
-//    levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
-//  * sign term: m16n8k32 int8 MMAs.  The stored sign bits are spread to 0/1
-//    bytes with one shift and mask per 4 bits; S q is quantized to 16-bit
-//    integers z, and sum_i s_i z_i = sum_i z_i - 2 sum_i beta_i z_i.
-// The MMA's N = 8 columns are the high and low slices of 4 queries.
-//
 // Two kernels per call, chained by programmatic dependent launch:
-//  1. prep_queries_kernel: one thread-block cluster per (KV group, tile of 4
-//     queries); each CTA computes 32 (or 64) rows of [Pi q ; S q] for the 4
-//     queries, the CTAs exchange their partial maxima through distributed
-//     shared memory, and each writes its rows as MMA B-fragment bytes.
-//  2. logits_kernel: every warp owns a set of 16-key tiles and copies them
-//     (as many as its ring holds) into shared memory with cp.async before it
-//     waits for the query fragments, so the cache stream is in flight while
-//     the queries are prepared.  Thread t of an MMA quad owns chunk t of every
-//     record.
+//  * prep_queries_kernel: one thread-block cluster per (KV group, tile of 4
+//    query heads); each CTA computes its rows of [Pi q ; S q] on the tensor
+//    cores (bf16 hi + lo fragments of [Pi ; S], pre-swizzled in the
+//    codebook, times the bf16 hi + lo split of the queries, fp32
+//    accumulation), the CTAs exchange their per-query maxima through
+//    distributed shared memory, and each writes its rows as MMA B-fragment
+//    bytes to the workspace.
+//  * logits_kernel: every CTA owns an equal share of one sequence's keys;
+//    its warps stream 32-key units into shared-memory rings with bulk copies
+//    (the first ones in flight before the query fragments exist) and run them
+//    through the tensor cores with the key operand built in registers:
+//     - codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer
+//       of at most 16 bits for every level, so a key element is two int8
+//       slices; eight stored codes form one byte-permute selector after a
+//       single mask, and two permutes of 8-byte tables give the high and low
+//       slices of four elements.  (Pi q) is quantized to 16-bit integers
+//       scaled by its largest entry, also as two int8 slices; the slice
+//       products are accumulated exactly in int32 and combined at the end.
+//     - codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
+//       levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
+//     - sign term: m16n8k32 int8 MMAs.  The stored sign bits enter in place
+//       as 0 / 2^p bytes (one mask per operand register); S q is quantized to
+//       integers z, and sum_i s_i z_i = sum_i z_i - 2 sum_i beta_i z_i.
+//    The MMA's N = 8 columns are the high and low slices of 4 queries.
 // HBM traffic is the packed records plus the logits.
 
 #include "tq_internal.cuh"
 
 namespace tqd {
 
-// ---- query preparation ------------------------------------------------------
-// Workspace: codebook fragments uint2 [gq][KC][32] (KC = E/8 int8 k-steps, or
-// E/4 fp16 k-steps for b = 4), QJL fragments uint2 [gq][F/8][32]
-// (gq = group x query tile), per-query scalars float4 [batch * n_q_heads] =
-// {codebook scale, QJL step, 0, 0}.  Lane (2 * query + slice) * 4 + t of
-// an int8 fragment holds the slice (0 high, 1 low) of chunk t's elements.
-
-constexpr int kSliceMax = 32639;   // |z| bound: the high int8 slice stays in [-128, 127]
+constexpr int kSliceMax = 32639;   // |z| bound of Pi q: the high int8 slice stays in [-128, 127]
 constexpr int kSliceMaxQ = 16319;  // |z| bound of S q: 2 z still splits into int8 slices
-constexpr int kPrepThreads = 128;
-constexpr int kMaxClusterCtas = 8;
+constexpr int kLogitsWarps = 4;    // warps per CTA
+constexpr int kCtaPages = 64;      // block-table entries staged per CTA
+constexpr int kMaxCluster = 8;     // CTAs per cluster (portable limit)
 
-struct PrepParams {
-  const void* q;
-  tq_dtype dtype;
-  int d, d_pad, m_pad, E, F;   // E, F: coordinates / QJL rows per chunk
-  int n_q_heads, n_kv_heads, G, qtiles;
-  int cb_int8;           // codebook fragments as int8 slices (b <= 3) or fp16 hi/lo (b = 4)
-  float cb_unscale;      // 2^-f: c16 * 2^f are the integer table entries
-  const float* pi32;     // Pi [d_pad][d], rows >= d zero
-  const float* s32;      // S  [m_pad][d], rows >= m zero
-  uint2* frag;
-  uint2* qfrag;
-  float4* scal;
-};
+// CTAs resident per SM (65536 registers / (128 x this) per thread)
+__host__ __device__ constexpr int logits_min_blocks(int bits, int E) { return E >= 48 ? 4 : bits == 4 ? 4 : 5; }
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-// Stores v into the same shared variable of CTA `rank` of this cluster.
-__device__ __forceinline__ void st_cluster(const void* local, uint32_t rank, float v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote), "f"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster(const void* local, uint32_t rank, int v) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(remote), "r"(v) : "memory");
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() {
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
-// Sums 32 per-lane partial values across the warp so that lane l ends with
-// the total of value l (a butterfly that halves the values each round).
-__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool upper = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < o; ++i) {
-      const float send = upper ? v[i] : v[i + o];
-      const float keep = upper ? v[i + o] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-  return v[0];
-}
-
-// Rotates and sketches each query once (TQ §How it works: the query is
-// pre-rotated once and reused over the whole context).
-// grid: (nblk, groups * qtiles), cluster (nblk, 1, 1); CTA `rank` computes
-// rows [rank * RB, rank * RB + RB) of [Pi q ; S q] for the 4 queries of its
-// tile (RB = 4 * RPW rows; d_pad is a multiple of RB, so a block never
-// straddles Pi q / S q).  The block's RB x d matrix rows are copied into
-// shared memory with every cp.async in flight while the queries load.  Warp
-// w: rows w * RPW .. w * RPW + RPW - 1 of the block, lanes split the sum over
-// k.  The CTAs of the cluster exchange their per-query maxima through
-// distributed shared memory; every fragment byte of the tile is written
-// (zeros for padding rows and for query slots past G), so the workspace
-// needs no clearing.
-// QJL fragments: in the MMA k-step of rows 8 kk .. 8 kk + 7 of a chunk, the
-// slots of rows 8 kk .. 8 kk + 3 hold the slices of 2 z and those of rows
-// 8 kk + 4 .. 8 kk + 7 the slices of z (|z| <= kSliceMaxQ), matching the key
-// operand of the logits kernel, whose sign bytes there are 2^(2 kk) beta and
-// 2^(2 kk + 1) beta.
-template <int RPW>
-__global__ void __launch_bounds__(kPrepThreads) prep_queries_kernel(PrepParams p) {
-  asm volatile("griddepcontrol.launch_dependents;");
-  cluster_arrive_relaxed();          // phase 1: every CTA of the cluster has started
-  constexpr int RB = 4 * RPW;        // rows per CTA
-  extern __shared__ __align__(16) float mrows[];   // [RB][d]
-  __shared__ float qs[4][256];
-  __shared__ float qnorm2[4];
-  __shared__ float wred[4][4];
-  __shared__ float pmax[kMaxClusterCtas][4];   // partial maxima pushed by each rank
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rank = blockIdx.x, nblk = gridDim.x;
-  const int gq = blockIdx.y;
-  const int gi = gq / p.qtiles, qt = gq % p.qtiles;
-  const int b = gi / p.n_kv_heads, kv = gi % p.n_kv_heads;
-  const int d = p.d;
-  const int64_t qbase = (int64_t)b * p.n_q_heads + kv * p.G + qt * 4;   // first query row of the tile
-  const int nq = min(4, p.G - qt * 4);
-
-  const int row0 = rank * RB;
-  const bool sk = row0 >= p.d_pad;                 // this block holds S q rows
-  const int prow0 = sk ? row0 - p.d_pad : row0;    // first row within its part
-  {
-    const float4* src = reinterpret_cast<const float4*>((sk ? p.s32 : p.pi32) + (size_t)prow0 * d);
-    const uint32_t dst = smem_addr(mrows);
-    for (int c = threadIdx.x; c < RB * d / 4; c += kPrepThreads)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + 16 * c), "l"(src + c) : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  }
-  // the 4 queries of the tile (zeros for slots past G) and their squared norms
-  {
-    float s2 = 0.0f;
-    for (int k = lane; k < d; k += 32) {
-      const float x = warp < nq ? load_elem(p.q, (qbase + warp) * d + k, p.dtype) : 0.0f;
-      qs[warp][k] = x;
-      s2 = fmaf(x, x, s2);
-    }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-    if (lane == 0) qnorm2[warp] = s2;
-  }
-  asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
-
-  // val[h]: lane l holds row prow0 + w * RPW + 8 h + l / 4 of query slot l % 4
-  float val[RPW / 8];
-#pragma unroll
-  for (int h = 0; h < RPW / 8; ++h) {
-    float acc[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.0f;
-    const float* Mh = mrows + (warp * RPW + 8 * h) * d;
-    for (int k = lane; k < d; k += 32) {
-      const float x0 = qs[0][k], x1 = qs[1][k], x2 = qs[2][k], x3 = qs[3][k];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float m = Mh[j * d + k];
-        acc[4 * j] = fmaf(m, x0, acc[4 * j]);
-        acc[4 * j + 1] = fmaf(m, x1, acc[4 * j + 1]);
-        acc[4 * j + 2] = fmaf(m, x2, acc[4 * j + 2]);
-        acc[4 * j + 3] = fmaf(m, x3, acc[4 * j + 3]);
-      }
-    }
-    val[h] = reduce_scatter32(acc, lane);
-  }
-  const int qi = lane & 3;           // this lane's query slot
-
-  // partial max |v| of this block per query slot
-  float mx = 0.0f;
-#pragma unroll
-  for (int h = 0; h < RPW / 8; ++h) mx = fmaxf(mx, fabsf(val[h]));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-  if (lane < 4) wred[warp][lane] = mx;
-  __syncthreads();
-  cluster_wait();                    // phase 1 complete: the peers' shared memory exists
-  if (threadIdx.x < 4 * nblk) {
-    const int dst = threadIdx.x >> 2, qq = threadIdx.x & 3;
-    const float m4 = fmaxf(fmaxf(wred[0][qq], wred[1][qq]), fmaxf(wred[2][qq], wred[3][qq]));
-    st_cluster(&pmax[rank][qq], (uint32_t)dst, m4);
-  }
-  cluster_sync();                    // phase 2: every partial maximum delivered; no remote access after this
-
-  const int nb_pi = p.d_pad / RB;    // ranks [0, nb_pi) hold Pi q rows
-  float mpi = 0.0f, msk = 0.0f;
-  for (int r = 0; r < nblk; ++r) {
-    if (r < nb_pi) mpi = fmaxf(mpi, pmax[r][qi]);
-    else msk = fmaxf(msk, pmax[r][qi]);
-  }
-  int e2 = 0;                        // b = 4: 2^(14 - e2) puts |(Pi q)_j| <= ||q|| below 2^14
-  {
-    const float qn = sqrtf(qnorm2[qi]);
-    if (qn > 0.0f) frexpf(qn, &e2);
-  }
-  const float step = sk ? (msk > 0.0f ? msk / (float)kSliceMaxQ : 0.0f)
-                        : (mpi > 0.0f ? mpi / (float)kSliceMax : 0.0f);
-#pragma unroll
-  for (int h = 0; h < RPW / 8; ++h) {
-    const int l = prow0 + warp * RPW + 8 * h + (lane >> 2);   // row within its part
-    const float v = val[h];
-    if (!sk && !p.cb_int8) {
-      const float vs = v * ldexpf(1.0f, 14 - e2);
-      const __half hi = __float2half_rn(vs);
-      const __half lo = __float2half_rn(vs - __half2float(hi));
-      const int t = l / p.E, e4 = l % p.E;
-      __half* fr = reinterpret_cast<__half*>(p.frag + ((int64_t)gq * (p.E / 4) + e4 / 4) * 32);
-      const int half_idx = ((e4 >> 1) & 1) * 2 + (e4 & 1);
-      fr[((2 * qi) * 4 + t) * 4 + half_idx] = hi;
-      fr[((2 * qi + 1) * 4 + t) * 4 + half_idx] = lo;
-      continue;
-    }
-    const int Ep = sk ? p.F : p.E;
-    const int t = l / Ep, e = l % Ep;
-    const int kk = e / 8, hreg = (e >> 2) & 1, by = e & 3;
-    const int zmax = sk ? kSliceMaxQ : kSliceMax;
-    int z = 0;
-    if (step > 0.0f) z = max(-zmax, min(zmax, __float2int_rn(v / step)));
-    if (sk && hreg == 0) z *= 2;              // rows 8 kk .. 8 kk + 3: 2 z
-    const int zh = (z + 128) >> 8;            // floor((z + 128) / 256)
-    const int zl = z - 256 * zh;              // in [-128, 127]
-    int8_t* fr = reinterpret_cast<int8_t*>((sk ? p.qfrag : p.frag) + ((int64_t)gq * (Ep / 8) + kk) * 32);
-    fr[((2 * qi) * 4 + t) * 8 + hreg * 4 + by] = (int8_t)zh;
-    fr[((2 * qi + 1) * 4 + t) * 8 + hreg * 4 + by] = (int8_t)zl;
-  }
-  if (rank == 0 && threadIdx.x < nq) {
-    const int qq = threadIdx.x;
-    float m0 = 0.0f, m1 = 0.0f;
-    for (int r = 0; r < nblk; ++r) {
-      if (r < nb_pi) m0 = fmaxf(m0, pmax[r][qq]);
-      else m1 = fmaxf(m1, pmax[r][qq]);
-    }
-    float c0;
-    if (p.cb_int8) {
-      c0 = (m0 > 0.0f ? m0 / (float)kSliceMax : 0.0f) * p.cb_unscale;
-    } else {
-      int e = 0;
-      const float qn = sqrtf(qnorm2[qq]);
-      if (qn > 0.0f) frexpf(qn, &e);
-      c0 = ldexpf(1.0f, e - 14);
-    }
-    const float zstep = m1 > 0.0f ? m1 / (float)kSliceMaxQ : 0.0f;
-    p.scal[qbase + qq] = make_float4(c0, zstep, 0.0f, 0.0f);
-  }
-}
-
-// ---- logits ---------------------------------------------------------------------
-
-constexpr int kLogitsWarps = 4;     // warps per CTA
-constexpr int kLogitsMinBlocks = 6; // CTAs resident per SM (registers <= 80 per thread)
-constexpr int kCtaPages = 64;       // block-table entries staged per CTA
+// rows of [Pi q ; S q] per CTA of a query-preparation cluster: R / C with C <= 8
+__host__ __device__ constexpr int prep_rows_per_cta(int E, int F) { return 4 * (E + F) <= 256 ? 32 : 64; }
 
 // Per-warp shared-memory ring: a stage holds one 32-key unit, two 16-key
 // tiles of 16 consecutive records each (16 * 16W bytes, contiguous in its
@@ -289,17 +63,54 @@ struct LogitsParams {
   int page_shift;            // log2(page_tokens)
   const int32_t* ctx_len;
   int n_kv_heads, n_q_heads, G, qtiles;
-  int keys_per_cta;          // a multiple of 32
+  int n_chunks;              // CTAs per (group, query tile) along the keys
+  int units;                 // 32-key units of max_ctx
   int max_ctx;               // ctx_len values are clamped to [0, max_ctx]
-  const uint2* frag;
+  const uint2* frag;         // workspace: query fragments and scales (prep_queries_kernel)
   const uint2* qfrag;
-  const float4* scal;
+  const float2* scal;
   float* out;
   int64_t out_stride;
   uint32_t th0, th1, tl0, tl1;  // b <= 3: high / low int8 slices of c16 * 2^f, levels 0..7
   uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
-  float qjl_scale;
 };
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// ---- cluster helpers ------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t n;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
+  return n;
+}
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_sync() {
+  cluster_arrive_release();
+  cluster_wait_acquire();
+}
+__device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  return remote;
+}
+
+// ---- MMA wrappers -------------------------------------------------------------------
 
 __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                         uint32_t a3, uint2 b) {
@@ -308,6 +119,14 @@ __device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1,
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], uint4 a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a.x), "r"(a.y), "r"(a.z), "r"(a.w), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void mma_s8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -327,6 +146,8 @@ __device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, 
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
 }
+
+// ---- key operand decoding ---------------------------------------------------------
 
 // Byte-permute selector of the codes of local elements 8 kk .. 8 kk + 7 of a
 // chunk (layout version 3, b <= 3): nibble i holds the code of element 8 kk + i.
@@ -361,13 +182,37 @@ __device__ __forceinline__ void decode_nibble_pair(const uint32_t* w, int ks, co
   h1 = prmt(lo, hi, 0x7351u) | ((x << 8) & 0x80008000u);
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+// ---- copies -------------------------------------------------------------------------
+
+constexpr long long kWaitCycles = 2000000000LL;   // ~1 s: a bounded mbarrier wait gives up after this
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+// Waits for the phase of the given parity; false after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done) : "r"(smem_addr(bar)), "r"(parity) : "memory");
+    if (done) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+}
+// Bulk copy (no multicast) of `bytes` global -> shared, completing on `bar`;
+// both addresses 16-byte aligned, bytes a multiple of 16.  L2 evict-first:
+// the cache is streamed once per call.
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                          uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol) : "memory");
 }
 
 // The W words of one chunk from shared memory (4W-byte aligned).
@@ -397,18 +242,242 @@ __device__ __forceinline__ float lo_half(uint32_t v) {
 __device__ __forceinline__ float hi_half(uint32_t v) {
   return __half2float(__ushort_as_half((unsigned short)(v >> 16)));
 }
+__device__ __forceinline__ uint16_t bf16_bits(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
 
-// grid: (chunks of keys, batch * n_kv_heads, query tiles of 4); block 128;
-// dynamic smem kLogitsWarps * S * stage bytes.
-// Warp w of a CTA takes the CTA's 32-key units w, w + 4, w + 8, ...; unit i of
-// the warp goes to ring stage i % S.  The block-table entries of the CTA's
-// key range are staged first (loaded together with ctx_len; page_tokens is
-// a power of two, so page and slot are a shift and a mask); then each warp
-// puts its first S units in flight (one cp.async group per unit, empty groups
-// keep the count uniform) and only then waits for the query preparation
-// kernel (griddepcontrol.wait).  A unit's copy and its reads are by the same
-// warp: wait_group + __syncwarp order them, and a __syncwarp after the reads
-// precedes the copy that reuses the stage.  The two tiles of a unit are read
+// ---- query preparation -----------------------------------------------------------
+//
+// Workspace: codebook fragments uint2 [gq][KC][32] (gq = group x query tile;
+// KC = E/8 int8 k-steps, or E/4 fp16 k-steps for b = 4), QJL fragments uint2
+// [gq][F/8][32], per-query scales float2 [batch * n_q_heads] = {c0, c1}.
+// Lane (2 q + s) * 4 + t of a fragment holds slice s (0 high, 1 low) of
+// query slot q for chunk t; byte e % 8 (half e % 4 for fp16) of it is row e
+// of the k-step.  In the QJL part rows 8 kk .. 8 kk + 3 of a k-step hold the
+// slices of 2 z, rows 8 kk + 4 .. 8 kk + 7 those of z (|z| <= kSliceMaxQ),
+// matching the key operand of the logits kernel (sign bytes 2^(2 kk) beta
+// and 2^(2 kk + 1) beta).
+
+struct PrepParams {
+  const void* q;             // [batch][n_q_heads][d]
+  tq_dtype dtype;
+  int d, E, F;               // d_pad = 4E, m_pad = 4F
+  int n_q_heads, n_kv_heads, G, qtiles;
+  int cb_int8;               // codebook fragments as int8 slices (b <= 3) or fp16 hi / lo (b = 4)
+  float cb_unscale;          // 2^-f
+  float qjl_scale;           // sqrt(pi/2) / m
+  const uint4* qprep;        // [Pi ; S] bf16 hi + lo A fragments (tq_codebook::qprep_frag)
+  uint2* frag;
+  uint2* qfrag;
+  float2* scal;
+};
+
+// Rotates and sketches each query once (TQ §How it works: the query is
+// pre-rotated once and reused over the whole context).
+// grid: (C, groups * qtiles), cluster (C, 1, 1), block 128.  CTA `rank`
+// computes rows [rank RB, rank RB + RB) of [Pi q ; S q] for the 4 query
+// slots of its tile (R = d_pad + m_pad = C RB rows; d_pad is a multiple of RB)
+// on the tensor cores: bf16 hi + lo fragments of [Pi ; S] times the bf16
+// hi + lo split of the queries, fp32 accumulation (warp w: 16-row tile
+// w % MT, k split w / MT).  The CTAs exchange their per-slot maxima through
+// distributed shared memory, then quantize their own rows into the workspace
+// fragments; every fragment byte of the tile is written (zeros for padding
+// rows and slots past G), so the workspace needs no clearing.
+template <int RB>
+__global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepParams p) {
+  constexpr int MT = RB / 16;                 // 16-row tiles per CTA (2 or 4)
+  constexpr int KSPL = kLogitsWarps / MT;     // k splits (2 or 1)
+  constexpr int QROW = 256 + 8;               // bf16 per staged query row (padding: no bank conflicts)
+  __shared__ __align__(16) uint16_t qsb[8][QROW];   // column 2 q + s: bf16 slice s of query slot q
+  __shared__ float4 ksum[MT][32];
+  __shared__ float wmax[MT][4];
+  __shared__ float pmax[kMaxCluster][4];      // per-rank maxima, pushed by every rank
+  __shared__ float qn2s[4];
+  asm volatile("griddepcontrol.launch_dependents;");
+  cluster_arrive_relaxed();                   // phase 0 of the cluster barrier
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const uint32_t rank = cluster_rank();
+  const int C = (int)cluster_size();
+  const int gq = blockIdx.y;
+  const int gi = gq / p.qtiles, qt = gq % p.qtiles;
+  const int b = gi / p.n_kv_heads, kv = gi % p.n_kv_heads;
+  const int64_t qbase = (int64_t)b * p.n_q_heads + kv * p.G + qt * 4;   // first query row of the tile
+  const int nq = min(4, p.G - qt * 4);
+  const int d = p.d, d16 = (d + 15) >> 4;
+
+  const int mt = warp % MT, ksp = warp / MT;
+  const int kb = ksp * d16 / KSPL, ke = (ksp + 1) * d16 / KSPL;     // this warp's k-steps
+  const uint4* afr = p.qprep + (size_t)(rank * MT + mt) * d16 * 64 + lane;
+  uint4 af[4][2];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    if (kb + u < ke) {
+      af[u][0] = __ldg(afr + ((kb + u) * 2) * 32);
+      af[u][1] = __ldg(afr + ((kb + u) * 2 + 1) * 32);
+    }
+  {
+    // warp w: query slot w, lanes over k; every load in flight before any use
+    float x[8];
+    const int64_t qoff = (qbase + warp) * d;
+    const bool valid = warp < nq;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+    if (valid) {
+      if (p.dtype == TQ_BF16) {
+        const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(p.q) + qoff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (lane + 32 * i < d) x[i] = __bfloat162float(qp[lane + 32 * i]);
+      } else if (p.dtype == TQ_F16) {
+        const __half* qp = reinterpret_cast<const __half*>(p.q) + qoff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (lane + 32 * i < d) x[i] = __half2float(qp[lane + 32 * i]);
+      } else {
+        const float* qp = reinterpret_cast<const float*>(p.q) + qoff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (lane + 32 * i < d) x[i] = qp[lane + 32 * i];
+      }
+    }
+    float s2 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int k = lane + 32 * i;
+      if (k < 16 * d16) {
+        const uint16_t hb = bf16_bits(x[i]);
+        qsb[2 * warp][k] = hb;
+        qsb[2 * warp + 1][k] = bf16_bits(x[i] - __bfloat162float(__ushort_as_bfloat16(hb)));
+      }
+      s2 = fmaf(x[i], x[i], s2);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    if (lane == 0) qn2s[warp] = s2;
+  }
+  __syncthreads();
+
+  // column pair (2t, 2t+1) of the accumulator is (A q_hi, A q_lo) of query
+  // slot t: rows g and g + 8 of tile mt are acc[0] + acc[1], acc[2] + acc[3]
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int kc = kb; kc < ke; kc += 4) {
+    if (kc != kb) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (kc + u < ke) {
+          af[u][0] = __ldg(afr + ((kc + u) * 2) * 32);
+          af[u][1] = __ldg(afr + ((kc + u) * 2 + 1) * 32);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (kc + u < ke) {
+        const int k = kc + u;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&qsb[g][16 * k + 2 * t]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&qsb[g][16 * k + 2 * t + 8]);
+        mma_bf16(acc, af[u][0], b0, b1);
+        mma_bf16(acc, af[u][1], b0, b1);
+      }
+  }
+  if constexpr (KSPL == 2) {
+    if (ksp == 1) ksum[mt][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    __syncthreads();
+    if (ksp == 0) {
+      const float4 o = ksum[mt][lane];
+      acc[0] += o.x; acc[1] += o.y; acc[2] += o.z; acc[3] += o.w;
+    }
+  }
+  const float va = acc[0] + acc[1], vb = acc[2] + acc[3];
+  if (warp < MT) {
+    float mx = fmaxf(fabsf(va), fabsf(vb));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    if (g == 0) wmax[mt][t] = mx;
+  }
+  __syncthreads();
+  cluster_wait_acquire();            // phase 0 complete: every CTA of the cluster exists
+  if ((int)threadIdx.x < 4 * C) {
+    const int qq = threadIdx.x & 3;
+    float m = wmax[0][qq];
+#pragma unroll
+    for (int u = 1; u < MT; ++u) m = fmaxf(m, wmax[u][qq]);
+    asm volatile("st.shared::cluster.f32 [%0], %1;"
+                 ::"r"(map_rank(&pmax[rank][qq], (uint32_t)(threadIdx.x >> 2))), "f"(m) : "memory");
+  }
+  cluster_sync();                    // phase 1: every rank's maxima delivered; no remote access after this
+
+  const int nb_pi = 4 * p.E / RB;    // ranks [0, nb_pi) hold Pi q rows
+  float mpi = 0.0f, msk = 0.0f;      // maxima of query slot t
+  for (int r = 0; r < C; ++r) {
+    const float m = pmax[r][t];
+    if (r < nb_pi) mpi = fmaxf(mpi, m);
+    else msk = fmaxf(msk, m);
+  }
+  int e2 = 0;                        // b = 4: ||q|| in [2^(e2-1), 2^e2)
+  {
+    const float qn = sqrtf(qn2s[t]);
+    if (qn > 0.0f) frexpf(qn, &e2);
+  }
+  const bool sk = (int)rank >= nb_pi;
+  if (warp < MT) {
+    const int Ep = sk ? p.F : p.E;
+    const float mxp = sk ? msk : mpi;
+    const int zmax = sk ? kSliceMaxQ : kSliceMax;
+    const float scale = mxp > 0.0f ? (float)zmax * __frcp_rn(mxp) : 0.0f;
+    const float f16scale = ldexpf(1.0f, 14 - e2);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int l = (int)rank * RB - (sk ? 4 * p.E : 0) + 16 * mt + g + 8 * hh;   // row within its part
+      const float v = hh ? vb : va;
+      const int tc = l / Ep, e = l % Ep;        // chunk, row within the chunk
+      if (!sk && !p.cb_int8) {
+        const float vs = v * f16scale;
+        const __half hi = __float2half_rn(vs);
+        const __half lo = __float2half_rn(vs - __half2float(hi));
+        __half* fr = reinterpret_cast<__half*>(p.frag + ((int64_t)gq * (p.E / 4) + e / 4) * 32);
+        fr[((2 * t) * 4 + tc) * 4 + (e & 3)] = hi;
+        fr[((2 * t + 1) * 4 + tc) * 4 + (e & 3)] = lo;
+      } else {
+        int z = max(-zmax, min(zmax, __float2int_rn(v * scale)));
+        if (sk && (e & 7) < 4) z *= 2;          // rows 8 kk .. 8 kk + 3 of a QJL k-step: 2 z
+        const int zh = (z + 128) >> 8;          // floor((z + 128) / 256)
+        const int zl = z - 256 * zh;            // in [-128, 127]
+        int8_t* fr = reinterpret_cast<int8_t*>((sk ? p.qfrag : p.frag) + ((int64_t)gq * (Ep / 8) + e / 8) * 32);
+        fr[((2 * t) * 4 + tc) * 8 + (e & 7)] = (int8_t)zh;
+        fr[((2 * t + 1) * 4 + tc) * 8 + (e & 7)] = (int8_t)zl;
+      }
+    }
+  }
+  if (rank == 0 && (int)threadIdx.x < nq) {
+    const int qq = threadIdx.x;
+    float m0 = 0.0f, m1 = 0.0f;
+    for (int r = 0; r < C; ++r) {
+      if (r < nb_pi) m0 = fmaxf(m0, pmax[r][qq]);
+      else m1 = fmaxf(m1, pmax[r][qq]);
+    }
+    int e = 0;
+    const float qn = sqrtf(qn2s[qq]);
+    if (qn > 0.0f) frexpf(qn, &e);
+    const float c0 = p.cb_int8 ? m0 * (1.0f / (float)kSliceMax) * p.cb_unscale : ldexpf(1.0f, e - 14);
+    const float c1 = p.qjl_scale * m1 * (1.0f / (float)kSliceMaxQ);
+    p.scal[qbase + qq] = make_float2(c0, c1);
+  }
+}
+
+// ---- logits -----------------------------------------------------------------------
+//
+// grid: (n_chunks, batch * n_kv_heads, query tiles of 4), block 128, dynamic
+// smem kLogitsWarps * S * stage bytes.  CTA x of a (group, query tile) owns
+// the 32-key units [x U / n_chunks, (x + 1) U / n_chunks) of the sequence
+// (U = ceil(max_ctx / 32)): every CTA gets the same work to within one unit.
+// Before it waits for the query preparation kernel (griddepcontrol.wait) a
+// CTA stages its block-table entries (page_tokens is a power of two: page
+// and slot are a shift and a mask) and every warp puts its first S units in
+// flight: lane 0 issues bulk copies of the unit's 32 records and 32 norm
+// slots into ring stage i % S, completing on that stage's mbarrier.  Warp w
+// takes the CTA's units w, w + 4, ...  The two tiles of a unit are read
 // before either is computed, so their MMA chains interleave; a tile whose
 // page is bad or that lies past the context computes on stale bytes and
 // stores nothing.
@@ -418,7 +487,7 @@ __device__ __forceinline__ float hi_half(uint32_t v) {
 // every k-step of a word to weight 2^(2 n - 1) (n k-steps in the word), and
 // words are scaled to the common weight 128.
 template <int BITS, int E, int F>
-__global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5 : kLogitsMinBlocks) logits_kernel(LogitsParams p) {
+__global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E)) logits_kernel(LogitsParams p) {
   constexpr bool kInt8 = BITS <= 3;
   constexpr int KC = kInt8 ? E / 8 : E / 4;   // codebook MMA k-steps
   constexpr int KQ = F / 8;                   // sign-term MMA k-steps
@@ -432,68 +501,94 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5
   constexpr int TILE = RS::kTileCode;
   constexpr int STAGE = RS::kStageBytes;
   extern __shared__ __align__(16) uint8_t ring_smem[];
-  __shared__ int64_t page_base[kCtaPages];   // byte offset of this head's block, -1 if bad
+  __shared__ int64_t page_base[kCtaPages];    // byte offset of this head's block, -1 if bad
+  __shared__ uint64_t ring_bar[kLogitsWarps][4];   // one per ring stage (S <= 4)
 
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
   const int gi = blockIdx.y;
   const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
   const int qt = blockIdx.z;
-  const int k0 = blockIdx.x * p.keys_per_cta;          // < max_ctx
-  const int kend = min(k0 + p.keys_per_cta, p.max_ctx);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
+  const int u0 = (int)((int64_t)blockIdx.x * p.units / p.n_chunks);
+  const int u1 = (int)((int64_t)(blockIdx.x + 1) * p.units / p.n_chunks);
+  const int k0 = 32 * u0;
+  const int kend = min(32 * u1, p.max_ctx);
   const int ps = p.page_shift;
   const int P = 1 << ps;
   const int first_page = k0 >> ps;
+  const int n_pgx = k0 < kend ? ((kend - 1) >> ps) - first_page + 1 : 0;   // <= kCtaPages
   const int ctx = min(p.ctx_len[b], p.max_ctx);
-  {
-    const int n_pg = ((kend - 1) >> ps) - first_page + 1;
-    for (int j = threadIdx.x; j < n_pg; j += blockDim.x) {
-      const int64_t page = p.cv.block_table[(int64_t)b * p.cv.max_pages + first_page + j];
-      page_base[j] = (page >= 0 && page < p.cv.n_pages)
-                         ? page * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes : -1;
+  const int jt = threadIdx.x;
+  static_assert(kCtaPages <= kLogitsWarps * 32, "one block-table entry per thread");
+  const int64_t pg = jt < n_pgx ? p.cv.block_table[(int64_t)b * p.cv.max_pages + first_page + jt] : 0;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) mbar_init(&ring_bar[warp][s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const int k1 = min(kend, ctx);     // keys [k0, k1) of this CTA (none when k1 <= k0)
+  const bool has_keys = k0 < k1;
+  bool bad = false;
+  if (jt < n_pgx) {
+    const bool valid = pg >= 0 && pg < p.cv.n_pages;
+    page_base[jt] = valid ? pg * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes : -1;
+    // pages past the context are not used: an invalid entry there is no error
+    if (!valid && has_keys && jt <= ((k1 - 1) >> ps) - first_page) {
+      bad = true;
+      report(p.cv.err, TQ_DEV_ERR_PAGE);
     }
   }
-  if (k0 >= ctx) return;
-  const int k1 = min(kend, ctx);
-  __syncthreads();
+  // fast path: every used page valid and 32-key units never straddle a page
+  const bool fast = !__syncthreads_or(bad) && P >= 32;   // also publishes the barriers' init
 
-  const int n_units = (k1 - k0 + 31) >> 5;
+  const int n_units = has_keys ? (k1 - k0 + 31) >> 5 : 0;
   const int n_my = warp < n_units ? (n_units - warp + kLogitsWarps - 1) / kLogitsWarps : 0;
   const uint8_t* ring = ring_smem + warp * S * STAGE;
   const uint32_t ring_s = smem_addr(ring);
   const int64_t norm_off = (int64_t)P * (16 * W);   // norm slots follow the P records
+  uint64_t pol;                      // the cache is streamed once per call: evict it first from L2
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
 
-  // copies unit i of this warp (2 x (16 records + 16 norm slots)) into stage i % S
+  // lane 0 copies unit i of this warp (32 records + 32 norm slots) into stage
+  // i % S with bulk copies completing on that stage's barrier
   auto issue = [&](int i) {
+    if (lane != 0) return;
+    uint64_t* bar = &ring_bar[warp][i & (S - 1)];
     const uint32_t dst = ring_s + (i & (S - 1)) * STAGE;
+    const int ubase = k0 + 32 * (warp + kLogitsWarps * i);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads of the stage first
+    if (fast) {
+      // one page holds the whole unit (records past the context are read and not used)
+      const int slot = ubase & (P - 1);
+      const uint8_t* hb = p.cv.pages + page_base[(ubase >> ps) - first_page];
+      mbar_arrive_tx(bar, 2 * TILE + 32 * NB);
+      bulk_copy(dst, hb + (int64_t)slot * (16 * W), 2 * TILE, bar, pol);
+      bulk_copy(dst + 2 * TILE, hb + norm_off + slot * NB, 32 * NB, bar, pol);
+      return;
+    }
+    uint32_t bytes = 0;
+    int64_t off[2] = {-1, -1};
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
-      const int base = k0 + 32 * (warp + kLogitsWarps * i) + 16 * hf;
-      if (base >= k1) break;
-      const int64_t off = page_base[(base >> ps) - first_page];
-      if (off < 0) {
-        report(p.cv.err, TQ_DEV_ERR_PAGE);
-        continue;
-      }
-      const int slot = base & (P - 1);
-      const uint8_t* hb = p.cv.pages + off;
-      const uint8_t* src = hb + (int64_t)slot * (16 * W);
+      const int base = ubase + 16 * hf;
+      if (base < k1) off[hf] = page_base[(base >> ps) - first_page];
+      if (off[hf] >= 0) bytes += TILE + 16 * NB;
+    }
+    mbar_arrive_tx(bar, bytes);        // 0 bytes: the phase completes on the arrival alone
 #pragma unroll
-      for (int j = 0; j < (16 * W + 31) / 32; ++j) {
-        const int c = lane + 32 * j;
-        if (c < 16 * W) cp_async16(dst + hf * TILE + 16 * c, src + 16 * c);
-      }
-      if (lane < NB) cp_async16(dst + 2 * TILE + 64 * hf + 16 * lane, hb + norm_off + slot * NB + 16 * lane);
+    for (int hf = 0; hf < 2; ++hf) {
+      if (off[hf] < 0) continue;
+      const int slot = (ubase + 16 * hf) & (P - 1);
+      const uint8_t* hb = p.cv.pages + off[hf];
+      bulk_copy(dst + hf * TILE, hb + (int64_t)slot * (16 * W), TILE, bar, pol);
+      bulk_copy(dst + 2 * TILE + 16 * NB * hf, hb + norm_off + slot * NB, 16 * NB, bar, pol);
     }
   };
-
 #pragma unroll
-  for (int s = 0; s < S; ++s) {
+  for (int s = 0; s < S; ++s)
     if (s < n_my) issue(s);
-    cp_async_commit();
-  }
 
-  // the query fragments come from the preparation kernel
+  // the query fragments and scales come from the preparation kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int gq = gi * p.qtiles + qt;
   uint2 bq[KC];
@@ -516,11 +611,10 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5
   const int qidx = qt * 4 + t;                  // this thread's query within the group
   const bool qvalid = qidx < p.G;
   const int hq = h * p.G + (qvalid ? qidx : 0);
-  const float4 sc = p.scal[(int64_t)b * p.n_q_heads + hq];
+  const float2 sc = p.scal[(int64_t)b * p.n_q_heads + hq];
   const float c0 = sc.x;
-  const float c1 = F > 0 ? p.qjl_scale * sc.y : 0.0f;
+  const float c1 = F > 0 ? sc.y : 0.0f;
   float* orow = p.out + ((int64_t)b * p.n_q_heads + hq) * p.out_stride;
-
   // logits of rows g (la) and g + 8 (lb) of one tile, for query t
   auto tile = [&](const uint32_t (&wa)[W], const uint32_t (&wb)[W], uint32_t na, uint32_t nb,
                   float& la, float& lb) {
@@ -560,23 +654,22 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5
       int qa[4] = {0, 0, 0, 0};                 // 128 sum beta z (hi, lo columns)
 #pragma unroll
       for (int w = 0; w < QW; ++w) {
-        constexpr int rows_full = 32;
-        const int nk = min(4, (F - rows_full * w) / 8);   // k-steps of this word (4, or 2 for a half word)
-        int acc[4] = {0, 0, 0, 0};
+        const int nk = min(4, (F - 32 * w) / 8);   // k-steps of this word (4, or 2 for a half word)
+        int a4[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           if (k < nk) {
             if (k > 0) {
 #pragma unroll
-              for (int r = 0; r < 4; ++r) acc[r] *= 4;
+              for (int r = 0; r < 4; ++r) a4[r] *= 4;
             }
             const uint32_t m0 = 0x01010101u << (2 * k), m1 = m0 << 1;
-            mma_u8s8(acc, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, bz[4 * w + k]);
+            mma_u8s8(a4, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, bz[4 * w + k]);
           }
         }
         const int sh = 6 - 2 * (nk - 1);           // weight 2^(2 nk - 1) -> 128
 #pragma unroll
-        for (int r = 0; r < 4; ++r) qa[r] += acc[r] << sh;
+        for (int r = 0; r < 4; ++r) qa[r] += a4[r] << sh;
       }
       // sum_i s_i z_i = sum z - 2 sum beta z
       const float ta = fmaf(-1.0f / 64.0f, (float)(256 * qa[0] + qa[1]), zsumf);
@@ -589,9 +682,13 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5
     }
   };
 
+  bool timed_out = false;
+  int issued = min(S, n_my);         // units whose copies were issued
   for (int i = 0; i < n_my; ++i) {
-    cp_async_wait<S - 1>();
-    __syncwarp();
+    if (!mbar_wait(&ring_bar[warp][i & (S - 1)], (uint32_t)(i / S) & 1u)) {
+      timed_out = true;
+      break;
+    }
     const int ubase = k0 + 32 * (warp + kLogitsWarps * i);
     const uint8_t* stg = ring + (i & (S - 1)) * STAGE;
     uint32_t wa0[W], wb0[W], wa1[W], wb1[W];
@@ -607,24 +704,43 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, E >= 48 ? 4 : BITS == 4 ? 5
       const uint8_t* nsl = stg + 2 * TILE;
       na0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * g);
       nb0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * (g + 8));
-      na1 = *reinterpret_cast<const unsigned short*>(nsl + 64 + 2 * g);
-      nb1 = *reinterpret_cast<const unsigned short*>(nsl + 64 + 2 * (g + 8));
+      na1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * g);
+      nb1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * (g + 8));
     }
-    const bool ok0 = page_base[(ubase >> ps) - first_page] >= 0;
-    const bool ok1 = ubase + 16 < k1 && page_base[((ubase + 16) >> ps) - first_page] >= 0;
+    bool ok0 = true, ok1 = ubase + 16 < k1;
+    if (!fast) {
+      ok0 = page_base[(ubase >> ps) - first_page] >= 0;
+      ok1 = ok1 && page_base[((ubase + 16) >> ps) - first_page] >= 0;
+    }
     __syncwarp();                    // every read of this stage precedes its reuse
-    if (i + S < n_my) issue(i + S);
-    cp_async_commit();
+    if (i + S < n_my) {
+      issue(i + S);
+      issued = i + S + 1;
+    }
     float la0, lb0, la1, lb1;
     tile(wa0, wb0, na0, nb0, la0, lb0);
     tile(wa1, wb1, na1, nb1, la1, lb1);
     if (qvalid) {
       const int r = ubase + g;
-      if (ok0 && r < k1) __stcs(orow + r, la0);
-      if (ok0 && r + 8 < k1) __stcs(orow + r + 8, lb0);
-      if (ok1 && r + 16 < k1) __stcs(orow + r + 16, la1);
-      if (ok1 && r + 24 < k1) __stcs(orow + r + 24, lb1);
+      if (fast && ubase + 32 <= k1) {
+        __stcs(orow + r, la0);
+        __stcs(orow + r + 8, lb0);
+        __stcs(orow + r + 16, la1);
+        __stcs(orow + r + 24, lb1);
+      } else {
+        if (ok0 && r < k1) __stcs(orow + r, la0);
+        if (ok0 && r + 8 < k1) __stcs(orow + r + 8, lb0);
+        if (ok1 && r + 16 < k1) __stcs(orow + r + 16, la1);
+        if (ok1 && r + 24 < k1) __stcs(orow + r + 24, lb1);
+      }
     }
+  }
+  if (timed_out) {
+    // report, then let the copies already issued land (the last unit issued
+    // into each stage; each wait bounded) before the CTA's shared memory is
+    // released
+    if (lane == 0) report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+    for (int u = max(0, issued - S); u < issued; ++u) mbar_wait(&ring_bar[warp][u & (S - 1)], (uint32_t)(u / S) & 1u);
   }
 }
 
@@ -636,15 +752,14 @@ struct LogitsWs {
   size_t frag, qfrag, scal, total;
 };
 
-static int codebook_ksteps(const Layout& L) { return L.bits <= 3 ? L.E / 8 : L.E / 4; }
-
 static LogitsWs logits_ws_layout(const tq_codebook* cb, int64_t groups, int G, int64_t batch_heads) {
   auto al = [](size_t n) { return (n + 255) / 256 * 256; };
   const int qtiles = (G + 3) / 4;
+  const int kc = cb->lay.bits <= 3 ? cb->lay.E / 8 : cb->lay.E / 4;
   LogitsWs w;
-  w.frag = al((size_t)groups * qtiles * codebook_ksteps(cb->lay) * 32 * sizeof(uint2));
+  w.frag = al((size_t)groups * qtiles * kc * 32 * sizeof(uint2));
   w.qfrag = al((size_t)groups * qtiles * (cb->lay.F / 8) * 32 * sizeof(uint2));
-  w.scal = al((size_t)batch_heads * sizeof(float4));
+  w.scal = al((size_t)batch_heads * sizeof(float2));
   w.total = w.frag + w.qfrag + w.scal;
   return w;
 }
@@ -654,7 +769,7 @@ size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
 }
 
 template <int BITS, int E, int F>
-static cudaError_t run_logits(const tqd::LogitsParams& p, dim3 grid, cudaStream_t st) {
+static tq_status run_logits(const tqd::LogitsParams& p, int64_t groups, int qtiles, cudaStream_t st) {
   constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
                    : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
   constexpr int W = q0 + (F + 31) / 32;
@@ -664,11 +779,11 @@ static cudaError_t run_logits(const tqd::LogitsParams& p, dim3 grid, cudaStream_
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(tqd::logits_kernel<BITS, E, F>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) return cuda_fail(e, "tq_logits: smem attribute");
     attr = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
+  cfg.gridDim = dim3((unsigned)p.n_chunks, (unsigned)groups, (unsigned)qtiles);
   cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
@@ -677,46 +792,40 @@ static cudaError_t run_logits(const tqd::LogitsParams& p, dim3 grid, cudaStream_
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
+  if (e != cudaSuccess) return cuda_fail(e, "tq_logits launch");
+  return TQ_OK;
 }
 
 template <int BITS>
-static bool dispatch_logits(const Layout& L, const tqd::LogitsParams& p, dim3 grid, cudaStream_t st,
-                            cudaError_t& err) {
-  if (L.E == 32 && L.F == 32) return err = run_logits<BITS, 32, 32>(p, grid, st), true;
-  if (L.E == 32 && L.F == 0) return err = run_logits<BITS, 32, 0>(p, grid, st), true;
-  if (L.E == 16 && L.F == 16) return err = run_logits<BITS, 16, 16>(p, grid, st), true;
-  if (L.E == 16 && L.F == 0) return err = run_logits<BITS, 16, 0>(p, grid, st), true;
-  if (L.E == 64 && L.F == 64) return err = run_logits<BITS, 64, 64>(p, grid, st), true;
-  if (L.E == 64 && L.F == 0) return err = run_logits<BITS, 64, 0>(p, grid, st), true;
-  if (L.E == 48 && L.F == 48) return err = run_logits<BITS, 48, 48>(p, grid, st), true;
-  if (L.E == 48 && L.F == 0) return err = run_logits<BITS, 48, 0>(p, grid, st), true;
-  return false;
+static tq_status dispatch_logits(const Layout& L, const tqd::LogitsParams& p, int64_t groups, int qtiles,
+                                 cudaStream_t st) {
+  if (L.E == 32 && L.F == 32) return run_logits<BITS, 32, 32>(p, groups, qtiles, st);
+  if (L.E == 32 && L.F == 0) return run_logits<BITS, 32, 0>(p, groups, qtiles, st);
+  if (L.E == 16 && L.F == 16) return run_logits<BITS, 16, 16>(p, groups, qtiles, st);
+  if (L.E == 16 && L.F == 0) return run_logits<BITS, 16, 0>(p, groups, qtiles, st);
+  if (L.E == 64 && L.F == 64) return run_logits<BITS, 64, 64>(p, groups, qtiles, st);
+  if (L.E == 64 && L.F == 0) return run_logits<BITS, 64, 0>(p, groups, qtiles, st);
+  if (L.E == 48 && L.F == 48) return run_logits<BITS, 48, 48>(p, groups, qtiles, st);
+  if (L.E == 48 && L.F == 0) return run_logits<BITS, 48, 0>(p, groups, qtiles, st);
+  return fail(TQ_EUNSUPPORTED, "tq_logits: no kernel for this (d, m)");
 }
 
-template <int RPW>
-static cudaError_t run_prep(const tqd::PrepParams& pp, int nblk, int64_t units, cudaStream_t st) {
-  const int smem = 4 * RPW * pp.d * (int)sizeof(float);   // the block's matrix rows
-  static bool attr = false;            // per template instance
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(tqd::prep_queries_kernel<RPW>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * RPW * 256 * 4);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+template <int RB>
+static cudaError_t run_prep(const tqd::PrepParams& pp, int cluster, int64_t units, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)nblk, (unsigned)units);
-  cfg.blockDim = dim3(tqd::kPrepThreads);
-  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.gridDim = dim3((unsigned)cluster, (unsigned)units);
+  cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeClusterDimension;
-  attrs[0].val.clusterDim.x = (unsigned)nblk;
+  attrs[0].val.clusterDim.x = (unsigned)cluster;
   attrs[0].val.clusterDim.y = 1;
   attrs[0].val.clusterDim.z = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tqd::prep_queries_kernel<RPW>, pp);
+  return cudaLaunchKernelEx(&cfg, tqd::prep_queries_kernel<RB>, pp);
 }
 
 tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* q, tq_dtype dt,
@@ -728,20 +837,18 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   const int qtiles = (G + 3) / 4;
   const int64_t groups = batch * cv.n_kv_heads;
   const LogitsWs wl = logits_ws_layout(cb, groups, G, batch * n_q_heads);
-  if (ws_bytes < wl.total) return fail(TQ_EINVAL, "tq_logits: workspace too small");
+  if (ws_bytes < wl.total || !ws) return fail(TQ_EINVAL, "tq_logits: workspace too small");
   if (max_ctx == 0 || batch == 0) return TQ_OK;
-  if (groups * qtiles > 65535) return fail(TQ_EINVAL, "tq_logits: batch * n_kv_heads * query tiles > 65535");
+  if (groups > 65535 || groups * qtiles > 65535) return fail(TQ_EINVAL, "tq_logits: batch * n_kv_heads too large");
   uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
   uint2* frag = reinterpret_cast<uint2*>(wsb);
   uint2* qfrag = reinterpret_cast<uint2*>(wsb + wl.frag);
-  float4* scal = reinterpret_cast<float4*>(wsb + wl.frag + wl.qfrag);
+  float2* scal = reinterpret_cast<float2*>(wsb + wl.frag + wl.qfrag);
 
   tqd::PrepParams pp;
   pp.q = q;
   pp.dtype = dt;
   pp.d = L.d;
-  pp.d_pad = L.d_pad;
-  pp.m_pad = L.m_pad;
   pp.E = L.E;
   pp.F = L.F;
   pp.n_q_heads = n_q_heads;
@@ -750,18 +857,16 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   pp.qtiles = qtiles;
   pp.cb_int8 = L.bits <= 3 ? 1 : 0;
   pp.cb_unscale = std::ldexp(1.0f, -cb->table_exp);
-  pp.pi32 = cb->pi32;
-  pp.s32 = cb->s32;
+  pp.qjl_scale = (float)cb->qjl_scale;
+  pp.qprep = cb->qprep_frag;
   pp.frag = frag;
   pp.qfrag = qfrag;
   pp.scal = scal;
-  // rows of [Pi q ; S q] per CTA: 32, or 64 when that keeps the cluster at
-  // most kMaxClusterCtas CTAs (d_pad and m_pad are multiples of 64)
   const int rows = L.d_pad + L.m_pad;
-  const int rb = rows <= 32 * tqd::kMaxClusterCtas ? 32 : 64;
-  const int nblk = rows / rb;
-  cudaError_t e = rb == 32 ? run_prep<8>(pp, nblk, groups * qtiles, st)
-                           : run_prep<16>(pp, nblk, groups * qtiles, st);
+  const int rb = tqd::prep_rows_per_cta(L.E, L.F);
+  const int cluster = rows / rb;                 // 2 .. 8
+  cudaError_t e = rb == 32 ? run_prep<32>(pp, cluster, groups * qtiles, st)
+                           : run_prep<64>(pp, cluster, groups * qtiles, st);
   if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
 
   tqd::LogitsParams lp;
@@ -774,21 +879,18 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   lp.n_q_heads = n_q_heads;
   lp.G = G;
   lp.qtiles = qtiles;
-  // Split the context so that the grid fills every CTA slot of the GPU once
-  // (148 SMs x kLogitsMinBlocks), each CTA a whole number of 32-key units.
-  const int64_t units = groups * qtiles;
-  const int64_t slots = 148LL * tqd::kLogitsMinBlocks;
-  const int64_t chunks = (slots + units - 1) / units;
-  int64_t kpc = (max_ctx + chunks - 1) / chunks;
-  kpc = ((kpc + 31) / 32) * 32;
-  if (kpc < 32 * tqd::kLogitsWarps) kpc = 32 * tqd::kLogitsWarps;
-  // a CTA stages at most kCtaPages block-table entries (its range may start
-  // inside a page, hence the 2 spare entries)
-  const int64_t kpc_cap = ((int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 32) * 32;
-  if (kpc > kpc_cap) kpc = kpc_cap;
-  const int64_t n_chunks = (max_ctx + kpc - 1) / kpc;
+  // Every CTA slot of the GPU (148 SMs x resident CTAs) gets one CTA, each
+  // an equal share (to one 32-key unit) of one sequence's keys; more CTAs
+  // when a share would need more than kCtaPages - 2 block-table entries.
+  const int64_t units = (max_ctx + 31) / 32;
+  const int64_t slots = 148LL * tqd::logits_min_blocks(L.bits, L.E);
+  int64_t n_chunks = std::max<int64_t>(1, slots / (groups * qtiles));
+  const int64_t max_units_cta = (int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 32;
+  n_chunks = std::max<int64_t>(n_chunks, (units + max_units_cta - 1) / max_units_cta);
+  n_chunks = std::min<int64_t>(n_chunks, units);
   if (n_chunks > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_logits: context too long");
-  lp.keys_per_cta = (int)kpc;
+  lp.n_chunks = (int)n_chunks;
+  lp.units = (int)units;
   lp.max_ctx = (int)max_ctx;
   lp.frag = frag;
   lp.qfrag = qfrag;
@@ -809,19 +911,13 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
       lp.hi1 |= (uint32_t)(M[4 + i] >> 8) << (8 * i);
     }
   }
-  lp.qjl_scale = (float)cb->qjl_scale;
-  dim3 grid((unsigned)n_chunks, (unsigned)groups, (unsigned)qtiles);
-  bool ok = false;
-  cudaError_t le = cudaSuccess;
   switch (L.bits) {
-    case 1: ok = dispatch_logits<1>(L, lp, grid, st, le); break;
-    case 2: ok = dispatch_logits<2>(L, lp, grid, st, le); break;
-    case 3: ok = dispatch_logits<3>(L, lp, grid, st, le); break;
-    case 4: ok = dispatch_logits<4>(L, lp, grid, st, le); break;
+    case 1: return dispatch_logits<1>(L, lp, groups, qtiles, st);
+    case 2: return dispatch_logits<2>(L, lp, groups, qtiles, st);
+    case 3: return dispatch_logits<3>(L, lp, groups, qtiles, st);
+    case 4: return dispatch_logits<4>(L, lp, groups, qtiles, st);
   }
-  if (!ok) return fail(TQ_EUNSUPPORTED, "tq_logits: no kernel for this (d, m)");
-  if (le != cudaSuccess) return cuda_fail(le, "tq_logits launch");
-  return cuda_fail(cudaGetLastError(), "tq_logits launch");
+  return fail(TQ_EUNSUPPORTED, "tq_logits: bits");
 }
 
 }  // namespace tq

@@ -75,6 +75,10 @@ struct tq_codebook {
   float* cent32;      // [2^b]        float(fp16(c))
   __nv_bfloat16* pi_bf;    // tensor-core operands: [2][d_pad][d_pad] hi, lo of Pi
   __nv_bfloat16* srot_bf;  // [2][m_pad][d_pad] hi, lo of S Pi^T
+  // [Pi ; S] (R = d_pad + m_pad rows, d columns padded to d16 = ceil(d/16)
+  // blocks of 16) as bf16 hi + lo in mma.m16n8k16 A-fragment order:
+  // uint4 [R/16 row tiles][d16][2: hi, lo][32 lanes]
+  uint4* qprep_frag;
   // fp16 bit patterns of the reconstruction magnitudes M[mu] = c16[H + mu]
   uint16_t mag16[8];
   uint16_t cent16[16];
