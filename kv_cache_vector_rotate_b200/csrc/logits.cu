@@ -32,7 +32,7 @@
 //    The MMA's N = 8 columns are the high and low slices of 4 queries.
 // HBM traffic is the packed records plus the logits.
 
-#include "tq_internal.cuh"
+#include "stream.cuh"
 
 namespace tqd {
 
@@ -75,10 +75,6 @@ struct LogitsParams {
   uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
 };
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
 // ---- cluster helpers ------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -111,15 +107,6 @@ __device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
 }
 
 // ---- MMA wrappers -------------------------------------------------------------------
-
-__device__ __forceinline__ void mma_f16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                        uint32_t a3, uint2 b) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b.x), "r"(b.y));
-}
 
 __device__ __forceinline__ void mma_bf16(float (&c)[4], uint4 a, uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -183,37 +170,6 @@ __device__ __forceinline__ void decode_nibble_pair(const uint32_t* w, int ks, co
 }
 
 // ---- copies -------------------------------------------------------------------------
-
-constexpr long long kWaitCycles = 2000000000LL;   // ~1 s: a bounded mbarrier wait gives up after this
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
-               : "memory");
-}
-// Waits for the phase of the given parity; false after kWaitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const long long t0 = clock64();
-  while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-        : "=r"(done) : "r"(smem_addr(bar)), "r"(parity) : "memory");
-    if (done) return true;
-    if (clock64() - t0 > kWaitCycles) return false;
-  }
-}
-// Bulk copy (no multicast) of `bytes` global -> shared, completing on `bar`;
-// both addresses 16-byte aligned, bytes a multiple of 16.  L2 evict-first:
-// the cache is streamed once per call.
-__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar,
-                                          uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
-      ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol) : "memory");
-}
 
 // The W words of one chunk from shared memory (4W-byte aligned).
 template <int W>
@@ -546,8 +502,7 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E))
   const uint8_t* ring = ring_smem + warp * S * STAGE;
   const uint32_t ring_s = smem_addr(ring);
   const int64_t norm_off = (int64_t)P * (16 * W);   // norm slots follow the P records
-  uint64_t pol;                      // the cache is streamed once per call: evict it first from L2
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  const uint64_t pol = evict_first_policy();   // the cache is streamed once per call
 
   // lane 0 copies unit i of this warp (32 records + 32 norm slots) into stage
   // i % S with bulk copies completing on that stage's barrier

@@ -5,12 +5,18 @@
 //  * mode A writes v_hat for every token;
 //  * mode B forms o_h = sum_t w_{h,t} v_hat_t for the query heads of a KV head.
 //    The sum is accumulated in the rotated space (acc_h = sum_t w_{h,t}
-//    ||v_t|| c16[idx_t]) and rotated back once per head (o_h = Pi^T acc_h),
-//    so the per-token work is a decode and G multiply-adds per coordinate.
-//    Partial sums of context chunks go to the workspace; a second kernel adds
-//    them and applies Pi^T.
+//    ||v_t|| c16[idx_t]) and rotated back once per head (o_h = Pi^T acc_h).
+//    Per KV group that is ACC^T = C^T (w ||v||)^T, a contraction over the
+//    tokens, run on the tensor cores: each warp streams 32-token units of
+//    records into a shared-memory ring with bulk copies, each lane decodes
+//    one token's coordinates into fp16 c16 values of a [token][coordinate]
+//    tile, ldmatrix.trans turns the tile into MMA A fragments (coordinates x
+//    tokens), and the weights times the norms, split into fp16 hi + lo, are
+//    the B columns (4 query heads x 2).  Partial sums of context chunks go to
+//    the workspace; a second kernel adds them and applies Pi^T.
 
 #include "pack.cuh"
+#include "stream.cuh"
 
 namespace tqd {
 
@@ -26,9 +32,6 @@ struct ValuesParams {
   void* out;
   tq_dtype odt;
   int64_t out_stride;
-  float* partial;           // mode B: [chunks][groups][G][d_pad]
-  int tokens_per_cta;
-  int n_chunks;
   int max_ctx;              // ctx_len values are clamped to [0, max_ctx]
 };
 
@@ -115,70 +118,319 @@ __global__ void __launch_bounds__(128) dequant_kernel(ValuesParams p) {
   }
 }
 
-// Mode B, pass 1.  grid: (n_chunks, batch * n_kv_heads); block 128.
-// Dynamic shared memory: acc [G][4E] floats and weights [16][G].
+// ---- mode B on the tensor cores ----------------------------------------------------
+
+constexpr int kValWarps = 4;       // warps per CTA of the accumulate kernel
+constexpr int kValCtaPages = 64;   // block-table entries staged per CTA
+constexpr int kValStages = 2;      // ring stages per warp
+
+struct ValuesTcParams {
+  tq::CacheView cv;
+  int page_shift;                  // log2(page_tokens)
+  const int32_t* ctx_len;
+  int n_kv_heads, n_q_heads, G, qtiles;
+  int n_chunks;                    // CTAs per (group, query tile) along the tokens
+  int units;                       // 32-token units of max_ctx
+  int max_ctx;                     // ctx_len values are clamped to [0, max_ctx]
+  int d;
+  const float* w;                  // [batch][n_q_heads][w_stride]
+  int64_t w_stride;
+  float* partial;                  // [n_chunks][groups * qtiles][4][4E]
+  const float* pi32;               // [d_pad][d]
+  float* out;                      // [batch][n_q_heads][d]
+  uint32_t tlo0, tlo1, thi0, thi1; // low / high bytes of c16 (b <= 3: levels 0..7; b = 4: magnitudes)
+};
+
+template <int W, int E>
+struct ValShape {
+  static constexpr int kRec = 16 * W;                  // bytes per record
+  static constexpr int kStage = 32 * kRec + 64;        // 32 records + 32 fp16 norms
+  static constexpr int kTile = 32 * 4 * E * 2;         // fp16 [32 tokens][4E coordinates]
+  static constexpr int kWarpBytes = kValStages * kStage + kTile + 32 * 16;   // + w ||v|| [32][4] fp32
+};
+
+// fp16 c16 values of the 8 coordinates 8 kk .. 8 kk + 7 of a chunk, as four
+// fp16 pairs (b <= 3: level selector and two byte permutes per 4 values; b =
+// 4: sign-magnitude nibbles).
 template <int BITS, int E>
-__global__ void __launch_bounds__(128) accumulate_kernel(ValuesParams p) {
-  constexpr int DP = 4 * E;
-  __shared__ float cs[16][DP + 1];
-  __shared__ float sc[16];
-  extern __shared__ float dyn[];
-  const int G = p.G;
-  float* acc = dyn;                 // [G][DP]
-  float* ws = dyn + G * DP;         // [16][G]
-  const int gi = blockIdx.y, b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
-  const int ctx = min(p.ctx_len[b], p.max_ctx);
-  const int k0 = blockIdx.x * p.tokens_per_cta;
-  const int k1 = min(k0 + p.tokens_per_cta, ctx);
-  for (int i = threadIdx.x; i < G * DP; i += 128) acc[i] = 0.0f;
-  if (threadIdx.x < (1 << BITS)) sc[threadIdx.x] = p.cent32[threadIdx.x];
-  __syncthreads();
-  for (int base = k0; base < k1; base += 16) {
-    stage_tokens<BITS, E>(p, b, h, base, k1, cs, sc);
-    for (int i = threadIdx.x; i < 16 * G; i += 128) {
-      const int tok = i / G, hh = i % G;
-      const int pos = base + tok;
-      ws[i] = pos < k1 ? __ldg(p.w + ((int64_t)b * p.n_q_heads + h * G + hh) * p.w_stride + pos) : 0.0f;
-    }
-    __syncthreads();
-    for (int j = threadIdx.x; j < DP; j += 128) {
-      for (int hh = 0; hh < G; ++hh) {
-        float a = acc[hh * DP + j];
-#pragma unroll
-        for (int tok = 0; tok < 16; ++tok) a = fmaf(ws[tok * G + hh], cs[tok][j], a);
-        acc[hh * DP + j] = a;
+__device__ __forceinline__ uint4 decode8(const uint32_t* cw, int kk, const ValuesTcParams& p) {
+  uint4 r;
+  if constexpr (BITS <= 3) {
+    uint32_t sel;
+    if constexpr (BITS == 1) sel = (cw[kk / 4] >> (kk % 4)) & 0x11111111u;
+    else if constexpr (BITS == 2) sel = (cw[kk / 2] >> (2 * (kk % 2))) & 0x33333333u;
+    else {
+      constexpr int full = E / 32;
+      const int gg = kk / 4, j = kk % 4;
+      if (gg < full) {
+        sel = j < 3 ? cw[3 * gg + j] & 0x77777777u
+                    : ((cw[3 * gg] >> 3) & 0x11111111u) | ((cw[3 * gg + 1] >> 2) & 0x22222222u) |
+                          ((cw[3 * gg + 2] >> 1) & 0x44444444u);
+      } else {
+        sel = cw[3 * full + (kk - 4 * full)] & 0x77777777u;
       }
     }
-    __syncthreads();
+    const uint32_t lo = prmt(p.tlo0, p.tlo1, sel), hi = prmt(p.thi0, p.thi1, sel);
+    const uint32_t lo2 = prmt(p.tlo0, p.tlo1, sel >> 16), hi2 = prmt(p.thi0, p.thi1, sel >> 16);
+    r.x = prmt(lo, hi, 0x5140u);
+    r.y = prmt(lo, hi, 0x7362u);
+    r.z = prmt(lo2, hi2, 0x5140u);
+    r.w = prmt(lo2, hi2, 0x7362u);
+  } else {
+    // word kk: nibble a holds element 2a, nibble a + 4 element 2a + 1 (a < 4)
+    const uint32_t x = cw[kk];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t y = x >> (8 * half);           // elements 4 half .. 4 half + 3
+      const uint32_t sel = (y & 0x77u) | ((y >> 8) & 0x7700u);
+      const uint32_t lo = prmt(p.tlo0, p.tlo1, sel), hi = prmt(p.thi0, p.thi1, sel);
+      const uint32_t h0 = prmt(lo, hi, 0x6240u) | ((y << 12) & 0x80008000u);
+      const uint32_t h1 = prmt(lo, hi, 0x7351u) | ((y << 8) & 0x80008000u);
+      if (half == 0) { r.x = h0; r.y = h1; } else { r.z = h0; r.w = h1; }
+    }
   }
-  float* dst = p.partial + (((int64_t)blockIdx.x * gridDim.y + gi) * G) * DP;
-  for (int i = threadIdx.x; i < G * DP; i += 128) dst[i] = acc[i];
+  return r;
 }
 
-// Mode B, pass 2: sum the chunk partials and rotate back, o = Pi^T acc.
-// grid: (batch * n_q_heads); block 128.
-template <int E>
-__global__ void __launch_bounds__(128) finish_kernel(ValuesParams p) {
-  constexpr int DP = 4 * E;
-  __shared__ float a[DP];
-  const int qrow = blockIdx.x;
-  const int b = qrow / p.n_q_heads, hq = qrow % p.n_q_heads;
-  const int h = hq / p.G, hh = hq % p.G;
-  const int gi = b * p.n_kv_heads + h;
-  const int groups = gridDim.x / p.n_q_heads * p.n_kv_heads;
-  for (int j = threadIdx.x; j < DP; j += 128) {
-    float s = 0.0f;
-    for (int c = 0; c < p.n_chunks; ++c)
-      s += p.partial[(((int64_t)c * groups + gi) * p.G + hh) * DP + j];
-    a[j] = s;
+// Mode B, pass 1.  grid: (n_chunks, batch * n_kv_heads, query tiles of 4);
+// block 128; dynamic smem kValWarps * ValShape::kWarpBytes.
+// CTA x of a (group, query tile) owns the 32-token units [x U / n_chunks,
+// (x + 1) U / n_chunks) (U = ceil(max_ctx / 32)); warp w takes its units w,
+// w + 4, ...; lane 0 bulk-copies a unit (32 records, 32 norms) into ring
+// stage i % 2 (mbarrier, bounded wait).  Lane l decodes token l into row l
+// of the warp's fp16 tile (16-byte pieces XOR-swizzled by row: conflict-free
+// stores and ldmatrix reads) and forms w ||v|| for the 4 query slots; then
+// per 16 tokens and 16 coordinates one ldmatrix.x4.trans and one
+// m16n8k16 MMA.  Column pair (2q, 2q + 1) of the accumulators is the hi / lo
+// part of query slot q.  Tokens past the context, on a bad page, or query
+// slots past G get weight 0 (the tile then holds finite table values).  The
+// warps' sums meet in shared memory; the CTA writes one partial.
+template <int BITS, int E>
+__global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcParams p) {
+  constexpr int W = ChunkWords<BITS, E, 0>::W;
+  using VS = ValShape<W, E>;
+  constexpr int REC = VS::kRec, STAGE = VS::kStage, S = kValStages;
+  constexpr int DP = 4 * E;        // padded coordinates
+  constexpr int MT = DP / 16;      // 16-coordinate tiles
+  constexpr int PIECES = DP / 8;   // 16-byte pieces per tile row
+  extern __shared__ __align__(16) uint8_t vsm[];
+  __shared__ int64_t page_base[kValCtaPages];
+  __shared__ uint64_t bars[kValWarps][S];
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int gi = blockIdx.y;
+  const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
+  const int qt = blockIdx.z;
+  const int u0 = (int)((int64_t)blockIdx.x * p.units / p.n_chunks);
+  const int u1 = (int)((int64_t)(blockIdx.x + 1) * p.units / p.n_chunks);
+  const int k0 = 32 * u0;
+  const int kend = min(32 * u1, p.max_ctx);
+  const int ps = p.page_shift;
+  const int P = 1 << ps;
+  const int first_page = k0 >> ps;
+  const int n_pgx = k0 < kend ? ((kend - 1) >> ps) - first_page + 1 : 0;   // <= kValCtaPages
+  const int ctx = min(p.ctx_len[b], p.max_ctx);
+  const int jt = threadIdx.x;
+  static_assert(kValCtaPages <= kValWarps * 32, "one block-table entry per thread");
+  const int64_t pg = jt < n_pgx ? p.cv.block_table[(int64_t)b * p.cv.max_pages + first_page + jt] : 0;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < S; ++s) mbar_init(&bars[warp][s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const int k1 = min(kend, ctx);
+  const bool has_keys = k0 < k1;
+  bool bad = false;
+  if (jt < n_pgx) {
+    const bool valid = pg >= 0 && pg < p.cv.n_pages;
+    page_base[jt] = valid ? pg * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes : -1;
+    if (!valid && has_keys && jt <= ((k1 - 1) >> ps) - first_page) {
+      bad = true;
+      report(p.cv.err, TQ_DEV_ERR_PAGE);
+    }
+  }
+  const bool fast = !__syncthreads_or(bad) && P >= 32;
+
+  const int n_units = has_keys ? (k1 - k0 + 31) >> 5 : 0;
+  const int n_my = warp < n_units ? (n_units - warp + kValWarps - 1) / kValWarps : 0;
+  uint8_t* wbase = vsm + warp * VS::kWarpBytes;
+  const uint32_t ring_s = smem_addr(wbase);
+  uint8_t* tile = wbase + S * STAGE;
+  float4* wn = reinterpret_cast<float4*>(tile + VS::kTile);
+  const int64_t norm_off = (int64_t)P * REC;
+  const uint64_t pol = evict_first_policy();
+
+  auto issue = [&](int i) {
+    if (lane != 0) return;
+    uint64_t* bar = &bars[warp][i & (S - 1)];
+    const uint32_t dst = ring_s + (i & (S - 1)) * STAGE;
+    const int ubase = k0 + 32 * (warp + kValWarps * i);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (fast) {
+      const int slot = ubase & (P - 1);
+      const uint8_t* hb = p.cv.pages + page_base[(ubase >> ps) - first_page];
+      mbar_arrive_tx(bar, 32 * REC + 64);
+      bulk_copy(dst, hb + (int64_t)slot * REC, 32 * REC, bar, pol);
+      bulk_copy(dst + 32 * REC, hb + norm_off + slot * 2, 64, bar, pol);
+      return;
+    }
+    uint32_t bytes = 0;
+    int64_t off[2] = {-1, -1};
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const int base = ubase + 16 * hf;
+      if (base < k1) off[hf] = page_base[(base >> ps) - first_page];
+      if (off[hf] >= 0) bytes += 16 * REC + 32;
+    }
+    mbar_arrive_tx(bar, bytes);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      if (off[hf] < 0) continue;
+      const int slot = (ubase + 16 * hf) & (P - 1);
+      const uint8_t* hb = p.cv.pages + off[hf];
+      bulk_copy(dst + hf * 16 * REC, hb + (int64_t)slot * REC, 16 * REC, bar, pol);
+      bulk_copy(dst + 32 * REC + 32 * hf, hb + norm_off + slot * 2, 32, bar, pol);
+    }
+  };
+#pragma unroll
+  for (int s = 0; s < S; ++s)
+    if (s < n_my) issue(s);
+
+  const int64_t wrow0 = ((int64_t)b * p.n_q_heads + h * p.G + qt * 4) * p.w_stride;
+  const int nq = min(4, p.G - qt * 4);
+  float acc[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+  bool timed_out = false;
+  int issued = min(S, n_my);
+  for (int i = 0; i < n_my; ++i) {
+    const int ubase = k0 + 32 * (warp + kValWarps * i);
+    const int pos = ubase + lane;                 // this lane's token
+    bool tok_ok = pos < k1;
+    if (tok_ok && !fast) tok_ok = page_base[(pos >> ps) - first_page] >= 0;
+    float wv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) wv[q] = (tok_ok && q < nq) ? __ldg(p.w + wrow0 + q * p.w_stride + pos) : 0.0f;
+    if (!mbar_wait(&bars[warp][i & (S - 1)], (uint32_t)(i / S) & 1u)) {
+      timed_out = true;
+      break;
+    }
+    // decode token `lane` into row `lane` of the tile
+    const uint8_t* stg = wbase + (i & (S - 1)) * STAGE;
+    uint32_t rec[4 * W];
+#pragma unroll
+    for (int x = 0; x < W; ++x) {
+      const uint4 v = reinterpret_cast<const uint4*>(stg + lane * REC)[x];
+      rec[4 * x] = v.x; rec[4 * x + 1] = v.y; rec[4 * x + 2] = v.z; rec[4 * x + 3] = v.w;
+    }
+    const float nrm = __half2float(reinterpret_cast<const __half*>(stg + 32 * REC)[lane]);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int kk = 0; kk < E / 8; ++kk) {
+        const int piece = c * (E / 8) + kk;     // coordinates 8 piece .. 8 piece + 7
+        reinterpret_cast<uint4*>(tile + lane * (DP * 2))[piece ^ (lane & 7)] =
+            decode8<BITS, E>(rec + c * W, kk, p);
+      }
+    wn[lane] = make_float4(wv[0] * nrm, wv[1] * nrm, wv[2] * nrm, wv[3] * nrm);
+    __syncwarp();                                 // the tile, wn, and every read of the stage
+    if (i + S < n_my) {
+      issue(i + S);
+      issued = i + S + 1;
+    }
+    // 2 k-steps of 16 tokens: B column g = slice g & 1 of query slot g >> 1
+    const float* wnf = reinterpret_cast<const float*>(wn);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      uint32_t bw[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int tk = 16 * j + 2 * t + 8 * r;
+        const float x0 = wnf[tk * 4 + (g >> 1)], x1 = wnf[(tk + 1) * 4 + (g >> 1)];
+        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+        const __half v0 = (g & 1) ? __float2half_rn(x0 - __half2float(h0)) : h0;
+        const __half v1 = (g & 1) ? __float2half_rn(x1 - __half2float(h1)) : h1;
+        bw[r] = (uint32_t)__half_as_ushort(v0) | ((uint32_t)__half_as_ushort(v1) << 16);
+      }
+      const int mi = lane >> 3, rr = lane & 7;
+      const int row = 16 * j + 8 * (mi >> 1) + rr;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int piece = 2 * mt + (mi & 1);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_trans(smem_addr(tile + row * (DP * 2) + 16 * (piece ^ rr)), a0, a1, a2, a3);
+        mma_f16(acc[mt], a0, a1, a2, a3, make_uint2(bw[0], bw[1]));
+      }
+    }
+    __syncwarp();                                 // the tile is rewritten by the next unit
+  }
+  if (timed_out) {
+    if (lane == 0) report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+    for (int u = max(0, issued - S); u < issued; ++u) mbar_wait(&bars[warp][u & (S - 1)], (uint32_t)(u / S) & 1u);
+  }
+  // the warps' sums meet in shared memory (the rings are free now)
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(vsm);     // [kValWarps][4][DP]
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    red[(warp * 4 + t) * DP + 16 * mt + g] = acc[mt][0] + acc[mt][1];
+    red[(warp * 4 + t) * DP + 16 * mt + g + 8] = acc[mt][2] + acc[mt][3];
   }
   __syncthreads();
-  const int d = p.d;
-  float* o = reinterpret_cast<float*>(p.out) + (int64_t)qrow * d;
-  for (int k = threadIdx.x; k < d; k += 128) {
+  const int gq = gi * p.qtiles + qt;
+  float* dst = p.partial + ((int64_t)blockIdx.x * gridDim.y * gridDim.z + gq) * 4 * DP;
+  for (int i = threadIdx.x; i < 4 * DP; i += kValWarps * 32) {
     float s = 0.0f;
-    for (int j = 0; j < d; ++j) s = fmaf(__ldg(p.pi32 + (size_t)j * d + k), a[j], s);
-    o[k] = s;
+#pragma unroll
+    for (int w2 = 0; w2 < kValWarps; ++w2) s += red[w2 * 4 * DP + i];
+    dst[i] = s;
+  }
+}
+
+// Mode B, pass 2: o = Pi^T sum_chunks partial, one CTA per (query tile,
+// query slot < G); CL x DP threads (CL = 1024 / DP chunk lanes).
+// Launched by programmatic dependent launch: waits for pass 1 first.
+template <int E>
+__global__ void __launch_bounds__(1024) values_finish_kernel(ValuesTcParams p) {
+  constexpr int DP = 4 * E;
+  constexpr int CL = 1024 / DP;    // chunk lanes
+  __shared__ float red[CL][DP];
+  __shared__ float a[DP];
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int gq = blockIdx.x / 4, q = blockIdx.x % 4;
+  const int gi = gq / p.qtiles, qt = gq % p.qtiles;
+  const int hql = qt * 4 + q;                     // query within the group
+  if (hql >= p.G) return;
+  const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
+  const int k = threadIdx.x % DP, cl = threadIdx.x / DP;
+  const int nq = gridDim.x;                       // groups * qtiles * 4
+  float s = 0.0f;
+  const float* src = p.partial + ((int64_t)gq * 4 + q) * DP + k;
+#pragma unroll 4
+  for (int c = cl; c < p.n_chunks; c += CL) s += src[(int64_t)c * nq * DP];
+  red[cl][k] = s;
+  __syncthreads();
+  if (cl == 0) {
+    float t2 = 0.0f;
+#pragma unroll
+    for (int x = 0; x < CL; ++x) t2 += red[x][k];
+    a[k] = t2;
+  }
+  __syncthreads();
+  // o_k' = sum_j Pi[j][k'] a_j: CL lanes each take every CL-th j
+  const int d = p.d;
+  float o = 0.0f;
+  if (k < d)
+    for (int j = cl; j < d; j += CL) o = fmaf(__ldg(p.pi32 + (size_t)j * d + k), a[j], o);
+  __syncthreads();
+  red[cl][k] = o;
+  __syncthreads();
+  if (cl == 0 && k < d) {
+    float t2 = 0.0f;
+#pragma unroll
+    for (int x = 0; x < CL; ++x) t2 += red[x][k];
+    p.out[((int64_t)b * p.n_q_heads + h * p.G + hql) * d + k] = t2;
   }
 }
 
@@ -186,55 +438,71 @@ __global__ void __launch_bounds__(128) finish_kernel(ValuesParams p) {
 
 namespace tq {
 
-static int values_chunks(int64_t groups, int64_t max_ctx, int* tokens_per_cta) {
-  int64_t target = 2 * 148;
-  int64_t chunks = (target + groups - 1) / groups;
-  int64_t tpc = (max_ctx + chunks - 1) / chunks;
-  tpc = ((tpc + 15) / 16) * 16;
-  if (tpc < 16) tpc = 16;
-  *tokens_per_cta = (int)tpc;
-  return (int)((max_ctx + tpc - 1) / tpc);
+// Mode B chunking: every CTA slot of the GPU (148 SMs x 4) gets one CTA, each
+// an equal share (to one 32-token unit) of a sequence; more CTAs when a share
+// would need more than kValCtaPages - 2 block-table entries.
+static int64_t values_chunks(int64_t units_gq, int64_t max_ctx, int page_tokens) {
+  const int64_t units = (max_ctx + 31) / 32;
+  int64_t n = std::max<int64_t>(1, 148LL * 4 / std::max<int64_t>(1, units_gq));
+  const int64_t max_units_cta = (int64_t)(tqd::kValCtaPages - 2) * page_tokens / 32;
+  n = std::max<int64_t>(n, (units + max_units_cta - 1) / max_units_cta);
+  return std::min<int64_t>(n, units);
 }
 
+// The workspace is sized for the smallest page (16 tokens), so it covers
+// every cache of these sizes.
 size_t values_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, int n_q_heads,
                         int64_t max_ctx) {
   if (n_kv_heads <= 0 || n_q_heads <= 0 || max_ctx <= 0) return 0;
-  int tpc;
-  const int64_t groups = batch * n_kv_heads;
-  const int chunks = values_chunks(groups, max_ctx, &tpc);
   const int G = n_q_heads / n_kv_heads;
-  return (size_t)chunks * groups * G * cb->lay.d_pad * sizeof(float);
+  const int64_t gq = batch * n_kv_heads * ((G + 3) / 4);
+  const int64_t chunks = values_chunks(gq, max_ctx, 16);
+  return (size_t)chunks * gq * 4 * cb->lay.d_pad * sizeof(float);
 }
 
 template <int BITS, int E>
-static tq_status run_values(tqd::ValuesParams p, int64_t batch, int64_t max_ctx, bool mode_b,
-                            cudaStream_t st) {
+static tq_status run_values(tqd::ValuesParams p, const tqd::ValuesTcParams& tp, int64_t batch,
+                            int64_t max_ctx, bool mode_b, cudaStream_t st) {
   const int64_t groups = batch * p.n_kv_heads;
   if (!mode_b) {
     dim3 grid((unsigned)((max_ctx + 15) / 16), (unsigned)groups);
     tqd::dequant_kernel<BITS, E><<<grid, 128, 0, st>>>(p);
     return TQ_OK;
   }
-  const size_t dyn = ((size_t)p.G * 4 * E + 16 * p.G) * sizeof(float);
-  if (dyn > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(tqd::accumulate_kernel<BITS, E>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  constexpr int W = tqd::ChunkWords<BITS, E, 0>::W;
+  const int smem = tqd::kValWarps * tqd::ValShape<W, E>::kWarpBytes;
+  static bool attr = false;            // per template instance
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(tqd::values_acc_kernel<BITS, E>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "values: smem attribute");
+    attr = true;
   }
-  dim3 grid((unsigned)p.n_chunks, (unsigned)groups);
-  tqd::accumulate_kernel<BITS, E><<<grid, 128, dyn, st>>>(p);
-  tqd::finish_kernel<E><<<(unsigned)(batch * p.n_q_heads), 128, 0, st>>>(p);
+  dim3 grid((unsigned)tp.n_chunks, (unsigned)groups, (unsigned)tp.qtiles);
+  tqd::values_acc_kernel<BITS, E><<<grid, tqd::kValWarps * 32, smem, st>>>(tp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(groups * tp.qtiles * 4));
+  cfg.blockDim = dim3((1024 / (4 * E)) * (4 * E));   // whole chunk lanes of 4E coordinates
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::values_finish_kernel<E>, tp);
+  if (e != cudaSuccess) return cuda_fail(e, "values: finish launch");
   return TQ_OK;
 }
 
 template <int BITS>
-static int dispatch_values(const Layout& L, const tqd::ValuesParams& p, int64_t batch,
-                           int64_t max_ctx, bool mode_b, cudaStream_t st, tq_status* s) {
+static int dispatch_values(const Layout& L, const tqd::ValuesParams& p, const tqd::ValuesTcParams& tp,
+                           int64_t batch, int64_t max_ctx, bool mode_b, cudaStream_t st, tq_status* s) {
   switch (L.E) {
-    case 16: *s = run_values<BITS, 16>(p, batch, max_ctx, mode_b, st); return 1;
-    case 32: *s = run_values<BITS, 32>(p, batch, max_ctx, mode_b, st); return 1;
-    case 48: *s = run_values<BITS, 48>(p, batch, max_ctx, mode_b, st); return 1;
-    case 64: *s = run_values<BITS, 64>(p, batch, max_ctx, mode_b, st); return 1;
+    case 16: *s = run_values<BITS, 16>(p, tp, batch, max_ctx, mode_b, st); return 1;
+    case 32: *s = run_values<BITS, 32>(p, tp, batch, max_ctx, mode_b, st); return 1;
+    case 48: *s = run_values<BITS, 48>(p, tp, batch, max_ctx, mode_b, st); return 1;
+    case 64: *s = run_values<BITS, 64>(p, tp, batch, max_ctx, mode_b, st); return 1;
   }
   return 0;
 }
@@ -261,18 +529,48 @@ tq_status launch_values(const tq_codebook* cb, const CacheView& cv, const float*
   p.out = out;
   p.odt = odt;
   p.out_stride = out_stride;
-  p.partial = reinterpret_cast<float*>(ws);
-  p.n_chunks = values_chunks(batch * cv.n_kv_heads, max_ctx, &p.tokens_per_cta);
   p.max_ctx = (int)max_ctx;
-  if (mode_b && ws_bytes < values_workspace(cb, batch, cv.n_kv_heads, n_q_heads, max_ctx))
+  tqd::ValuesTcParams tp;
+  tp.cv = cv;
+  int ps = 0;
+  while ((1 << ps) < cv.page_tokens) ++ps;
+  tp.page_shift = ps;
+  tp.ctx_len = ctx_len;
+  tp.n_kv_heads = cv.n_kv_heads;
+  tp.n_q_heads = n_q_heads;
+  tp.G = n_q_heads / cv.n_kv_heads;
+  tp.qtiles = (tp.G + 3) / 4;
+  const int64_t gq = batch * cv.n_kv_heads * tp.qtiles;
+  if (mode_b && (batch * cv.n_kv_heads > 65535 || tp.qtiles > 65535 || gq * 4 > 0x7fffffffLL))
+    return fail(TQ_EINVAL, "tq_dequant_values: batch * n_kv_heads too large");
+  tp.n_chunks = (int)values_chunks(gq, max_ctx, cv.page_tokens);
+  tp.units = (int)((max_ctx + 31) / 32);
+  tp.max_ctx = (int)max_ctx;
+  tp.d = L.d;
+  tp.w = w;
+  tp.w_stride = w_stride;
+  tp.partial = reinterpret_cast<float*>(ws);
+  tp.pi32 = cb->pi32;
+  tp.out = reinterpret_cast<float*>(out);
+  tp.tlo0 = tp.tlo1 = tp.thi0 = tp.thi1 = 0u;
+  {
+    const uint16_t* T = L.bits == 4 ? cb->mag16 : cb->cent16;   // 8 entries
+    for (int i = 0; i < 4; ++i) {
+      tp.tlo0 |= (uint32_t)(T[i] & 0xFF) << (8 * i);
+      tp.tlo1 |= (uint32_t)(T[4 + i] & 0xFF) << (8 * i);
+      tp.thi0 |= (uint32_t)(T[i] >> 8) << (8 * i);
+      tp.thi1 |= (uint32_t)(T[4 + i] >> 8) << (8 * i);
+    }
+  }
+  if (mode_b && ws_bytes < (size_t)tp.n_chunks * gq * 4 * L.d_pad * sizeof(float))
     return fail(TQ_EINVAL, "tq_dequant_values: workspace too small");
   tq_status s = TQ_OK;
   int ok = 0;
   switch (L.bits) {
-    case 1: ok = dispatch_values<1>(L, p, batch, max_ctx, mode_b, st, &s); break;
-    case 2: ok = dispatch_values<2>(L, p, batch, max_ctx, mode_b, st, &s); break;
-    case 3: ok = dispatch_values<3>(L, p, batch, max_ctx, mode_b, st, &s); break;
-    case 4: ok = dispatch_values<4>(L, p, batch, max_ctx, mode_b, st, &s); break;
+    case 1: ok = dispatch_values<1>(L, p, tp, batch, max_ctx, mode_b, st, &s); break;
+    case 2: ok = dispatch_values<2>(L, p, tp, batch, max_ctx, mode_b, st, &s); break;
+    case 3: ok = dispatch_values<3>(L, p, tp, batch, max_ctx, mode_b, st, &s); break;
+    case 4: ok = dispatch_values<4>(L, p, tp, batch, max_ctx, mode_b, st, &s); break;
   }
   if (!ok) return fail(TQ_EUNSUPPORTED, "tq_dequant_values: no kernel for this d");
   if (s != TQ_OK) return s;
