@@ -190,10 +190,10 @@ def run_reference(args):
         if rank != 0:
             _barrier(ws)
             return
-    # calibrate one step to fit the whole run in ~90 s
-    nb, dt = oracle_logits_sample(2048)
-    per_key = dt / 2048
-    n_keys = int(max(256, min(CTX, 90.0 / (args.steps + args.warmup) / max(per_key, 1e-9))))
+    # calibrate one step to fit the whole run in about --ref-budget-s seconds
+    nb, dt = oracle_logits_sample(512)
+    per_key = dt / 512
+    n_keys = int(max(256, min(CTX, args.ref_budget_s / (args.steps + args.warmup) / max(per_key, 1e-9))))
     for _ in range(args.warmup):
         oracle_logits_sample(n_keys)
     tot_b, tot_t = 0, 0.0
@@ -440,6 +440,8 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of extra warm-up steps (clock samples)")
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="seconds of oracle work for --impl reference (all timed and warm-up steps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
