@@ -9,7 +9,7 @@ import pytest
 
 from kv_cache_vector_rotate_b200 import synth
 from oracle import tq_oracle as O
-from parity import compare_codes
+from parity import compare_codes, fp16_ulp
 
 pytestmark = pytest.mark.gpu
 
@@ -147,3 +147,60 @@ def test_empty_append_is_a_no_op(tqm):
     tqm.quantize_append(cb, x, torch.zeros(1, dtype=torch.int32, device="cuda"), cache)
     torch.cuda.synchronize()
     assert not cache.pages.any()
+
+
+@pytest.mark.parametrize("bits,m", [(3, 128), (3, 0), (4, 128), (1, 128)])
+def test_prefill_batch_tensor_core_path(tqm, bits, m):
+    """A prefill-shaped append (bf16, d = 128, thousands of vectors: the
+    tensor-core kernel) against the oracle on every vector of 2 of the 16
+    (sequence, head) pairs and on the norms of all of them."""
+    d, pt = 128, 64
+    batch, heads, n_new = 4, 4, 1024
+    rng = np.random.default_rng(16 + bits + m)
+    xf = rng.standard_normal((batch, heads, n_new, d)).astype(np.float32)
+    xf[rng.random(xf.shape) < 0.01] *= 30.0             # outliers, as in the append workload
+    bits16, vals = synth.to_bf16(xf)
+    bt = synth.block_table(17, batch, n_new // pt)
+    cb, cache = _run_append(tqm, d, bits, m, _dev_tensor(bits16, "bf16"), [0] * batch, batch * n_new // pt, pt, bt)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    for b, h in [(0, 0), (3, 2)]:
+        pos = np.arange(n_new)
+        idx, qneg, n16, r16 = _read_back(lay, cache, bt, b, h, pos)
+        X = vals[b, h]
+        compare_codes(codec, X, O.encode(codec, X), idx, qneg, n16, r16)
+    for b in range(batch):
+        for h in range(heads):
+            _, _, n16, _ = _read_back(lay, cache, bt, b, h, np.arange(n_new))
+            ref = O.fp16(np.linalg.norm(vals[b, h], axis=-1))
+            dn = np.abs(n16.astype(np.float64) - ref.astype(np.float64))
+            assert np.all(dn <= fp16_ulp(ref) + 1e-30)     # fp32 vs fp64 sums: within one fp16 ulp
+    assert cache.errors() == 0
+
+
+def test_tensor_core_path_matches_small_appends(tqm):
+    """The same 2048 bf16 vectors appended at once (tensor-core kernel) and in
+    appends of 8 (CUDA-core kernel) give records that agree except where both
+    are within the oracle's windows."""
+    d, bits, m, pt = 128, 3, 128, 64
+    rng = np.random.default_rng(18)
+    bits16, vals = synth.to_bf16(rng.standard_normal((1, 2, 1024, d)).astype(np.float32))
+    bt = synth.block_table(19, 1, 1024 // pt)
+    x = _dev_tensor(bits16, "bf16")
+    cb, big = _run_append(tqm, d, bits, m, x, [0], 1024 // pt, pt, bt)
+    small = tqm.PagedCache.allocate(cb, 1024 // pt, pt, 2, torch.from_numpy(bt))
+    for s in range(0, 1024, 8):
+        tqm.quantize_append(cb, x[:, :, s:s + 8].contiguous(), torch.tensor([s], dtype=torch.int32, device="cuda"),
+                            small)
+    torch.cuda.synchronize()
+    lay = O.Layout(d, bits, m, pt, 2)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    for h in range(2):
+        pos = np.arange(1024)
+        a = O.read_pages(lay, big.pages.cpu().numpy(), bt, 0, h, pos)
+        c = O.read_pages(lay, small.pages.cpu().numpy(), bt, 0, h, pos)
+        ora = O.encode(codec, vals[0, h])
+        for got in (a, c):
+            compare_codes(codec, vals[0, h], ora, *got)
+        same_idx = (a[0] == c[0]).mean()
+        assert same_idx > 0.9999
