@@ -219,6 +219,51 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def long_context_phase(dev, ws, steps: int = 20):
+    """tq_logits on the long-context decode workload: batch 4, 8 KV / 32
+    query heads, d = 128, context 131072, keys b + QJL m = 128 for b = 2, 3, 4
+    (one cache of 218 - 352 MB, larger than L2, so no replicas).  Device time
+    of a CUDA graph of `steps` calls, max over ranks; algorithmic bytes as in
+    the headline."""
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    batch, hkv, hq, ctx, d, m, pt = 4, 8, 32, 131072, 128, 128, 64
+    out = {"workload": "batch 4, 8 KV / 32 query heads, d 128, context 131072, keys b + QJL m=128, bf16"}
+    K, q = synth.decode_keys_device(1003, batch, hkv, hq, ctx, d, device=dev)
+    pps = ctx // pt
+    bt = torch.from_numpy(synth.block_table(1004, batch, pps))
+    ctx_t = torch.full((batch,), ctx, dtype=torch.int32, device=dev)
+    Lout = torch.empty(batch, hq, ctx, dtype=torch.float32, device=dev)
+    cs = torch.cuda.Stream(device=dev)
+    for bits in (2, 3, 4):
+        cb = tq.Codebook(d, bits, m, synth.SEED_PI, synth.SEED_S)
+        cache = tq.PagedCache.allocate(cb, batch * pps, pt, hkv, bt, device=dev)
+        tq.quantize_append(cb, K, torch.zeros(batch, dtype=torch.int32, device=dev), cache)
+        ws_t = torch.empty(max(16, tq.logits_workspace_bytes(cb, batch, hkv, hq)), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            tq.logits(cb, cache, q, ctx_t, ctx, out=Lout, workspace=ws_t)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            for _ in range(steps):
+                tq.logits(cb, cache, q, ctx_t, ctx, out=Lout, workspace=ws_t)
+        g.replay()
+        torch.cuda.synchronize()
+        _barrier(ws)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record()
+        g.replay()
+        b_.record()
+        torch.cuda.synchronize()
+        ms = _max_over_ranks(a_.elapsed_time(b_), ws, dev) / steps
+        rec = (bits * d + m) // 8 + 4
+        nbytes = batch * hkv * ctx * rec + batch * hq * ctx * 4 + batch * hq * d * 2
+        out[f"b{bits}"] = {"us_per_call": 1e3 * ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "record_bytes": rec}
+        del g, cache
+    return out
+
+
 def run_ours(args):
     import torch
 
@@ -361,6 +406,10 @@ def run_ours(args):
     kq = None
     if not args.no_append_phase:
         kq = append_phase(args, dev, ws)
+    # long-context decode (batch 4, context 131072, b = 2, 3, 4): logits GB/s
+    lc = None
+    if not args.no_long:
+        lc = long_context_phase(dev, ws)
 
     n = ws
     steps = args.steps
@@ -389,6 +438,8 @@ def run_ours(args):
     }
     if kq is not None:
         line["keys_quantized"] = kq
+    if lc is not None:
+        line["long_context"] = lc
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
@@ -440,6 +491,7 @@ def main():
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of extra warm-up steps (clock samples)")
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="seconds of oracle work for --impl reference (all timed and warm-up steps)")
     args = ap.parse_args()

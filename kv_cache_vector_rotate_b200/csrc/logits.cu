@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
     else msk = fmaxf(msk, m);
   }
   int e2 = 0;                        // b = 4: ||q|| in [2^(e2-1), 2^e2)
-  {
+  if (!p.cb_int8) {
     const float qn = sqrtf(qn2s[t]);
     if (qn > 0.0f) frexpf(qn, &e2);
   }
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
     const float mxp = sk ? msk : mpi;
     const int zmax = sk ? kSliceMaxQ : kSliceMax;
     const float scale = mxp > 0.0f ? (float)zmax * __frcp_rn(mxp) : 0.0f;
-    const float f16scale = ldexpf(1.0f, 14 - e2);
+    const float f16scale = p.cb_int8 ? 1.0f : ldexpf(1.0f, 14 - e2);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int l = (int)rank * RB - (sk ? 4 * p.E : 0) + 16 * mt + g + 8 * hh;   // row within its part

@@ -92,3 +92,20 @@ def anisotropic_unit(seed: int, n: int, d: int = 200, chunk: int = 65536) -> np.
         x = rng.standard_normal((e - s, d), dtype=np.float32) * sd[None, :]
         out[s:e] = x / np.linalg.norm(x, axis=1, keepdims=True)
     return out
+
+
+def decode_keys_device(seed: int, batch: int, n_kv_heads: int, n_q_heads: int, ctx: int, d: int = 128,
+                       device="cuda"):
+    """The decode-step laws of decode_step, drawn on the device with torch's
+    seeded generator (for contexts too large to draw on the host): bf16 K
+    [batch, n_kv_heads, ctx, d] ~ N(0, 1) * scale[h, c] (log-uniform [0.1, 10]
+    per (KV head, channel)) and bf16 queries [batch, n_q_heads, d] ~ N(0, 1)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    lo, hi = float(np.log(0.1)), float(np.log(10.0))
+    scale = torch.exp(torch.rand((n_kv_heads, d), generator=g, device=device) * (hi - lo) + lo)
+    k = torch.randn((batch, n_kv_heads, ctx, d), generator=g, device=device)
+    k.mul_(scale[None, :, None, :])
+    q = torch.randn((batch, n_q_heads, d), generator=g, device=device)
+    return k.to(torch.bfloat16), q.to(torch.bfloat16)

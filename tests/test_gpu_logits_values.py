@@ -10,7 +10,7 @@ import pytest
 
 from kv_cache_vector_rotate_b200 import synth
 from oracle import tq_oracle as O
-from parity import LOGIT_TOL, VALUE_TOL, logit_error, oracle_pages
+from parity import LOGIT_TOL, VALUE_TOL, compare_codes, logit_error, oracle_pages
 
 pytestmark = pytest.mark.gpu
 
@@ -157,3 +157,46 @@ def test_values_mode_a_and_b(tqm, d, bits):
         scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
         assert np.all(np.abs(B[b, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None])
     assert cache.errors() == 0
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_long_context_config_sampled(tqm, bits):
+    """Long-context decode: batch 4, 8 KV / 32 query heads, d = 128, context
+    131072, keys b + QJL m = 128, written by the GPU append.  On 256 sampled
+    positions of every (sequence, KV head): the codes against the oracle's
+    encoding of the same vectors, and the GPU logits at those positions
+    against the oracle estimator given the codes read back."""
+    batch, hkv, hq, ctx, d, m, pt = 4, 8, 32, 131072, 128, 128, 64
+    G = hq // hkv
+    K, q = synth.decode_keys_device(1003 + bits, batch, hkv, hq, ctx, d)
+    pps = ctx // pt
+    bt = synth.block_table(25 + bits, batch, pps)
+    cb = tqm.Codebook(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, batch * pps, pt, hkv, torch.from_numpy(bt))
+    tqm.quantize_append(cb, K, torch.zeros(batch, dtype=torch.int32, device="cuda"), cache)
+    ctx_t = torch.full((batch,), ctx, dtype=torch.int32, device="cuda")
+    L = tqm.logits(cb, cache, q, ctx_t, ctx)
+    torch.cuda.synchronize()
+    assert cache.errors() == 0
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, hkv)
+    pages = cache.pages.cpu().numpy()
+    rng = np.random.default_rng(26 + bits)
+    qf = q.float().cpu().numpy().astype(np.float64)
+    worst = 0.0
+    got = {"X": [], "idx": [], "qneg": [], "n16": [], "r16": []}
+    for b in range(batch):
+        for h in range(hkv):
+            pos = np.sort(rng.choice(ctx, 256, replace=False))
+            X = K[b, h, torch.from_numpy(pos).cuda()].float().cpu().numpy().astype(np.float64)
+            idx, qneg, n16, r16 = O.read_pages(lay, pages, bt, b, h, pos)
+            for k_, v_ in zip(got, (X, idx, qneg, n16, r16)):
+                got[k_].append(v_)
+            Qg = qf[b, h * G:(h + 1) * G]
+            Lo = O.logits_from_codes(codec, Qg, idx, qneg, n16, r16)
+            Lg = L[b, h * G:(h + 1) * G][:, torch.from_numpy(pos).cuda()].cpu().numpy()
+            worst = max(worst, logit_error(Lg, Lo, np.linalg.norm(Qg, axis=1), n16, d))
+    assert worst <= LOGIT_TOL, worst
+    # the mismatch rate is a statistic of the whole sample (8192 vectors)
+    X = np.concatenate(got["X"])
+    compare_codes(codec, X, O.encode(codec, X), *(np.concatenate(got[k_]) for k_ in ("idx", "qneg", "n16", "r16")))
