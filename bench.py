@@ -47,12 +47,10 @@ LOGIT_BYTES = B * HKV * CTX * KEY_REC + B * HQ * CTX * 4 + B * HQ * D * 2
 VALUE_BYTES = B * HKV * CTX * VAL_REC + B * HQ * CTX * 4 + B * HQ * D * 4
 APPEND_BYTES = 2 * B * HKV * D * 2 + B * HKV * (KEY_REC + VAL_REC)
 APPEND_CFG = dict(batch=16, heads=8, n_new=4096)
-# DRAM bytes (read + write) of one tq_logits call of this workload, from one
-# ncu capture of the current kernels (--set full, one launch each):
-# logits_kernel<3,32,32> 17,874,176 + 0 and prep_queries_kernel<32> 162,304 + 0.
-LOGITS_DRAM_BYTES = 17874176 + 162304
-LOGITS_DRAM_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, logits_kernel<3,32,32> + "
-                      "prep_queries_kernel<32>, one launch each")
+# DRAM bytes (read + write) of one tq_logits call of this workload as ncu
+# counted them (None until the current kernels have been captured).
+LOGITS_DRAM_BYTES = None
+LOGITS_DRAM_SOURCE = "not captured for the current kernels"
 WORKLOAD = "decode step: batch 1, 8 KV / 32 query heads, head_dim 128, context 32768, keys b=3 + QJL m=128, values b=3"
 
 
@@ -428,7 +426,7 @@ def run_ours(args):
                      "frac": logits_gbs / n / hbm_peak, "traffic": LOGITS_DRAM_BYTES,
                      "traffic_source": LOGITS_DRAM_SOURCE,
                      "peak_source": f"{peak_src} hbm_gbs (copy, burst)",
-                     "kernel": "tq_logits (query prep + fused logits), per launch"},
+                     "kernel": "tq_logits (query preparation + fused logits), per call"},
         "e2e": {"value": n * LOGIT_BYTES * steps / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": q.numel() * 2 + knew.numel() * 2 + vnew.numel() * 2,
                 "d2h_bytes_per_step": Lout.numel() * 4 + Oout.numel() * 4,

@@ -170,9 +170,10 @@ size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n
  * t >= ctx_len[b] are not written.  q: device [batch, n_q_heads, d] of dtype.
  * ctx_len: device int32 [batch], each <= max_ctx <= out_stride.  workspace:
  * device, at least tq_logits_workspace_bytes(), 16-byte aligned (the rotated,
- * sketched queries as tensor-core fragments).  Two kernel launches: the
- * query preparation, then the logits kernel by programmatic dependent
- * launch (it streams the cache while the queries are prepared). */
+ * sketched queries as tensor-core fragments; every call rewrites what it
+ * reads, so it needs no clearing).  Two kernel launches: the query
+ * preparation, then the logits kernel by programmatic dependent launch (it
+ * streams the cache while the queries are prepared). */
 tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
                     tq_dtype dtype, int64_t batch, int32_t n_q_heads,
                     const int32_t* ctx_len, int64_t max_ctx, float* out,

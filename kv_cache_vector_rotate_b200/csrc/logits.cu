@@ -6,30 +6,33 @@
 // evaluated from the indices and sign bits without dequantizing the key.
 //
 // Two kernels per call, chained by programmatic dependent launch:
-//  * prep_queries_kernel: one thread-block cluster per (KV group, tile of 4
-//    query heads); each CTA computes its rows of [Pi q ; S q] on the tensor
-//    cores (bf16 hi + lo fragments of [Pi ; S], pre-swizzled in the
-//    codebook, times the bf16 hi + lo split of the queries, fp32
-//    accumulation), the CTAs exchange their per-query maxima through
-//    distributed shared memory, and each writes its rows as MMA B-fragment
-//    bytes to the workspace.
-//  * logits_kernel: every CTA owns an equal share of one sequence's keys;
-//    its warps stream 32-key units into shared-memory rings with bulk copies
-//    (the first ones in flight before the query fragments exist) and run them
-//    through the tensor cores with the key operand built in registers:
-//     - codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer
-//       of at most 16 bits for every level, so a key element is two int8
-//       slices; eight stored codes form one byte-permute selector after a
-//       single mask, and two permutes of 8-byte tables give the high and low
-//       slices of four elements.  (Pi q) is quantized to 16-bit integers
-//       scaled by its largest entry, also as two int8 slices; the slice
-//       products are accumulated exactly in int32 and combined at the end.
-//     - codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
-//       levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
-//     - sign term: m16n8k32 int8 MMAs.  The stored sign bits enter in place
-//       as 0 / 2^p bytes (one mask per operand register); S q is quantized to
-//       integers z, and sum_i s_i z_i = sum_i z_i - 2 sum_i beta_i z_i.
-//    The MMA's N = 8 columns are the high and low slices of 4 queries.
+//  * prep_queries_kernel: [Pi q ; S q] is split into parts of 32 rows; a
+//    part is computed by one CTA on the tensor cores (bf16 hi + lo fragments
+//    of [Pi ; S], pre-swizzled in the codebook, times the bf16 hi + lo split
+//    of the queries, fp32 accumulation) and written as MMA B-fragment bytes
+//    to the workspace.  Every part quantizes with a scale that needs no
+//    other part: |(Pi q)_j| <= ||q|| (Pi is orthogonal) and
+//    |(S q)_i| <= max_i ||S_i|| ||q||.
+//  * logits_kernel (below), which streams the cache while the queries are
+//    prepared.
+//
+// The logits kernel: every CTA owns an equal share of one sequence's keys;
+// its warps stream 32-key units into shared-memory rings with bulk copies
+// and run them through the tensor cores with the key operand built in
+// registers:
+//  - codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer of
+//    at most 16 bits for every level, so a key element is two int8 slices;
+//    eight stored codes form one byte-permute selector after a single mask,
+//    and two permutes of 8-byte tables give the high and low slices of four
+//    elements.  (Pi q) is quantized to 16-bit integers, also as two int8
+//    slices; the slice products are accumulated exactly in int32 and
+//    combined at the end.
+//  - codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
+//    levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
+//  - sign term: m16n8k32 int8 MMAs.  The stored sign bits enter in place as
+//    0 / 2^p bytes (one mask per operand register); S q is quantized to
+//    integers z, and sum_i s_i z_i = sum_i z_i - 2 sum_i beta_i z_i.
+// The MMA's N = 8 columns are the high and low slices of 4 queries.
 // HBM traffic is the packed records plus the logits.
 
 #include "stream.cuh"
@@ -40,13 +43,17 @@ constexpr int kSliceMax = 32639;   // |z| bound of Pi q: the high int8 slice sta
 constexpr int kSliceMaxQ = 16319;  // |z| bound of S q: 2 z still splits into int8 slices
 constexpr int kLogitsWarps = 4;    // warps per CTA
 constexpr int kCtaPages = 64;      // block-table entries staged per CTA
-constexpr int kMaxCluster = 8;     // CTAs per cluster (portable limit)
+constexpr int kPartRows = 32;      // rows of [Pi q ; S q] per preparation part
 
-// CTAs resident per SM (65536 registers / (128 x this) per thread)
+// CTAs of the logits kernel resident per SM, and its registers per thread:
+// for d <= 128 few enough that a preparation CTA (128 threads x 64
+// registers) still fits beside them (a warp scheduler's share of the
+// register file is 16384: 5 x 88 x 32 + 64 x 32, or 4 x 104 x 32 + 64 x 32),
+// so that no logits CTA has to wait for a preparation CTA to finish
 __host__ __device__ constexpr int logits_min_blocks(int bits, int E) { return E >= 48 ? 4 : bits == 4 ? 4 : 5; }
-
-// rows of [Pi q ; S q] per CTA of a query-preparation cluster: R / C with C <= 8
-__host__ __device__ constexpr int prep_rows_per_cta(int E, int F) { return 4 * (E + F) <= 256 ? 32 : 64; }
+__host__ __device__ constexpr int logits_max_regs(int bits, int E) {
+  return E >= 48 ? 128 : logits_min_blocks(bits, E) == 5 ? 88 : 104;
+}
 
 // Per-warp shared-memory ring: a stage holds one 32-key unit, two 16-key
 // tiles of 16 consecutive records each (16 * 16W bytes, contiguous in its
@@ -58,6 +65,21 @@ struct RingShape {
   static constexpr int kStages = kStageBytes <= 2304 ? 4 : 2;   // a power of two
 };
 
+struct PrepParams {
+  const void* q;             // [batch][n_q_heads][d]
+  tq_dtype dtype;
+  int d, E, F;               // d_pad = 4E, m_pad = 4F
+  int n_q_heads, n_kv_heads, G, qtiles;
+  int cb_int8;               // codebook fragments as int8 slices (b <= 3) or fp16 hi / lo (b = 4)
+  float cb_unscale;          // 2^-f
+  float qjl_scale;           // sqrt(pi/2) / m
+  float s_rowmax;            // >= max_i ||S_i||
+  const uint4* qprep;        // [Pi ; S] bf16 hi + lo A fragments (tq_codebook::qprep_frag)
+  uint2* frag;
+  uint2* qfrag;
+  float2* scal;
+};
+
 struct LogitsParams {
   tq::CacheView cv;
   int page_shift;            // log2(page_tokens)
@@ -66,44 +88,27 @@ struct LogitsParams {
   int n_chunks;              // CTAs per (group, query tile) along the keys
   int units;                 // 32-key units of max_ctx
   int max_ctx;               // ctx_len values are clamped to [0, max_ctx]
-  const uint2* frag;         // workspace: query fragments and scales (prep_queries_kernel)
+  const uint2* frag;         // workspace: query fragments and scales
   const uint2* qfrag;
   const float2* scal;
   float* out;
   int64_t out_stride;
   uint32_t th0, th1, tl0, tl1;  // b <= 3: high / low int8 slices of c16 * 2^f, levels 0..7
   uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
+  int pre_stages;            // ring stages filled before the query fragments are ready (1 .. 4)
 };
 
-// ---- cluster helpers ------------------------------------------------------------
+// ---- loads of the workspace written by the preparation kernel (L2) ------------
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
+__device__ __forceinline__ uint2 ld_cg(const uint2* p) {
+  uint2 v;
+  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
 }
-__device__ __forceinline__ uint32_t cluster_size() {
-  uint32_t n;
-  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(n));
-  return n;
-}
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_arrive_release() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait_acquire() {
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_sync() {
-  cluster_arrive_release();
-  cluster_wait_acquire();
-}
-__device__ __forceinline__ uint32_t map_rank(const void* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
-  return remote;
+__device__ __forceinline__ float2 ld_cg(const float2* p) {
+  float2 v;
+  asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
 }
 
 // ---- MMA wrappers -------------------------------------------------------------------
@@ -214,57 +219,32 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
 // matching the key operand of the logits kernel (sign bytes 2^(2 kk) beta
 // and 2^(2 kk + 1) beta).
 
-struct PrepParams {
-  const void* q;             // [batch][n_q_heads][d]
-  tq_dtype dtype;
-  int d, E, F;               // d_pad = 4E, m_pad = 4F
-  int n_q_heads, n_kv_heads, G, qtiles;
-  int cb_int8;               // codebook fragments as int8 slices (b <= 3) or fp16 hi / lo (b = 4)
-  float cb_unscale;          // 2^-f
-  float qjl_scale;           // sqrt(pi/2) / m
-  const uint4* qprep;        // [Pi ; S] bf16 hi + lo A fragments (tq_codebook::qprep_frag)
-  uint2* frag;
-  uint2* qfrag;
-  float2* scal;
+// Shared memory of one preparation part.
+struct PrepSmem {
+  uint16_t qsb[8][256 + 8];   // column 2 q + s: bf16 slice s of query slot q (padded rows: no bank conflicts)
+  float4 ksum[2][32];         // k-split partial sums
+  float qn2[4];               // ||q||^2 of the 4 query slots
 };
 
-// Rotates and sketches each query once (TQ §How it works: the query is
-// pre-rotated once and reused over the whole context).
-// grid: (C, groups * qtiles), cluster (C, 1, 1), block 128.  CTA `rank`
-// computes rows [rank RB, rank RB + RB) of [Pi q ; S q] for the 4 query
-// slots of its tile (R = d_pad + m_pad = C RB rows; d_pad is a multiple of RB)
-// on the tensor cores: bf16 hi + lo fragments of [Pi ; S] times the bf16
-// hi + lo split of the queries, fp32 accumulation (warp w: 16-row tile
-// w % MT, k split w / MT).  The CTAs exchange their per-slot maxima through
-// distributed shared memory, then quantize their own rows into the workspace
-// fragments; every fragment byte of the tile is written (zeros for padding
-// rows and slots past G), so the workspace needs no clearing.
-template <int RB>
-__global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepParams p) {
-  constexpr int MT = RB / 16;                 // 16-row tiles per CTA (2 or 4)
-  constexpr int KSPL = kLogitsWarps / MT;     // k splits (2 or 1)
-  constexpr int QROW = 256 + 8;               // bf16 per staged query row (padding: no bank conflicts)
-  __shared__ __align__(16) uint16_t qsb[8][QROW];   // column 2 q + s: bf16 slice s of query slot q
-  __shared__ float4 ksum[MT][32];
-  __shared__ float wmax[MT][4];
-  __shared__ float pmax[kMaxCluster][4];      // per-rank maxima, pushed by every rank
-  __shared__ float qn2s[4];
-  asm volatile("griddepcontrol.launch_dependents;");
-  cluster_arrive_relaxed();                   // phase 0 of the cluster barrier
+// Part `r` of query tile gq (TQ §How it works: the query is pre-rotated once
+// and reused over the whole context): rows [32 r, 32 r + 32) of
+// [Pi q ; S q] for the 4 query slots of the tile, on the tensor cores
+// (warp w: 16-row tile w % 2, k half w / 2), quantized and written as
+// fragment bytes.  Every fragment byte of the part is written (zeros for
+// padding rows and slots past G).  Part 0 also writes the slots' scales.
+// All 128 threads of the CTA call it.
+__device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, PrepSmem& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t rank = cluster_rank();
-  const int C = (int)cluster_size();
-  const int gq = blockIdx.y;
   const int gi = gq / p.qtiles, qt = gq % p.qtiles;
   const int b = gi / p.n_kv_heads, kv = gi % p.n_kv_heads;
   const int64_t qbase = (int64_t)b * p.n_q_heads + kv * p.G + qt * 4;   // first query row of the tile
   const int nq = min(4, p.G - qt * 4);
   const int d = p.d, d16 = (d + 15) >> 4;
 
-  const int mt = warp % MT, ksp = warp / MT;
-  const int kb = ksp * d16 / KSPL, ke = (ksp + 1) * d16 / KSPL;     // this warp's k-steps
-  const uint4* afr = p.qprep + (size_t)(rank * MT + mt) * d16 * 64 + lane;
+  const int mt = warp & 1, ksp = warp >> 1;
+  const int kb = ksp * d16 / 2, ke = (ksp + 1) * d16 / 2;     // this warp's k-steps
+  const uint4* afr = p.qprep + (size_t)(r * 2 + mt) * d16 * 64 + lane;
   uint4 af[4][2];
 #pragma unroll
   for (int u = 0; u < 4; ++u)
@@ -303,14 +283,14 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
       const int k = lane + 32 * i;
       if (k < 16 * d16) {
         const uint16_t hb = bf16_bits(x[i]);
-        qsb[2 * warp][k] = hb;
-        qsb[2 * warp + 1][k] = bf16_bits(x[i] - __bfloat162float(__ushort_as_bfloat16(hb)));
+        sm.qsb[2 * warp][k] = hb;
+        sm.qsb[2 * warp + 1][k] = bf16_bits(x[i] - __bfloat162float(__ushort_as_bfloat16(hb)));
       }
       s2 = fmaf(x[i], x[i], s2);
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-    if (lane == 0) qn2s[warp] = s2;
+    if (lane == 0) sm.qn2[warp] = s2;
   }
   __syncthreads();
 
@@ -330,62 +310,29 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
     for (int u = 0; u < 4; ++u)
       if (kc + u < ke) {
         const int k = kc + u;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&qsb[g][16 * k + 2 * t]);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&qsb[g][16 * k + 2 * t + 8]);
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&sm.qsb[g][16 * k + 2 * t]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&sm.qsb[g][16 * k + 2 * t + 8]);
         mma_bf16(acc, af[u][0], b0, b1);
         mma_bf16(acc, af[u][1], b0, b1);
       }
   }
-  if constexpr (KSPL == 2) {
-    if (ksp == 1) ksum[mt][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    __syncthreads();
-    if (ksp == 0) {
-      const float4 o = ksum[mt][lane];
-      acc[0] += o.x; acc[1] += o.y; acc[2] += o.z; acc[3] += o.w;
-    }
-  }
-  const float va = acc[0] + acc[1], vb = acc[2] + acc[3];
-  if (warp < MT) {
-    float mx = fmaxf(fabsf(va), fabsf(vb));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    if (g == 0) wmax[mt][t] = mx;
-  }
+  if (ksp == 1) sm.ksum[mt][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   __syncthreads();
-  cluster_wait_acquire();            // phase 0 complete: every CTA of the cluster exists
-  if ((int)threadIdx.x < 4 * C) {
-    const int qq = threadIdx.x & 3;
-    float m = wmax[0][qq];
-#pragma unroll
-    for (int u = 1; u < MT; ++u) m = fmaxf(m, wmax[u][qq]);
-    asm volatile("st.shared::cluster.f32 [%0], %1;"
-                 ::"r"(map_rank(&pmax[rank][qq], (uint32_t)(threadIdx.x >> 2))), "f"(m) : "memory");
-  }
-  cluster_sync();                    // phase 1: every rank's maxima delivered; no remote access after this
-
-  const int nb_pi = 4 * p.E / RB;    // ranks [0, nb_pi) hold Pi q rows
-  float mpi = 0.0f, msk = 0.0f;      // maxima of query slot t
-  for (int r = 0; r < C; ++r) {
-    const float m = pmax[r][t];
-    if (r < nb_pi) mpi = fmaxf(mpi, m);
-    else msk = fmaxf(msk, m);
-  }
-  int e2 = 0;                        // b = 4: ||q|| in [2^(e2-1), 2^e2)
-  if (!p.cb_int8) {
-    const float qn = sqrtf(qn2s[t]);
-    if (qn > 0.0f) frexpf(qn, &e2);
-  }
-  const bool sk = (int)rank >= nb_pi;
-  if (warp < MT) {
+  const float qn = sqrtf(sm.qn2[t]);
+  const bool sk = r * kPartRows >= 4 * p.E;   // the part holds S q rows
+  if (warp < 2) {
+    const float4 o = sm.ksum[mt][lane];
+    const float va = acc[0] + acc[1] + o.x + o.y, vb = acc[2] + acc[3] + o.z + o.w;
     const int Ep = sk ? p.F : p.E;
-    const float mxp = sk ? msk : mpi;
     const int zmax = sk ? kSliceMaxQ : kSliceMax;
-    const float scale = mxp > 0.0f ? (float)zmax * __frcp_rn(mxp) : 0.0f;
+    const float bound = sk ? p.s_rowmax * qn : qn;
+    const float scale = bound > 0.0f ? (float)zmax * __frcp_rn(bound) : 0.0f;
+    int e2 = 0;                       // b = 4: ||q|| in [2^(e2-1), 2^e2)
+    if (!p.cb_int8 && qn > 0.0f) frexpf(qn, &e2);
     const float f16scale = p.cb_int8 ? 1.0f : ldexpf(1.0f, 14 - e2);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      const int l = (int)rank * RB - (sk ? 4 * p.E : 0) + 16 * mt + g + 8 * hh;   // row within its part
+      const int l = r * kPartRows - (sk ? 4 * p.E : 0) + 16 * mt + g + 8 * hh;   // row within its half
       const float v = hh ? vb : va;
       const int tc = l / Ep, e = l % Ep;        // chunk, row within the chunk
       if (!sk && !p.cb_int8) {
@@ -406,20 +353,23 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
       }
     }
   }
-  if (rank == 0 && (int)threadIdx.x < nq) {
-    const int qq = threadIdx.x;
-    float m0 = 0.0f, m1 = 0.0f;
-    for (int r = 0; r < C; ++r) {
-      if (r < nb_pi) m0 = fmaxf(m0, pmax[r][qq]);
-      else m1 = fmaxf(m1, pmax[r][qq]);
-    }
+  if (r == 0 && (int)threadIdx.x < nq) {
+    const float qq = sqrtf(sm.qn2[threadIdx.x]);
     int e = 0;
-    const float qn = sqrtf(qn2s[qq]);
-    if (qn > 0.0f) frexpf(qn, &e);
-    const float c0 = p.cb_int8 ? m0 * (1.0f / (float)kSliceMax) * p.cb_unscale : ldexpf(1.0f, e - 14);
-    const float c1 = p.qjl_scale * m1 * (1.0f / (float)kSliceMaxQ);
-    p.scal[qbase + qq] = make_float2(c0, c1);
+    if (qq > 0.0f) frexpf(qq, &e);
+    const float c0 = p.cb_int8 ? qq * (1.0f / (float)kSliceMax) * p.cb_unscale : ldexpf(1.0f, e - 14);
+    const float c1 = p.qjl_scale * (p.s_rowmax * qq) * (1.0f / (float)kSliceMaxQ);
+    p.scal[qbase + threadIdx.x] = make_float2(c0, c1);
   }
+  __syncthreads();                  // the shared buffers may be reused
+}
+
+// Two-launch form: grid (parts, groups * qtiles), block 128; the logits
+// kernel follows by programmatic dependent launch.
+__global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepParams p) {
+  __shared__ PrepSmem sm;
+  asm volatile("griddepcontrol.launch_dependents;");
+  prep_part(p, blockIdx.y, blockIdx.x, sm);
 }
 
 // ---- logits -----------------------------------------------------------------------
@@ -428,11 +378,12 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
 // smem kLogitsWarps * S * stage bytes.  CTA x of a (group, query tile) owns
 // the 32-key units [x U / n_chunks, (x + 1) U / n_chunks) of the sequence
 // (U = ceil(max_ctx / 32)): every CTA gets the same work to within one unit.
-// Before it waits for the query preparation kernel (griddepcontrol.wait) a
-// CTA stages its block-table entries (page_tokens is a power of two: page
-// and slot are a shift and a mask) and every warp puts its first S units in
-// flight: lane 0 issues bulk copies of the unit's 32 records and 32 norm
-// slots into ring stage i % S, completing on that stage's mbarrier.  Warp w
+// Before it needs the query fragments a CTA stages its block-table entries
+// (page_tokens is a power of two: page and slot are a shift and a mask) and
+// every warp puts its first S units in flight: lane 0 issues bulk copies of
+// the unit's 32 records and 32 norm slots into ring stage i % S, completing
+// on that stage's mbarrier; then it waits for the preparation kernel
+// (griddepcontrol.wait).  Warp w
 // takes the CTA's units w, w + 4, ...  The two tiles of a unit are read
 // before either is computed, so their MMA chains interleave; a tile whose
 // page is bad or that lies past the context computes on stale bytes and
@@ -443,7 +394,7 @@ __global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepPar
 // every k-step of a word to weight 2^(2 n - 1) (n k-steps in the word), and
 // words are scaled to the common weight 128.
 template <int BITS, int E, int F>
-__global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E)) logits_kernel(LogitsParams p) {
+__global__ void __maxnreg__(logits_max_regs(BITS, E)) logits_kernel(LogitsParams p) {
   constexpr bool kInt8 = BITS <= 3;
   constexpr int KC = kInt8 ? E / 8 : E / 4;   // codebook MMA k-steps
   constexpr int KQ = F / 8;                   // sign-term MMA k-steps
@@ -539,23 +490,26 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E))
       bulk_copy(dst + 2 * TILE + 16 * NB * hf, hb + norm_off + slot * NB, 16 * NB, bar, pol);
     }
   };
+  // the first p.pre_stages units now, the rest of the ring once the query
+  // fragments are in registers (they would queue behind the copies at the SM)
+  int issued = 0;                    // units whose copies were issued
 #pragma unroll
   for (int s = 0; s < S; ++s)
-    if (s < n_my) issue(s);
+    if (s < n_my && s < p.pre_stages) issue(issued++);
 
+  const int gq = gi * p.qtiles + qt;
   // the query fragments and scales come from the preparation kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int gq = gi * p.qtiles + qt;
   uint2 bq[KC];
   const uint2* fsrc = p.frag + (int64_t)gq * KC * 32 + lane;
 #pragma unroll
-  for (int kk = 0; kk < KC; ++kk) bq[kk] = fsrc[kk * 32];
+  for (int kk = 0; kk < KC; ++kk) bq[kk] = ld_cg(fsrc + kk * 32);
   uint2 bz[KQ > 0 ? KQ : 1];
   float zsumf = 0.0f;
   if constexpr (KQ > 0) {
     const uint2* qsrc = p.qfrag + (int64_t)gq * KQ * 32 + lane;
 #pragma unroll
-    for (int kk = 0; kk < KQ; ++kk) bz[kk] = qsrc[kk * 32];
+    for (int kk = 0; kk < KQ; ++kk) bz[kk] = ld_cg(qsrc + kk * 32);
     // sum_i z_i of query t from its own fragments: weights 1 on the 2 z
     // slots and 2 on the z slots give 2 sum z in columns (2t, 2t+1)
     int zs[4] = {0, 0, 0, 0};
@@ -566,7 +520,7 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E))
   const int qidx = qt * 4 + t;                  // this thread's query within the group
   const bool qvalid = qidx < p.G;
   const int hq = h * p.G + (qvalid ? qidx : 0);
-  const float2 sc = p.scal[(int64_t)b * p.n_q_heads + hq];
+  const float2 sc = ld_cg(p.scal + (int64_t)b * p.n_q_heads + hq);
   const float c0 = sc.x;
   const float c1 = F > 0 ? sc.y : 0.0f;
   float* orow = p.out + ((int64_t)b * p.n_q_heads + hq) * p.out_stride;
@@ -637,8 +591,10 @@ __global__ void __launch_bounds__(kLogitsWarps * 32, logits_min_blocks(BITS, E))
     }
   };
 
+#pragma unroll
+  for (int s = 1; s < S; ++s)
+    if (issued == s && s < n_my) issue(issued++);
   bool timed_out = false;
-  int issued = min(S, n_my);         // units whose copies were issued
   for (int i = 0; i < n_my; ++i) {
     if (!mbar_wait(&ring_bar[warp][i & (S - 1)], (uint32_t)(i / S) & 1u)) {
       timed_out = true;
@@ -723,8 +679,16 @@ size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
   return logits_ws_layout(cb, groups, G, groups * G).total;
 }
 
+static int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
 template <int BITS, int E, int F>
-static tq_status run_logits(const tqd::LogitsParams& p, int64_t groups, int qtiles, cudaStream_t st) {
+static tq_status run_logits(const tqd::LogitsParams& p, const tqd::PrepParams& pp, int parts, int64_t groups,
+                            int qtiles, cudaStream_t st) {
   constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
                    : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
   constexpr int W = q0 + (F + 31) / 32;
@@ -735,8 +699,15 @@ static tq_status run_logits(const tqd::LogitsParams& p, int64_t groups, int qtil
     cudaError_t e = cudaFuncSetAttribute(tqd::logits_kernel<BITS, E, F>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "tq_logits: smem attribute");
+    // the preparation kernel asks for the logits kernel's shared-memory
+    // split, or its CTAs would keep logits CTAs off their SMs
+    e = cudaFuncSetAttribute(tqd::prep_queries_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_logits: carveout attribute");
     attr = true;
   }
+  tqd::prep_queries_kernel<<<dim3((unsigned)parts, (unsigned)(groups * qtiles)), tqd::kLogitsWarps * 32, 0, st>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.n_chunks, (unsigned)groups, (unsigned)qtiles);
   cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
@@ -747,40 +718,23 @@ static tq_status run_logits(const tqd::LogitsParams& p, int64_t groups, int qtil
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
+  e = cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
   if (e != cudaSuccess) return cuda_fail(e, "tq_logits launch");
   return TQ_OK;
 }
 
 template <int BITS>
-static tq_status dispatch_logits(const Layout& L, const tqd::LogitsParams& p, int64_t groups, int qtiles,
-                                 cudaStream_t st) {
-  if (L.E == 32 && L.F == 32) return run_logits<BITS, 32, 32>(p, groups, qtiles, st);
-  if (L.E == 32 && L.F == 0) return run_logits<BITS, 32, 0>(p, groups, qtiles, st);
-  if (L.E == 16 && L.F == 16) return run_logits<BITS, 16, 16>(p, groups, qtiles, st);
-  if (L.E == 16 && L.F == 0) return run_logits<BITS, 16, 0>(p, groups, qtiles, st);
-  if (L.E == 64 && L.F == 64) return run_logits<BITS, 64, 64>(p, groups, qtiles, st);
-  if (L.E == 64 && L.F == 0) return run_logits<BITS, 64, 0>(p, groups, qtiles, st);
-  if (L.E == 48 && L.F == 48) return run_logits<BITS, 48, 48>(p, groups, qtiles, st);
-  if (L.E == 48 && L.F == 0) return run_logits<BITS, 48, 0>(p, groups, qtiles, st);
+static tq_status dispatch_logits(const Layout& L, const tqd::LogitsParams& p, const tqd::PrepParams& pp,
+                                 int parts, int64_t groups, int qtiles, cudaStream_t st) {
+  if (L.E == 32 && L.F == 32) return run_logits<BITS, 32, 32>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 32 && L.F == 0) return run_logits<BITS, 32, 0>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 16 && L.F == 16) return run_logits<BITS, 16, 16>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 16 && L.F == 0) return run_logits<BITS, 16, 0>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 64 && L.F == 64) return run_logits<BITS, 64, 64>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 64 && L.F == 0) return run_logits<BITS, 64, 0>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 48 && L.F == 48) return run_logits<BITS, 48, 48>(p, pp, parts, groups, qtiles, st);
+  if (L.E == 48 && L.F == 0) return run_logits<BITS, 48, 0>(p, pp, parts, groups, qtiles, st);
   return fail(TQ_EUNSUPPORTED, "tq_logits: no kernel for this (d, m)");
-}
-
-template <int RB>
-static cudaError_t run_prep(const tqd::PrepParams& pp, int cluster, int64_t units, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cluster, (unsigned)units);
-  cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = st;
-  cudaLaunchAttribute attrs[1];
-  attrs[0].id = cudaLaunchAttributeClusterDimension;
-  attrs[0].val.clusterDim.x = (unsigned)cluster;
-  attrs[0].val.clusterDim.y = 1;
-  attrs[0].val.clusterDim.z = 1;
-  cfg.attrs = attrs;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tqd::prep_queries_kernel<RB>, pp);
 }
 
 tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* q, tq_dtype dt,
@@ -813,16 +767,13 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   pp.cb_int8 = L.bits <= 3 ? 1 : 0;
   pp.cb_unscale = std::ldexp(1.0f, -cb->table_exp);
   pp.qjl_scale = (float)cb->qjl_scale;
+  // |(S q)_i| <= ||S_i|| ||q||: the float bound is rounded up
+  pp.s_rowmax = (float)(cb->s_row_norm_max * (1.0 + 1e-6));
   pp.qprep = cb->qprep_frag;
   pp.frag = frag;
   pp.qfrag = qfrag;
   pp.scal = scal;
-  const int rows = L.d_pad + L.m_pad;
-  const int rb = tqd::prep_rows_per_cta(L.E, L.F);
-  const int cluster = rows / rb;                 // 2 .. 8
-  cudaError_t e = rb == 32 ? run_prep<32>(pp, cluster, groups * qtiles, st)
-                           : run_prep<64>(pp, cluster, groups * qtiles, st);
-  if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
+  const int parts = (L.d_pad + L.m_pad) / tqd::kPartRows;
 
   tqd::LogitsParams lp;
   lp.cv = cv;
@@ -834,15 +785,20 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   lp.n_q_heads = n_q_heads;
   lp.G = G;
   lp.qtiles = qtiles;
-  // Every CTA slot of the GPU (148 SMs x resident CTAs) gets one CTA, each
-  // an equal share (to one 32-key unit) of one sequence's keys; more CTAs
-  // when a share would need more than kCtaPages - 2 block-table entries.
+  // Every CTA slot of the GPU (SMs x resident CTAs) gets one CTA, each an
+  // equal share (to one 32-key unit) of one sequence's keys; more CTAs when a
+  // share would need more than kCtaPages - 2 block-table entries, and then as
+  // many as fill whole waves of the slots (a last, partly filled wave would
+  // run at a fraction of the GPU for as long as a full one).
   const int64_t units = (max_ctx + 31) / 32;
-  const int64_t slots = 148LL * tqd::logits_min_blocks(L.bits, L.E);
-  int64_t n_chunks = std::max<int64_t>(1, slots / (groups * qtiles));
+  const int64_t tiles = groups * qtiles;
+  const int64_t slots = (int64_t)std::max(1, device_sms()) * tqd::logits_min_blocks(L.bits, L.E);
+  int64_t n_chunks = std::max<int64_t>(1, slots / tiles);
   const int64_t max_units_cta = (int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 32;
   n_chunks = std::max<int64_t>(n_chunks, (units + max_units_cta - 1) / max_units_cta);
   n_chunks = std::min<int64_t>(n_chunks, units);
+  const int64_t waves = (n_chunks * tiles + slots - 1) / slots;
+  n_chunks = std::min<int64_t>(std::max<int64_t>(n_chunks, waves * slots / tiles), units);
   if (n_chunks > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_logits: context too long");
   lp.n_chunks = (int)n_chunks;
   lp.units = (int)units;
@@ -852,6 +808,7 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   lp.scal = scal;
   lp.out = out;
   lp.out_stride = out_stride;
+  lp.pre_stages = 1;
   lp.th0 = cb->int8_hi[0];
   lp.th1 = cb->int8_hi[1];
   lp.tl0 = cb->int8_lo[0];
@@ -867,10 +824,10 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
     }
   }
   switch (L.bits) {
-    case 1: return dispatch_logits<1>(L, lp, groups, qtiles, st);
-    case 2: return dispatch_logits<2>(L, lp, groups, qtiles, st);
-    case 3: return dispatch_logits<3>(L, lp, groups, qtiles, st);
-    case 4: return dispatch_logits<4>(L, lp, groups, qtiles, st);
+    case 1: return dispatch_logits<1>(L, lp, pp, parts, groups, qtiles, st);
+    case 2: return dispatch_logits<2>(L, lp, pp, parts, groups, qtiles, st);
+    case 3: return dispatch_logits<3>(L, lp, pp, parts, groups, qtiles, st);
+    case 4: return dispatch_logits<4>(L, lp, pp, parts, groups, qtiles, st);
   }
   return fail(TQ_EUNSUPPORTED, "tq_logits: bits");
 }

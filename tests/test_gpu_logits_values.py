@@ -200,3 +200,42 @@ def test_long_context_config_sampled(tqm, bits):
     # the mismatch rate is a statistic of the whole sample (8192 vectors)
     X = np.concatenate(got["X"])
     compare_codes(codec, X, O.encode(codec, X), *(np.concatenate(got[k_]) for k_ in ("idx", "qneg", "n16", "r16")))
+
+
+def _small_case(tqm, batch, heads, G, ctx, pt, seed, d=128, bits=3, m=128):
+    rng = np.random.default_rng(seed)
+    keys = rng.standard_normal((batch, heads, max(ctx), d))
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, lay, keys, ctx, pt, seed + 1)
+    _, q = synth.to_bf16(rng.standard_normal((batch, heads * G, d)).astype(np.float32))
+    return codec, cb, cache, encs, q
+
+
+def test_logits_workspace_reused_across_shapes(tqm):
+    # One workspace serves calls of three shapes in turn (stale fragments of
+    # a larger shape left in it); each call is exact against the oracle.
+    cases = [(2, 2, 4, [700, 129], 32), (1, 4, 8, [1500], 64), (3, 1, 2, [64, 1, 300], 16)]
+    built = [_small_case(tqm, *c, seed=40 + i) for i, c in enumerate(cases)]
+    need = max(tqm.logits_workspace_bytes(cb, len(c[3]), c[1], c[1] * c[2])
+               for c, (_, cb, _, _, _) in zip(cases, built))
+    ws = torch.full((need,), 0x5A, dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        for (batch, heads, G, ctx, pt), (codec, cb, cache, encs, q) in zip(cases, built):
+            ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+            L = tqm.logits(cb, cache, _q_tensor(q, "bf16"), ctx_t, max(ctx), workspace=ws)
+            torch.cuda.synchronize()
+            _check_logits(codec, q, encs, L.cpu().numpy(), ctx, heads, G)
+            assert cache.errors() == 0
+
+
+def test_logits_more_query_tiles_than_cta_slots(tqm):
+    # 128 sequences x 8 KV heads = 1024 query tiles, short ragged contexts:
+    # more tiles than CTA slots on the GPU (148 SMs x 5), one CTA per tile.
+    ctx = [40 + (i * 7) % 25 for i in range(128)]
+    codec, cb, cache, encs, q = _small_case(tqm, 128, 8, 4, ctx, 16, 50)
+    L = tqm.logits(cb, cache, _q_tensor(q, "bf16"), torch.tensor(ctx, dtype=torch.int32, device="cuda"),
+                   max(ctx))
+    torch.cuda.synchronize()
+    _check_logits(codec, q, encs, L.cpu().numpy(), ctx, 8, 4)
+    assert cache.errors() == 0
