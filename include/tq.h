@@ -76,6 +76,7 @@ typedef enum { TQ_BF16 = 0, TQ_F16 = 1, TQ_F32 = 2 } tq_dtype;
 #define TQ_DEV_ERR_PAGE 1u     /* block-table entry outside [0, n_pages) */
 #define TQ_DEV_ERR_RANGE 2u    /* a norm >= 65520 became +inf in fp16 */
 #define TQ_DEV_ERR_TIMEOUT 4u  /* a bounded mbarrier wait gave up */
+#define TQ_DEV_ERR_CONFIG 8u   /* a kernel found its shared memory misaligned and did nothing */
 
 /* Codec parameters.  d: head dimension, a multiple of 8 with 8 <= d <= 256.
  * bits: Lloyd-Max bits per coordinate, 1..4 on the GPU path (TQ §Stage 1).

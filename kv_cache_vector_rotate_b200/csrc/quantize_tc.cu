@@ -10,26 +10,36 @@
 // run as tcgen05 MMAs (M = N = 128, K = 16, bf16 operands from shared memory,
 // fp32 accumulators in tensor memory).  Pi and S_rot are split into bf16 hi +
 // lo (the input is bf16, so X Pi^T = X Pi_hi + X Pi_lo to fp32 rounding); R
-// is split as well, and P = R_hi S_hi + R_hi S_lo + R_lo S_hi.  One CTA per SM
-// keeps Pi and S_rot resident (128 KB) and walks 128-vector tiles; every
-// thread owns one vector in the epilogues: it reads its row of Y from tensor
-// memory, quantizes, forms the residual (written back as the next MMA's
-// operand), reads its row of P, and assembles its whole record in registers.
+// is split as well, and P = R_hi S_hi + R_hi S_lo + R_lo S_hi.
+//
+// One persistent CTA of 16 warps per SM keeps Pi and S_rot resident (128 KB)
+// and walks 128-vector tiles.  X tiles arrive by TMA (two boxes of 64
+// columns, 128-byte swizzle) into one of two buffers; Y is double-buffered in
+// tensor memory, so the rotation of the next tile runs while this tile's
+// epilogue does.  Warp w reads rows 32 (w % 4) .. + 31 (its tensor-memory
+// lanes) and chunk w / 4 (32 coordinates) of each: the thread quantizes its
+// 32 coordinates, writes their residual into the operand tiles of the
+// sketch (R hi over the spent X buffer, R lo in its own tile), later turns
+// its 32 entries of P into sign bits, and stores its chunk of the record.
 //
 // Shared-memory operands use the K-major 128-byte-swizzle canonical layout:
 // a 128 x 128 bf16 operand is two K-atoms of 128 rows x 128 bytes (16 KB,
-// 1024-byte aligned); 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+// 1024-byte aligned); 16-byte chunk c of row r sits at chunk c ^ (r % 8),
+// which is the layout a TMA box of 64 bf16 columns with 128-byte swizzle
+// writes.
+
+#include <cudaTypedefs.h>
 
 #include "pack.cuh"
 #include "stream.cuh"
 
 namespace tqd {
 
-constexpr int kQtcThreads = 128;                  // 4 warps: warp w owns rows 32w .. 32w + 31
+constexpr int kQtcThreads = 512;                  // 16 warps: rows 32 (w % 4) .., chunk w / 4
 constexpr int kOpBytes = 128 * 128 * 2;           // one 128 x 128 bf16 operand
+constexpr int kAtomBytes = 128 * 128;             // one K-atom: 128 rows x 64 bf16
 
 struct QuantizeTcParams {
-  const __nv_bfloat16* x;    // [rows][128]
   int64_t rows, n_new;       // rows = batch * n_kv_heads * n_new
   int n_kv_heads;
   const int32_t* start_pos;
@@ -95,125 +105,183 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// grid: min(tiles, SMs) persistent CTAs; block 128; dynamic smem
-// (3 + 4 * has_qjl) operands + 1 KB alignment slack.  CTA k takes the
-// 128-row tiles k, k + gridDim.x, ...; thread 32 w + l owns row 32 w + l of
-// the tile, which lives in tensor-memory lane 32 w + l (columns 0..127: Y,
-// 128..255: P).  One elected thread issues the MMAs; every wait on their
-// completion is bounded.
+// One 64-column x 128-row box of the bf16 input (a K-atom of the operand),
+// no multicast, completing on `bar`.
+__device__ __forceinline__ void tma_load_box(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)) : "memory");
+}
+
+// bf16 pair (lo element first) and the bf16 pair of what it leaves of (a, b).
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Small shared state, after the operands in the dynamic shared memory.
+struct QtcState {
+  uint64_t bar_x[2], bar_y[2], bar_p;
+  uint32_t tmem_base;
+  int fail;
+  float sb[16], sc[16];     // boundaries (sb[0] unused) and centroids
+  float part[4][128];       // per-chunk sums of squares of a row: ||x||^2, then ||r||^2
+};
+
+// grid: min(tiles, SMs) persistent CTAs; block 512; dynamic smem (1024-byte
+// aligned): Pi hi/lo, (S_rot hi/lo,) two X/R-hi buffers, (R lo,) QtcState.  CTA c
+// takes the 128-row tiles c, c + gridDim.x, ...  Tensor memory: Y of tile k
+// in columns 128 (k % 2) .. + 127, P in 256 .. 383.  One thread issues the
+// TMA loads and the MMAs; every wait on a copy or an MMA is bounded, and a
+// CTA whose wait gives up reports TQ_DEV_ERR_TIMEOUT, waits (bounded) for
+// what it has in flight and frees its tensor memory.
 template <int BITS, int F>
-__global__ void __launch_bounds__(kQtcThreads, 1) quantize_tc_kernel(QuantizeTcParams p) {
+__global__ void __launch_bounds__(kQtcThreads, 1)
+    quantize_tc_kernel(const __grid_constant__ CUtensorMap tmx, QuantizeTcParams p) {
   constexpr int E = 32;
   constexpr int K = 1 << BITS;
   using CW = ChunkWords<BITS, E, F>;
   constexpr int W = CW::W;
   constexpr bool kQjl = F > 0;
-  constexpr uint32_t kCols = kQjl ? 256 : 128;   // tensor-memory columns (a power of two >= 32)
-  extern __shared__ uint8_t qsm_raw[];
-  __shared__ uint64_t bar_mma;
-  __shared__ uint32_t tmem_base_s;
-  __shared__ float sb[16], sc[16];
-  __shared__ int abort_all;
-
+  constexpr uint32_t kCols = kQjl ? 512 : 256;   // tensor-memory columns (a power of two >= 32)
+  extern __shared__ __align__(1024) uint8_t qsm_raw[];
+  constexpr int kRes = kQjl ? 4 : 2;             // resident operands
+  constexpr int kOps = kRes + (kQjl ? 3 : 2);    // + X/R-hi buffers, R lo
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t base_s = (smem_addr(qsm_raw) + 1023u) & ~1023u;    // SW128 atoms: 1024-byte aligned
-  uint8_t* const base_g = qsm_raw + (base_s - smem_addr(qsm_raw));
-  const uint32_t pi_s = base_s, xt_s = base_s + 2 * kOpBytes, sr_s = base_s + 3 * kOpBytes,
-                 rt_s = base_s + 5 * kOpBytes;
-  uint8_t* const rt_g = base_g + 5 * kOpBytes;
-  uint8_t* const xt_g = base_g + 2 * kOpBytes;
+  const int ch = warp >> 2;                      // chunk: coordinates 32 ch .. 32 ch + 31
+  const int r = 32 * (warp & 3) + lane;          // row of the tile (tensor-memory lane)
+  const uint32_t base_s = smem_addr(qsm_raw);
+  uint8_t* const base_g = qsm_raw;
+  if (base_s & 1023u) {                          // the SW128 atoms need 1024-byte alignment
+    if (tid == 0) report(p.cv.err, TQ_DEV_ERR_CONFIG);
+    return;
+  }
+  QtcState& st = *reinterpret_cast<QtcState*>(qsm_raw + kOps * kOpBytes);
+  uint64_t* const bar_x = st.bar_x;
+  uint64_t* const bar_y = st.bar_y;
+  uint64_t& bar_p = st.bar_p;
+  float* const sb = st.sb;
+  float* const sc = st.sc;
+  const uint32_t pi_s = base_s, sr_s = base_s + 2 * kOpBytes, xr_s = base_s + kRes * kOpBytes,
+                 rl_s = base_s + (kRes + 2) * kOpBytes;
+  uint8_t* const xr_g = base_g + kRes * kOpBytes;
+  uint8_t* const rl_g = base_g + (kRes + 2) * kOpBytes;
+  const int64_t n_my = p.n_tiles > blockIdx.x ? (p.n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
   if (tid == 0) {
-    mbar_init(&bar_mma, 1);
+    mbar_init(&bar_x[0], 1);
+    mbar_init(&bar_x[1], 1);
+    mbar_init(&bar_y[0], 1);
+    mbar_init(&bar_y[1], 1);
+    mbar_init(&bar_p, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    abort_all = 0;
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
+    st.fail = 0;
   }
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                 ::"r"(smem_addr(&tmem_base_s)), "r"(kCols) : "memory");
+                 ::"r"(smem_addr(&st.tmem_base)), "r"(kCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid < K) sc[tid] = p.cent32[tid];
   if (tid < K - 1) sb[tid + 1] = p.bound32[tid];
   if (tid == 0) sb[0] = 0.0f;
   // resident operands: Pi hi / lo (and S_rot hi / lo) in the swizzled layout
-  {
-    const int n_ops = kQjl ? 4 : 2;
-    for (int q = tid; q < n_ops * 128 * 16; q += kQtcThreads) {
-      const int op = q / 2048, r = (q / 16) % 128, c = q % 16;
-      const __nv_bfloat16* src = (op < 2 ? p.pi_bf + (size_t)op * 16384 : p.srot_bf + (size_t)(op - 2) * 16384) +
-                                 (size_t)r * 128 + 8 * c;
-      const uint32_t dst = (op < 2 ? pi_s + op * kOpBytes : sr_s + (op - 2) * kOpBytes) + sw128_offset(r, 8 * c);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int q = tid; q < kRes * 128 * 16; q += kQtcThreads) {
+    const int op = q / 2048, rr = (q / 16) % 128, c = q % 16;
+    const __nv_bfloat16* src = (op < 2 ? p.pi_bf + (size_t)op * 16384 : p.srot_bf + (size_t)(op - 2) * 16384) +
+                               (size_t)rr * 128 + 8 * c;
+    const uint32_t dst = base_s + op * kOpBytes + sw128_offset(rr, 8 * c);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
   }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the copies, visible to the MMAs
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = tmem_base_s;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;     // this warp's tensor-memory lanes
-  uint32_t phase = 0;
+  const uint32_t tmem = st.tmem_base;
+  const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's tensor-memory lanes
 
-  for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
-    const int64_t row0 = tile * 128;
-    // X tile: 128 rows x 16 chunks of 16 bytes, zero past the last row
-    for (int q = tid; q < 128 * 16; q += kQtcThreads) {
-      const int r = q >> 4, c = q & 15;
-      const bool ok = row0 + r < p.rows;
-      const __nv_bfloat16* src = p.x + (ok ? (row0 + r) * 128 + 8 * c : 0);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
-                   ::"r"(xt_s + sw128_offset(r, 8 * c)), "l"(src), "r"(ok ? 16 : 0) : "memory");
-    }
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the copies, visible to the MMAs
-    tc_fence_before();
-    __syncthreads();
+  // Thread 0 issues every copy and MMA and counts, per barrier, the phases
+  // it started and the completions it has seen (the n-th completion of a
+  // barrier has parity n % 2), so that a failed CTA can wait out what is in
+  // flight.  Every thread knows the parities of the waits in the loop from k.
+  int x_iss[2] = {0, 0}, x_done[2] = {0, 0}, y_iss[2] = {0, 0}, y_done[2] = {0, 0}, p_iss = 0, p_done = 0;
+  auto issue_x = [&](int64_t k) {                // TMA of tile k into buffer k % 2
+    const int bb = (int)(k & 1);
+    const int y = (int)((blockIdx.x + k * gridDim.x) * 128);
+    mbar_arrive_tx(&bar_x[bb], kOpBytes);
+    tma_load_box(xr_s + bb * kOpBytes, &tmx, 0, y, &bar_x[bb]);
+    tma_load_box(xr_s + bb * kOpBytes + kAtomBytes, &tmx, 64, y, &bar_x[bb]);
+    ++x_iss[bb];
+  };
+  auto issue_y = [&](int64_t k) -> bool {        // Y(k) = X(k) Pi^T once X(k) has landed
+    const int bb = (int)(k & 1);
+    if (!mbar_wait(&bar_x[bb], (uint32_t)(x_done[bb] & 1))) return false;
+    ++x_done[bb];
     tc_fence_after();
+    const uint32_t xs = xr_s + bb * kOpBytes, d = tmem + 128 * bb;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const uint32_t koff = (ks >> 2) * kAtomBytes + (ks & 3) * 32;
+      const uint64_t ad = sw128_desc(xs + koff);
+      tc_mma(d, ad, sw128_desc(pi_s + koff), ks > 0);
+      tc_mma(d, ad, sw128_desc(pi_s + kOpBytes + koff), 1);
+    }
+    tc_commit(&bar_y[bb]);
+    ++y_iss[bb];
+    return true;
+  };
+  if (tid == 0) {
+    for (int64_t k = 0; k < n_my && k < 2; ++k) issue_x(k);
+    if (n_my > 0 && !issue_y(0)) st.fail = 1;
+  }
+  __syncthreads();                               // st.fail
 
-    // Y = X Pi^T (X Pi_hi + X Pi_lo), 8 K-steps of 16
-    if (tid == 0) {
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-        const uint64_t ad = sw128_desc(xt_s + koff);
-        tc_mma(tmem, ad, sw128_desc(pi_s + koff), ks > 0);
-        tc_mma(tmem, ad, sw128_desc(pi_s + kOpBytes + koff), 1);
-      }
-      tc_commit(&bar_mma);
-    }
-    // this thread's row: ||x|| from the tile (while the MMAs run)
-    const int r = tid;
+  bool aborted = false;
+  for (int64_t k = 0; k < n_my; ++k) {
+    const int bb = (int)(k & 1);
+    const int64_t row0 = (blockIdx.x + k * gridDim.x) * 128;
+    // X(k) landed (this thread reads it) and Y(k) is complete
+    bool ok = st.fail == 0 && mbar_wait(&bar_x[bb], (uint32_t)((k >> 1) & 1)) &&
+              mbar_wait(&bar_y[bb], (uint32_t)((k >> 1) & 1));
+    if (ok && tid == 0) ++y_done[bb];
+    // ||x||^2 of this thread's 32 coordinates, from the X tile
     float n2 = 0.0f;
+    {
+      const uint8_t* xt = xr_g + bb * kOpBytes;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(xt_g + sw128_offset(r, 8 * c));
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128_offset(r, 32 * ch + 8 * c));
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = __uint_as_float(w4[e] << 16), b2 = __uint_as_float(w4[e] & 0xFFFF0000u);
-        n2 = fmaf(a, a, fmaf(b2, b2, n2));
+        for (int e = 0; e < 4; ++e) {
+          const float a = __uint_as_float(w4[e] << 16), b2 = __uint_as_float(w4[e] & 0xFFFF0000u);
+          n2 = fmaf(a, a, fmaf(b2, b2, n2));
+        }
       }
     }
-    const float nrm = sqrtf(n2);
-    const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
-    bool ok = mbar_wait(&bar_mma, phase);
-    phase ^= 1u;
-    if (__syncthreads_or(!ok)) {
-      if (tid == 0) abort_all = 1;
+    st.part[ch][r] = n2;
+    tc_fence_before();
+    if (__syncthreads_or(!ok)) {                 // every X read of the buffer is done past this point
+      aborted = true;
       break;
     }
     tc_fence_after();
+    const float nrm = sqrtf(st.part[0][r] + st.part[1][r] + st.part[2][r] + st.part[3][r]);
+    const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
 
-    // quantize: indices, residual (as the next MMA's operand), record words
-    uint32_t rec[4 * W];
+    // quantize this chunk: index bits, residual (the sketch operand)
+    uint32_t rec[W];
 #pragma unroll
-    for (int i = 0; i < 4 * W; ++i) rec[i] = 0u;
+    for (int i = 0; i < W; ++i) rec[i] = 0u;
     float rr2 = 0.0f;
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
+    {
       float y[32];
-      tmem_ld32(tmem + lane_base + 32 * t, y);
+      tmem_ld32(tmem + lane_base + 128 * bb + 32 * ch, y);
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
         const float u = y[e] * inv;
@@ -223,69 +291,72 @@ __global__ void __launch_bounds__(kQtcThreads, 1) quantize_tc_kernel(QuantizeTcP
           if (u >= sb[idx + step]) idx += step;
         const uint32_t code = stored_code<BITS>(idx);
 #pragma unroll
-        for (int k = 0; k < (BITS == 4 ? 4 : BITS); ++k)
-          rec[t * W + code_word<BITS, E>(e, k)] |= ((code >> k) & 1u) << code_bit<BITS, E>(e, k);
+        for (int kb = 0; kb < (BITS == 4 ? 4 : BITS); ++kb)
+          rec[code_word<BITS, E>(e, kb)] |= ((code >> kb) & 1u) << code_bit<BITS, E>(e, kb);
         y[e] = u - sc[idx];                       // residual, rotated space
         rr2 = fmaf(y[e], y[e], rr2);
       }
       if constexpr (kQjl) {
-        // residual as bf16 hi / lo, 8 values per 16-byte chunk
+        // residual as bf16 hi (over the spent X tile) / lo, 8 values per 16-byte chunk
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t hw[4], lw[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float a0 = y[8 * c + 2 * e], a1 = y[8 * c + 2 * e + 1];
-            const __nv_bfloat16 h0 = __float2bfloat16_rn(a0), h1 = __float2bfloat16_rn(a1);
-            const __nv_bfloat16 l0 = __float2bfloat16_rn(a0 - __bfloat162float(h0));
-            const __nv_bfloat16 l1 = __float2bfloat16_rn(a1 - __bfloat162float(h1));
-            hw[e] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-            lw[e] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
-          }
-          const uint32_t off = sw128_offset(r, 32 * t + 8 * c);
-          *reinterpret_cast<uint4*>(rt_g + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(rt_g + kOpBytes + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          for (int e = 0; e < 4; ++e) split_bf16x2(y[8 * c + 2 * e], y[8 * c + 2 * e + 1], hw[e], lw[e]);
+          const uint32_t off = sw128_offset(r, 32 * ch + 8 * c);
+          *reinterpret_cast<uint4*>(xr_g + bb * kOpBytes + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(rl_g + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
         }
       }
     }
-    const float rn = sqrtf(rr2);
-
-    if constexpr (kQjl) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the residual tile, visible to the MMAs
-      tc_fence_before();
-      __syncthreads();
-      tc_fence_after();
-      // P = R S_rot^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
-      if (tid == 0) {
+    // R (and the reads of X) ordered before the copies and MMAs that come next
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();                             // R complete; every read of Y(k) and of the ||x|| sums done
+    tc_fence_after();
+    st.part[ch][r] = rr2;                        // read after the next CTA barrier
+    if (tid == 0) {
+      if constexpr (kQjl) {
+        // P = R S_rot^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
+        const uint32_t rh_s = xr_s + bb * kOpBytes;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-          const uint64_t rh = sw128_desc(rt_s + koff), rl = sw128_desc(rt_s + kOpBytes + koff);
-          tc_mma(tmem + 128, rh, sw128_desc(sr_s + koff), ks > 0);
-          tc_mma(tmem + 128, rh, sw128_desc(sr_s + kOpBytes + koff), 1);
-          tc_mma(tmem + 128, rl, sw128_desc(sr_s + koff), 1);
+          const uint32_t koff = (ks >> 2) * kAtomBytes + (ks & 3) * 32;
+          const uint64_t rh = sw128_desc(rh_s + koff), rl = sw128_desc(rl_s + koff);
+          tc_mma(tmem + 256, rh, sw128_desc(sr_s + koff), ks > 0);
+          tc_mma(tmem + 256, rh, sw128_desc(sr_s + kOpBytes + koff), 1);
+          tc_mma(tmem + 256, rl, sw128_desc(sr_s + koff), 1);
         }
-        tc_commit(&bar_mma);
+        tc_commit(&bar_p);
+        ++p_iss;
       }
-      ok = mbar_wait(&bar_mma, phase);
-      phase ^= 1u;
+      // the next tile's rotation, behind the sketch in the tensor pipe
+      if (k + 1 < n_my && !issue_y(k + 1)) st.fail = 1;
+      // without a sketch the X buffer is free once Y(k) was read
+      if constexpr (!kQjl) {
+        if (k + 2 < n_my) issue_x(k + 2);
+      }
+    }
+    if constexpr (kQjl) {
+      ok = mbar_wait(&bar_p, (uint32_t)(k & 1));
+      if (ok && tid == 0) ++p_done;
+      tc_fence_before();
       if (__syncthreads_or(!ok)) {
-        if (tid == 0) abort_all = 1;
+        aborted = true;
         break;
       }
       tc_fence_after();
+      // R hi of this tile is spent: the buffer takes tile k + 2
+      if (tid == 0 && k + 2 < n_my) issue_x(k + 2);
+      float pv[32];
+      tmem_ld32(tmem + lane_base + 256 + 32 * ch, pv);
+      uint32_t qw = 0u;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float pv[32];
-        tmem_ld32(tmem + 128 + lane_base + 32 * t, pv);
-        uint32_t qw = 0u;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) qw |= (pv[e] < 0.0f ? 1u : 0u) << qjl_bit(e);
-        rec[t * W + CW::q0] = qw;
-      }
+      for (int e = 0; e < 32; ++e) qw |= (pv[e] < 0.0f ? 1u : 0u) << qjl_bit(e);
+      rec[CW::q0] = qw;
     }
 
-    // store the record and the norm slot
+    // store this chunk of the record (and, chunk 0, the norm slot)
     const int64_t row = row0 + r;
     if (row < p.rows) {
       const int64_t per_seq = (int64_t)p.n_kv_heads * p.n_new;
@@ -295,33 +366,44 @@ __global__ void __launch_bounds__(kQtcThreads, 1) quantize_tc_kernel(QuantizeTcP
       const int64_t hb = head_block_offset(p.cv, b, h, pos);
       if (hb >= 0) {
         const int slot = (int)(pos % p.cv.page_tokens);
-        uint8_t* recp = p.cv.pages + hb + (int64_t)slot * 16 * W;
+        uint8_t* recp = p.cv.pages + hb + (int64_t)slot * 16 * W + ch * 4 * W;
         if constexpr (W % 4 == 0) {
 #pragma unroll
-          for (int i = 0; i < W; ++i)
-            reinterpret_cast<uint4*>(recp)[i] =
-                make_uint4(rec[4 * i], rec[4 * i + 1], rec[4 * i + 2], rec[4 * i + 3]);
+          for (int i = 0; i < W / 4; ++i)
+            reinterpret_cast<uint4*>(recp)[i] = make_uint4(rec[4 * i], rec[4 * i + 1], rec[4 * i + 2], rec[4 * i + 3]);
+        } else if constexpr (W % 2 == 0) {
+#pragma unroll
+          for (int i = 0; i < W / 2; ++i) reinterpret_cast<uint2*>(recp)[i] = make_uint2(rec[2 * i], rec[2 * i + 1]);
         } else {
 #pragma unroll
-          for (int i = 0; i < 4 * W; ++i) reinterpret_cast<uint32_t*>(recp)[i] = rec[i];
+          for (int i = 0; i < W; ++i) reinterpret_cast<uint32_t*>(recp)[i] = rec[i];
         }
-        const __half nh = __float2half_rn(nrm);
-        if (__hisinf(nh)) report(p.cv.err, TQ_DEV_ERR_RANGE);
-        __half* ns = reinterpret_cast<__half*>(p.cv.pages + hb + (int64_t)p.cv.page_tokens * 16 * W +
-                                               (int64_t)slot * (kQjl ? 4 : 2));
-        ns[0] = nh;
-        if constexpr (kQjl) ns[1] = __float2half_rn(rn);
+        if (ch == 0) {
+          const __half nh = __float2half_rn(nrm);
+          if (__hisinf(nh)) report(p.cv.err, TQ_DEV_ERR_RANGE);
+          __half* ns = reinterpret_cast<__half*>(p.cv.pages + hb + (int64_t)p.cv.page_tokens * 16 * W +
+                                                 (int64_t)slot * (kQjl ? 4 : 2));
+          ns[0] = nh;
+          if constexpr (kQjl) ns[1] = __float2half_rn(sqrtf(st.part[0][r] + st.part[1][r] + st.part[2][r] + st.part[3][r]));
+        }
       }
     }
     tc_fence_before();
-    __syncthreads();                               // tensor memory and the tiles are reused
+    __syncthreads();                             // partial sums, R lo and P are reused
     tc_fence_after();
   }
 
-  if (abort_all) {
-    // a completion wait gave up: report, wait (bounded) for the MMAs in flight
-    if (tid == 0) report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
-    mbar_wait(&bar_mma, phase);
+  if (__syncthreads_or(st.fail != 0 || aborted)) {
+    // a wait gave up: report, then wait (bounded) for every copy and MMA this
+    // CTA put in flight before its shared and tensor memory are released
+    if (tid == 0) {
+      report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+      for (int bb = 0; bb < 2; ++bb) {
+        while (x_done[bb] < x_iss[bb] && mbar_wait(&bar_x[bb], (uint32_t)(x_done[bb] & 1))) ++x_done[bb];
+        while (y_done[bb] < y_iss[bb] && mbar_wait(&bar_y[bb], (uint32_t)(y_done[bb] & 1))) ++y_done[bb];
+      }
+      while (p_done < p_iss && mbar_wait(&bar_p, (uint32_t)(p_done & 1))) ++p_done;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -333,9 +415,27 @@ __global__ void __launch_bounds__(kQtcThreads, 1) quantize_tc_kernel(QuantizeTcP
 
 namespace tq {
 
+// cuTensorMapEncodeTiled from the driver, through the runtime (no link
+// against libcuda).
+static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    looked = true;
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }
+  return fn;
+}
+
 template <int BITS, int F>
-static tq_status run_quantize_tc(const tqd::QuantizeTcParams& p, int sms, cudaStream_t st) {
-  const int smem = (F > 0 ? 7 : 3) * tqd::kOpBytes + 1024;
+static tq_status run_quantize_tc(const CUtensorMap& map, const tqd::QuantizeTcParams& p, int sms,
+                                 cudaStream_t st) {
+  constexpr int ops = F > 0 ? 7 : 4;
+  const int smem = ops * tqd::kOpBytes + (int)sizeof(tqd::QtcState);
   static bool attr = false;            // per template instance
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(tqd::quantize_tc_kernel<BITS, F>,
@@ -344,7 +444,7 @@ static tq_status run_quantize_tc(const tqd::QuantizeTcParams& p, int sms, cudaSt
     attr = true;
   }
   const int64_t grid = p.n_tiles < sms ? p.n_tiles : sms;
-  tqd::quantize_tc_kernel<BITS, F><<<(unsigned)grid, tqd::kQtcThreads, smem, st>>>(p);
+  tqd::quantize_tc_kernel<BITS, F><<<(unsigned)grid, tqd::kQtcThreads, smem, st>>>(map, p);
   return cuda_fail(cudaGetLastError(), "quantize_tc launch");
 }
 
@@ -360,16 +460,28 @@ tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, 
   *handled = false;
   const int64_t rows = batch * n_kv_heads * n_new;
   if (dt != TQ_BF16 || L.d != 128 || L.d_pad != 128 || !(L.m_pad == 0 || L.m_pad == 128) ||
-      rows < kMinRows || (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
+      rows < kMinRows || rows > 0x7fffff00LL || (reinterpret_cast<uintptr_t>(x) & 15u) != 0)
     return TQ_OK;
+  const PFN_cuTensorMapEncodeTiled_v12000 encode = encode_tiled_fn();
+  if (!encode) return TQ_OK;
   static int sms = 0;
   if (!sms) {
     int dev = 0;
     cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
   }
+  // X as a 2-D bf16 tensor [rows][128]; a box is 64 columns (128 bytes) x
+  // 128 rows, written with the 128-byte swizzle; rows past the end read as 0
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {128 * sizeof(__nv_bfloat16)};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  if (encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return fail(TQ_ECUDA, "quantize_tc: cuTensorMapEncodeTiled");
   tqd::QuantizeTcParams p;
-  p.x = reinterpret_cast<const __nv_bfloat16*>(x);
   p.rows = rows;
   p.n_new = n_new;
   p.n_kv_heads = n_kv_heads;
@@ -383,10 +495,10 @@ tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, 
   tq_status s = TQ_OK;
   const bool q = L.m_pad == 128;
   switch (L.bits) {
-    case 1: s = q ? run_quantize_tc<1, 32>(p, sms, st) : run_quantize_tc<1, 0>(p, sms, st); break;
-    case 2: s = q ? run_quantize_tc<2, 32>(p, sms, st) : run_quantize_tc<2, 0>(p, sms, st); break;
-    case 3: s = q ? run_quantize_tc<3, 32>(p, sms, st) : run_quantize_tc<3, 0>(p, sms, st); break;
-    case 4: s = q ? run_quantize_tc<4, 32>(p, sms, st) : run_quantize_tc<4, 0>(p, sms, st); break;
+    case 1: s = q ? run_quantize_tc<1, 32>(map, p, sms, st) : run_quantize_tc<1, 0>(map, p, sms, st); break;
+    case 2: s = q ? run_quantize_tc<2, 32>(map, p, sms, st) : run_quantize_tc<2, 0>(map, p, sms, st); break;
+    case 3: s = q ? run_quantize_tc<3, 32>(map, p, sms, st) : run_quantize_tc<3, 0>(map, p, sms, st); break;
+    case 4: s = q ? run_quantize_tc<4, 32>(map, p, sms, st) : run_quantize_tc<4, 0>(map, p, sms, st); break;
     default: return TQ_OK;
   }
   *handled = true;

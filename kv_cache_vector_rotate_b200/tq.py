@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "_lib", "libtq.so")
 
 TQ_OK, TQ_EINVAL, TQ_EUNSUPPORTED, TQ_ERANGE, TQ_ETIMEOUT, TQ_ECUDA, TQ_ENOMEM = range(7)
 TQ_BF16, TQ_F16, TQ_F32 = 0, 1, 2
-DEV_ERR_PAGE, DEV_ERR_RANGE, DEV_ERR_TIMEOUT = 1, 2, 4
+DEV_ERR_PAGE, DEV_ERR_RANGE, DEV_ERR_TIMEOUT, DEV_ERR_CONFIG = 1, 2, 4, 8
 
 # Every entry point declared in include/tq.h.
 EXPORTS = (

@@ -204,3 +204,59 @@ def test_tensor_core_path_matches_small_appends(tqm):
             compare_codes(codec, vals[0, h], ora, *got)
         same_idx = (a[0] == c[0]).mean()
         assert same_idx > 0.9999
+
+
+def test_tensor_core_many_tiles_ragged(tqm):
+    """4 x 8 x 1999 bf16 vectors: 500 tiles of 128 (the last one 96 rows), so
+    each persistent CTA walks 3-4 tiles through both X buffers and both
+    tensor-memory Y buffers; 3 (sequence, head) pairs against the oracle,
+    every norm within one fp16 ulp."""
+    d, bits, m, pt = 128, 3, 128, 64
+    batch, heads, n_new = 4, 8, 1999
+    rng = np.random.default_rng(26)
+    xf = rng.standard_normal((batch, heads, n_new, d)).astype(np.float32)
+    xf[rng.random(xf.shape) < 0.01] *= 30.0
+    bits16, vals = synth.to_bf16(xf)
+    pps = (n_new + pt - 1) // pt
+    bt = synth.block_table(27, batch, pps)
+    cb, cache = _run_append(tqm, d, bits, m, _dev_tensor(bits16, "bf16"), [0] * batch, batch * pps, pt, bt)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    pages = cache.pages.cpu().numpy()
+    for b, h in [(0, 0), (1, 5), (3, 7)]:
+        idx, qneg, n16, r16 = O.read_pages(lay, pages, bt, b, h, np.arange(n_new))
+        compare_codes(codec, vals[b, h], O.encode(codec, vals[b, h]), idx, qneg, n16, r16)
+    for b in range(batch):
+        for h in range(heads):
+            _, _, n16, _ = O.read_pages(lay, pages, bt, b, h, np.arange(n_new))
+            ref = O.fp16(np.linalg.norm(vals[b, h], axis=-1))
+            assert np.all(np.abs(n16.astype(np.float64) - ref.astype(np.float64)) <= fp16_ulp(ref) + 1e-30)
+    assert cache.errors() == 0
+
+
+def test_append_workload_full_size_sampled(tqm):
+    """The online-append workload at full size (16 x 8 KV heads x 4096 new
+    bf16 tokens, 1% outliers x30, 64-token pages, b = 3 + QJL m = 128), in
+    the launch the benchmark times: 2048 sampled records against the
+    oracle."""
+    d, bits, m, pt = 128, 3, 128, 64
+    batch, heads, n_new = 16, 8, 4096
+    bits16, vals = synth.append_batch(1005, batch, heads, n_new, d)
+    pps = n_new // pt
+    bt = synth.block_table(1006, batch, pps)
+    cb, cache = _run_append(tqm, d, bits, m, _dev_tensor(bits16, "bf16"), [0] * batch, batch * pps, pt, bt)
+    codec = O.make_codec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, m, pt, heads)
+    pages = cache.pages.cpu().numpy()
+    rng = np.random.default_rng(28)
+    X, got = [], [[], [], [], []]
+    for _ in range(16):
+        b, h = int(rng.integers(batch)), int(rng.integers(heads))
+        pos = np.sort(rng.choice(n_new, 128, replace=False))
+        for acc, part in zip(got, O.read_pages(lay, pages, bt, b, h, pos)):
+            acc.append(part)
+        X.append(vals[b, h, pos].astype(np.float64))
+    X = np.concatenate(X)
+    idx, qneg, n16, r16 = (np.concatenate(a) for a in got)
+    compare_codes(codec, X, O.encode(codec, X), idx, qneg, n16, r16)
+    assert cache.errors() == 0
