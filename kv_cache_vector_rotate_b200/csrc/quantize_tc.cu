@@ -113,6 +113,16 @@ __device__ __forceinline__ void tma_load_box(uint32_t dst, const CUtensorMap* ma
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)) : "memory");
 }
 
+// True when the stored code of local element e occupies consecutive bits of
+// one chunk word (then it is ORed in with one shift).
+template <int BITS, int E>
+__host__ __device__ constexpr bool code_contiguous(int e) {
+  for (int k = 1; k < (BITS == 4 ? 4 : BITS); ++k)
+    if (code_word<BITS, E>(e, k) != code_word<BITS, E>(e, 0) || code_bit<BITS, E>(e, k) != code_bit<BITS, E>(e, 0) + k)
+      return false;
+  return true;
+}
+
 // bf16 pair (lo element first) and the bf16 pair of what it leaves of (a, b).
 __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -124,20 +134,37 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
 
 // Small shared state, after the operands in the dynamic shared memory.
 struct QtcState {
-  uint64_t bar_x[2], bar_y[2], bar_p;
+  uint64_t bar_x, bar_y, bar_p[2];
   uint32_t tmem_base;
   int fail;
   float sb[16], sc[16];     // boundaries (sb[0] unused) and centroids
-  float part[4][128];       // per-chunk sums of squares of a row: ||x||^2, then ||r||^2
+  float part_x[4][128];     // per-chunk sums of squares of a row (||x||^2)
 };
 
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
+__device__ __forceinline__ float tmem_ld4_sum(uint32_t taddr) {
+  uint32_t a, b, c, d;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(taddr) : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  return (__uint_as_float(a) + __uint_as_float(b)) + (__uint_as_float(c) + __uint_as_float(d));
+}
+
 // grid: min(tiles, SMs) persistent CTAs; block 512; dynamic smem (1024-byte
-// aligned): Pi hi/lo, (S_rot hi/lo,) two X/R-hi buffers, (R lo,) QtcState.  CTA c
-// takes the 128-row tiles c, c + gridDim.x, ...  Tensor memory: Y of tile k
-// in columns 128 (k % 2) .. + 127, P in 256 .. 383.  One thread issues the
-// TMA loads and the MMAs; every wait on a copy or an MMA is bounded, and a
-// CTA whose wait gives up reports TQ_DEV_ERR_TIMEOUT, waits (bounded) for
-// what it has in flight and frees its tensor memory.
+// aligned): Pi hi/lo, (S_rot hi/lo,) the X tile, (R hi, R lo,) QtcState.
+// CTA c takes the 128-row tiles c, c + gridDim.x, ...  Tensor memory: Y in
+// columns 0..127; with a sketch, P of tile k in 128 + 128 (k % 2) .. + 127 and
+// the four per-chunk ||r||^2 of each row in 384 + 4 (k % 2) .. + 3.
+// Iteration k: ||x|| from X(k); the X tile is then free and the copy of
+// X(k + 1) starts; the thread quantizes its chunk of Y(k) and, once the
+// sketch of tile k - 1 is done with R, writes its residual to R; after a CTA
+// barrier one thread issues the sketch of tile k and another the rotation of
+// tile k + 1, while every thread turns P(k - 1) into sign bits and stores the
+// records of tile k - 1.  Every wait on a copy or an MMA is bounded; a CTA
+// whose wait gives up reports TQ_DEV_ERR_TIMEOUT, waits (bounded) for what it
+// has in flight and frees its tensor memory.
 template <int BITS, int F>
 __global__ void __launch_bounds__(kQtcThreads, 1)
     quantize_tc_kernel(const __grid_constant__ CUtensorMap tmx, QuantizeTcParams p) {
@@ -146,37 +173,32 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
   using CW = ChunkWords<BITS, E, F>;
   constexpr int W = CW::W;
   constexpr bool kQjl = F > 0;
-  constexpr uint32_t kCols = kQjl ? 512 : 256;   // tensor-memory columns (a power of two >= 32)
+  constexpr uint32_t kCols = kQjl ? 512 : 128;   // tensor-memory columns (a power of two >= 32)
+  constexpr uint32_t kColP = 128, kColR = 384;
   extern __shared__ __align__(1024) uint8_t qsm_raw[];
   constexpr int kRes = kQjl ? 4 : 2;             // resident operands
-  constexpr int kOps = kRes + (kQjl ? 3 : 2);    // + X/R-hi buffers, R lo
+  constexpr int kOps = kRes + (kQjl ? 3 : 1);    // + X, R hi, R lo
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ch = warp >> 2;                      // chunk: coordinates 32 ch .. 32 ch + 31
   const int r = 32 * (warp & 3) + lane;          // row of the tile (tensor-memory lane)
   const uint32_t base_s = smem_addr(qsm_raw);
-  uint8_t* const base_g = qsm_raw;
   if (base_s & 1023u) {                          // the SW128 atoms need 1024-byte alignment
     if (tid == 0) report(p.cv.err, TQ_DEV_ERR_CONFIG);
     return;
   }
   QtcState& st = *reinterpret_cast<QtcState*>(qsm_raw + kOps * kOpBytes);
-  uint64_t* const bar_x = st.bar_x;
-  uint64_t* const bar_y = st.bar_y;
-  uint64_t& bar_p = st.bar_p;
-  float* const sb = st.sb;
-  float* const sc = st.sc;
-  const uint32_t pi_s = base_s, sr_s = base_s + 2 * kOpBytes, xr_s = base_s + kRes * kOpBytes,
-                 rl_s = base_s + (kRes + 2) * kOpBytes;
-  uint8_t* const xr_g = base_g + kRes * kOpBytes;
-  uint8_t* const rl_g = base_g + (kRes + 2) * kOpBytes;
+  const uint32_t pi_s = base_s, sr_s = base_s + 2 * kOpBytes, x_s = base_s + kRes * kOpBytes,
+                 rh_s = x_s + kOpBytes, rl_s = x_s + 2 * kOpBytes;
+  const uint8_t* const x_g = qsm_raw + kRes * kOpBytes;
+  uint8_t* const rh_g = qsm_raw + (kRes + 1) * kOpBytes;
+  uint8_t* const rl_g = qsm_raw + (kRes + 2) * kOpBytes;
   const int64_t n_my = p.n_tiles > blockIdx.x ? (p.n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
   if (tid == 0) {
-    mbar_init(&bar_x[0], 1);
-    mbar_init(&bar_x[1], 1);
-    mbar_init(&bar_y[0], 1);
-    mbar_init(&bar_y[1], 1);
-    mbar_init(&bar_p, 1);
+    mbar_init(&st.bar_x, 1);
+    mbar_init(&st.bar_y, 1);
+    mbar_init(&st.bar_p[0], 1);
+    mbar_init(&st.bar_p[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
     st.fail = 0;
@@ -186,9 +208,9 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
                  ::"r"(smem_addr(&st.tmem_base)), "r"(kCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tid < K) sc[tid] = p.cent32[tid];
-  if (tid < K - 1) sb[tid + 1] = p.bound32[tid];
-  if (tid == 0) sb[0] = 0.0f;
+  if (tid < K) st.sc[tid] = p.cent32[tid];
+  if (tid < K - 1) st.sb[tid + 1] = p.bound32[tid];
+  if (tid == 0) st.sb[0] = 0.0f;
   // resident operands: Pi hi / lo (and S_rot hi / lo) in the swizzled layout
   for (int q = tid; q < kRes * 128 * 16; q += kQtcThreads) {
     const int op = q / 2048, rr = (q / 16) % 128, c = q % 16;
@@ -204,206 +226,243 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
   tc_fence_after();
   const uint32_t tmem = st.tmem_base;
   const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;   // this warp's tensor-memory lanes
+  const float* const sb = st.sb;
+  const float* const sc = st.sc;
 
-  // Thread 0 issues every copy and MMA and counts, per barrier, the phases
-  // it started and the completions it has seen (the n-th completion of a
-  // barrier has parity n % 2), so that a failed CTA can wait out what is in
-  // flight.  Every thread knows the parities of the waits in the loop from k.
-  int x_iss[2] = {0, 0}, x_done[2] = {0, 0}, y_iss[2] = {0, 0}, y_done[2] = {0, 0}, p_iss = 0, p_done = 0;
-  auto issue_x = [&](int64_t k) {                // TMA of tile k into buffer k % 2
-    const int bb = (int)(k & 1);
+  // Thread kIssueY (warp 4) issues the copies and the rotation MMAs, thread
+  // kIssueP (warp 8) the sketch MMAs; each counts, per barrier it issues
+  // to, the phases it started and the completions it has seen (the n-th
+  // completion of a barrier has parity n % 2), so that a failed CTA can wait
+  // out what is in flight.  Every thread knows the parities of the waits in
+  // the loop from k.  Descriptors of consecutive K-steps differ only in the
+  // start-address field (address >> 4, 14 bits, never carried out of).
+  constexpr int kIssueY = 128, kIssueP = 256;
+  int x_iss = 0, x_done = 0, y_iss = 0, y_done = 0, p_iss[2] = {0, 0}, p_done[2] = {0, 0};
+  const uint64_t d_pih = sw128_desc(pi_s), d_pil = sw128_desc(pi_s + kOpBytes), d_x = sw128_desc(x_s);
+  const uint64_t d_srh = sw128_desc(sr_s), d_srl = sw128_desc(sr_s + kOpBytes);
+  const uint64_t d_rh = sw128_desc(rh_s), d_rl = sw128_desc(rl_s);
+  auto issue_x = [&](int64_t k) {                // TMA of tile k (two 64-column boxes)
     const int y = (int)((blockIdx.x + k * gridDim.x) * 128);
-    mbar_arrive_tx(&bar_x[bb], kOpBytes);
-    tma_load_box(xr_s + bb * kOpBytes, &tmx, 0, y, &bar_x[bb]);
-    tma_load_box(xr_s + bb * kOpBytes + kAtomBytes, &tmx, 64, y, &bar_x[bb]);
-    ++x_iss[bb];
+    mbar_arrive_tx(&st.bar_x, kOpBytes);
+    tma_load_box(x_s, &tmx, 0, y, &st.bar_x);
+    tma_load_box(x_s + kAtomBytes, &tmx, 64, y, &st.bar_x);
+    ++x_iss;
   };
-  auto issue_y = [&](int64_t k) -> bool {        // Y(k) = X(k) Pi^T once X(k) has landed
-    const int bb = (int)(k & 1);
-    if (!mbar_wait(&bar_x[bb], (uint32_t)(x_done[bb] & 1))) return false;
-    ++x_done[bb];
+  auto issue_y = [&]() -> bool {                 // Y = X Pi^T once the X tile has landed
+    if (!mbar_wait(&st.bar_x, (uint32_t)(x_done & 1))) return false;
+    ++x_done;
     tc_fence_after();
-    const uint32_t xs = xr_s + bb * kOpBytes, d = tmem + 128 * bb;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const uint32_t koff = (ks >> 2) * kAtomBytes + (ks & 3) * 32;
-      const uint64_t ad = sw128_desc(xs + koff);
-      tc_mma(d, ad, sw128_desc(pi_s + koff), ks > 0);
-      tc_mma(d, ad, sw128_desc(pi_s + kOpBytes + koff), 1);
+      const uint32_t ko = ((ks >> 2) * kAtomBytes + (ks & 3) * 32) >> 4;
+      tc_mma(tmem, d_x + ko, d_pih + ko, ks > 0);
+      tc_mma(tmem, d_x + ko, d_pil + ko, 1);
     }
-    tc_commit(&bar_y[bb]);
-    ++y_iss[bb];
+    tc_commit(&st.bar_y);
+    ++y_iss;
     return true;
   };
-  if (tid == 0) {
-    for (int64_t k = 0; k < n_my && k < 2; ++k) issue_x(k);
-    if (n_my > 0 && !issue_y(0)) st.fail = 1;
+  if (tid == kIssueY && n_my > 0) {
+    issue_x(0);
+    if (!issue_y()) st.fail = 1;
   }
   __syncthreads();                               // st.fail
 
+  // the tile whose signs and record are still to be done (sketch form)
+  uint32_t rec_prev[W];
+  int64_t hb_prev = -1;
+  int slot_prev = 0;
+  float nrm_prev = 0.0f;
   bool aborted = false;
-  for (int64_t k = 0; k < n_my; ++k) {
-    const int bb = (int)(k & 1);
-    const int64_t row0 = (blockIdx.x + k * gridDim.x) * 128;
-    // X(k) landed (this thread reads it) and Y(k) is complete
-    bool ok = st.fail == 0 && mbar_wait(&bar_x[bb], (uint32_t)((k >> 1) & 1)) &&
-              mbar_wait(&bar_y[bb], (uint32_t)((k >> 1) & 1));
-    if (ok && tid == 0) ++y_done[bb];
-    // ||x||^2 of this thread's 32 coordinates, from the X tile
-    float n2 = 0.0f;
-    {
-      const uint8_t* xt = xr_g + bb * kOpBytes;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(xt + sw128_offset(r, 32 * ch + 8 * c));
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float a = __uint_as_float(w4[e] << 16), b2 = __uint_as_float(w4[e] & 0xFFFF0000u);
-          n2 = fmaf(a, a, fmaf(b2, b2, n2));
-        }
-      }
-    }
-    st.part[ch][r] = n2;
-    tc_fence_before();
-    if (__syncthreads_or(!ok)) {                 // every X read of the buffer is done past this point
-      aborted = true;
-      break;
-    }
-    tc_fence_after();
-    const float nrm = sqrtf(st.part[0][r] + st.part[1][r] + st.part[2][r] + st.part[3][r]);
-    const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
 
-    // quantize this chunk: index bits, residual (the sketch operand)
-    uint32_t rec[W];
-#pragma unroll
-    for (int i = 0; i < W; ++i) rec[i] = 0u;
-    float rr2 = 0.0f;
-    {
-      float y[32];
-      tmem_ld32(tmem + lane_base + 128 * bb + 32 * ch, y);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float u = y[e] * inv;
-        int idx = 0;
-#pragma unroll
-        for (int step = K / 2; step >= 1; step >>= 1)
-          if (u >= sb[idx + step]) idx += step;
-        const uint32_t code = stored_code<BITS>(idx);
-#pragma unroll
-        for (int kb = 0; kb < (BITS == 4 ? 4 : BITS); ++kb)
-          rec[code_word<BITS, E>(e, kb)] |= ((code >> kb) & 1u) << code_bit<BITS, E>(e, kb);
-        y[e] = u - sc[idx];                       // residual, rotated space
-        rr2 = fmaf(y[e], y[e], rr2);
-      }
-      if constexpr (kQjl) {
-        // residual as bf16 hi (over the spent X tile) / lo, 8 values per 16-byte chunk
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t hw[4], lw[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) split_bf16x2(y[8 * c + 2 * e], y[8 * c + 2 * e + 1], hw[e], lw[e]);
-          const uint32_t off = sw128_offset(r, 32 * ch + 8 * c);
-          *reinterpret_cast<uint4*>(xr_g + bb * kOpBytes + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(rl_g + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        }
-      }
-    }
-    // R (and the reads of X) ordered before the copies and MMAs that come next
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();                             // R complete; every read of Y(k) and of the ||x|| sums done
-    tc_fence_after();
-    st.part[ch][r] = rr2;                        // read after the next CTA barrier
-    if (tid == 0) {
-      if constexpr (kQjl) {
-        // P = R S_rot^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
-        const uint32_t rh_s = xr_s + bb * kOpBytes;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * kAtomBytes + (ks & 3) * 32;
-          const uint64_t rh = sw128_desc(rh_s + koff), rl = sw128_desc(rl_s + koff);
-          tc_mma(tmem + 256, rh, sw128_desc(sr_s + koff), ks > 0);
-          tc_mma(tmem + 256, rh, sw128_desc(sr_s + kOpBytes + koff), 1);
-          tc_mma(tmem + 256, rl, sw128_desc(sr_s + koff), 1);
-        }
-        tc_commit(&bar_p);
-        ++p_iss;
-      }
-      // the next tile's rotation, behind the sketch in the tensor pipe
-      if (k + 1 < n_my && !issue_y(k + 1)) st.fail = 1;
-      // without a sketch the X buffer is free once Y(k) was read
-      if constexpr (!kQjl) {
-        if (k + 2 < n_my) issue_x(k + 2);
-      }
-    }
+  // P(j) into sign bits, then the record of tile j (and its norm slot)
+  auto finish = [&](int64_t j) {
     if constexpr (kQjl) {
-      ok = mbar_wait(&bar_p, (uint32_t)(k & 1));
-      if (ok && tid == 0) ++p_done;
-      tc_fence_before();
-      if (__syncthreads_or(!ok)) {
-        aborted = true;
-        break;
-      }
-      tc_fence_after();
-      // R hi of this tile is spent: the buffer takes tile k + 2
-      if (tid == 0 && k + 2 < n_my) issue_x(k + 2);
       float pv[32];
-      tmem_ld32(tmem + lane_base + 256 + 32 * ch, pv);
+      tmem_ld32(tmem + lane_base + kColP + 128 * (uint32_t)(j & 1) + 32 * ch, pv);
       uint32_t qw = 0u;
 #pragma unroll
       for (int e = 0; e < 32; ++e) qw |= (pv[e] < 0.0f ? 1u : 0u) << qjl_bit(e);
-      rec[CW::q0] = qw;
+      rec_prev[CW::q0] = qw;
     }
+    float rn = 0.0f;
+    if (kQjl && ch == 0) rn = sqrtf(tmem_ld4_sum(tmem + lane_base + kColR + 4 * (uint32_t)(j & 1)));
+    if (hb_prev >= 0) {
+      uint8_t* recp = p.cv.pages + hb_prev + (int64_t)slot_prev * 16 * W + ch * 4 * W;
+      if constexpr (W % 4 == 0) {
+#pragma unroll
+        for (int i = 0; i < W / 4; ++i)
+          reinterpret_cast<uint4*>(recp)[i] =
+              make_uint4(rec_prev[4 * i], rec_prev[4 * i + 1], rec_prev[4 * i + 2], rec_prev[4 * i + 3]);
+      } else if constexpr (W % 2 == 0) {
+#pragma unroll
+        for (int i = 0; i < W / 2; ++i) reinterpret_cast<uint2*>(recp)[i] = make_uint2(rec_prev[2 * i], rec_prev[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < W; ++i) reinterpret_cast<uint32_t*>(recp)[i] = rec_prev[i];
+      }
+      if (ch == 0) {
+        const __half nh = __float2half_rn(nrm_prev);
+        if (__hisinf(nh)) report(p.cv.err, TQ_DEV_ERR_RANGE);
+        __half* ns = reinterpret_cast<__half*>(p.cv.pages + hb_prev + (int64_t)p.cv.page_tokens * 16 * W +
+                                               (int64_t)slot_prev * (kQjl ? 4 : 2));
+        ns[0] = nh;
+        if constexpr (kQjl) ns[1] = __float2half_rn(rn);
+      }
+    }
+  };
 
-    // store this chunk of the record (and, chunk 0, the norm slot)
+  for (int64_t k = 0; k < n_my; ++k) {
+    const int64_t row0 = (blockIdx.x + k * gridDim.x) * 128;
+    // where this row's record goes (the block-table read overlaps the waits)
     const int64_t row = row0 + r;
+    int64_t hb = -1;
+    int slot = 0;
     if (row < p.rows) {
       const int64_t per_seq = (int64_t)p.n_kv_heads * p.n_new;
       const int64_t b = row / per_seq;
       const int h = (int)((row / p.n_new) % p.n_kv_heads);
       const int64_t pos = p.start_pos[b] + row % p.n_new;
-      const int64_t hb = head_block_offset(p.cv, b, h, pos);
-      if (hb >= 0) {
-        const int slot = (int)(pos % p.cv.page_tokens);
-        uint8_t* recp = p.cv.pages + hb + (int64_t)slot * 16 * W + ch * 4 * W;
-        if constexpr (W % 4 == 0) {
+      hb = head_block_offset(p.cv, b, h, pos);
+      slot = (int)(pos % p.cv.page_tokens);
+    }
+    // X(k) landed (this thread reads it) and Y(k) is complete
+    bool ok = st.fail == 0 && mbar_wait(&st.bar_x, (uint32_t)(k & 1)) && mbar_wait(&st.bar_y, (uint32_t)(k & 1));
+    if (ok && tid == kIssueY) ++y_done;
+    float n2 = 0.0f;
 #pragma unroll
-          for (int i = 0; i < W / 4; ++i)
-            reinterpret_cast<uint4*>(recp)[i] = make_uint4(rec[4 * i], rec[4 * i + 1], rec[4 * i + 2], rec[4 * i + 3]);
-        } else if constexpr (W % 2 == 0) {
+    for (int c = 0; c < 4; ++c) {
+      const uint4 v = *reinterpret_cast<const uint4*>(x_g + sw128_offset(r, 32 * ch + 8 * c));
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int i = 0; i < W / 2; ++i) reinterpret_cast<uint2*>(recp)[i] = make_uint2(rec[2 * i], rec[2 * i + 1]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < W; ++i) reinterpret_cast<uint32_t*>(recp)[i] = rec[i];
-        }
-        if (ch == 0) {
-          const __half nh = __float2half_rn(nrm);
-          if (__hisinf(nh)) report(p.cv.err, TQ_DEV_ERR_RANGE);
-          __half* ns = reinterpret_cast<__half*>(p.cv.pages + hb + (int64_t)p.cv.page_tokens * 16 * W +
-                                                 (int64_t)slot * (kQjl ? 4 : 2));
-          ns[0] = nh;
-          if constexpr (kQjl) ns[1] = __float2half_rn(sqrtf(st.part[0][r] + st.part[1][r] + st.part[2][r] + st.part[3][r]));
-        }
+      for (int e = 0; e < 4; ++e) {
+        const float a = __uint_as_float(w4[e] << 16), b2 = __uint_as_float(w4[e] & 0xFFFF0000u);
+        n2 = fmaf(a, a, fmaf(b2, b2, n2));
       }
     }
+    st.part_x[ch][r] = n2;
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the reads of X before the next copy
     tc_fence_before();
-    __syncthreads();                             // partial sums, R lo and P are reused
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
     tc_fence_after();
+    if (tid == kIssueY && k + 1 < n_my) issue_x(k + 1);   // X(k) was read by Y(k) and by every thread
+    const float nrm = sqrtf((st.part_x[0][r] + st.part_x[1][r]) + (st.part_x[2][r] + st.part_x[3][r]));
+    const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
+
+    // quantize this chunk of Y(k): index bits and residual
+    uint32_t rec[W];
+#pragma unroll
+    for (int i = 0; i < W; ++i) rec[i] = 0u;
+    float rr2 = 0.0f;
+    float y[32];
+    tmem_ld32(tmem + lane_base + 32 * ch, y);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float u = y[e] * inv;
+      int idx = 0;
+#pragma unroll
+      for (int step = K / 2; step >= 1; step >>= 1)
+        if (u >= sb[idx + step]) idx += step;
+      const uint32_t code = stored_code<BITS>(idx);
+      if (code_contiguous<BITS, E>(e)) {
+        rec[code_word<BITS, E>(e, 0)] |= code << code_bit<BITS, E>(e, 0);
+      } else {
+#pragma unroll
+        for (int kb = 0; kb < (BITS == 4 ? 4 : BITS); ++kb)
+          rec[code_word<BITS, E>(e, kb)] |= ((code >> kb) & 1u) << code_bit<BITS, E>(e, kb);
+      }
+      y[e] = u - sc[idx];                       // residual, rotated space
+      rr2 = fmaf(y[e], y[e], rr2);
+    }
+    bool ok2 = true;
+    if constexpr (kQjl) {
+      tmem_st1(tmem + lane_base + kColR + 4 * (uint32_t)(k & 1) + ch, rr2);
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      // R is free once the sketch of tile k - 1 is done (its P is read below)
+      if (k > 0) {
+        ok2 = mbar_wait(&st.bar_p[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1));
+        if (ok2 && tid == kIssueP) ++p_done[(k - 1) & 1];
+      }
+      // residual as bf16 hi / lo, 8 values per 16-byte chunk
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_bf16x2(y[8 * c + 2 * e], y[8 * c + 2 * e + 1], hw[e], lw[e]);
+        const uint32_t off = sw128_offset(r, 32 * ch + 8 * c);
+        *reinterpret_cast<uint4*>(rh_g + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(rl_g + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // R, visible to the MMAs
+    }
+    tc_fence_before();
+    if (__syncthreads_or(!ok2)) {                // R complete; every read of Y(k) done
+      aborted = true;
+      break;
+    }
+    tc_fence_after();
+    if constexpr (kQjl) {
+      if (tid == kIssueP) {
+        // P(k) = R S_rot^T: R_hi S_hi + R_hi S_lo + R_lo S_hi
+        const uint32_t dcol = tmem + kColP + 128 * (uint32_t)(k & 1);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ko = ((ks >> 2) * kAtomBytes + (ks & 3) * 32) >> 4;
+          tc_mma(dcol, d_rh + ko, d_srh + ko, ks > 0);
+          tc_mma(dcol, d_rh + ko, d_srl + ko, 1);
+          tc_mma(dcol, d_rl + ko, d_srh + ko, 1);
+        }
+        tc_commit(&st.bar_p[k & 1]);
+        ++p_iss[k & 1];
+      }
+    }
+    // the next tile's rotation (Y(k) has been read)
+    if (tid == kIssueY && k + 1 < n_my && !issue_y()) st.fail = 1;
+    if constexpr (kQjl) {
+      if (k > 0) finish(k - 1);                  // P(k - 1) completed before R was written
+      hb_prev = hb;
+      slot_prev = slot;
+      nrm_prev = nrm;
+#pragma unroll
+      for (int i = 0; i < W; ++i) rec_prev[i] = rec[i];
+    } else {
+      hb_prev = hb;
+      slot_prev = slot;
+      nrm_prev = nrm;
+#pragma unroll
+      for (int i = 0; i < W; ++i) rec_prev[i] = rec[i];
+      finish(k);
+    }
+  }
+  if constexpr (kQjl) {
+    // the last tile's signs and record
+    if (!aborted && n_my > 0) {
+      const int64_t j = n_my - 1;
+      const bool ok = mbar_wait(&st.bar_p[j & 1], (uint32_t)((j >> 1) & 1));
+      if (ok && tid == kIssueP) ++p_done[j & 1];
+      tc_fence_before();
+      if (__syncthreads_or(!ok)) aborted = true;
+      else {
+        tc_fence_after();
+        finish(j);
+      }
+    }
   }
 
   if (__syncthreads_or(st.fail != 0 || aborted)) {
     // a wait gave up: report, then wait (bounded) for every copy and MMA this
     // CTA put in flight before its shared and tensor memory are released
-    if (tid == 0) {
+    if (tid == kIssueY) {
       report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
-      for (int bb = 0; bb < 2; ++bb) {
-        while (x_done[bb] < x_iss[bb] && mbar_wait(&bar_x[bb], (uint32_t)(x_done[bb] & 1))) ++x_done[bb];
-        while (y_done[bb] < y_iss[bb] && mbar_wait(&bar_y[bb], (uint32_t)(y_done[bb] & 1))) ++y_done[bb];
-      }
-      while (p_done < p_iss && mbar_wait(&bar_p, (uint32_t)(p_done & 1))) ++p_done;
+      while (x_done < x_iss && mbar_wait(&st.bar_x, (uint32_t)(x_done & 1))) ++x_done;
+      while (y_done < y_iss && mbar_wait(&st.bar_y, (uint32_t)(y_done & 1))) ++y_done;
     }
+    if (tid == kIssueP)
+      for (int bb = 0; bb < 2; ++bb)
+        while (p_done[bb] < p_iss[bb] && mbar_wait(&st.bar_p[bb], (uint32_t)(p_done[bb] & 1))) ++p_done[bb];
   }
   tc_fence_before();
   __syncthreads();
@@ -434,7 +493,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
 template <int BITS, int F>
 static tq_status run_quantize_tc(const CUtensorMap& map, const tqd::QuantizeTcParams& p, int sms,
                                  cudaStream_t st) {
-  constexpr int ops = F > 0 ? 7 : 4;
+  constexpr int ops = F > 0 ? 7 : 3;
   const int smem = ops * tqd::kOpBytes + (int)sizeof(tqd::QtcState);
   static bool attr = false;            // per template instance
   if (!attr) {
