@@ -30,6 +30,9 @@ tq_status cuda_fail(cudaError_t e, const char* what) {
 tq_status launch_quantize_simt(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
                                int n_kv_heads, int64_t n_new, const int32_t* start_pos,
                                const CacheView& cv, cudaStream_t st);
+tq_status launch_quantize_small(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
+                                int n_kv_heads, int64_t n_new, const int32_t* start_pos,
+                                const CacheView& cv, cudaStream_t st, bool* handled);
 tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
                              int n_kv_heads, int64_t n_new, const int32_t* start_pos,
                              const CacheView& cv, cudaStream_t st, bool* handled);
@@ -132,16 +135,18 @@ static tq_status upload(tq_codebook* cb) {
   const size_t sz_pi = al((size_t)dp * d * 4), sz_s = al((size_t)mp * d * 4 + 4),
                sz_srott = al((size_t)dp * mp * 4 + 4), sz_b = al(16 * 4), sz_c = al(16 * 4),
                sz_pibf = al((size_t)2 * dp * dp * 2), sz_srbf = al((size_t)2 * mp * dp * 2 + 4);
-  const size_t sz_pit = al((size_t)d * dp * 4), sz_st = al((size_t)d * mp * 4 + 4);
+  const size_t sz_pit = al((size_t)d * dp * 4), sz_st = al((size_t)d * mp * 4 + 4),
+               sz_srot = al((size_t)mp * dp * 4 + 4);
   const int R = dp + mp, d16 = (d + 15) / 16;
   const size_t sz_qf = al((size_t)(R / 16) * d16 * 2 * 32 * 16);
-  const size_t total = sz_pi + sz_s + sz_srott + sz_b + sz_c + sz_pibf + sz_srbf + sz_pit + sz_st + sz_qf;
+  const size_t total =
+      sz_pi + sz_s + sz_srott + sz_b + sz_c + sz_pibf + sz_srbf + sz_pit + sz_st + sz_qf + sz_srot;
   std::vector<uint8_t> host(total, 0);
   size_t off = 0;
   auto take = [&](size_t n) { size_t o = off; off += n; return o; };
   const size_t o_pi = take(sz_pi), o_s = take(sz_s), o_srott = take(sz_srott), o_b = take(sz_b),
                o_c = take(sz_c), o_pibf = take(sz_pibf), o_srbf = take(sz_srbf),
-               o_pit = take(sz_pit), o_st = take(sz_st), o_qf = take(sz_qf);
+               o_pit = take(sz_pit), o_st = take(sz_st), o_qf = take(sz_qf), o_srot = take(sz_srot);
   float* pi32 = reinterpret_cast<float*>(host.data() + o_pi);
   float* s32 = reinterpret_cast<float*>(host.data() + o_s);
   float* srott32 = reinterpret_cast<float*>(host.data() + o_srott);
@@ -151,6 +156,7 @@ static tq_status upload(tq_codebook* cb) {
   __nv_bfloat16* srbf = reinterpret_cast<__nv_bfloat16*>(host.data() + o_srbf);
   float* pit32 = reinterpret_cast<float*>(host.data() + o_pit);
   float* st32 = reinterpret_cast<float*>(host.data() + o_st);
+  float* srot32 = reinterpret_cast<float*>(host.data() + o_srot);
   for (int j = 0; j < d; ++j)
     for (int k = 0; k < d; ++k) {
       pi32[(size_t)j * d + k] = (float)cb->pi[(size_t)j * d + k];
@@ -167,6 +173,7 @@ static tq_status upload(tq_codebook* cb) {
       double acc = 0.0;
       for (int k = 0; k < d; ++k) acc += cb->s[(size_t)i * d + k] * cb->pi[(size_t)j * d + k];
       srott32[(size_t)j * mp + i] = (float)acc;
+      srot32[(size_t)i * dp + j] = (float)acc;
       const __nv_bfloat16 hi = __double2bfloat16(acc);
       srbf[(size_t)i * dp + j] = hi;
       srbf[(size_t)mp * dp + (size_t)i * dp + j] = __double2bfloat16(acc - (double)__bfloat162float(hi));
@@ -232,6 +239,7 @@ static tq_status upload(tq_codebook* cb) {
   cb->pit32 = reinterpret_cast<float*>(base + o_pit);
   cb->st32 = reinterpret_cast<float*>(base + o_st);
   cb->qprep_frag = reinterpret_cast<uint4*>(base + o_qf);
+  cb->srot32 = reinterpret_cast<float*>(base + o_srot);
   return TQ_OK;
 }
 
@@ -371,6 +379,8 @@ tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtyp
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   bool handled = false;
   s = launch_quantize_tc(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st, &handled);
+  if (handled || s != TQ_OK) return s;
+  s = launch_quantize_small(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st, &handled);
   if (handled || s != TQ_OK) return s;
   return launch_quantize_simt(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st);
 }

@@ -71,6 +71,7 @@ struct tq_codebook {
   float* srott32;     // [d_pad][m_pad] (S Pi^T)^T, zero padded    (residual sketch, coalesced)
   float* pit32;       // [d][d_pad]   Pi^T, columns >= d zero     (query rotation, coalesced)
   float* st32;        // [d][m_pad]   S^T, columns >= m zero      (query sketch, coalesced)
+  float* srot32;      // [m_pad][d_pad] S Pi^T row-major, zero padded (residual sketch, small appends)
   float* bound32;     // [2^b - 1]    boundaries (fp32)
   float* cent32;      // [2^b]        float(fp16(c))
   __nv_bfloat16* pi_bf;    // tensor-core operands: [2][d_pad][d_pad] hi, lo of Pi
