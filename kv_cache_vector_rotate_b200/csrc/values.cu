@@ -212,11 +212,12 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
   constexpr int REC = VS::kRec, STAGE = VS::kStage, S = kValStages;
   constexpr int DP = 4 * E;        // padded coordinates
   constexpr int MT = DP / 16;      // 16-coordinate tiles
-  constexpr int PIECES = DP / 8;   // 16-byte pieces per tile row
   extern __shared__ __align__(16) uint8_t vsm[];
   __shared__ int64_t page_base[kValCtaPages];
   __shared__ uint64_t bars[kValWarps][S];
 
+  // the finish kernel may start now: it prefetches Pi and then waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int gi = blockIdx.y;
@@ -304,14 +305,21 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
   for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
   bool timed_out = false;
   int issued = min(S, n_my);
-  for (int i = 0; i < n_my; ++i) {
-    const int ubase = k0 + 32 * (warp + kValWarps * i);
-    const int pos = ubase + lane;                 // this lane's token
-    bool tok_ok = pos < k1;
+  // the weights of unit i (this lane's token, 4 query slots), loaded one unit ahead
+  auto load_w = [&](int i, float (&wv)[4]) {
+    const int pos = k0 + 32 * (warp + kValWarps * i) + lane;
+    bool tok_ok = i < n_my && pos < k1;
     if (tok_ok && !fast) tok_ok = page_base[(pos >> ps) - first_page] >= 0;
-    float wv[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) wv[q] = (tok_ok && q < nq) ? __ldg(p.w + wrow0 + q * p.w_stride + pos) : 0.0f;
+  };
+  float wnext[4];
+  load_w(0, wnext);
+  for (int i = 0; i < n_my; ++i) {
+    float wv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) wv[q] = wnext[q];
+    load_w(i + 1, wnext);
     if (!mbar_wait(&bars[warp][i & (S - 1)], (uint32_t)(i / S) & 1u)) {
       timed_out = true;
       break;
@@ -389,27 +397,47 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
 }
 
 // Mode B, pass 2: o = Pi^T sum_chunks partial, one CTA per (query tile,
-// query slot < G); CL x DP threads (CL = 1024 / DP chunk lanes).
-// Launched by programmatic dependent launch: waits for pass 1 first.
+// query slot < G); CL x DP threads (CL = 1024 / DP chunk lanes).  Thread
+// (cl, k) loads its entries Pi[j][k] (j = cl, cl + CL, ...) before it waits
+// for pass 1 (programmatic dependent launch; pass 1 lets it start early), then
+// sums its chunks of the partials with independent accumulators.
 template <int E>
 __global__ void __launch_bounds__(1024) values_finish_kernel(ValuesTcParams p) {
   constexpr int DP = 4 * E;
   constexpr int CL = 1024 / DP;    // chunk lanes
+  constexpr int JN = (DP + CL - 1) / CL;   // rows of Pi per thread
   __shared__ float red[CL][DP];
   __shared__ float a[DP];
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int gq = blockIdx.x / 4, q = blockIdx.x % 4;
   const int gi = gq / p.qtiles, qt = gq % p.qtiles;
   const int hql = qt * 4 + q;                     // query within the group
-  if (hql >= p.G) return;
   const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
   const int k = threadIdx.x % DP, cl = threadIdx.x / DP;
+  const int d = p.d;
+  constexpr bool kPre = JN <= 16;              // Pi entries held in registers across the wait
+  float pij[kPre ? JN : 1];
+  if constexpr (kPre) {
+#pragma unroll
+    for (int n = 0; n < JN; ++n) {
+      const int j = cl + CL * n;
+      pij[n] = (k < d && j < d) ? __ldg(p.pi32 + (size_t)j * d + k) : 0.0f;
+    }
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (hql >= p.G) return;
   const int nq = gridDim.x;                       // groups * qtiles * 4
-  float s = 0.0f;
   const float* src = p.partial + ((int64_t)gq * 4 + q) * DP + k;
-#pragma unroll 4
-  for (int c = cl; c < p.n_chunks; c += CL) s += src[(int64_t)c * nq * DP];
-  red[cl][k] = s;
+  const int64_t cs = (int64_t)nq * DP;            // stride between chunks
+  float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+  int c = cl;
+  for (; c + 3 * CL < p.n_chunks; c += 4 * CL) {
+    s0 += src[(int64_t)c * cs];
+    s1 += src[(int64_t)(c + CL) * cs];
+    s2 += src[(int64_t)(c + 2 * CL) * cs];
+    s3 += src[(int64_t)(c + 3 * CL) * cs];
+  }
+  for (; c < p.n_chunks; c += CL) s0 += src[(int64_t)c * cs];
+  red[cl][k] = (s0 + s1) + (s2 + s3);
   __syncthreads();
   if (cl == 0) {
     float t2 = 0.0f;
@@ -418,11 +446,18 @@ __global__ void __launch_bounds__(1024) values_finish_kernel(ValuesTcParams p) {
     a[k] = t2;
   }
   __syncthreads();
-  // o_k' = sum_j Pi[j][k'] a_j: CL lanes each take every CL-th j
-  const int d = p.d;
+  // o_k = sum_j Pi[j][k] a_j over this lane's rows j
   float o = 0.0f;
-  if (k < d)
-    for (int j = cl; j < d; j += CL) o = fmaf(__ldg(p.pi32 + (size_t)j * d + k), a[j], o);
+  if constexpr (kPre) {
+#pragma unroll
+    for (int n = 0; n < JN; ++n) {
+      const int j = cl + CL * n;
+      if (j < DP) o = fmaf(pij[n], a[j], o);
+    }
+  } else {
+    for (int j = cl; j < d; j += CL)
+      if (k < d) o = fmaf(__ldg(p.pi32 + (size_t)j * d + k), a[j], o);
+  }
   __syncthreads();
   red[cl][k] = o;
   __syncthreads();
