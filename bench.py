@@ -47,10 +47,12 @@ LOGIT_BYTES = B * HKV * CTX * KEY_REC + B * HQ * CTX * 4 + B * HQ * D * 2
 VALUE_BYTES = B * HKV * CTX * VAL_REC + B * HQ * CTX * 4 + B * HQ * D * 4
 APPEND_BYTES = 2 * B * HKV * D * 2 + B * HKV * (KEY_REC + VAL_REC)
 APPEND_CFG = dict(batch=16, heads=8, n_new=4096)
-# DRAM bytes (read + write) of one tq_logits call of this workload as ncu
-# counted them (None until the current kernels have been captured).
-LOGITS_DRAM_BYTES = None
-LOGITS_DRAM_SOURCE = "not captured for the current kernels"
+# DRAM bytes (read + write) of one tq_logits call of this workload, from one
+# ncu capture of the current kernels (--set full, one launch each):
+# logits_kernel<3,32,32> 17,882,368 + 0 and prep_queries_kernel 156,416 + 0.
+LOGITS_DRAM_BYTES = 17882368 + 156416
+LOGITS_DRAM_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, logits_kernel<3,32,32> + "
+                      "prep_queries_kernel, one launch each")
 WORKLOAD = "decode step: batch 1, 8 KV / 32 query heads, head_dim 128, context 32768, keys b=3 + QJL m=128, values b=3"
 
 
@@ -260,6 +262,66 @@ def long_context_phase(dev, ws, steps: int = 20):
         out[f"b{bits}"] = {"us_per_call": 1e3 * ms, "gbs": nbytes / (ms * 1e-3) / 1e9, "record_bytes": rec}
         del g, cache
     return out
+
+
+def profile_phase(args):
+    """Sets up one workload and makes three eager calls of one entry point, for
+    ncu captures (no timing, no JSON line):
+      append        tq_quantize_append of the online-append batch (16 x 8 x 4096 bf16 keys)
+      decode        tq_logits and tq_dequant_values of the decode step (batch 1, ctx 32768)
+      long_b{2,3,4} tq_logits of the long-context workload (batch 4, ctx 131072) at b bits"""
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    tq.load_library()
+    ph = args.profile_phase
+    if ph == "append":
+        c = APPEND_CFG
+        bits16, _ = synth.append_batch(1005, c["batch"], c["heads"], c["n_new"], D)
+        X = torch.from_numpy(bits16.view(np.int16)).view(torch.bfloat16).to(dev)
+        cb = tq.Codebook(D, BITS, M, synth.SEED_PI, synth.SEED_S)
+        pps = c["n_new"] // PT
+        cache = tq.PagedCache.allocate(cb, c["batch"] * pps, PT, c["heads"],
+                                       torch.from_numpy(synth.block_table(1006, c["batch"], pps)), device=dev)
+        start = torch.zeros(c["batch"], dtype=torch.int32, device=dev)
+        for _ in range(3):
+            tq.quantize_append(cb, X, start, cache)
+    elif ph == "decode":
+        data = synth.decode_step(1002, B, HKV, HQ, CTX, D)
+        as_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        kcb = tq.Codebook(D, BITS, M, synth.SEED_PI, synth.SEED_S)
+        vcb = tq.Codebook(D, BITS, 0, synth.SEED_PI, 0)
+        pps = CTX // PT
+        bt = torch.from_numpy(synth.block_table(1003, B, pps))
+        zero = torch.zeros(B, dtype=torch.int32, device=dev)
+        kc = tq.PagedCache.allocate(kcb, pps, PT, HKV, bt, device=dev)
+        vc = tq.PagedCache.allocate(vcb, pps, PT, HKV, bt, device=dev)
+        tq.quantize_append(kcb, as_bf16(data["k"][0]), zero, kc)
+        tq.quantize_append(vcb, as_bf16(data["v"][0]), zero, vc)
+        q = as_bf16(data["q"][0])
+        W = torch.from_numpy(synth.softmax_like_weights(1004, B, HQ, CTX)).to(dev)
+        ctx_t = torch.full((B,), CTX, dtype=torch.int32, device=dev)
+        for _ in range(3):
+            tq.logits(kcb, kc, q, ctx_t, CTX)
+            tq.dequant_values(vcb, vc, ctx_t, CTX, B, weights=W)
+    else:
+        bits = int(ph[-1])
+        batch, hkv, hq, ctx, d, m, pt = 4, 8, 32, 131072, 128, 128, 64
+        K, q = synth.decode_keys_device(1003, batch, hkv, hq, ctx, d, device=dev)
+        pps = ctx // pt
+        cb = tq.Codebook(d, bits, m, synth.SEED_PI, synth.SEED_S)
+        cache = tq.PagedCache.allocate(cb, batch * pps, pt, hkv, torch.from_numpy(synth.block_table(1004, batch, pps)),
+                                       device=dev)
+        tq.quantize_append(cb, K, torch.zeros(batch, dtype=torch.int32, device=dev), cache)
+        del K
+        ctx_t = torch.full((batch,), ctx, dtype=torch.int32, device=dev)
+        Lout = torch.empty(batch, hq, ctx, dtype=torch.float32, device=dev)
+        for _ in range(3):
+            tq.logits(cb, cache, q, ctx_t, ctx, out=Lout)
+    torch.cuda.synchronize()
+    print("profile phase", ph, "done", flush=True)
 
 
 def run_ours(args):
@@ -490,12 +552,16 @@ def main():
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")
+    ap.add_argument("--profile-phase", choices=["append", "decode", "long_b2", "long_b3", "long_b4"],
+                    help="set up one workload and make three eager calls (for ncu captures)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="seconds of oracle work for --impl reference (all timed and warm-up steps)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile_phase:
+        profile_phase(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)
