@@ -264,6 +264,49 @@ def long_context_phase(dev, ws, steps: int = 20):
     return out
 
 
+def vector_search_phase(dev, n: int = 1_000_000, nq: int = 1000, d: int = 200):
+    """Nearest-neighbour search from the codes (stands in for the GloVe d = 200
+    evaluation of the method's benchmarks; GloVe is not available here): 10^6
+    unit rows ~ N(0, diag(1/i)) and 1000 queries of the same law, coded at
+    b in {2, 4} with QJL m = 200, scored by tq_logits (one sequence of one KV
+    head, the queries as its query heads). Recall@10 and 1@10 of the code
+    scores against the exact top 10 (fp64 brute force on the GPU, outside the
+    product path); the quantize and scoring calls are timed with CUDA events."""
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    m, pt = d, 64
+    X = torch.from_numpy(synth.anisotropic_unit(2005, n, d)).to(dev)
+    Q = torch.from_numpy(synth.anisotropic_unit(3005, nq, d)).to(dev)
+    top_exact = []
+    for s0 in range(0, nq, 100):
+        top_exact.append(torch.topk(Q[s0:s0 + 100].double() @ X.double().T, 10, dim=1).indices)
+    top_exact = torch.cat(top_exact)
+    out = {"workload": f"{n} unit rows d={d} ~ N(0, diag(1/i)), {nq} queries, QJL m={m}, scores from codes"}
+    pps = (n + pt - 1) // pt
+    bt = torch.from_numpy(synth.block_table(2006, 1, pps))
+    ctx_t = torch.tensor([n], dtype=torch.int32, device=dev)
+    scores = torch.empty(1, nq, n, dtype=torch.float32, device=dev)
+    for bits in (2, 4):
+        cb = tq.Codebook(d, bits, m, synth.SEED_PI, synth.SEED_S)
+        cache = tq.PagedCache.allocate(cb, pps, pt, 1, bt, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        tq.quantize_append(cb, X.view(1, 1, n, d), torch.zeros(1, dtype=torch.int32, device=dev), cache)
+        ev[1].record()
+        tq.logits(cb, cache, Q.view(1, nq, d), ctx_t, n, out=scores)
+        ev[2].record()
+        torch.cuda.synchronize()
+        top = torch.topk(scores[0], 10, dim=1).indices
+        hit = (top.unsqueeze(2) == top_exact.unsqueeze(1)).any(dim=2).float()
+        best_in = (top == top_exact[:, :1]).any(dim=1).float()
+        out[f"b{bits}"] = {"recall_at_10": float(hit.mean()), "one_at_10": float(best_in.mean()),
+                           "quantize_ms": ev[0].elapsed_time(ev[1]), "score_ms": ev[1].elapsed_time(ev[2]),
+                           "errors": cache.errors()}
+        del cache
+    return out
+
+
 def profile_phase(args):
     """Sets up one workload and makes three eager calls of one entry point, for
     ncu captures (no timing, no JSON line):
@@ -470,6 +513,10 @@ def run_ours(args):
     lc = None
     if not args.no_long:
         lc = long_context_phase(dev, ws)
+    # vector search at d = 200 (10^6 rows, 1000 queries): recall from the codes
+    vs = None
+    if not args.no_search:
+        vs = vector_search_phase(dev)
 
     n = ws
     steps = args.steps
@@ -500,6 +547,8 @@ def run_ours(args):
         line["keys_quantized"] = kq
     if lc is not None:
         line["long_context"] = lc
+    if vs is not None:
+        line["vector_search"] = vs
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:
@@ -552,6 +601,7 @@ def main():
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")
+    ap.add_argument("--no-search", action="store_true", help="skip the vector-search (10^6 x d 200) phase")
     ap.add_argument("--profile-phase", choices=["append", "decode", "long_b2", "long_b3", "long_b4"],
                     help="set up one workload and make three eager calls (for ncu captures)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
