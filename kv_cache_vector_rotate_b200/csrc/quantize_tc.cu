@@ -189,7 +189,6 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
   QtcState& st = *reinterpret_cast<QtcState*>(qsm_raw + kOps * kOpBytes);
   const uint32_t pi_s = base_s, sr_s = base_s + 2 * kOpBytes, x_s = base_s + kRes * kOpBytes,
                  rh_s = x_s + kOpBytes, rl_s = x_s + 2 * kOpBytes;
-  const uint8_t* const x_g = qsm_raw + kRes * kOpBytes;
   uint8_t* const rh_g = qsm_raw + (kRes + 1) * kOpBytes;
   uint8_t* const rl_g = qsm_raw + (kRes + 2) * kOpBytes;
   const int64_t n_my = p.n_tiles > blockIdx.x ? (p.n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
@@ -282,7 +281,7 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
       tmem_ld32(tmem + lane_base + kColP + 128 * (uint32_t)(j & 1) + 32 * ch, pv);
       uint32_t qw = 0u;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) qw |= (pv[e] < 0.0f ? 1u : 0u) << qjl_bit(e);
+      for (int e = 0; e < 32; ++e) qw |= (__float_as_uint(pv[e]) >> 31) << qjl_bit(e);
       rec_prev[CW::q0] = qw;
     }
     float rn = 0.0f;
@@ -326,29 +325,25 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
       hb = head_block_offset(p.cv, b, h, pos);
       slot = (int)(pos % p.cv.page_tokens);
     }
-    // X(k) landed (this thread reads it) and Y(k) is complete
-    bool ok = st.fail == 0 && mbar_wait(&st.bar_x, (uint32_t)(k & 1)) && mbar_wait(&st.bar_y, (uint32_t)(k & 1));
+    // Y(k) is complete (so its MMAs are done reading X(k))
+    bool ok = st.fail == 0 && mbar_wait(&st.bar_y, (uint32_t)(k & 1));
     if (ok && tid == kIssueY) ++y_done;
+    tc_fence_after();
+    // this thread's 32 coordinates of Y(k); ||x|| = ||Pi x|| from the row of Y
+    // (Pi is orthogonal; Y carries the input to fp32 rounding)
+    float y[32];
+    tmem_ld32(tmem + lane_base + 32 * ch, y);
     float n2 = 0.0f;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(x_g + sw128_offset(r, 32 * ch + 8 * c));
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float a = __uint_as_float(w4[e] << 16), b2 = __uint_as_float(w4[e] & 0xFFFF0000u);
-        n2 = fmaf(a, a, fmaf(b2, b2, n2));
-      }
-    }
+    for (int e = 0; e < 32; ++e) n2 = fmaf(y[e], y[e], n2);
     st.part_x[ch][r] = n2;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the reads of X before the next copy
     tc_fence_before();
     if (__syncthreads_or(!ok)) {
       aborted = true;
       break;
     }
     tc_fence_after();
-    if (tid == kIssueY && k + 1 < n_my) issue_x(k + 1);   // X(k) was read by Y(k) and by every thread
+    if (tid == kIssueY && k + 1 < n_my) issue_x(k + 1);   // X(k) was read by Y(k)
     const float nrm = sqrtf((st.part_x[0][r] + st.part_x[1][r]) + (st.part_x[2][r] + st.part_x[3][r]));
     const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
 
@@ -357,8 +352,6 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
 #pragma unroll
     for (int i = 0; i < W; ++i) rec[i] = 0u;
     float rr2 = 0.0f;
-    float y[32];
-    tmem_ld32(tmem + lane_base + 32 * ch, y);
 #pragma unroll
     for (int e = 0; e < 32; ++e) {
       const float u = y[e] * inv;
