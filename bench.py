@@ -264,6 +264,64 @@ def long_context_phase(dev, ws, steps: int = 20):
     return out
 
 
+def budget_phase(dev, steps: int = 20):
+    """Key codecs side by side on the decode-step keys (batch 1, 8 KV / 32
+    query heads, d 128, ctx 32768): Lloyd-Max bits b with or without the QJL
+    sketch (m = 128), so that equal totals can be compared (e.g. b = 3 alone
+    against b = 2 + 1 QJL bit per coordinate). Per codec: record bytes, bits
+    per coordinate, tq_logits time (CUDA graph of `steps` calls), and the
+    estimator against the exact fp32 <q, k>: bias = sum(L est * L exact) /
+    sum(L exact^2) - 1 (0 for an unbiased estimator) and rms error in units of
+    ||q|| ||k|| / sqrt(d)."""
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    data = synth.decode_step(1002, B, HKV, HQ, CTX, D)
+    as_bf16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+    K = as_bf16(data["k"][0])
+    q = as_bf16(data["q"][0])
+    G = HQ // HKV
+    kf = K.float()[0]                                           # [HKV, CTX, D]
+    qf = q.float()[0].view(HKV, G, D)                           # [HKV, G, D]
+    exact = torch.einsum("hgd,hcd->hgc", qf, kf)                # [HKV, G, CTX]
+    scale = (qf.norm(dim=2, keepdim=True) * kf.norm(dim=2).unsqueeze(1)) / D ** 0.5
+    pps = CTX // PT
+    bt = torch.from_numpy(synth.block_table(1003, B, pps))
+    ctx_t = torch.full((B,), CTX, dtype=torch.int32, device=dev)
+    Lout = torch.empty(B, HQ, CTX, dtype=torch.float32, device=dev)
+    cs = torch.cuda.Stream(device=dev)
+    out = {"workload": "decode-step keys (batch 1, 8 KV / 32 query heads, d 128, ctx 32768), one cache (no replicas)"}
+    for bits, m in ((1, 128), (2, 0), (2, 128), (3, 0), (3, 128), (4, 0)):
+        cb = tq.Codebook(D, bits, m, synth.SEED_PI, synth.SEED_S if m else 0)
+        cache = tq.PagedCache.allocate(cb, pps, PT, HKV, bt, device=dev)
+        tq.quantize_append(cb, K, torch.zeros(B, dtype=torch.int32, device=dev), cache)
+        ws_t = torch.empty(max(16, tq.logits_workspace_bytes(cb, B, HKV, HQ)), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            tq.logits(cb, cache, q, ctx_t, CTX, out=Lout, workspace=ws_t)
+        torch.cuda.synchronize()
+        est = Lout[0].view(HKV, G, CTX).clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cs):
+            for _ in range(steps):
+                tq.logits(cb, cache, q, ctx_t, CTX, out=Lout, workspace=ws_t)
+        g.replay()
+        torch.cuda.synchronize()
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record()
+        g.replay()
+        b_.record()
+        torch.cuda.synchronize()
+        us = 1e3 * a_.elapsed_time(b_) / steps
+        rec = (bits * D + m) // 8 + (4 if m else 2)
+        nbytes = B * HKV * CTX * rec + B * HQ * CTX * 4 + B * HQ * D * 2
+        bias = float((est * exact).sum() / (exact * exact).sum()) - 1.0
+        rms = float((((est - exact) / scale) ** 2).mean().sqrt())
+        out[f"b{bits}_m{m}"] = {"record_bytes": rec, "bits_per_coord": round(8 * rec / D, 3), "us_per_call": us,
+                                "gbs": nbytes / (us * 1e-6) / 1e9, "bias": bias, "rms_err": rms}
+        del g, cache
+    return out
+
+
 def vector_search_phase(dev, n: int = 1_000_000, nq: int = 1000, d: int = 200):
     """Nearest-neighbour search from the codes (stands in for the GloVe d = 200
     evaluation of the method's benchmarks; GloVe is not available here): 10^6
@@ -513,6 +571,10 @@ def run_ours(args):
     lc = None
     if not args.no_long:
         lc = long_context_phase(dev, ws)
+    # key codecs side by side at equal bit budgets (Lloyd-Max bits vs QJL bits)
+    bud = None
+    if not args.no_budget:
+        bud = budget_phase(dev)
     # vector search at d = 200 (10^6 rows, 1000 queries): recall from the codes
     vs = None
     if not args.no_search:
@@ -547,6 +609,8 @@ def run_ours(args):
         line["keys_quantized"] = kq
     if lc is not None:
         line["long_context"] = lc
+    if bud is not None:
+        line["key_codecs"] = bud
     if vs is not None:
         line["vector_search"] = vs
     if rank == 0 and not args.no_cpu_baseline:
@@ -602,6 +666,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")
     ap.add_argument("--no-search", action="store_true", help="skip the vector-search (10^6 x d 200) phase")
+    ap.add_argument("--no-budget", action="store_true", help="skip the key-codec comparison phase")
     ap.add_argument("--profile-phase", choices=["append", "decode", "long_b2", "long_b3", "long_b4"],
                     help="set up one workload and make three eager calls (for ncu captures)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
