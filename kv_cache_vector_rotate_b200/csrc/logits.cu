@@ -583,8 +583,10 @@ __global__ void __maxnreg__(logits_max_regs(BITS, E)) logits_kernel(LogitsParams
       // sum_i s_i z_i = sum z - 2 sum beta z
       const float ta = fmaf(-1.0f / 64.0f, (float)(256 * qa[0] + qa[1]), zsumf);
       const float tb = fmaf(-1.0f / 64.0f, (float)(256 * qa[2] + qa[3]), zsumf);
-      la = lo_half(na) * fmaf(c1 * hi_half(na), ta, c0 * cba);
-      lb = lo_half(nb) * fmaf(c1 * hi_half(nb), tb, c0 * cbb);
+      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&na));   // ||k||, ||r||
+      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&nb));
+      la = fa.x * fmaf(c1 * fa.y, ta, c0 * cba);
+      lb = fb.x * fmaf(c1 * fb.y, tb, c0 * cbb);
     } else {
       la = lo_half(na) * (c0 * cba);
       lb = lo_half(nb) * (c0 * cbb);
