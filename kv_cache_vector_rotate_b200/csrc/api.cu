@@ -243,6 +243,22 @@ static tq_status upload(tq_codebook* cb) {
   return TQ_OK;
 }
 
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return dev;
+}
+
+int device_sm_count() {
+  static int cache[64] = {};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
 static tq_status make_view(const tq_codebook* cb, const tq_cache* c, CacheView* v) {
   if (!c) return fail(TQ_EINVAL, "cache is NULL");
   if (!c->pages || !c->block_table) return fail(TQ_EINVAL, "cache pages / block_table is NULL");

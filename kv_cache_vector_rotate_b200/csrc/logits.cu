@@ -681,13 +681,6 @@ size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
   return logits_ws_layout(cb, groups, G, groups * G).total;
 }
 
-static int device_sms() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 template <int BITS, int E, int F>
 static tq_status run_logits(const tqd::LogitsParams& p, const tqd::PrepParams& pp, int parts, int64_t groups,
                             int qtiles, cudaStream_t st) {
@@ -696,8 +689,8 @@ static tq_status run_logits(const tqd::LogitsParams& p, const tqd::PrepParams& p
   constexpr int W = q0 + (F + 31) / 32;
   using RS = tqd::RingShape<W>;
   const int smem = tqd::kLogitsWarps * RS::kStages * RS::kStageBytes;
-  static bool attr = false;            // per template instance
-  if (!attr) {
+  static PerDeviceOnce attr;           // per template instance
+  if (const int dev_ = current_device(); attr.need(dev_)) {
     cudaError_t e = cudaFuncSetAttribute(tqd::logits_kernel<BITS, E, F>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "tq_logits: smem attribute");
@@ -705,7 +698,7 @@ static tq_status run_logits(const tqd::LogitsParams& p, const tqd::PrepParams& p
     // split, or its CTAs would keep logits CTAs off their SMs
     e = cudaFuncSetAttribute(tqd::prep_queries_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return cuda_fail(e, "tq_logits: carveout attribute");
-    attr = true;
+    attr.mark(dev_);
   }
   tqd::prep_queries_kernel<<<dim3((unsigned)parts, (unsigned)(groups * qtiles)), tqd::kLogitsWarps * 32, 0, st>>>(pp);
   cudaError_t e = cudaGetLastError();
@@ -794,7 +787,7 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   // run at a fraction of the GPU for as long as a full one).
   const int64_t units = (max_ctx + 31) / 32;
   const int64_t tiles = groups * qtiles;
-  const int64_t slots = (int64_t)std::max(1, device_sms()) * tqd::logits_min_blocks(L.bits, L.E);
+  const int64_t slots = (int64_t)device_sm_count() * tqd::logits_min_blocks(L.bits, L.E);
   int64_t n_chunks = std::max<int64_t>(1, slots / tiles);
   const int64_t max_units_cta = (int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 32;
   n_chunks = std::max<int64_t>(n_chunks, (units + max_units_cta - 1) / max_units_cta);

@@ -191,19 +191,19 @@ namespace tq {
 template <int BITS, int E, int F>
 static tq_status launch_simt(tqd::QuantizeSimtParams p, cudaStream_t st) {
   // one vector per CTA while the GPU is not full, up to kSimtRows after that
-  const int64_t sms = 148;
+  const int64_t sms = device_sm_count();
   int rpc = (int)((p.rows + sms * 4 - 1) / (sms * 4));
   rpc = rpc < 1 ? 1 : rpc > tqd::kSimtRows ? tqd::kSimtRows : rpc;
   p.rows_per_cta = rpc;
   const int64_t ctas = (p.rows + rpc - 1) / rpc;
   const unsigned blocks = (unsigned)(ctas < sms * 8 ? ctas : sms * 8);
   const size_t smem = tqd::kSimtStageFloats * sizeof(float);
-  static bool attr_set = false;   // per instantiation; setting it twice is harmless
-  if (!attr_set) {
+  static PerDeviceOnce attr_set;   // per instantiation
+  if (const int dev_ = current_device(); attr_set.need(dev_)) {
     cudaError_t e = cudaFuncSetAttribute(tqd::quantize_simt_kernel<BITS, E, F>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "quantize_simt: smem attribute");
-    attr_set = true;
+    attr_set.mark(dev_);
   }
   tqd::quantize_simt_kernel<BITS, E, F><<<blocks, 4 * E, smem, st>>>(p);
   return TQ_OK;

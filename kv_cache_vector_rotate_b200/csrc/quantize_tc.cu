@@ -488,12 +488,12 @@ static tq_status run_quantize_tc(const CUtensorMap& map, const tqd::QuantizeTcPa
                                  cudaStream_t st) {
   constexpr int ops = F > 0 ? 7 : 3;
   const int smem = ops * tqd::kOpBytes + (int)sizeof(tqd::QtcState);
-  static bool attr = false;            // per template instance
-  if (!attr) {
+  static PerDeviceOnce attr;           // per template instance
+  if (const int dev_ = current_device(); attr.need(dev_)) {
     cudaError_t e = cudaFuncSetAttribute(tqd::quantize_tc_kernel<BITS, F>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "quantize_tc: smem attribute");
-    attr = true;
+    attr.mark(dev_);
   }
   const int64_t grid = p.n_tiles < sms ? p.n_tiles : sms;
   tqd::quantize_tc_kernel<BITS, F><<<(unsigned)grid, tqd::kQtcThreads, smem, st>>>(map, p);
@@ -516,12 +516,7 @@ tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, 
     return TQ_OK;
   const PFN_cuTensorMapEncodeTiled_v12000 encode = encode_tiled_fn();
   if (!encode) return TQ_OK;
-  static int sms = 0;
-  if (!sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
-  }
+  const int sms = device_sm_count();
   // X as a 2-D bf16 tensor [rows][128]; a box is 64 columns (128 bytes) x
   // 128 rows, written with the 128-byte swizzle; rows past the end read as 0
   CUtensorMap map;

@@ -92,6 +92,20 @@ struct tq_codebook {
 
 namespace tq {
 
+// The current device and its SM count (cached per device).
+int current_device();
+int device_sm_count();
+
+// A flag per device (up to 64) for per-device set-up such as kernel
+// attributes: need(dev) until mark(dev) (setting an attribute twice is harmless).
+struct PerDeviceOnce {
+  unsigned long long done = 0;
+  bool need(int dev) const { return dev < 0 || dev >= 64 || !(done & (1ull << dev)); }
+  void mark(int dev) {
+    if (dev >= 0 && dev < 64) done |= 1ull << dev;
+  }
+};
+
 // Error reporting (thread-local message for tq_last_error).
 void set_error(const std::string& msg);
 tq_status fail(tq_status st, const std::string& msg);

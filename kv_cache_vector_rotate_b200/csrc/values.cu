@@ -473,12 +473,12 @@ __global__ void __launch_bounds__(1024) values_finish_kernel(ValuesTcParams p) {
 
 namespace tq {
 
-// Mode B chunking: every CTA slot of the GPU (148 SMs x 4) gets one CTA, each
+// Mode B chunking: every CTA slot of the GPU (SMs x 4) gets one CTA, each
 // an equal share (to one 32-token unit) of a sequence; more CTAs when a share
 // would need more than kValCtaPages - 2 block-table entries.
 static int64_t values_chunks(int64_t units_gq, int64_t max_ctx, int page_tokens) {
   const int64_t units = (max_ctx + 31) / 32;
-  int64_t n = std::max<int64_t>(1, 148LL * 4 / std::max<int64_t>(1, units_gq));
+  int64_t n = std::max<int64_t>(1, (int64_t)device_sm_count() * 4 / std::max<int64_t>(1, units_gq));
   const int64_t max_units_cta = (int64_t)(tqd::kValCtaPages - 2) * page_tokens / 32;
   n = std::max<int64_t>(n, (units + max_units_cta - 1) / max_units_cta);
   return std::min<int64_t>(n, units);
@@ -506,12 +506,12 @@ static tq_status run_values(tqd::ValuesParams p, const tqd::ValuesTcParams& tp, 
   }
   constexpr int W = tqd::ChunkWords<BITS, E, 0>::W;
   const int smem = tqd::kValWarps * tqd::ValShape<W, E>::kWarpBytes;
-  static bool attr = false;            // per template instance
-  if (!attr) {
+  static PerDeviceOnce attr;           // per template instance
+  if (const int dev_ = current_device(); attr.need(dev_)) {
     cudaError_t e = cudaFuncSetAttribute(tqd::values_acc_kernel<BITS, E>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail(e, "values: smem attribute");
-    attr = true;
+    attr.mark(dev_);
   }
   dim3 grid((unsigned)tp.n_chunks, (unsigned)groups, (unsigned)tp.qtiles);
   tqd::values_acc_kernel<BITS, E><<<grid, tqd::kValWarps * 32, smem, st>>>(tp);
