@@ -223,6 +223,14 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache,
                             void* out, tq_dtype out_dtype, int64_t out_stride,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Self-test of the device-side failure path: one small kernel waits on an
+ * mbarrier that nothing completes, with the bounded wait every streaming
+ * kernel uses; after about a second the wait gives up and the kernel ORs
+ * TQ_DEV_ERR_TIMEOUT into *error_word (device, uint32) and returns.  No
+ * fault, trap or hang; asynchronous on the stream.  TQ_EINVAL for a NULL
+ * error_word.  The method has no counterpart: this checks the library. */
+tq_status tq_selftest_wait_timeout(uint32_t* error_word, void* stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 

@@ -24,7 +24,7 @@ EXPORTS = (
     "tq_codebook_build", "tq_codebook_build_host", "tq_codebook_free", "tq_codebook_export",
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
-    "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes",
+    "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
 )
 
 
@@ -80,6 +80,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     vp, i32, i64, vp, sz, vp]),
         "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
         "tq_logits_noalloc_scratch_bytes": (sz, []),
+        "tq_selftest_wait_timeout": (i32, [vp, vp]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_layout_version": (i32, []),
     }
@@ -266,3 +267,9 @@ def logits_noalloc(cb: Codebook, cache: PagedCache, q, ctx_len, max_ctx: int, ou
                                              _ptr(ctx_len), max_ctx, _ptr(out), out.stride(1),
                                              _stream(stream)))
     return out
+
+
+def selftest_wait_timeout(error_word, stream=None) -> None:
+    """tq_selftest_wait_timeout: a bounded wait that runs out (about 1 s) and
+    reports DEV_ERR_TIMEOUT into `error_word` (device int32 [1])."""
+    _check(load_library().tq_selftest_wait_timeout(_ptr(error_word), _stream(stream)))

@@ -260,3 +260,27 @@ def test_append_workload_full_size_sampled(tqm):
     idx, qneg, n16, r16 = (np.concatenate(a) for a in got)
     compare_codes(codec, X, O.encode(codec, X), idx, qneg, n16, r16)
     assert cache.errors() == 0
+
+
+def test_bounded_wait_runs_out_and_reports(tqm):
+    """The failure path of every streaming kernel: a wait on an mbarrier that
+    nothing completes gives up after about a second, reports
+    TQ_DEV_ERR_TIMEOUT in the error word and returns (the context stays
+    usable: an append afterwards is exact)."""
+    import time
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.time()
+    tqm.selftest_wait_timeout(err)
+    torch.cuda.synchronize()
+    dt = time.time() - t0
+    assert int(err.item()) & tqm.DEV_ERR_TIMEOUT
+    assert 0.05 < dt < 30.0, dt
+    rng = np.random.default_rng(29)
+    bits16, vals = synth.to_bf16(rng.standard_normal((1, 1, 64, 128)).astype(np.float32))
+    cb, cache = _run_append(tqm, 128, 3, 128, _dev_tensor(bits16, "bf16"), [0], 1, 64, synth.block_table(30, 1, 1))
+    codec = O.make_codec(128, 3, 128, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(128, 3, 128, 64, 1)
+    got = _read_back(lay, cache, synth.block_table(30, 1, 1), 0, 0, np.arange(64))
+    compare_codes(codec, vals[0, 0], O.encode(codec, vals[0, 0]), *got)
+    assert cache.errors() == 0
