@@ -223,6 +223,28 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache,
                             void* out, tq_dtype out_dtype, int64_t out_stride,
                             void* workspace, size_t workspace_bytes, void* stream);
 
+/* Workspace (device bytes) that tq_attend needs for these sizes. */
+size_t tq_attend_workspace_bytes(const tq_codebook* key_cb, const tq_codebook* value_cb, int64_t batch,
+                                 int32_t n_kv_heads, int32_t n_q_heads, int64_t max_ctx);
+
+/* Decode attention from the packed caches (TQ §How it works: logits from the
+ * compressed keys, values from their codes): for query head hq of sequence b
+ * (KV head hq / (n_q_heads / n_kv_heads)),
+ *   out[b, hq, :] = sum_{t < ctx_len[b]} softmax_t(scale * L[b, hq, t]) v_hat_t
+ * with L the tq_logits estimate and v_hat_t = ||v_t|| Pi_v^T c16[idx_t] (the
+ * value codebook's reconstruction); a row with ctx_len[b] = 0 is all zeros.
+ * key_cb / key_cache and value_cb / value_cache as for tq_logits and
+ * tq_dequant_values (same d and n_kv_heads; value_cb has m = 0).  q: device
+ * [batch, n_q_heads, d] of dtype; out: device fp32 [batch, n_q_heads, d];
+ * scale: usually 1/sqrt(d).  workspace: device, at least
+ * tq_attend_workspace_bytes(), 256-byte aligned (the scores, then the
+ * workspaces of the two passes).  Four kernel launches on the stream: query
+ * preparation, logits, row softmax, value accumulation (+ its finish). */
+tq_status tq_attend(const tq_codebook* key_cb, const tq_cache* key_cache, const tq_codebook* value_cb,
+                    const tq_cache* value_cache, const void* q, tq_dtype dtype, int64_t batch,
+                    int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx, float scale, float* out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
 /* Self-test of the device-side failure path: one small kernel waits on an
  * mbarrier that nothing completes, with the bounded wait every streaming
  * kernel uses; after about a second the wait gives up and the kernel ORs

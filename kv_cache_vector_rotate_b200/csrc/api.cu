@@ -469,4 +469,43 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache, const 
                        reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t tq_attend_workspace_bytes(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch,
+                                 int32_t n_kv_heads, int32_t n_q_heads, int64_t max_ctx) {
+  if (!kcb || !vcb || batch < 0 || max_ctx < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads ||
+      n_q_heads % n_kv_heads)
+    return 0;
+  return attend_workspace(kcb, vcb, batch, n_kv_heads, n_q_heads, max_ctx);
+}
+
+tq_status tq_attend(const tq_codebook* kcb, const tq_cache* kcache, const tq_codebook* vcb,
+                    const tq_cache* vcache, const void* q, tq_dtype dtype, int64_t batch, int32_t n_q_heads,
+                    const int32_t* ctx_len, int64_t max_ctx, float scale, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  tq_status s = check_cb(kcb);
+  if (s != TQ_OK) return s;
+  s = check_cb(vcb);
+  if (s != TQ_OK) return s;
+  CacheView kv, vv;
+  s = make_view(kcb, kcache, &kv);
+  if (s != TQ_OK) return s;
+  s = make_view(vcb, vcache, &vv);
+  if (s != TQ_OK) return s;
+  if (kcb->lay.d != vcb->lay.d) return fail(TQ_EINVAL, "tq_attend: key and value codebooks differ in d");
+  if (vcb->lay.m != 0) return fail(TQ_EINVAL, "tq_attend: the value codebook must have m = 0");
+  if (kv.n_kv_heads != vv.n_kv_heads) return fail(TQ_EINVAL, "tq_attend: caches differ in n_kv_heads");
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_attend: bad dtype");
+  if (batch < 0 || max_ctx < 0 || max_ctx > INT32_MAX) return fail(TQ_EINVAL, "tq_attend: bad size");
+  if (n_q_heads < kv.n_kv_heads || n_q_heads % kv.n_kv_heads)
+    return fail(TQ_EINVAL, "tq_attend: n_q_heads must be a multiple of the caches' n_kv_heads");
+  if (max_ctx > kv.max_pages * kv.page_tokens || max_ctx > vv.max_pages * vv.page_tokens)
+    return fail(TQ_EINVAL, "tq_attend: max_ctx exceeds a block table");
+  if (!std::isfinite(scale)) return fail(TQ_EINVAL, "tq_attend: scale is not finite");
+  if (batch == 0 || max_ctx == 0) return TQ_OK;
+  if (!q || !ctx_len || !out || !workspace) return fail(TQ_EINVAL, "tq_attend: NULL pointer");
+  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 256))
+    return fail(TQ_EINVAL, "tq_attend: misaligned pointer");
+  return launch_attend(kcb, kv, vcb, vv, q, dtype, batch, n_q_heads, ctx_len, max_ctx, scale, out, workspace,
+                       workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

@@ -131,6 +131,12 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
                         float* out, int64_t out_stride, void* ws, size_t ws_bytes,
                         cudaStream_t st);
 
+size_t attend_workspace(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch, int n_kv_heads,
+                        int n_q_heads, int64_t max_ctx);
+tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,
+                        const void* q, tq_dtype dt, int64_t batch, int n_q_heads, const int32_t* ctx_len,
+                        int64_t max_ctx, float scale, float* out, void* ws, size_t ws_bytes, cudaStream_t st);
+
 size_t values_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, int n_q_heads,
                         int64_t max_ctx);
 tq_status launch_values(const tq_codebook* cb, const CacheView& cv, const float* w,

@@ -25,6 +25,7 @@ EXPORTS = (
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
+    "tq_attend_workspace_bytes", "tq_attend",
 )
 
 
@@ -81,6 +82,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
         "tq_logits_noalloc_scratch_bytes": (sz, []),
         "tq_selftest_wait_timeout": (i32, [vp, vp]),
+        "tq_attend_workspace_bytes": (sz, [vp, vp, i64, i32, i32, i64]),
+        "tq_attend": (i32, [vp, ctypes.POINTER(CacheStruct), vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32,
+                            vp, i64, ctypes.c_float, vp, vp, sz, vp]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_layout_version": (i32, []),
     }
@@ -273,3 +277,30 @@ def selftest_wait_timeout(error_word, stream=None) -> None:
     """tq_selftest_wait_timeout: a bounded wait that runs out (about 1 s) and
     reports DEV_ERR_TIMEOUT into `error_word` (device int32 [1])."""
     _check(load_library().tq_selftest_wait_timeout(_ptr(error_word), _stream(stream)))
+
+
+def attend_workspace_bytes(key_cb: Codebook, value_cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int,
+                           max_ctx: int) -> int:
+    return int(load_library().tq_attend_workspace_bytes(key_cb.handle, value_cb.handle, batch, n_kv_heads,
+                                                        n_q_heads, max_ctx))
+
+
+def attend(key_cb: Codebook, key_cache: PagedCache, value_cb: Codebook, value_cache: PagedCache, q, ctx_len,
+           max_ctx: int, scale: float | None = None, out=None, workspace=None, stream=None):
+    """tq_attend: softmax(scale * logits) @ v_hat from the two caches;
+    q [batch, n_q_heads, d] -> out fp32 [batch, n_q_heads, d] (scale 1/sqrt(d) by default)."""
+    import torch
+    assert q.is_cuda and q.is_contiguous() and q.dim() == 3
+    b, hq, d = q.shape
+    if scale is None:
+        scale = 1.0 / d ** 0.5
+    if out is None:
+        out = torch.empty(b, hq, d, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = attend_workspace_bytes(key_cb, value_cb, b, key_cache.n_kv_heads, hq, max_ctx)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    ks, vs = key_cache.struct(), value_cache.struct()
+    _check(load_library().tq_attend(key_cb.handle, ctypes.byref(ks), value_cb.handle, ctypes.byref(vs), _ptr(q),
+                                    _dtype_code(q), b, hq, _ptr(ctx_len), max_ctx, float(scale), _ptr(out),
+                                    _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out

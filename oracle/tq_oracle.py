@@ -356,6 +356,28 @@ def weighted_values(codec: Codec, W: np.ndarray, idx: np.ndarray, norm16: np.nda
     return np.asarray(W, dtype=np.float64) @ dequantize(codec, idx, norm16)
 
 
+def attention_from_codes(kcodec: Codec, vcodec: Codec, Qv: np.ndarray, kenc, venc,
+                         scale: float) -> np.ndarray:
+    """Decode attention from the codes (TQ §How it works: attention logits
+    from the compressed keys, values from their codes), written out as its
+    definition: o_h = sum_t softmax_t(scale * L[h, t]) v_hat_t with L the
+    estimated logits of ``logits_from_codes`` and v_hat the reconstruction of
+    ``dequantize``.  READING: the softmax is the standard one over the valid
+    positions (the page names attention, not its normalization); an empty
+    context gives a zero row.  ``kenc`` / ``venc`` are (idx, qneg, norm16,
+    rnorm16) / (idx, norm16) of the same tokens."""
+    Qv = np.asarray(Qv, dtype=np.float64)
+    idx, qneg, n16, r16 = kenc
+    vidx, vn16 = venc
+    if len(idx) == 0:
+        return np.zeros((Qv.shape[0], vcodec.d))
+    L = scale * logits_from_codes(kcodec, Qv, idx, qneg, n16, r16)   # [nq, N]
+    L = L - L.max(axis=1, keepdims=True)
+    P = np.exp(L)
+    P /= P.sum(axis=1, keepdims=True)
+    return weighted_values(vcodec, P, vidx, vn16)
+
+
 def exact_logits(Qv: np.ndarray, K: np.ndarray) -> np.ndarray:
     """Brute force <q, k> in float64."""
     return np.asarray(Qv, np.float64) @ np.asarray(K, np.float64).T

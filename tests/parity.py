@@ -38,7 +38,8 @@ def oracle_pages(lay: O.Layout, n_pages: int, block_table: np.ndarray, encs: dic
     encs[(b, h)] = (positions, Encoded)."""
     pages = np.zeros(n_pages * lay.page_bytes, dtype=np.uint8)
     for (b, h), (pos, enc) in encs.items():
-        O.write_pages(lay, pages, block_table, b, h, pos, enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
+        if len(pos):                           # an empty sequence has no records
+            O.write_pages(lay, pages, block_table, b, h, pos, enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
     return pages
 
 

@@ -239,3 +239,42 @@ def test_logits_more_query_tiles_than_cta_slots(tqm):
     torch.cuda.synchronize()
     _check_logits(codec, q, encs, L.cpu().numpy(), ctx, 8, 4)
     assert cache.errors() == 0
+
+
+@pytest.mark.parametrize("kbits,m,vbits", [(3, 128, 3), (2, 128, 4), (4, 0, 2)])
+def test_attend_matches_oracle_attention(tqm, kbits, m, vbits):
+    """tq_attend (logits from the key codes, row softmax, values from their
+    codes) against the oracle's softmax attention given the same codes; a
+    sequence with an empty context gives a zero row.  The logit tolerance
+    (1e-3 of ||q|| ||k|| / sqrt(d)) moves the softmax weights by at most about
+    scale x that, so the output is checked to 2e-3 of its row scale."""
+    batch, heads, G, pt, d = 3, 2, 4, 32, 128
+    ctx = [700, 129, 0]
+    rng = np.random.default_rng(34 + kbits + vbits)
+    keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-1, 1, size=(1, heads, 1, d)))
+    vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
+    kcodec = O.make_codec(d, kbits, m, synth.SEED_PI, synth.SEED_S)
+    vcodec = O.make_codec(d, vbits, 0, synth.SEED_PI, synth.SEED_S)
+    kcb, kcache, kencs, _ = _oracle_cache(tqm, kcodec, O.Layout(d, kbits, m, pt, heads), keys, ctx, pt, 35)
+    vcb, vcache, vencs, _ = _oracle_cache(tqm, vcodec, O.Layout(d, vbits, 0, pt, heads), vals, ctx, pt, 36)
+    _, q = synth.to_bf16(rng.standard_normal((batch, heads * G, d)).astype(np.float32))
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    scale = 1.0 / np.sqrt(d)
+    out = tqm.attend(kcb, kcache, vcb, vcache, _q_tensor(q, "bf16"), ctx_t, max(ctx), scale=scale)
+    torch.cuda.synchronize()
+    O_gpu = out.cpu().numpy()
+    for b in range(batch):
+        for h in range(heads):
+            Qg = q[b, h * G:(h + 1) * G]
+            if ctx[b] == 0:
+                assert not O_gpu[b, h * G:(h + 1) * G].any()
+                continue
+            _, ke = kencs[(b, h)]
+            _, ve = vencs[(b, h)]
+            o = O.attention_from_codes(kcodec, vcodec, Qg, (ke.idx, ke.qneg, ke.norm16, ke.rnorm16),
+                                       (ve.idx, ve.norm16), scale)
+            vh = O.dequantize(vcodec, ve.idx, ve.norm16)
+            row_scale = np.maximum(np.abs(o).max(axis=1), np.linalg.norm(vh, axis=1).mean() / np.sqrt(d))
+            err = np.abs(O_gpu[b, h * G:(h + 1) * G] - o).max(axis=1)
+            assert np.all(err <= 2e-3 * row_scale), (b, h, err / row_scale)
+    assert kcache.errors() == 0 and vcache.errors() == 0

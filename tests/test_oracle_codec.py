@@ -292,3 +292,61 @@ def test_pages_round_trip_with_block_table():
     # head 0 of sequence 1 and everything of sequence 0 stay untouched
     for p in bt[0]:
         assert not pages[p * lay.page_bytes:(p + 1) * lay.page_bytes].any()
+
+
+def _attn_inputs(rng, d, n, bits_k=3, m=64, bits_v=3):
+    kc = O.make_codec(d, bits_k, m, 31, 32)
+    vc = O.make_codec(d, bits_v, 0, 33, 0)
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d)) * 2.0
+    ke, ve = O.encode(kc, K), O.encode(vc, V)
+    return kc, vc, K, (ke.idx, ke.qneg, ke.norm16, ke.rnorm16), (ve.idx, ve.norm16)
+
+
+def test_attention_uniform_weights_give_the_mean_value():
+    # a zero query (or scale 0) makes every logit equal: the output of every
+    # query row is the plain mean of the reconstructed values
+    rng = np.random.default_rng(40)
+    kc, vc, K, ke, ve = _attn_inputs(rng, 32, 40)
+    mean = O.dequantize(vc, *ve).mean(axis=0)
+    o0 = O.attention_from_codes(kc, vc, np.zeros((3, 32)), ke, ve, 0.2)
+    assert np.allclose(o0, mean[None, :], rtol=1e-12, atol=1e-12)
+    Qv = rng.standard_normal((3, 32))
+    o1 = O.attention_from_codes(kc, vc, Qv, ke, ve, 0.0)
+    assert np.allclose(o1, mean[None, :], rtol=1e-12, atol=1e-12)
+
+
+def test_attention_sharp_scale_selects_the_best_key():
+    # with a large scale the softmax concentrates on the key of the largest
+    # estimated logit: the output is that token's reconstructed value
+    rng = np.random.default_rng(41)
+    kc, vc, K, ke, ve = _attn_inputs(rng, 32, 40, bits_k=8, m=0)
+    Qv = rng.standard_normal((4, 32))
+    L = O.logits_from_codes(kc, Qv, ke[0], None, ke[2], None)
+    o = O.attention_from_codes(kc, vc, Qv, ke, ve, 1e4)
+    Vh = O.dequantize(vc, *ve)
+    assert np.allclose(o, Vh[np.argmax(L, axis=1)], rtol=1e-9, atol=1e-9)
+    # a query row's weights do not depend on the other rows
+    o_single = O.attention_from_codes(kc, vc, Qv[2:3], ke, ve, 1e4)
+    assert np.allclose(o_single[0], o[2], rtol=1e-12, atol=1e-12)
+
+
+def test_attention_weights_sum_to_one_and_shift_invariant():
+    # the output lies in the convex hull of the values: with all values equal
+    # to one vector the output is that vector, for any query and scale
+    rng = np.random.default_rng(42)
+    kc, vc, K, ke, _ = _attn_inputs(rng, 16, 25)
+    v = rng.standard_normal(16)
+    ve = O.encode(vc, np.repeat(v[None, :], 25, axis=0))
+    vh = O.dequantize(vc, ve.idx, ve.norm16)
+    o = O.attention_from_codes(kc, vc, rng.standard_normal((5, 16)) * 3.0, ke, (ve.idx, ve.norm16), 0.7)
+    assert np.allclose(o, vh[0][None, :], rtol=1e-12, atol=1e-12)
+
+
+def test_attention_empty_context_is_zero():
+    kc = O.make_codec(16, 3, 16, 31, 32)
+    vc = O.make_codec(16, 3, 0, 33, 0)
+    e = np.zeros((0, 16), dtype=np.int64)
+    o = O.attention_from_codes(kc, vc, np.ones((2, 16)), (e, np.zeros((0, 16), bool), np.zeros(0), np.zeros(0)),
+                               (e, np.zeros(0)), 0.25)
+    assert o.shape == (2, 16) and not o.any()
