@@ -19,8 +19,9 @@
 
 namespace tqd {
 
-constexpr int kSmaxThreads = 1024;
-constexpr int kSmaxUnroll = 8;      // independent loads in flight per thread
+constexpr int kSmaxCluster = 8;    // CTAs per row, one eighth of the row each
+constexpr int kSmaxThreads = 512;
+constexpr int kSmaxUnroll = 8;     // independent loads in flight per thread
 
 // Online (max, sum of exp) pair of two partial rows.
 __device__ __forceinline__ void smax_merge(float& m, float& l, float m2, float l2) {
@@ -32,29 +33,49 @@ __device__ __forceinline__ void smax_merge(float& m, float& l, float m2, float l
   }
 }
 
-// One CTA per row (sequence b, query head): the scores s[t] for t < ctx_len[b]
-// become exp(scale s[t] - max) / sum, in place; positions past the context are
-// left as they are (the value pass does not read them).  Each thread reads
-// kSmaxUnroll scores per step, all loads in flight before any is used.
-__global__ void __launch_bounds__(kSmaxThreads) softmax_rows_kernel(float* s, const int32_t* ctx_len, int n_q_heads,
-                                                                    int64_t stride, int max_ctx, float scale) {
+__device__ __forceinline__ uint32_t smax_cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// One cluster of kSmaxCluster CTAs per row (sequence b, query head): the
+// scores s[t] for t < ctx_len[b] become exp(scale s[t] - max) / sum, in place;
+// positions past the context are left as they are (the value pass does not
+// read them).  CTA c reduces its segment of the row to a (max, sum) pair and
+// stores it into slot c of every CTA of the cluster (distributed shared
+// memory); after the cluster barrier each CTA merges the eight pairs and
+// rewrites its segment, whose second read comes from L2.
+__global__ void __cluster_dims__(kSmaxCluster, 1, 1) __launch_bounds__(kSmaxThreads)
+    softmax_rows_kernel(float* s, const int32_t* ctx_len, int n_q_heads, int64_t stride, int max_ctx,
+                        float scale) {
   constexpr int kStep = kSmaxThreads * kSmaxUnroll;
-  __shared__ float sm[kSmaxThreads / 32], sl[kSmaxThreads / 32];
-  const int64_t row = blockIdx.x;
+  __shared__ float wm[kSmaxThreads / 32], wl[kSmaxThreads / 32];
+  __shared__ float pm[kSmaxCluster], pl[kSmaxCluster];
+  // phase 0 opens: every CTA of the cluster has started before any remote store
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+  const uint32_t c = smax_cluster_rank();
+  const int64_t row = blockIdx.x / kSmaxCluster;
   const int b = (int)(row / n_q_heads);
   const int n = max(0, min(ctx_len[b], max_ctx));
+  const int seg = ((n + kSmaxCluster - 1) / kSmaxCluster + 31) & ~31;
+  const int lo = min(n, (int)c * seg), hi = min(n, lo + seg);
   float* x = s + row * stride;
   float m = -INFINITY, l = 0.0f;
-  for (int t0 = threadIdx.x; t0 < n; t0 += kStep) {
+  for (int t0 = lo + (int)threadIdx.x; t0 < hi; t0 += kStep) {
     float v[kSmaxUnroll];
 #pragma unroll
     for (int i = 0; i < kSmaxUnroll; ++i) {
       const int t = t0 + i * kSmaxThreads;
-      v[i] = t < n ? scale * x[t] : -INFINITY;
+      v[i] = t < hi ? scale * x[t] : -INFINITY;
     }
+    float mv = v[0];
 #pragma unroll
-    for (int i = 0; i < kSmaxUnroll; ++i)
-      if (v[i] > -INFINITY) smax_merge(m, l, v[i], 1.0f);
+    for (int i = 1; i < kSmaxUnroll; ++i) mv = fmaxf(mv, v[i]);
+    float lv = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kSmaxUnroll; ++i) lv += expf(v[i] - mv);   // v[0] is finite: mv > -inf
+    smax_merge(m, l, mv, lv);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -63,26 +84,43 @@ __global__ void __launch_bounds__(kSmaxThreads) softmax_rows_kernel(float* s, co
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane == 0) {
-    sm[warp] = m;
-    sl[warp] = l;
+    wm[warp] = m;
+    wl[warp] = l;
   }
   __syncthreads();
-  m = sm[0];
-  l = sl[0];
+  m = wm[0];
+  l = wl[0];
 #pragma unroll
-  for (int w = 1; w < kSmaxThreads / 32; ++w) smax_merge(m, l, sm[w], sl[w]);
+  for (int w = 1; w < kSmaxThreads / 32; ++w) smax_merge(m, l, wm[w], wl[w]);
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+  if (threadIdx.x < kSmaxCluster) {
+    uint32_t am, al;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                 : "=r"(am) : "r"((uint32_t)__cvta_generic_to_shared(&pm[c])), "r"((uint32_t)threadIdx.x));
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+                 : "=r"(al) : "r"((uint32_t)__cvta_generic_to_shared(&pl[c])), "r"((uint32_t)threadIdx.x));
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(am), "f"(m) : "memory");
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(al), "f"(l) : "memory");
+  }
+  // phase 1: every pair delivered; no remote access after this
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  m = pm[0];
+  l = pl[0];
+#pragma unroll
+  for (int r = 1; r < kSmaxCluster; ++r) smax_merge(m, l, pm[r], pl[r]);
   const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-  for (int t0 = threadIdx.x; t0 < n; t0 += kStep) {
+  for (int t0 = lo + (int)threadIdx.x; t0 < hi; t0 += kStep) {
     float v[kSmaxUnroll];
 #pragma unroll
     for (int i = 0; i < kSmaxUnroll; ++i) {
       const int t = t0 + i * kSmaxThreads;
-      v[i] = t < n ? x[t] : 0.0f;
+      v[i] = t < hi ? x[t] : 0.0f;
     }
 #pragma unroll
     for (int i = 0; i < kSmaxUnroll; ++i) {
       const int t = t0 + i * kSmaxThreads;
-      if (t < n) x[t] = expf(scale * v[i] - m) * inv;
+      if (t < hi) x[t] = expf(scale * v[i] - m) * inv;
     }
   }
 }
@@ -123,8 +161,9 @@ tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_c
     tq_status s = launch_logits(kcb, kcv, q, dt, batch, n_q_heads, ctx_len, max_ctx, scores, max_ctx,
                                 base + w.scores, w.logits, st);
     if (s != TQ_OK) return s;
-    if (batch * n_q_heads > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_attend: batch * n_q_heads too large");
-    tqd::softmax_rows_kernel<<<(unsigned)(batch * n_q_heads), tqd::kSmaxThreads, 0, st>>>(
+    if (batch * n_q_heads > 0x7fffffffLL / tqd::kSmaxCluster || max_ctx > 0x7fff0000LL)
+      return fail(TQ_EINVAL, "tq_attend: batch * n_q_heads or max_ctx too large");
+    tqd::softmax_rows_kernel<<<(unsigned)(batch * n_q_heads * tqd::kSmaxCluster), tqd::kSmaxThreads, 0, st>>>(
         scores, ctx_len, n_q_heads, max_ctx, (int)max_ctx, scale);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "tq_attend: softmax launch");
