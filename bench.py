@@ -34,6 +34,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -73,10 +74,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, out_dir: str | None = None):
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        d = out_dir or tempfile.mkdtemp(prefix="tq_clocks_")
+        self.path = os.path.join(d, f"clocks_rank{gpu_index}.csv")
 
     def start(self):
         try:
@@ -513,7 +515,7 @@ def run_ours(args):
         g.replay()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, args.clocks_dir)
     clocks.start()
     # soak so the clock samples see the GPU under load
     t_end = time.time() + args.soak
@@ -669,6 +671,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of extra warm-up steps (clock samples)")
+    ap.add_argument("--clocks-dir", default=None,
+                    help="directory for the raw nvidia-smi clock samples (default: a temporary directory)")
     ap.add_argument("--no-append-phase", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")

@@ -256,7 +256,7 @@ tq_status tq_selftest_wait_timeout(uint32_t* error_word, void* stream);
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 
-/* Layout version of the packed records written and read by this build. */
+/* Layout version of the packed records this library writes and reads. */
 int32_t tq_layout_version(void);
 
 #ifdef __cplusplus

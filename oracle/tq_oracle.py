@@ -26,7 +26,7 @@ implement 6x LLM memory savings), a2a-mcp.org.  Sections cited:
 Everything is float64 numpy.  The library routines used as single steps are
 ``numpy.linalg.qr`` (Householder QR), ``numpy.polynomial.legendre.leggauss``
 (quadrature nodes) and matrix products.  Readings of points the page leaves
-open are marked READING and listed together in the design doc.
+open are marked READING where they are taken.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against published values, closed forms, textbook special cases or brute force.
