@@ -232,7 +232,8 @@ size_t tq_attend_workspace_bytes(const tq_codebook* key_cb, const tq_codebook* v
  * (KV head hq / (n_q_heads / n_kv_heads)),
  *   out[b, hq, :] = sum_{t < ctx_len[b]} softmax_t(scale * L[b, hq, t]) v_hat_t
  * with L the tq_logits estimate and v_hat_t = ||v_t|| Pi_v^T c16[idx_t] (the
- * value codebook's reconstruction); a row with ctx_len[b] = 0 is all zeros.
+ * value codebook's reconstruction); a row with ctx_len[b] = 0 is all zeros
+ * (with max_ctx = 0 the whole of out is cleared and nothing else runs).
  * key_cb / key_cache and value_cb / value_cache as for tq_logits and
  * tq_dequant_values (same d and n_kv_heads; value_cb has m = 0).  q: device
  * [batch, n_q_heads, d] of dtype; out: device fp32 [batch, n_q_heads, d];

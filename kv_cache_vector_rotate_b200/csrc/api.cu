@@ -500,7 +500,13 @@ tq_status tq_attend(const tq_codebook* kcb, const tq_cache* kcache, const tq_cod
   if (max_ctx > kv.max_pages * kv.page_tokens || max_ctx > vv.max_pages * vv.page_tokens)
     return fail(TQ_EINVAL, "tq_attend: max_ctx exceeds a block table");
   if (!std::isfinite(scale)) return fail(TQ_EINVAL, "tq_attend: scale is not finite");
-  if (batch == 0 || max_ctx == 0) return TQ_OK;
+  if (batch == 0) return TQ_OK;
+  if (max_ctx == 0) {                    // every context is empty: the rows are zeros
+    if (!out || !aligned(out, 4)) return fail(TQ_EINVAL, "tq_attend: out is NULL or misaligned");
+    return cuda_fail(cudaMemsetAsync(out, 0, (size_t)batch * n_q_heads * kcb->lay.d * sizeof(float),
+                                     reinterpret_cast<cudaStream_t>(stream)),
+                     "tq_attend: clearing out");
+  }
   if (!q || !ctx_len || !out || !workspace) return fail(TQ_EINVAL, "tq_attend: NULL pointer");
   if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 256))
     return fail(TQ_EINVAL, "tq_attend: misaligned pointer");

@@ -85,3 +85,30 @@ def test_integer_codebook_tables_fit_for_every_supported_d(bits):
     for d in range(8, 257, 8):
         cb = tq.Codebook(d, bits, 0, 3, 4, device=False)
         cb.close()
+
+
+def test_attend_workspace_is_scores_plus_both_passes():
+    # tq_attend's workspace: fp32 scores [batch, n_q_heads, max_ctx], then the
+    # logits and values workspaces, each rounded up to 256 bytes.
+    kcb = tq.Codebook(128, 3, 128, 1, 2, device=False)
+    vcb = tq.Codebook(128, 3, 0, 3, 4, device=False)
+    lib = tq.load_library()
+    al = lambda n: (n + 255) // 256 * 256
+    for batch, hkv, hq, ctx in [(1, 8, 32, 32768), (3, 2, 8, 700), (2, 4, 4, 17)]:
+        want = (al(batch * hq * ctx * 4) + al(lib.tq_logits_workspace_bytes(kcb.handle, batch, hkv, hq))
+                + al(lib.tq_values_workspace_bytes(vcb.handle, batch, hkv, hq, ctx)))
+        assert lib.tq_attend_workspace_bytes(kcb.handle, vcb.handle, batch, hkv, hq, ctx) == want
+    for args in [(1, 8, 30, 64), (1, 0, 8, 64), (-1, 2, 8, 64), (1, 2, 8, -1)]:
+        assert lib.tq_attend_workspace_bytes(kcb.handle, vcb.handle, *args) == 0
+    assert lib.tq_attend_workspace_bytes(None, vcb.handle, 1, 2, 8, 64) == 0
+
+
+def test_attend_refuses_host_only_codebooks():
+    kcb = tq.Codebook(128, 3, 128, 1, 2, device=False)
+    vcb = tq.Codebook(128, 3, 0, 3, 4, device=False)
+    lib = tq.load_library()
+    cs = tq.CacheStruct(None, 1, 64, 1, None, 1, None)
+    st = lib.tq_attend(kcb.handle, ctypes.byref(cs), vcb.handle, ctypes.byref(cs), None, 0, 1, 4, None, 64,
+                       0.1, None, None, 0, None)
+    assert st == tq.TQ_EINVAL
+    assert b"host-only" in lib.tq_last_error()

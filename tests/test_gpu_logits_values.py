@@ -278,3 +278,20 @@ def test_attend_matches_oracle_attention(tqm, kbits, m, vbits):
             err = np.abs(O_gpu[b, h * G:(h + 1) * G] - o).max(axis=1)
             assert np.all(err <= 2e-3 * row_scale), (b, h, err / row_scale)
     assert kcache.errors() == 0 and vcache.errors() == 0
+
+
+def test_attend_with_no_context_clears_out(tqm):
+    """max_ctx = 0: every context is empty, so tq_attend writes zero rows over
+    whatever out held."""
+    d, pt, heads, G, batch = 128, 32, 2, 4, 2
+    kcb = tqm.Codebook(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    vcb = tqm.Codebook(d, 3, 0, synth.SEED_PI, synth.SEED_S)
+    bt = torch.from_numpy(synth.block_table(37, batch, 1))
+    kcache = tqm.PagedCache.allocate(kcb, batch, pt, heads, bt)
+    vcache = tqm.PagedCache.allocate(vcb, batch, pt, heads, bt)
+    q = torch.randn(batch, heads * G, d, device="cuda").to(torch.bfloat16)
+    out = torch.full((batch, heads * G, d), float("nan"), device="cuda")
+    ctx_t = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    tqm.attend(kcb, kcache, vcb, vcache, q, ctx_t, 0, out=out)
+    torch.cuda.synchronize()
+    assert bool((out == 0).all())
