@@ -215,8 +215,10 @@ size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n
  * (weights != NULL, device fp32 [batch, n_q_heads, w_stride]): out device
  * fp32 [batch, n_q_heads, d] receives sum_{t < ctx_len[b]} weights[b,hq,t]
  * v_hat_t, accumulated in the rotated space and rotated back once.  For mode B
- * out_dtype must be TQ_F32 and out_stride is ignored.  workspace: device, at
- * least tq_values_workspace_bytes() (0 is enough for mode A). */
+ * out_dtype must be TQ_F32 and out_stride is ignored; with max_ctx = 0 out is
+ * cleared (every context is empty).  workspace: device, at least
+ * tq_values_workspace_bytes() (0 is enough for mode A).  out, weights and
+ * workspace must be aligned to their element size (TQ_EINVAL otherwise). */
 tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache,
                             const float* weights, int64_t w_stride, int64_t batch,
                             int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx,

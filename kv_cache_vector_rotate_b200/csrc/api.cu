@@ -461,9 +461,20 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache, const 
   } else if (out_stride < max_ctx) {
     return fail(TQ_EINVAL, "tq_dequant_values: out_stride < max_ctx");
   }
-  if (batch == 0 || max_ctx == 0) return TQ_OK;
+  if (batch == 0) return TQ_OK;
+  if (max_ctx == 0) {
+    if (!weights) return TQ_OK;          // mode A: no token to write
+    // mode B: every context is empty, so every output row is zero
+    if (!out || !aligned(out, 4)) return fail(TQ_EINVAL, "tq_dequant_values: out is NULL or misaligned");
+    return cuda_fail(cudaMemsetAsync(out, 0, (size_t)batch * n_q_heads * cb->lay.d * sizeof(float),
+                                     reinterpret_cast<cudaStream_t>(stream)),
+                     "tq_dequant_values: clearing out");
+  }
   if (!ctx_len || !out) return fail(TQ_EINVAL, "tq_dequant_values: NULL pointer");
   if (weights && !workspace) return fail(TQ_EINVAL, "tq_dequant_values: mode B needs a workspace");
+  const bool misaligned = weights ? !aligned(out, 4) || !aligned(weights, 4) || !aligned(workspace, 4)
+                                  : !aligned(out, dtype_size(out_dtype));
+  if (misaligned) return fail(TQ_EINVAL, "tq_dequant_values: misaligned pointer");
   return launch_values(cb, cv, weights, w_stride, batch, n_q_heads, ctx_len, max_ctx, out,
                        out_dtype, out_stride, workspace, workspace_bytes,
                        reinterpret_cast<cudaStream_t>(stream));

@@ -295,3 +295,17 @@ def test_attend_with_no_context_clears_out(tqm):
     tqm.attend(kcb, kcache, vcb, vcache, q, ctx_t, 0, out=out)
     torch.cuda.synchronize()
     assert bool((out == 0).all())
+
+
+def test_values_mode_b_with_no_context_clears_out(tqm):
+    """Mode B with max_ctx = 0: every weighted sum is over an empty context,
+    so out becomes zeros whatever it held."""
+    d, pt, heads, G, batch = 128, 32, 2, 4, 2
+    cb = tqm.Codebook(d, 3, 0, synth.SEED_PI, synth.SEED_S)
+    cache = tqm.PagedCache.allocate(cb, batch, pt, heads, torch.from_numpy(synth.block_table(38, batch, 1)))
+    w = torch.zeros(batch, heads * G, 1, device="cuda")
+    out = torch.full((batch, heads * G, d), float("nan"), device="cuda")
+    ctx_t = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    tqm.dequant_values(cb, cache, ctx_t, 0, batch, weights=w, out=out)
+    torch.cuda.synchronize()
+    assert bool((out == 0).all())
