@@ -107,7 +107,9 @@ typedef struct {
 /* A paged cache of packed records, owned by the caller.  pages: device,
  * n_pages * page_bytes bytes, 16-byte aligned.  block_table: device int32
  * [batch, max_pages_per_seq].  page_tokens: a power of two, 16..256.
- * error_word: device uint32 or NULL. */
+ * error_word: device uint32 or NULL.  Every int32 / uint32 / float array the
+ * entry points take (block_table, error_word, start_pos, ctx_len, weights,
+ * out) must be aligned to its element size; a misaligned one is TQ_EINVAL. */
 typedef struct {
   void* pages;
   int64_t n_pages;

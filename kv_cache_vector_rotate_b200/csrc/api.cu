@@ -263,6 +263,8 @@ static tq_status make_view(const tq_codebook* cb, const tq_cache* c, CacheView* 
   if (!c) return fail(TQ_EINVAL, "cache is NULL");
   if (!c->pages || !c->block_table) return fail(TQ_EINVAL, "cache pages / block_table is NULL");
   if (!aligned(c->pages, 16)) return fail(TQ_EINVAL, "cache pages must be 16-byte aligned");
+  if (!aligned(c->block_table, 4) || (c->error_word && !aligned(c->error_word, 4)))
+    return fail(TQ_EINVAL, "cache block_table / error_word must be 4-byte aligned");
   if (c->page_tokens < 16 || c->page_tokens > 256 || (c->page_tokens & (c->page_tokens - 1)) != 0)
     return fail(TQ_EINVAL, "page_tokens must be a power of two in [16, 256]");
   if (c->n_kv_heads < 1 || c->n_pages < 1 || c->max_pages_per_seq < 1)
@@ -391,7 +393,8 @@ tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtyp
     return fail(TQ_EINVAL, "tq_quantize_append: n_kv_heads differs from the cache's");
   if (batch == 0 || n_new == 0) return TQ_OK;
   if (!x || !start_pos) return fail(TQ_EINVAL, "tq_quantize_append: x / start_pos is NULL");
-  if (!aligned(x, dtype_size(dtype))) return fail(TQ_EINVAL, "tq_quantize_append: x misaligned");
+  if (!aligned(x, dtype_size(dtype)) || !aligned(start_pos, 4))
+    return fail(TQ_EINVAL, "tq_quantize_append: x / start_pos misaligned");
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   bool handled = false;
   s = launch_quantize_tc(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st, &handled);
@@ -426,7 +429,7 @@ tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
     return fail(TQ_EINVAL, "tq_logits: max_ctx exceeds the block table");
   if (batch == 0 || max_ctx == 0) return TQ_OK;
   if (!q || !ctx_len || !out || !workspace) return fail(TQ_EINVAL, "tq_logits: NULL pointer");
-  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 16))
+  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 16) || !aligned(ctx_len, 4))
     return fail(TQ_EINVAL, "tq_logits: misaligned pointer");
   return launch_logits(cb, cv, q, dtype, batch, n_q_heads, ctx_len, max_ctx, out, out_stride,
                        workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
@@ -471,6 +474,7 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache, const 
                      "tq_dequant_values: clearing out");
   }
   if (!ctx_len || !out) return fail(TQ_EINVAL, "tq_dequant_values: NULL pointer");
+  if (!aligned(ctx_len, 4)) return fail(TQ_EINVAL, "tq_dequant_values: ctx_len misaligned");
   if (weights && !workspace) return fail(TQ_EINVAL, "tq_dequant_values: mode B needs a workspace");
   const bool misaligned = weights ? !aligned(out, 4) || !aligned(weights, 4) || !aligned(workspace, 4)
                                   : !aligned(out, dtype_size(out_dtype));
@@ -519,7 +523,7 @@ tq_status tq_attend(const tq_codebook* kcb, const tq_cache* kcache, const tq_cod
                      "tq_attend: clearing out");
   }
   if (!q || !ctx_len || !out || !workspace) return fail(TQ_EINVAL, "tq_attend: NULL pointer");
-  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 256))
+  if (!aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 256) || !aligned(ctx_len, 4))
     return fail(TQ_EINVAL, "tq_attend: misaligned pointer");
   return launch_attend(kcb, kv, vcb, vv, q, dtype, batch, n_q_heads, ctx_len, max_ctx, scale, out, workspace,
                        workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
