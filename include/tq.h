@@ -258,6 +258,20 @@ tq_status tq_attend(const tq_codebook* key_cb, const tq_cache* key_cache, const 
  * error_word.  The method has no counterpart: this checks the library. */
 tq_status tq_selftest_wait_timeout(uint32_t* error_word, void* stream);
 
+/* Host-side tables of the recursive polar form of stage 1 ("TurboQuant
+ * explained", §Stage 1, PolarQuant paragraph): the rotated unit vector's
+ * coordinates are paired recursively into polar form, level 1 giving angles
+ * atan2(u[2i+1], u[2i]) in [-pi, pi] and level l > 1 angles atan2(rho[2i+1],
+ * rho[2i]) in [0, pi/2] of the previous level's radii.  For a uniform unit
+ * vector level-1 angles are uniform and a level-l angle has sin^2 phi ~
+ * Beta(k/2, k/2), k = 2^(l-1).  Writes the Lloyd-Max quantizer of that law
+ * with 2^bits levels: centroids (host, 2^bits doubles, ascending, symmetric
+ * about the middle of the support), boundaries (host, 2^bits - 1 midpoints,
+ * or NULL) and the mean squared angle error (or NULL).  level in [1, 8],
+ * bits in [1, 8] (TQ_EINVAL / TQ_EUNSUPPORTED otherwise).  No GPU needed. */
+tq_status tq_polar_angle_codebook(int32_t level, int32_t bits, double* centroids, double* boundaries,
+                                  double* distortion);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 

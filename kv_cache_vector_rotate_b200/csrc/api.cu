@@ -363,6 +363,18 @@ tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s, doubl
   return TQ_OK;
 }
 
+tq_status tq_polar_angle_codebook(int32_t level, int32_t bits, double* centroids, double* boundaries,
+                                  double* distortion) {
+  if (level < 1 || level > 8) return fail(TQ_EINVAL, "tq_polar_angle_codebook: level must be in [1, 8]");
+  if (bits < 1 || bits > 8) return fail(TQ_EUNSUPPORTED, "tq_polar_angle_codebook: bits must be in [1, 8]");
+  if (!centroids) return fail(TQ_EINVAL, "tq_polar_angle_codebook: centroids is NULL");
+  const tqhost::LloydMax lm = tqhost::polar_angle_lloyd_max(level, bits);
+  std::memcpy(centroids, lm.centroids.data(), lm.centroids.size() * sizeof(double));
+  if (boundaries) std::memcpy(boundaries, lm.boundaries.data(), lm.boundaries.size() * sizeof(double));
+  if (distortion) *distortion = lm.distortion;
+  return TQ_OK;
+}
+
 tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_heads,
                     tq_layout_info* info) {
   if (!cb || !info) return fail(TQ_EINVAL, "codebook / info is NULL");

@@ -117,12 +117,17 @@ struct Moments {
   double p, m1, m2;
 };
 
+// The coordinate law of §Stage 1.  Start cells: equal probability, from a
+// trapezoid CDF in theta.
 class BetaLaw {
  public:
   explicit BetaLaw(int d) : d_(d), gauss_(24) {
     c_ = std::exp(std::lgamma(d / 2.0) - 0.5 * std::log(3.14159265358979323846) -
                   std::lgamma((d - 1) / 2.0));
   }
+  double lo() const { return -1.0; }
+  double hi() const { return 1.0; }
+  double centre() const { return 0.0; }
   double density(double t) const {
     double s = 1.0 - t * t;
     if (s <= 0.0) return 0.0;
@@ -150,6 +155,26 @@ class BetaLaw {
     r.m2 *= c_;
     return r;
   }
+  std::vector<double> equiprobable_edges(int K) const {
+    const int G = 20001;
+    const double half_pi = 1.57079632679489661923;
+    std::vector<double> th(G), cdf(G, 0.0);
+    for (int i = 0; i < G; ++i) th[i] = -half_pi + 2.0 * half_pi * i / (G - 1);
+    for (int i = 1; i < G; ++i)
+      cdf[i] = cdf[i - 1] + 0.5 * (std::pow(std::cos(th[i]), d_ - 2) +
+                                   std::pow(std::cos(th[i - 1]), d_ - 2)) * (th[i] - th[i - 1]);
+    std::vector<double> qe(K + 1);
+    qe[0] = -1.0;
+    qe[K] = 1.0;
+    int j = 0;
+    for (int k = 1; k < K; ++k) {
+      double target = (double)k / K * cdf[G - 1];
+      while (j < G - 2 && cdf[j + 1] < target) ++j;
+      double fr = (target - cdf[j]) / (cdf[j + 1] - cdf[j]);
+      qe[k] = std::sin(th[j] + fr * (th[j + 1] - th[j]));
+    }
+    return qe;
+  }
 
  private:
   int d_;
@@ -157,40 +182,95 @@ class BetaLaw {
   Gauss gauss_;
 };
 
-}  // namespace
-
-LloydMax lloyd_max(int d, int bits) {
-  const int K = 1 << bits;
-  BetaLaw law(d);
-  // start: means of the K cells of equal probability (trapezoid CDF in theta)
-  std::vector<double> c(K), e(K + 1);
-  {
+// The law of a level-`level` angle of the recursive polar form of §Stage 1
+// for a uniform unit vector: level 1 uniform on [-pi, pi]; level l > 1, whose
+// radii each cover k = 2^(l-1) coordinates, 2 (sin phi cos phi)^(k-1) /
+// B(k/2, k/2) on [0, pi/2] (sin^2 phi follows Beta(k/2, k/2)).  Smooth on its
+// support, so cells are integrated in phi directly.
+class AngleLaw {
+ public:
+  explicit AngleLaw(int level) : level_(level), gauss_(24) {
+    const double pi = 3.14159265358979323846;
+    if (level == 1) {
+      lo_ = -pi;
+      hi_ = pi;
+      logc_ = -std::log(2.0 * pi);
+    } else {
+      const double k = std::ldexp(1.0, level - 1);
+      lo_ = 0.0;
+      hi_ = 0.5 * pi;
+      logc_ = std::log(2.0) + std::lgamma(k) - 2.0 * std::lgamma(0.5 * k);
+    }
+  }
+  double lo() const { return lo_; }
+  double hi() const { return hi_; }
+  double centre() const { return 0.5 * (lo_ + hi_); }
+  double density(double phi) const {
+    if (phi < lo_ || phi > hi_) return 0.0;
+    if (level_ == 1) return std::exp(logc_);
+    const double s = std::sin(phi) * std::cos(phi);
+    if (s <= 0.0) return 0.0;
+    return std::exp(logc_ + (std::ldexp(1.0, level_ - 1) - 1.0) * std::log(s));
+  }
+  Moments cell(double a, double b) const {
+    const int panels = 48;
+    const double h = (b - a) / panels;
+    Moments r{0.0, 0.0, 0.0};
+    for (int p = 0; p < panels; ++p) {
+      const double mid = a + (p + 0.5) * h, half = 0.5 * h;
+      for (size_t i = 0; i < gauss_.x.size(); ++i) {
+        const double x = mid + half * gauss_.x[i];
+        const double g = half * gauss_.w[i] * density(x);
+        r.p += g;
+        r.m1 += g * x;
+        r.m2 += g * x * x;
+      }
+    }
+    return r;
+  }
+  std::vector<double> equiprobable_edges(int K) const {
     const int G = 20001;
-    const double half_pi = 1.57079632679489661923;
-    std::vector<double> th(G), cdf(G, 0.0);
-    for (int i = 0; i < G; ++i) th[i] = -half_pi + 2.0 * half_pi * i / (G - 1);
-    for (int i = 1; i < G; ++i)
-      cdf[i] = cdf[i - 1] + 0.5 * (std::pow(std::cos(th[i]), d - 2) +
-                                   std::pow(std::cos(th[i - 1]), d - 2)) * (th[i] - th[i - 1]);
-    for (int i = 0; i < G; ++i) cdf[i] /= cdf[G - 1];
+    std::vector<double> x(G), cdf(G, 0.0);
+    for (int i = 0; i < G; ++i) x[i] = lo_ + (hi_ - lo_) * i / (G - 1);
+    for (int i = 1; i < G; ++i) cdf[i] = cdf[i - 1] + 0.5 * (density(x[i]) + density(x[i - 1])) * (x[i] - x[i - 1]);
     std::vector<double> qe(K + 1);
-    qe[0] = -1.0;
-    qe[K] = 1.0;
+    qe[0] = lo_;
+    qe[K] = hi_;
     int j = 0;
     for (int k = 1; k < K; ++k) {
-      double target = (double)k / K;
+      const double target = (double)k / K * cdf[G - 1];
       while (j < G - 2 && cdf[j + 1] < target) ++j;
-      double fr = (target - cdf[j]) / (cdf[j + 1] - cdf[j]);
-      qe[k] = std::sin(th[j] + fr * (th[j + 1] - th[j]));
+      const double fr = (target - cdf[j]) / (cdf[j + 1] - cdf[j]);
+      qe[k] = x[j] + fr * (x[j + 1] - x[j]);
     }
+    return qe;
+  }
+
+ private:
+  int level_;
+  double lo_, hi_, logc_;
+  Gauss gauss_;
+};
+
+// Lloyd-Max quantizer of a law symmetric about its centre (Lloyd 1957/1982,
+// Max 1960): centroids are the conditional means of their cells, boundaries
+// the midpoints.  Lloyd sweeps from the equal-probability cells, then Newton
+// on F_i(c) = c_i - mean_i(c) (tridiagonal Jacobian); the laws here are
+// log-concave, so the fixed point is unique.  The result is made exactly
+// symmetric about the centre.
+template <class Law>
+LloydMax lloyd_max_law(const Law& law, int K) {
+  std::vector<double> c(K), e(K + 1);
+  {
+    const std::vector<double> qe = law.equiprobable_edges(K);
     for (int k = 0; k < K; ++k) {
       Moments m = law.cell(qe[k], qe[k + 1]);
       c[k] = m.m1 / m.p;
     }
   }
   auto edges = [&](const std::vector<double>& cc) {
-    e[0] = -1.0;
-    e[K] = 1.0;
+    e[0] = law.lo();
+    e[K] = law.hi();
     for (int i = 1; i < K; ++i) e[i] = 0.5 * (cc[i - 1] + cc[i]);
   };
   std::vector<Moments> mo(K);
@@ -198,7 +278,6 @@ LloydMax lloyd_max(int d, int bits) {
     edges(c);
     for (int i = 0; i < K; ++i) mo[i] = law.cell(e[i], e[i + 1]);
   };
-  // Lloyd sweeps: centroid <- conditional mean of its cell.
   for (int it = 0; it < 300; ++it) {
     moments();
     double step = 0.0;
@@ -209,7 +288,6 @@ LloydMax lloyd_max(int d, int bits) {
     }
     if (step < 1e-15) break;
   }
-  // Newton on F_i(c) = c_i - mean_i(c); the Jacobian is tridiagonal.
   for (int it = 0; it < 60; ++it) {
     moments();
     std::vector<double> F(K), lower(K, 0.0), diag(K, 1.0), upper(K, 0.0);
@@ -241,16 +319,16 @@ LloydMax lloyd_max(int d, int bits) {
     for (int i = K - 2; i >= 0; --i) delta[i] = dp[i] - cp[i] * delta[i + 1];
     for (int i = 0; i < K; ++i) c[i] -= delta[i];
   }
-  // The law is symmetric: make the codebook exactly antisymmetric.
+  const double ctr = law.centre();
   std::vector<double> cs(K);
-  for (int i = 0; i < K; ++i) cs[i] = 0.5 * (c[i] - c[K - 1 - i]);
+  for (int i = 0; i < K; ++i) cs[i] = ctr + 0.5 * ((c[i] - ctr) - (c[K - 1 - i] - ctr));
   LloydMax out;
   out.centroids = cs;
   out.boundaries.resize(K - 1);
   for (int i = 1; i < K; ++i) out.boundaries[i - 1] = 0.5 * (cs[i - 1] + cs[i]);
   out.distortion = 0.0;
-  e[0] = -1.0;
-  e[K] = 1.0;
+  e[0] = law.lo();
+  e[K] = law.hi();
   for (int i = 1; i < K; ++i) e[i] = out.boundaries[i - 1];
   for (int i = 0; i < K; ++i) {
     Moments m = law.cell(e[i], e[i + 1]);
@@ -258,5 +336,11 @@ LloydMax lloyd_max(int d, int bits) {
   }
   return out;
 }
+
+}  // namespace
+
+LloydMax lloyd_max(int d, int bits) { return lloyd_max_law(BetaLaw(d), 1 << bits); }
+
+LloydMax polar_angle_lloyd_max(int level, int bits) { return lloyd_max_law(AngleLaw(level), 1 << bits); }
 
 }  // namespace tqhost

@@ -22,4 +22,9 @@ struct LloydMax {
 // Lloyd-Max quantizer of the Beta((d-1)/2,(d-1)/2) law on [-1, 1].
 LloydMax lloyd_max(int d, int bits);
 
+// Lloyd-Max quantizer of the level-`level` angle law of the recursive polar
+// form (level 1 uniform on [-pi, pi]; level l > 1 on [0, pi/2] with
+// sin^2 phi ~ Beta(k/2, k/2), k = 2^(l-1)); symmetric about the centre.
+LloydMax polar_angle_lloyd_max(int level, int bits);
+
 }  // namespace tqhost

@@ -25,7 +25,7 @@ EXPORTS = (
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
-    "tq_attend_workspace_bytes", "tq_attend",
+    "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook",
 )
 
 
@@ -85,6 +85,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_attend_workspace_bytes": (sz, [vp, vp, i64, i32, i32, i64]),
         "tq_attend": (i32, [vp, ctypes.POINTER(CacheStruct), vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32,
                             vp, i64, ctypes.c_float, vp, vp, sz, vp]),
+        "tq_polar_angle_codebook": (i32, [i32, i32, vp, vp, vp]),
         "tq_last_error": (ctypes.c_char_p, []),
         "tq_layout_version": (i32, []),
     }
@@ -277,6 +278,18 @@ def selftest_wait_timeout(error_word, stream=None) -> None:
     """tq_selftest_wait_timeout: a bounded wait that runs out (about 1 s) and
     reports DEV_ERR_TIMEOUT into `error_word` (device int32 [1])."""
     _check(load_library().tq_selftest_wait_timeout(_ptr(error_word), _stream(stream)))
+
+
+def polar_angle_codebook(level: int, bits: int):
+    """tq_polar_angle_codebook: (centroids, boundaries, distortion) of the
+    Lloyd-Max quantizer of the level-`level` angles of the polar form."""
+    import numpy as np
+    c = np.zeros(1 << bits, dtype=np.float64)
+    t = np.zeros((1 << bits) - 1, dtype=np.float64)
+    dist = ctypes.c_double(0.0)
+    _check(load_library().tq_polar_angle_codebook(level, bits, c.ctypes.data, t.ctypes.data if t.size else None,
+                                                   ctypes.addressof(dist)))
+    return c, t, dist.value
 
 
 def attend_workspace_bytes(key_cb: Codebook, value_cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int,

@@ -112,3 +112,23 @@ def test_attend_refuses_host_only_codebooks():
                        0.1, None, None, 0, None)
     assert st == tq.TQ_EINVAL
     assert b"host-only" in lib.tq_last_error()
+
+
+@pytest.mark.parametrize("level", [1, 2, 3, 5, 7, 8])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_polar_angle_tables_match_oracle(level, bits):
+    from oracle import polar_oracle as P
+    c, t, dist = tq.polar_angle_codebook(level, bits)
+    ref = P.angle_lloyd_max(level, bits)
+    assert np.allclose(c, ref.centroids, rtol=0, atol=1e-11)
+    assert np.allclose(t, ref.boundaries, rtol=0, atol=1e-11)
+    assert abs(dist - ref.distortion) <= 1e-12 + 1e-9 * ref.distortion
+
+
+def test_polar_angle_codebook_refuses_bad_arguments():
+    lib = tq.load_library()
+    buf = (ctypes.c_double * 512)()
+    assert lib.tq_polar_angle_codebook(0, 2, buf, None, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_angle_codebook(9, 2, buf, None, None) == tq.TQ_EINVAL
+    assert lib.tq_polar_angle_codebook(2, 9, buf, None, None) == tq.TQ_EUNSUPPORTED
+    assert lib.tq_polar_angle_codebook(2, 2, None, None, None) == tq.TQ_EINVAL
