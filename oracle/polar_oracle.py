@@ -32,6 +32,9 @@ the rest of the page supports:
 * P6 Decoding runs the recursion backwards from radius 1 with the centroids
   in place of the angles.  The key is ||x|| Pi^T u_hat and its logit against
   a query q is ||x|| <Pi q, u_hat>; the zero vector decodes to zero.
+* P7 Stage 2 (§Stage 2) applies unchanged on top: the residual
+  r = u - Pi^T u_hat (original space) keeps the signs of S r and the fp16
+  ||r||, and the logit gains ||x|| sqrt(pi/2)/m ||r|| <S q, sign(S r)>.
 
 Parity status: every function here is pinned by ``tests/test_oracle_polar.py``
 against closed forms, a library's Beta law and integrals, special vectors and
@@ -45,7 +48,7 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from .tq_oracle import fp16, rotation, unit_and_norm
+from .tq_oracle import fp16, qjl_matrix, qjl_scale, rotation, unit_and_norm
 
 # ---------------------------------------------------------------------------
 # The recursive polar transform (P2, P3) and its inverse (P6).
@@ -187,12 +190,15 @@ class PolarCodec:
     bits: int
     Pi: np.ndarray                 # d x d, the rotation of the scalar codec
     books: list[AngleCodebook]     # level 1 first
+    m: int = 0                     # QJL rows (0: stage 1 only)
+    S: np.ndarray | None = None    # m x d
 
 
-def make_polar_codec(d: int, bits: int, seed_pi: int) -> PolarCodec:
+def make_polar_codec(d: int, bits: int, seed_pi: int, m: int = 0, seed_s: int = 0) -> PolarCodec:
     L = n_levels(d)
     Pi, _, _ = rotation(d, seed_pi)
-    return PolarCodec(d, bits, Pi, [angle_lloyd_max(level, bits) for level in range(1, L + 1)])
+    S = qjl_matrix(m, d, seed_s) if m > 0 else None
+    return PolarCodec(d, bits, Pi, [angle_lloyd_max(level, bits) for level in range(1, L + 1)], m, S)
 
 
 @dataclass
@@ -200,6 +206,8 @@ class PolarEncoded:
     idx: list[np.ndarray]      # level l: [N, d / 2^l] int, 0 .. 2^b - 1
     norm16: np.ndarray         # [N] float16 ||x||
     angles: list[np.ndarray]   # the exact angles (for boundary windows)
+    qneg: np.ndarray | None = None     # [N, m] bool, True where (S r)_i < 0
+    rnorm16: np.ndarray | None = None  # [N] float16 ||r||
 
 
 def quantize_angles(angles: list[np.ndarray], books: list[AngleCodebook]) -> list[np.ndarray]:
@@ -210,7 +218,13 @@ def quantize_angles(angles: list[np.ndarray], books: list[AngleCodebook]) -> lis
 def polar_encode(codec: PolarCodec, X: np.ndarray) -> PolarEncoded:
     U, n = unit_and_norm(X)
     angles, _ = polar_forward(U @ codec.Pi.T)
-    return PolarEncoded(quantize_angles(angles, codec.books), fp16(n), angles)
+    idx = quantize_angles(angles, codec.books)
+    enc = PolarEncoded(idx, fp16(n), angles)
+    if codec.m > 0:
+        R = U - polar_decode_unit(codec, idx) @ codec.Pi     # residual, original space (P7)
+        enc.qneg = (R @ codec.S.T) < 0.0
+        enc.rnorm16 = fp16(np.sqrt(np.sum(R * R, axis=1)))
+    return enc
 
 
 def polar_decode_unit(codec: PolarCodec, idx: list[np.ndarray]) -> np.ndarray:
@@ -225,6 +239,11 @@ def polar_decode(codec: PolarCodec, enc: PolarEncoded) -> np.ndarray:
 
 
 def polar_logits(codec: PolarCodec, Qv: np.ndarray, enc: PolarEncoded) -> np.ndarray:
-    """[n_queries, N]: ||x|| <Pi q, u_hat>, the query rotated once."""
-    Qr = np.asarray(Qv, dtype=np.float64) @ codec.Pi.T
-    return (Qr @ polar_decode_unit(codec, enc.idx).T) * enc.norm16.astype(np.float64)[None, :]
+    """[n_queries, N]: ||x|| (<Pi q, u_hat> + sqrt(pi/2)/m ||r|| <S q, sign(S r)>),
+    the query rotated (and sketched) once; the second term only when m > 0."""
+    Qv = np.asarray(Qv, dtype=np.float64)
+    out = (Qv @ codec.Pi.T) @ polar_decode_unit(codec, enc.idx).T
+    if codec.m > 0:
+        signs = np.where(enc.qneg, -1.0, 1.0)
+        out = out + qjl_scale(codec.m) * enc.rnorm16.astype(np.float64)[None, :] * ((Qv @ codec.S.T) @ signs.T)
+    return out * enc.norm16.astype(np.float64)[None, :]

@@ -182,3 +182,51 @@ def test_zero_vector_decodes_to_zero():
     codec = P.make_polar_codec(8, 2, SEED_PI)
     enc = P.polar_encode(codec, np.zeros((2, 8)))
     assert np.array_equal(P.polar_decode(codec, enc), np.zeros((2, 8)))
+
+
+def test_qjl_on_the_polar_residual_is_unbiased_with_closed_form_variance():
+    # Stage 2 over the polar stage 1: with Pi fixed and 1000 seeds for S the
+    # mean error is within 3 sigma / sqrt(1000) of 0, and the variance matches
+    # ||k||^2 ||r||^2 (pi/2)/m (||q||^2 - (2/pi) <q, r/||r||>^2).
+    d, b, m = 64, 2, 64
+    rng = np.random.default_rng(16)
+    k = rng.standard_normal(d) * 1.5
+    q = rng.standard_normal(d)
+    base = P.make_polar_codec(d, b, SEED_PI)
+    est = []
+    for seed in range(1000):
+        codec = P.PolarCodec(d, b, base.Pi, base.books, m, np.random.default_rng(5000 + seed).standard_normal((m, d)))
+        enc = P.polar_encode(codec, k[None, :])
+        u = k / np.linalg.norm(k)
+        r = u - P.polar_decode_unit(codec, enc.idx)[0] @ codec.Pi
+        # un-rounded side values, so that only the sketch is random
+        enc.norm16 = np.array([np.linalg.norm(k)])
+        enc.rnorm16 = np.array([np.linalg.norm(r)])
+        est.append(P.polar_logits(codec, q[None, :], enc)[0, 0])
+    err = np.array(est) - q @ k
+    sigma = err.std(ddof=1)
+    assert abs(err.mean()) < 3 * sigma / math.sqrt(len(err))
+    rhat = r / np.linalg.norm(r)
+    var_cf = (k @ k) * (r @ r) * (math.pi / 2) / m * (q @ q - (2 / math.pi) * (q @ rhat) ** 2)
+    chi2 = (len(err) - 1) * sigma ** 2 / var_cf
+    lo, hi = stats.chi2.ppf([0.0005, 0.9995], len(err) - 1)
+    assert lo < chi2 < hi
+
+
+def test_stage_one_logit_is_biased_where_the_sketch_is_not():
+    # The stage-1 estimate <q, x_hat> alone is off by <q, ||x|| Pi^T r> for
+    # this key; averaging the sketch term over seeds removes that offset.
+    d, b, m = 32, 1, 32
+    rng = np.random.default_rng(17)
+    k, q = rng.standard_normal(d), rng.standard_normal(d)
+    base = P.make_polar_codec(d, b, SEED_PI)
+    stage1 = P.polar_logits(base, q[None, :], P.polar_encode(base, k[None, :]))[0, 0]
+    vals = []
+    for seed in range(600):
+        codec = P.PolarCodec(d, b, base.Pi, base.books, m, np.random.default_rng(7000 + seed).standard_normal((m, d)))
+        vals.append(P.polar_logits(codec, q[None, :], P.polar_encode(codec, k[None, :]))[0, 0])
+    vals = np.array(vals)
+    se = vals.std(ddof=1) / math.sqrt(len(vals))
+    exact = q @ k
+    assert abs(stage1 - exact) > 6 * se          # stage 1 alone misses by many standard errors
+    assert abs(vals.mean() - exact) < 4 * se + 2e-3 * abs(exact)   # fp16 side values only
