@@ -30,6 +30,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -137,6 +138,13 @@ def _max_over_ranks(x: float, ws: int, device) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _percentiles(xs) -> dict:
+    """p10 / p50 / p90 of a sample by the nearest-rank rule."""
+    s = sorted(xs)
+    pick = lambda p: s[min(len(s) - 1, max(0, math.ceil(p / 100.0 * len(s)) - 1))]
+    return {"p10": pick(10), "p50": pick(50), "p90": pick(90), "n": len(s)}
 
 
 def _barrier(ws):
@@ -579,6 +587,8 @@ def run_ours(args):
     log_ms = timed("logits")
     val_ms = timed("values")
     att_ms = timed("attend")
+    # spread of the headline call: per-call time over further replays of its graph
+    log_spread = _percentiles([timed("logits") / args.steps for _ in range(args.spread_replays)])
     del graphs
 
     # e2e: the same step through host buffers (pinned), copies inside the region
@@ -641,7 +651,8 @@ def run_ours(args):
                    "logits_ms_per_step": log_ms / steps, "values_ms_per_step": val_ms / steps,
                    "append_ms_per_step": app_ms / steps,
                    "values_gbs": n * VALUE_BYTES * steps / (val_ms * 1e-3) / 1e9,
-                   "attend_ms_per_step": att_ms / steps},
+                   "attend_ms_per_step": att_ms / steps,
+                   "logits_ms_per_step_spread": dict(log_spread, replays_of_steps=steps)},
         "roofline": {"bound": "hbm", "achieved": logits_gbs / n, "peak": hbm_peak, "unit": "GB/s",
                      "frac": logits_gbs / n / hbm_peak, "traffic": LOGITS_DRAM_BYTES,
                      "traffic_source": LOGITS_DRAM_SOURCE,
@@ -711,6 +722,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of extra warm-up steps (clock samples)")
+    ap.add_argument("--spread-replays", type=int, default=15,
+                    help="extra replays of the logits graph for its p10 / p50 / p90 (after the timed region)")
     ap.add_argument("--clocks-dir", default=None,
                     help="directory for the raw nvidia-smi clock samples (default: a temporary directory)")
     ap.add_argument("--no-append-phase", action="store_true")

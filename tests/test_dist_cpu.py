@@ -87,3 +87,12 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["metric"] == "fused 3-bit logits HBM GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_percentiles_nearest_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench._percentiles(range(1, 11)) == {"p10": 1, "p50": 5, "p90": 9, "n": 10}
+    assert bench._percentiles([2.5]) == {"p10": 2.5, "p50": 2.5, "p90": 2.5, "n": 1}
+    s = bench._percentiles([4, 1, 3, 2])
+    assert (s["p10"], s["p50"], s["p90"]) == (1, 2, 4)
