@@ -129,9 +129,12 @@ def test_logits_empty_context(tqm):
     assert torch.all(out == 7.0)
 
 
-@pytest.mark.parametrize("d,bits", [(128, 3), (128, 2), (200, 4), (64, 1)])
-def test_values_mode_a_and_b(tqm, d, bits):
-    batch, heads, G, pt = 2, 2, 4, 64
+@pytest.mark.parametrize("d,bits,pt", [(128, 3, 64), (128, 2, 64), (200, 4, 64), (64, 1, 64),
+                                       (128, 3, 16), (128, 3, 256)])
+def test_values_mode_a_and_b(tqm, d, bits, pt):
+    # pt = 16: 32-token units straddle pages (the kernels' per-half copies);
+    # pt = 256: several units per page
+    batch, heads, G = 2, 2, 4
     ctx = [700, 129]
     rng = np.random.default_rng(31)
     vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
@@ -241,14 +244,15 @@ def test_logits_more_query_tiles_than_cta_slots(tqm):
     assert cache.errors() == 0
 
 
-@pytest.mark.parametrize("kbits,m,vbits", [(3, 128, 3), (2, 128, 4), (4, 0, 2)])
-def test_attend_matches_oracle_attention(tqm, kbits, m, vbits):
+@pytest.mark.parametrize("kbits,m,vbits,pt", [(3, 128, 3, 32), (2, 128, 4, 32), (4, 0, 2, 32), (3, 128, 3, 16),
+                                              (3, 128, 3, 256)])
+def test_attend_matches_oracle_attention(tqm, kbits, m, vbits, pt):
     """tq_attend (logits from the key codes, row softmax, values from their
     codes) against the oracle's softmax attention given the same codes; a
     sequence with an empty context gives a zero row.  The logit tolerance
     (1e-3 of ||q|| ||k|| / sqrt(d)) moves the softmax weights by at most about
     scale x that, so the output is checked to 2e-3 of its row scale."""
-    batch, heads, G, pt, d = 3, 2, 4, 32, 128
+    batch, heads, G, d = 3, 2, 4, 128
     ctx = [700, 129, 0]
     rng = np.random.default_rng(34 + kbits + vbits)
     keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-1, 1, size=(1, heads, 1, d)))
