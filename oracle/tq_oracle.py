@@ -383,6 +383,22 @@ def exact_logits(Qv: np.ndarray, K: np.ndarray) -> np.ndarray:
     return np.asarray(Qv, np.float64) @ np.asarray(K, np.float64).T
 
 
+def exact_top_k(scores: np.ndarray, k: int) -> np.ndarray:
+    """[rows, k] column indices of the k largest scores of each row, best
+    first; equal scores go to the lower index.  READING: the page names no
+    tie rule for nearest-neighbour search."""
+    scores = np.asarray(scores, dtype=np.float64)
+    cols = np.arange(scores.shape[1])
+    # lexsort sorts by the last key first: score descending, then index ascending
+    order = np.array([np.lexsort((cols, -row))[:k] for row in scores], dtype=np.int64)
+    return order.reshape(scores.shape[0], min(k, scores.shape[1]))
+
+
+def recall_at_k(found: np.ndarray, exact: np.ndarray) -> float:
+    """Mean over rows of |found_row & exact_row| / k (TQ §Benchmarks, recall@k)."""
+    return float(np.mean([len(set(a.tolist()) & set(b.tolist())) / len(b) for a, b in zip(found, exact)]))
+
+
 # ---------------------------------------------------------------------------
 # Packed record layout, version 3 (the byte format the CUDA library reads and
 # writes; written here from its specification, independently of the library).

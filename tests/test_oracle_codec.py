@@ -350,3 +350,21 @@ def test_attention_empty_context_is_zero():
     o = O.attention_from_codes(kc, vc, np.ones((2, 16)), (e, np.zeros((0, 16), bool), np.zeros(0), np.zeros(0)),
                                (e, np.zeros(0)), 0.25)
     assert o.shape == (2, 16) and not o.any()
+
+
+def test_exact_top_k_against_brute_force_with_ties():
+    rng = np.random.default_rng(61)
+    S = rng.integers(0, 6, size=(20, 40)).astype(np.float64)   # many equal scores
+    for k in (1, 3, 10, 40):
+        got = O.exact_top_k(S, k)
+        for row, g in zip(S, got):
+            brute = [j for _, j in sorted((-row[j], j) for j in range(len(row)))][:k]
+            assert list(g) == brute
+    assert O.exact_top_k(S, 100).shape == (20, 40)
+
+
+def test_recall_at_k():
+    exact = np.array([[1, 2, 3, 4], [5, 6, 7, 8]])
+    found = np.array([[4, 3, 9, 10], [5, 6, 7, 8]])
+    assert O.recall_at_k(found, exact) == 0.75
+    assert O.recall_at_k(exact, exact) == 1.0
