@@ -203,7 +203,8 @@ __device__ __forceinline__ uint4 decode8(const uint32_t* cw, int kk, const Value
 // per 16 tokens and 16 coordinates one ldmatrix.x4.trans and one
 // m16n8k16 MMA.  Column pair (2q, 2q + 1) of the accumulators is the hi / lo
 // part of query slot q.  Tokens past the context, on a bad page, or query
-// slots past G get weight 0 (the tile then holds finite table values).  The
+// slots past G get weight 0, and such tokens norm 0 (the tile then holds
+// finite table values, and nothing read from those slots reaches the sums).  The
 // warps' sums meet in shared memory; the CTA writes one partial.
 template <int BITS, int E>
 __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcParams p) {
@@ -332,7 +333,12 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
       const uint4 v = reinterpret_cast<const uint4*>(stg + lane * REC)[x];
       rec[4 * x] = v.x; rec[4 * x + 1] = v.y; rec[4 * x + 2] = v.z; rec[4 * x + 3] = v.w;
     }
-    const float nrm = __half2float(reinterpret_cast<const __half*>(stg + 32 * REC)[lane]);
+    // a slot past the context or on a bad page may hold any bytes (a NaN
+    // norm times a zero weight would still poison the sums): its norm is 0
+    const int pos = k0 + 32 * (warp + kValWarps * i) + lane;
+    bool tok_ok = pos < k1;
+    if (tok_ok && !fast) tok_ok = page_base[(pos >> ps) - first_page] >= 0;
+    const float nrm = tok_ok ? __half2float(reinterpret_cast<const __half*>(stg + 32 * REC)[lane]) : 0.0f;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll

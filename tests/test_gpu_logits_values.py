@@ -313,3 +313,36 @@ def test_values_mode_b_with_no_context_clears_out(tqm):
     tqm.dequant_values(cb, cache, ctx_t, 0, batch, weights=w, out=out)
     torch.cuda.synchronize()
     assert bool((out == 0).all())
+
+
+def test_values_mode_b_ignores_bytes_past_the_context(tqm):
+    """Slots past a sequence's context may hold any bytes (here 0xFF: NaN
+    norms): mode B must not let them reach the sums (zero weight times a
+    NaN norm would)."""
+    d, bits, pt, batch, heads, G, n = 128, 3, 64, 2, 2, 4, 700
+    ctx = [700, 129]
+    cb = tqm.Codebook(d, bits, 0, synth.SEED_PI, synth.SEED_S)
+    pps = (n + pt - 1) // pt
+    bt = synth.block_table(39, batch, pps)
+    cache = tqm.PagedCache.allocate(cb, batch * pps, pt, heads, torch.from_numpy(bt))
+    cache.pages.fill_(0xFF)
+    V = np.random.default_rng(40).standard_normal((batch, heads, n, d)).astype(np.float32)
+    tqm.quantize_append(cb, torch.from_numpy(V).cuda(), torch.zeros(batch, dtype=torch.int32, device="cuda"), cache)
+    W = synth.softmax_like_weights(41, batch, heads * G, n)
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
+    out = tqm.dequant_values(cb, cache, ctx_t, n, batch, weights=torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    B = out.cpu().numpy()
+    assert np.all(np.isfinite(B))
+    codec = O.make_codec(d, bits, 0, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, bits, 0, pt, heads)
+    pages = cache.pages.cpu().numpy()
+    for b in range(batch):
+        for h in range(heads):
+            idx, _, n16, _ = O.read_pages(lay, pages, bt, b, h, np.arange(ctx[b]))
+            Vh = O.dequantize(codec, idx, n16)
+            Wg = W[b, h * G:(h + 1) * G, : ctx[b]].astype(np.float64)
+            o = Wg @ Vh
+            scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
+            assert np.all(np.abs(B[b, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None])
+    assert cache.errors() == 0
