@@ -536,7 +536,13 @@ def run_ours(args):
     # warm-up: W eager steps (every replica is touched, kernels and attributes set up)
     for i in range(max(args.warmup, R)):
         step(i % R)
-    tq.attend(kcb, kc[0], vcb, vc[0], q, ctx_t, CTX, out=Aout, workspace=aws)
+    # tq_attend is timed beside the step; an error status from it (a launch
+    # the device refuses) is reported in the line instead of ending the run
+    attend_error = None
+    try:
+        tq.attend(kcb, kc[0], vcb, vc[0], q, ctx_t, CTX, out=Aout, workspace=aws)
+    except tq.TqError as e:
+        attend_error = str(e)
     torch.cuda.synchronize()
 
     # The timed work runs as CUDA graphs: launching from Python through ctypes
@@ -551,6 +557,8 @@ def run_ours(args):
         "values": lambda r: tq.dequant_values(vcb, vc[r], ctx_t, CTX, B, weights=W, out=Oout, workspace=vws),
         "attend": lambda r: tq.attend(kcb, kc[r], vcb, vc[r], q, ctx_t, CTX, out=Aout, workspace=aws),
     }
+    if attend_error is not None:
+        del parts["attend"]
     graphs = {}
     cap_stream = torch.cuda.Stream()
     for name, fn in parts.items():
@@ -586,7 +594,7 @@ def run_ours(args):
     app_ms = timed("append")
     log_ms = timed("logits")
     val_ms = timed("values")
-    att_ms = timed("attend")
+    att_ms = timed("attend") if "attend" in graphs else None
     # spread of the headline call: per-call time over further replays of its graph
     log_spread = _percentiles([timed("logits") / args.steps for _ in range(args.spread_replays)])
     del graphs
@@ -651,7 +659,7 @@ def run_ours(args):
                    "logits_ms_per_step": log_ms / steps, "values_ms_per_step": val_ms / steps,
                    "append_ms_per_step": app_ms / steps,
                    "values_gbs": n * VALUE_BYTES * steps / (val_ms * 1e-3) / 1e9,
-                   "attend_ms_per_step": att_ms / steps,
+                   "attend_ms_per_step": att_ms / steps if att_ms is not None else None,
                    "logits_ms_per_step_spread": dict(log_spread, replays_of_steps=steps)},
         "roofline": {"bound": "hbm", "achieved": logits_gbs / n, "peak": hbm_peak, "unit": "GB/s",
                      "frac": logits_gbs / n / hbm_peak, "traffic": LOGITS_DRAM_BYTES,
@@ -665,6 +673,8 @@ def run_ours(args):
         "gpu_launches": 6 * steps,
         "clocks": clk,
     }
+    if attend_error is not None:
+        line["config"]["attend_error"] = attend_error
     if kq is not None:
         line["keys_quantized"] = kq
     if lc is not None:
