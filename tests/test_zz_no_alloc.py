@@ -5,8 +5,8 @@ serving loop whose memory is an arena carved up at start-up, a framework or
 plugin interface that gives an operator no workspace, or a hot path that must
 not call cudaMalloc/cudaFree because they can block or synchronize the
 device.  tq_logits_noalloc serves them from a static 1 MiB device array.  This
-file is collected last on purpose; it passes alone in a fresh process and
-after the other tests.
+file is collected after the kernels' parity tests on purpose; it passes alone
+in a fresh process and after the other tests.
 """
 
 import ctypes
