@@ -49,13 +49,12 @@ LOGIT_BYTES = B * HKV * CTX * KEY_REC + B * HQ * CTX * 4 + B * HQ * D * 2
 VALUE_BYTES = B * HKV * CTX * VAL_REC + B * HQ * CTX * 4 + B * HQ * D * 4
 APPEND_BYTES = 2 * B * HKV * D * 2 + B * HKV * (KEY_REC + VAL_REC)
 APPEND_CFG = dict(batch=16, heads=8, n_new=4096)
-# DRAM bytes (read + write) of one tq_logits call of this workload, from one
-# ncu capture of the current kernels (dram__bytes_read.sum /
-# dram__bytes_write.sum, one launch each, python bench.py --profile-phase decode):
-# logits_kernel<3,32,32> 17,882,624 + 0 and prep_queries_kernel 156,928 + 0.
-LOGITS_DRAM_BYTES = 17882624 + 156928
-LOGITS_DRAM_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum, logits_kernel<3,32,32> + "
-                      "prep_queries_kernel, one launch each")
+# DRAM bytes (read + write) of one tq_logits call of this workload from an ncu
+# capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum,
+# python bench.py --profile-phase decode); None until the kernel as built has
+# been captured.
+LOGITS_DRAM_BYTES = None
+LOGITS_DRAM_SOURCE = None
 WORKLOAD = "decode step: batch 1, 8 KV / 32 query heads, head_dim 128, context 32768, keys b=3 + QJL m=128, values b=3"
 
 

@@ -142,6 +142,18 @@ void tq_codebook_free(tq_codebook* cb);
 tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s,
                              double* centroids, double* boundaries);
 
+/* Copies the reconstruction levels the library decodes with (host, 2^bits
+ * doubles, ascending) into `levels`, and their scale exponent into
+ * *scale_exp (may be NULL).  TQ §Stage 1 gives the Lloyd-Max centroids; how
+ * they are stored is this library's choice: for bits <= 3 every level is an
+ * 8-bit integer k times 2^-f (k = round(c 2^f), half to even, f the largest
+ * integer with max|c| 2^f <= 127; *scale_exp = f), so that a decoded
+ * coordinate is one signed byte; for bits = 4 the levels are the fp16
+ * roundings of the centroids (*scale_exp = INT32_MIN).  The residual of the
+ * QJL stage, the logits and the value path all use these levels.  Works on
+ * host-only codebooks too. */
+tq_status tq_codebook_levels(const tq_codebook* cb, double* levels, int32_t* scale_exp);
+
 /* Fills *info with the packed-format sizes for this codebook. */
 tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_heads,
                     tq_layout_info* info);
@@ -151,7 +163,7 @@ tq_status tq_layout(const tq_codebook* cb, int32_t page_tokens, int32_t n_kv_hea
  * d] of dtype.  start_pos: device int32 [batch], position of x[b, :, 0].
  * For every vector: ||x|| (fp32, stored fp16), y = Pi x / ||x||, indices
  * by threshold search over the Lloyd-Max boundaries, and when m > 0 the
- * residual r = y - c16[idx] (rotated space), ||r|| (fp16) and the m signs of
+ * residual r = y - c[idx] (rotated space; c = the reconstruction levels, see tq_codebook_levels), ||r|| (fp16) and the m signs of
  * S r; the packed record is written into its page slot.  Each token owns its
  * bytes, so appends that start inside a page are safe; calls on one stream
  * are ordered.  Returns TQ_EINVAL for bad shapes, dtype or pointers. */
@@ -167,7 +179,7 @@ size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n
 /* Fused logits from the packed keys (TQ §Stage 2 and §How it works): for
  * query head hq of sequence b (KV head hq / (n_q_heads / n_kv_heads)) and
  * every key position t < ctx_len[b],
- *   out[(b * n_q_heads + hq) * out_stride + t] = ||k|| ( <Pi q, c16[idx]>
+ *   out[(b * n_q_heads + hq) * out_stride + t] = ||k|| ( <Pi q, c[idx]>
  *        + sqrt(pi/2)/m ||r|| <S q, sign> )   (sign_i = -1 where the bit is 1)
  * with the query rotated once.  No 1/sqrt(d) scale, no softmax.  Positions
  * t >= ctx_len[b] are not written.  q: device [batch, n_q_heads, d] of dtype.
@@ -212,7 +224,7 @@ size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n
                                  int32_t n_q_heads, int64_t max_ctx);
 
 /* Value path from packed records (MSE reconstruction v_hat = ||v|| Pi^T
- * c16[idx]).  Mode A (weights == NULL): out device [batch, n_kv_heads,
+ * c[idx], c the reconstruction levels).  Mode A (weights == NULL): out device [batch, n_kv_heads,
  * out_stride, d] of out_dtype receives v_hat for t < ctx_len[b].  Mode B
  * (weights != NULL, device fp32 [batch, n_q_heads, w_stride]): out device
  * fp32 [batch, n_q_heads, d] receives sum_{t < ctx_len[b]} weights[b,hq,t]
@@ -235,7 +247,7 @@ size_t tq_attend_workspace_bytes(const tq_codebook* key_cb, const tq_codebook* v
  * compressed keys, values from their codes): for query head hq of sequence b
  * (KV head hq / (n_q_heads / n_kv_heads)),
  *   out[b, hq, :] = sum_{t < ctx_len[b]} softmax_t(scale * L[b, hq, t]) v_hat_t
- * with L the tq_logits estimate and v_hat_t = ||v_t|| Pi_v^T c16[idx_t] (the
+ * with L the tq_logits estimate and v_hat_t = ||v_t|| Pi_v^T c[idx_t] (the
  * value codebook's reconstruction); a row with ctx_len[b] = 0 is all zeros
  * (with max_ctx = 0 the whole of out is cleared and nothing else runs).
  * key_cb / key_cache and value_cb / value_cache as for tq_logits and

@@ -95,37 +95,29 @@ static void build_host_tables(tq_codebook* cb, const tq_params* p) {
   const int K = 1 << p->bits, H = K / 2;
   for (int i = 0; i < 16; ++i) cb->cent16[i] = 0;
   for (int i = 0; i < 8; ++i) cb->mag16[i] = 0;
-  for (int i = 0; i < K; ++i) cb->cent16[i] = f64_to_f16_bits(cb->centroids[i]);
-  for (int mu = 0; mu < H; ++mu) cb->mag16[mu] = cb->cent16[H + mu];
   cb->table_exp = 0;
-  cb->int8_hi[0] = cb->int8_hi[1] = cb->int8_lo[0] = cb->int8_lo[1] = 0u;
-}
-
-// b <= 3: the smallest f for which every c16 level times 2^f is an integer
-// (the finest fp16 spacing among the levels), and the int8 slices of those
-// integers.  Fails when an integer would not fit 16 bits.
-static bool make_int8_tables(tq_codebook* cb) {
-  const int K = 1 << cb->lay.bits;
-  int f = -30;
-  for (int i = 0; i < K; ++i) {
-    const float c = f16_bits_to_float(cb->cent16[i]);
-    if (c == 0.0f) continue;
-    int e;
-    std::frexp(std::fabs((double)c), &e);            // |c| in [2^(e-1), 2^e)
-    const int spacing_exp = std::max(e - 1, -14) - 10;  // fp16 spacing at |c|
-    f = std::max(f, -spacing_exp);
+  cb->int8_levels[0] = cb->int8_levels[1] = 0u;
+  cb->levels.assign(K, 0.0);
+  // Reconstruction levels (TQ §Stage 1 gives the centroids, not how they are
+  // stored): up to 8 levels in 8-bit fixed point on one power-of-two scale,
+  // level i = k_i 2^-f with k_i = round(c_i 2^f) (half to even) and f the
+  // largest integer with max |c| 2^f <= 127, so that a decoded coordinate is
+  // one signed byte; 16 levels in fp16.
+  if (K <= 8) {
+    double cmax = 0.0;
+    for (int i = 0; i < K; ++i) cmax = std::max(cmax, std::fabs(cb->centroids[i]));
+    const int f = (int)std::floor(std::log2(127.0 / cmax));
+    for (int i = 0; i < K; ++i) {
+      const double k = std::nearbyint(std::ldexp(cb->centroids[i], f));
+      cb->levels[i] = std::ldexp(k, -f);
+      cb->int8_levels[i / 4] |= (uint32_t)(uint8_t)(int8_t)k << (8 * (i % 4));
+    }
+    cb->table_exp = f;
+  } else {
+    for (int i = 0; i < K; ++i) cb->levels[i] = f16_bits_to_float(f64_to_f16_bits(cb->centroids[i]));
   }
-  for (int i = 0; i < K; ++i) {
-    const double v = std::ldexp((double)f16_bits_to_float(cb->cent16[i]), f);
-    if (v != std::nearbyint(v) || std::fabs(v) > 32639.0) return false;
-    const int iv = (int)v;
-    const int hi = (iv + 128) >> 8;
-    const int lo = iv - 256 * hi;
-    cb->int8_hi[i / 4] |= (uint32_t)(uint8_t)(int8_t)hi << (8 * (i % 4));
-    cb->int8_lo[i / 4] |= (uint32_t)(uint8_t)(int8_t)lo << (8 * (i % 4));
-  }
-  cb->table_exp = f;
-  return true;
+  for (int i = 0; i < K; ++i) cb->cent16[i] = f64_to_f16_bits(cb->levels[i]);   // exact
+  for (int mu = 0; mu < H; ++mu) cb->mag16[mu] = cb->cent16[H + mu];
 }
 
 static tq_status upload(tq_codebook* cb) {
@@ -317,10 +309,6 @@ static tq_status build_common(const tq_params* params, tq_codebook** out, bool d
   cb->device = -1;
   cb->dev_block = nullptr;
   build_host_tables(cb, params);
-  if (params->bits <= 3 && !make_int8_tables(cb)) {
-    delete cb;
-    return fail(TQ_EUNSUPPORTED, "codebook levels do not fit the 16-bit integer tables");
-  }
   if (device) {
     cudaError_t e = cudaGetDevice(&cb->device);
     if (e != cudaSuccess) {
@@ -350,6 +338,13 @@ void tq_codebook_free(tq_codebook* cb) {
   if (!cb) return;
   if (cb->dev_block) cudaFree(cb->dev_block);
   delete cb;
+}
+
+tq_status tq_codebook_levels(const tq_codebook* cb, double* levels, int32_t* scale_exp) {
+  if (!cb || !levels) return fail(TQ_EINVAL, "tq_codebook_levels: codebook / levels is NULL");
+  std::memcpy(levels, cb->levels.data(), cb->levels.size() * sizeof(double));
+  if (scale_exp) *scale_exp = cb->lay.bits <= 3 ? cb->table_exp : INT32_MIN;
+  return TQ_OK;
 }
 
 tq_status tq_codebook_export(const tq_codebook* cb, double* pi, double* s, double* centroids,

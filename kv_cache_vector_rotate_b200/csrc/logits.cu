@@ -2,7 +2,7 @@
 //
 // "TurboQuant explained" (a2a-mcp.org), §Stage 2 and §How it works: the
 // query is rotated once (Pi q) and sketched once (S q); every logit is then
-//   L = ||k|| ( sum_j (Pi q)_j c16[idx_j] + sqrt(pi/2)/m ||r|| sum_i (S q)_i s_i )
+//   L = ||k|| ( sum_j (Pi q)_j c[idx_j] + sqrt(pi/2)/m ||r|| sum_i (S q)_i s_i )
 // evaluated from the indices and sign bits without dequantizing the key.
 //
 // Two kernels per call, chained by programmatic dependent launch:
@@ -13,20 +13,18 @@
 //    to the workspace.  Every part quantizes with a scale that needs no
 //    other part: |(Pi q)_j| <= ||q|| (Pi is orthogonal) and
 //    |(S q)_i| <= max_i ||S_i|| ||q||.
-//  * logits_kernel (below), which streams the cache while the queries are
-//    prepared.
+//  * logits_kernel, which pulls the cache into L2 while the queries are
+//    prepared and then streams it through shared memory.
 //
-// The logits kernel: every CTA owns an equal share of one sequence's keys;
-// its warps stream 32-key units into shared-memory rings with bulk copies
-// and run them through the tensor cores with the key operand built in
+// The key side: every CTA owns a contiguous share of 32-key units; its
+// warps run them through the tensor cores with the key operand built in
 // registers:
-//  - codebook term, b <= 3: m16n8k32 int8 MMAs.  c16 * 2^f is an integer of
-//    at most 16 bits for every level, so a key element is two int8 slices;
-//    eight stored codes form one byte-permute selector after a single mask,
-//    and two permutes of 8-byte tables give the high and low slices of four
-//    elements.  (Pi q) is quantized to 16-bit integers, also as two int8
-//    slices; the slice products are accumulated exactly in int32 and
-//    combined at the end.
+//  - codebook term, b <= 3: m16n8k32 int8 MMAs.  The reconstruction levels
+//    are k 2^-f with k an 8-bit integer, so a key element is one signed
+//    byte; eight stored codes form one byte-permute selector after a single
+//    mask, and one permute of the 8-byte level table gives four elements.
+//    (Pi q) is quantized to 16-bit integers as two int8 slices; the products
+//    are accumulated exactly in int32 and combined at the end.
 //  - codebook term, b = 4: m16n8k16 fp16 MMAs on sign-magnitude codes (16
 //    levels do not fit one 8-byte permute table), the query as fp16 hi + lo.
 //  - sign term: m16n8k32 int8 MMAs.  The stored sign bits enter in place as
@@ -41,36 +39,21 @@ namespace tqd {
 
 constexpr int kSliceMax = 32639;   // |z| bound of Pi q: the high int8 slice stays in [-128, 127]
 constexpr int kSliceMaxQ = 16319;  // |z| bound of S q: 2 z still splits into int8 slices
-constexpr int kLogitsWarps = 4;    // warps per CTA
-constexpr int kCtaPages = 64;      // block-table entries staged per CTA
+constexpr int kPrepThreads = 128;  // threads of a preparation CTA
 constexpr int kPartRows = 32;      // rows of [Pi q ; S q] per preparation part
 
-// CTAs of the logits kernel resident per SM, and its registers per thread:
-// for d <= 128 few enough that a preparation CTA (128 threads x 64
-// registers) still fits beside them (a warp scheduler's share of the
-// register file is 16384: 5 x 88 x 32 + 64 x 32, or 4 x 104 x 32 + 64 x 32),
-// so that no logits CTA has to wait for a preparation CTA to finish
-__host__ __device__ constexpr int logits_min_blocks(int bits, int E) { return E >= 48 ? 4 : bits == 4 ? 4 : 5; }
-__host__ __device__ constexpr int logits_max_regs(int bits, int E) {
-  return E >= 48 ? 128 : logits_min_blocks(bits, E) == 5 ? 88 : 104;
-}
 
-// Per-warp shared-memory ring: a stage holds one 32-key unit, two 16-key
-// tiles of 16 consecutive records each (16 * 16W bytes, contiguous in its
-// page), then the two tiles' 16 norm slots (16 * NB <= 64 bytes each).
-template <int W>
-struct RingShape {
-  static constexpr int kTileCode = 256 * W;
-  static constexpr int kStageBytes = 2 * 256 * W + 128;
-  static constexpr int kStages = kStageBytes <= 2304 ? 4 : 2;   // a power of two
+// Byte-permute tables of the reconstruction levels (kernel parameters).
+struct KeyTables {
+  uint32_t t0, t1;              // b <= 3: the int8 levels k_i (level i = k_i 2^-f), levels 0..7
+  uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
 };
 
 struct PrepParams {
   const void* q;             // [batch][n_q_heads][d]
   tq_dtype dtype;
-  int d, E, F;               // d_pad = 4E, m_pad = 4F
+  int d;
   int n_q_heads, n_kv_heads, G, qtiles;
-  int cb_int8;               // codebook fragments as int8 slices (b <= 3) or fp16 hi / lo (b = 4)
   float cb_unscale;          // 2^-f
   float qjl_scale;           // sqrt(pi/2) / m
   float s_rowmax;            // >= max_i ||S_i||
@@ -80,23 +63,6 @@ struct PrepParams {
   float2* scal;
 };
 
-struct LogitsParams {
-  tq::CacheView cv;
-  int page_shift;            // log2(page_tokens)
-  const int32_t* ctx_len;
-  int n_kv_heads, n_q_heads, G, qtiles;
-  int n_chunks;              // CTAs per (group, query tile) along the keys
-  int units;                 // 32-key units of max_ctx
-  int max_ctx;               // ctx_len values are clamped to [0, max_ctx]
-  const uint2* frag;         // workspace: query fragments and scales
-  const uint2* qfrag;
-  const float2* scal;
-  float* out;
-  int64_t out_stride;
-  uint32_t th0, th1, tl0, tl1;  // b <= 3: high / low int8 slices of c16 * 2^f, levels 0..7
-  uint32_t lo0, lo1, hi0, hi1;  // b = 4: low / high bytes of the 8 fp16 magnitudes
-  int pre_stages;            // ring stages filled before the query fragments are ready (1 .. 4)
-};
 
 // ---- loads of the workspace written by the preparation kernel (L2) ------------
 
@@ -108,6 +74,15 @@ __device__ __forceinline__ uint2 ld_cg(const uint2* p) {
 __device__ __forceinline__ float2 ld_cg(const float2* p) {
   float2 v;
   asm volatile("ld.global.cg.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "l"(p));
+  return v;
+}
+
+// A read-only 16-byte load that the compiler keeps in program order with the
+// other volatile instructions (the table loads must be issued before the
+// dependent-launch wait, not sunk to their use).
+__device__ __forceinline__ uint4 ldg_early(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
   return v;
 }
 
@@ -164,7 +139,7 @@ __device__ __forceinline__ uint32_t code_selector(const uint32_t* w, int kk) {
 // b = 4: the two fp16 pairs (elements 4ks, 4ks+1 and 4ks+2, 4ks+3) of k-step
 // ks from the sign-magnitude nibbles (magnitude bytes by permute, sign ORed
 // into bit 15 of each half).
-__device__ __forceinline__ void decode_nibble_pair(const uint32_t* w, int ks, const LogitsParams& p,
+__device__ __forceinline__ void decode_nibble_pair(const uint32_t* w, int ks, const KeyTables& p,
                                                    uint32_t& h0, uint32_t& h1) {
   const uint32_t x = w[ks / 2] >> (8 * (ks % 2));
   const uint32_t sel = (x & 0x77u) | ((x >> 8) & 0x7700u);
@@ -207,17 +182,206 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(x));
 }
 
+// ---- one 16-key tile --------------------------------------------------------------
+
+// Words of a record chunk and MMA k-steps for (b, E, F).
+template <int BITS, int E, int F>
+struct TileShape {
+  static constexpr bool kInt8 = BITS <= 3;
+  static constexpr int KC = kInt8 ? E / 8 : E / 4;   // codebook MMA k-steps
+  static constexpr int KQ = F / 8;                   // sign-term MMA k-steps
+  static constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
+                          : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
+  static constexpr int QW = (F + 31) / 32;           // QJL words per chunk
+  static constexpr int W = q0 + QW;
+  static constexpr int NB = F > 0 ? 4 : 2;           // bytes of a norm slot
+};
+
+// The query side of a tile: fragments and scales of one query tile (4
+// query slots x high / low slices in the N = 8 columns).
+template <int KC, int KQ>
+struct QueryFrags {
+  uint2 bq[KC];
+  uint2 bz[KQ > 0 ? KQ : 1];
+  float c0, c1, zsum;
+};
+
+// sum_i z_i of query t from its own sign-term fragments: weights 1 on the 2 z
+// slots and 2 on the z slots give 2 sum z in columns (2t, 2t+1).
+template <int KQ>
+__device__ __forceinline__ float query_zsum(const uint2 (&bz)[KQ > 0 ? KQ : 1]) {
+  if constexpr (KQ == 0) {
+    return 0.0f;
+  } else {
+    int zs[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int kk = 0; kk < KQ; ++kk) mma_s8s8(zs, 0x01010101u, 0x01010101u, 0x02020202u, 0x02020202u, bz[kk]);
+    return 0.5f * (float)(256 * zs[0] + zs[1]);
+  }
+}
+
+// Logits of rows g (la) and g + 8 (lb) of one 16-key tile for this thread's
+// query t.  wa / wb: the W words of chunk t of the two keys; na / nb: their
+// norm slots (fp16 ||k||, then fp16 ||r|| when F > 0).
+// Sign term: k-step kk of a QJL word uses bit planes 2 kk and 2 kk + 1 in
+// place (one mask per operand register), weighted 2^(2 kk + 1) after the
+// query side's 2 z / z slots; a Horner step (x 4) between k-steps brings
+// every k-step of a word to weight 2^(2 n - 1) (n k-steps in the word), and
+// words are scaled to the common weight 128.
+template <int BITS, int E, int F>
+__device__ __forceinline__ void tile_logits(const uint32_t* wa, const uint32_t* wb, uint32_t na, uint32_t nb,
+                                            const QueryFrags<TileShape<BITS, E, F>::KC, TileShape<BITS, E, F>::KQ>& qf,
+                                            const KeyTables& kt, float& la, float& lb) {
+  using TS = TileShape<BITS, E, F>;
+  constexpr int KC = TS::KC, q0 = TS::q0, QW = TS::QW;
+  float cba, cbb;
+  if constexpr (TS::kInt8) {
+    // codebook term: the int8 levels k against the int8 slices of (Pi q)
+    int ah[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int kk = 0; kk < KC; ++kk) {
+      const uint32_t sa = code_selector<BITS, E>(wa, kk);
+      const uint32_t sb = code_selector<BITS, E>(wb, kk);
+      const uint32_t sa2 = sa >> 16, sb2 = sb >> 16;
+      mma_s8s8(ah, prmt(kt.t0, kt.t1, sa), prmt(kt.t0, kt.t1, sb), prmt(kt.t0, kt.t1, sa2),
+               prmt(kt.t0, kt.t1, sb2), qf.bq[kk]);
+    }
+    // columns 2t / 2t+1: high / low slice of query t; 256 hi + lo stays below
+    // 2^31 (|k| <= 127, |z| <= 32639, d <= 256)
+    cba = (float)(256 * ah[0] + ah[1]);
+    cbb = (float)(256 * ah[2] + ah[3]);
+  } else {
+    float acc0[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int ks = 0; ks < KC; ++ks) {
+      uint32_t a0, a2, a1, a3;
+      decode_nibble_pair(wa, ks, kt, a0, a2);
+      decode_nibble_pair(wb, ks, kt, a1, a3);
+      mma_f16(acc0, a0, a1, a2, a3, qf.bq[ks]);
+    }
+    // columns 2t (hi) and 2t+1 (lo) belong to query t of this tile
+    cba = acc0[0] + acc0[1];
+    cbb = acc0[2] + acc0[3];
+  }
+  if constexpr (F > 0) {
+    // sign term: in-place bit planes against the int8 slices of 2 z / z
+    int qa[4] = {0, 0, 0, 0};                 // 128 sum beta z (hi, lo columns)
+#pragma unroll
+    for (int w = 0; w < QW; ++w) {
+      const int nk = min(4, (F - 32 * w) / 8);   // k-steps of this word (4, or 2 for a half word)
+      int a4[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        if (k < nk) {
+          if (k > 0) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a4[r] *= 4;
+          }
+          const uint32_t m0 = 0x01010101u << (2 * k), m1 = m0 << 1;
+          mma_u8s8(a4, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, qf.bz[4 * w + k]);
+        }
+      }
+      const int sh = 6 - 2 * (nk - 1);           // weight 2^(2 nk - 1) -> 128
+#pragma unroll
+      for (int r = 0; r < 4; ++r) qa[r] += a4[r] << sh;
+    }
+    // sum_i s_i z_i = sum z - 2 sum beta z
+    const float ta = fmaf(-1.0f / 64.0f, (float)(256 * qa[0] + qa[1]), qf.zsum);
+    const float tb = fmaf(-1.0f / 64.0f, (float)(256 * qa[2] + qa[3]), qf.zsum);
+    const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&na));   // ||k||, ||r||
+    const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&nb));
+    la = fa.x * fmaf(qf.c1 * fa.y, ta, qf.c0 * cba);
+    lb = fb.x * fmaf(qf.c1 * fb.y, tb, qf.c0 * cbb);
+  } else {
+    la = lo_half(na) * (qf.c0 * cba);
+    lb = lo_half(nb) * (qf.c0 * cbb);
+  }
+}
+
+// The two norm slots of the rows g, g + 8 of each 16-key tile of a staged unit.
+template <int NB>
+__device__ __forceinline__ void unit_norms(const uint8_t* nsl, int g, uint32_t& na0, uint32_t& nb0, uint32_t& na1,
+                                           uint32_t& nb1) {
+  if constexpr (NB == 4) {
+    const uint32_t* n = reinterpret_cast<const uint32_t*>(nsl);
+    na0 = n[g]; nb0 = n[g + 8]; na1 = n[16 + g]; nb1 = n[24 + g];
+  } else {
+    na0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * g);
+    nb0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * (g + 8));
+    na1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * g);
+    nb1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * (g + 8));
+  }
+}
+
 // ---- query preparation -----------------------------------------------------------
 //
-// Workspace: codebook fragments uint2 [gq][KC][32] (gq = group x query tile;
-// KC = E/8 int8 k-steps, or E/4 fp16 k-steps for b = 4), QJL fragments uint2
-// [gq][F/8][32], per-query scales float2 [batch * n_q_heads] = {c0, c1}.
-// Lane (2 q + s) * 4 + t of a fragment holds slice s (0 high, 1 low) of
-// query slot q for chunk t; byte e % 8 (half e % 4 for fp16) of it is row e
-// of the k-step.  In the QJL part rows 8 kk .. 8 kk + 3 of a k-step hold the
-// slices of 2 z, rows 8 kk + 4 .. 8 kk + 7 those of z (|z| <= kSliceMaxQ),
-// matching the key operand of the logits kernel (sign bytes 2^(2 kk) beta
-// and 2^(2 kk + 1) beta).
+// Fragment bytes: codebook fragments uint2 [KC][32] per query tile (KC = E/8
+// int8 k-steps, or E/4 fp16 k-steps for b = 4), QJL fragments uint2
+// [F/8][32], per-query scales float2 {c0, c1}.  Lane (2 q + s) * 4 + t of a
+// fragment holds slice s (0 high, 1 low) of query slot q for chunk t; byte
+// e % 8 (half e % 4 for fp16) of it is row e of the k-step.  In the QJL part
+// rows 8 kk .. 8 kk + 3 of a k-step hold the slices of 2 z, rows 8 kk + 4 ..
+// 8 kk + 7 those of z (|z| <= kSliceMaxQ), matching the key operand of the
+// tile (sign bytes 2^(2 kk) beta and 2^(2 kk + 1) beta).
+
+// What the quantization of a prepared row needs of the codebook.
+struct PrepConsts {
+  float cb_unscale;          // 2^-f
+  float qjl_scale;           // sqrt(pi/2) / m
+  float s_rowmax;            // >= max_i ||S_i||
+};
+
+// Quantizes v = row `row` of [Pi q ; S q] for query slot `qs` (norm qn) into
+// its fragment bytes: codebook fragments `fr` ([KC][32] uint2 of this query
+// tile; int8 slices for b <= 3, fp16 hi / lo for b = 4), sign-term
+// fragments `fz` ([F/8][32]).  Global or shared memory.
+template <int E, int F, bool INT8>
+__device__ __forceinline__ void put_prepared(float v, int row, int qs, float qn, const PrepConsts& pc, uint2* fr,
+                                             uint2* fz) {
+  const bool sk = row >= 4 * E;                 // an S q row
+  const int l = sk ? row - 4 * E : row;         // row within its half
+  int tc, e;                                    // chunk, row within the chunk
+  if (sk) {
+    tc = l / (F > 0 ? F : 1);
+    e = l - tc * F;
+  } else {
+    tc = l / E;
+    e = l - tc * E;
+  }
+  if (!sk && !INT8) {
+    int e2 = 0;                                 // ||q|| in [2^(e2-1), 2^e2)
+    if (qn > 0.0f) frexpf(qn, &e2);
+    const float vs = v * ldexpf(1.0f, 14 - e2);
+    const __half hi = __float2half_rn(vs);
+    const __half lo = __float2half_rn(vs - __half2float(hi));
+    __half* h = reinterpret_cast<__half*>(fr + (e / 4) * 32);
+    h[((2 * qs) * 4 + tc) * 4 + (e & 3)] = hi;
+    h[((2 * qs + 1) * 4 + tc) * 4 + (e & 3)] = lo;
+    return;
+  }
+  const int zmax = sk ? kSliceMaxQ : kSliceMax;
+  const float bound = sk ? pc.s_rowmax * qn : qn;
+  const float scale = bound > 0.0f ? (float)zmax * __frcp_rn(bound) : 0.0f;
+  int z = max(-zmax, min(zmax, __float2int_rn(v * scale)));
+  if (sk && (e & 7) < 4) z *= 2;                // rows 8 kk .. 8 kk + 3 of a QJL k-step: 2 z
+  const int zh = (z + 128) >> 8;                // floor((z + 128) / 256)
+  const int zl = z - 256 * zh;                  // in [-128, 127]
+  int8_t* b8 = reinterpret_cast<int8_t*>((sk ? fz : fr) + (e / 8) * 32);
+  b8[((2 * qs) * 4 + tc) * 8 + (e & 7)] = (int8_t)zh;
+  b8[((2 * qs + 1) * 4 + tc) * 8 + (e & 7)] = (int8_t)zl;
+}
+
+// Per-query scales {c0, c1} of a query with norm qn: c0 undoes the codebook
+// fragments' scale (and 2^f of the int8 tables), c1 = sqrt(pi/2)/m times the
+// sketch fragments' scale.
+template <bool INT8>
+__device__ __forceinline__ float2 prep_scales(float qn, const PrepConsts& pc) {
+  int e = 0;
+  if (!INT8 && qn > 0.0f) frexpf(qn, &e);
+  const float c0 = INT8 ? qn * (1.0f / (float)kSliceMax) * pc.cb_unscale : ldexpf(1.0f, e - 14);
+  const float c1 = pc.qjl_scale * (pc.s_rowmax * qn) * (1.0f / (float)kSliceMaxQ);
+  return make_float2(c0, c1);
+}
 
 // Shared memory of one preparation part.
 struct PrepSmem {
@@ -233,6 +397,7 @@ struct PrepSmem {
 // fragment bytes.  Every fragment byte of the part is written (zeros for
 // padding rows and slots past G).  Part 0 also writes the slots' scales.
 // All 128 threads of the CTA call it.
+template <int E, int F, bool INT8>
 __device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, PrepSmem& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -241,6 +406,10 @@ __device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, Pr
   const int64_t qbase = (int64_t)b * p.n_q_heads + kv * p.G + qt * 4;   // first query row of the tile
   const int nq = min(4, p.G - qt * 4);
   const int d = p.d, d16 = (d + 15) >> 4;
+  PrepConsts pc;
+  pc.cb_unscale = p.cb_unscale;
+  pc.qjl_scale = p.qjl_scale;
+  pc.s_rowmax = p.s_rowmax;
 
   const int mt = warp & 1, ksp = warp >> 1;
   const int kb = ksp * d16 / 2, ke = (ksp + 1) * d16 / 2;     // this warp's k-steps
@@ -260,22 +429,9 @@ __device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, Pr
 #pragma unroll
     for (int i = 0; i < 8; ++i) x[i] = 0.0f;
     if (valid) {
-      if (p.dtype == TQ_BF16) {
-        const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(p.q) + qoff;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (lane + 32 * i < d) x[i] = __bfloat162float(qp[lane + 32 * i]);
-      } else if (p.dtype == TQ_F16) {
-        const __half* qp = reinterpret_cast<const __half*>(p.q) + qoff;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (lane + 32 * i < d) x[i] = __half2float(qp[lane + 32 * i]);
-      } else {
-        const float* qp = reinterpret_cast<const float*>(p.q) + qoff;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (lane + 32 * i < d) x[i] = qp[lane + 32 * i];
-      }
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < d) x[i] = load_elem(p.q, qoff + lane + 32 * i, p.dtype);
     }
     float s2 = 0.0f;
 #pragma unroll
@@ -319,341 +475,505 @@ __device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, Pr
   if (ksp == 1) sm.ksum[mt][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   __syncthreads();
   const float qn = sqrtf(sm.qn2[t]);
-  const bool sk = r * kPartRows >= 4 * p.E;   // the part holds S q rows
   if (warp < 2) {
     const float4 o = sm.ksum[mt][lane];
     const float va = acc[0] + acc[1] + o.x + o.y, vb = acc[2] + acc[3] + o.z + o.w;
-    const int Ep = sk ? p.F : p.E;
-    const int zmax = sk ? kSliceMaxQ : kSliceMax;
-    const float bound = sk ? p.s_rowmax * qn : qn;
-    const float scale = bound > 0.0f ? (float)zmax * __frcp_rn(bound) : 0.0f;
-    int e2 = 0;                       // b = 4: ||q|| in [2^(e2-1), 2^e2)
-    if (!p.cb_int8 && qn > 0.0f) frexpf(qn, &e2);
-    const float f16scale = p.cb_int8 ? 1.0f : ldexpf(1.0f, 14 - e2);
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int l = r * kPartRows - (sk ? 4 * p.E : 0) + 16 * mt + g + 8 * hh;   // row within its half
-      const float v = hh ? vb : va;
-      const int tc = l / Ep, e = l % Ep;        // chunk, row within the chunk
-      if (!sk && !p.cb_int8) {
-        const float vs = v * f16scale;
-        const __half hi = __float2half_rn(vs);
-        const __half lo = __float2half_rn(vs - __half2float(hi));
-        __half* fr = reinterpret_cast<__half*>(p.frag + ((int64_t)gq * (p.E / 4) + e / 4) * 32);
-        fr[((2 * t) * 4 + tc) * 4 + (e & 3)] = hi;
-        fr[((2 * t + 1) * 4 + tc) * 4 + (e & 3)] = lo;
-      } else {
-        int z = max(-zmax, min(zmax, __float2int_rn(v * scale)));
-        if (sk && (e & 7) < 4) z *= 2;          // rows 8 kk .. 8 kk + 3 of a QJL k-step: 2 z
-        const int zh = (z + 128) >> 8;          // floor((z + 128) / 256)
-        const int zl = z - 256 * zh;            // in [-128, 127]
-        int8_t* fr = reinterpret_cast<int8_t*>((sk ? p.qfrag : p.frag) + ((int64_t)gq * (Ep / 8) + e / 8) * 32);
-        fr[((2 * t) * 4 + tc) * 8 + (e & 7)] = (int8_t)zh;
-        fr[((2 * t + 1) * 4 + tc) * 8 + (e & 7)] = (int8_t)zl;
-      }
-    }
+    constexpr int kcs = INT8 ? E / 8 : E / 4;
+    uint2* fr = p.frag + (int64_t)gq * kcs * 32;
+    uint2* fz = p.qfrag + (int64_t)gq * (F / 8) * 32;
+    put_prepared<E, F, INT8>(va, r * kPartRows + 16 * mt + g, t, qn, pc, fr, fz);
+    put_prepared<E, F, INT8>(vb, r * kPartRows + 16 * mt + g + 8, t, qn, pc, fr, fz);
   }
-  if (r == 0 && (int)threadIdx.x < nq) {
-    const float qq = sqrtf(sm.qn2[threadIdx.x]);
-    int e = 0;
-    if (qq > 0.0f) frexpf(qq, &e);
-    const float c0 = p.cb_int8 ? qq * (1.0f / (float)kSliceMax) * p.cb_unscale : ldexpf(1.0f, e - 14);
-    const float c1 = p.qjl_scale * (p.s_rowmax * qq) * (1.0f / (float)kSliceMaxQ);
-    p.scal[qbase + threadIdx.x] = make_float2(c0, c1);
-  }
+  if (r == 0 && (int)threadIdx.x < nq) p.scal[qbase + threadIdx.x] = prep_scales<INT8>(sqrtf(sm.qn2[threadIdx.x]), pc);
   __syncthreads();                  // the shared buffers may be reused
 }
 
 // Two-launch form: grid (parts, groups * qtiles), block 128; the logits
 // kernel follows by programmatic dependent launch.
-__global__ void __launch_bounds__(kLogitsWarps * 32) prep_queries_kernel(PrepParams p) {
+template <int E, int F, bool INT8>
+__global__ void __launch_bounds__(kPrepThreads) prep_queries_kernel(PrepParams p) {
   __shared__ PrepSmem sm;
   asm volatile("griddepcontrol.launch_dependents;");
-  prep_part(p, blockIdx.y, blockIdx.x, sm);
+  prep_part<E, F, INT8>(p, blockIdx.y, blockIdx.x, sm);
 }
 
-// ---- logits -----------------------------------------------------------------------
+// ---- logits ------------------------------------------------------------------------
 //
-// grid: (n_chunks, batch * n_kv_heads, query tiles of 4), block 128, dynamic
-// smem kLogitsWarps * S * stage bytes.  CTA x of a (group, query tile) owns
-// the 32-key units [x U / n_chunks, (x + 1) U / n_chunks) of the sequence
-// (U = ceil(max_ctx / 32)): every CTA gets the same work to within one unit.
-// Before it needs the query fragments a CTA stages its block-table entries
-// (page_tokens is a power of two: page and slot are a shift and a mask) and
-// every warp puts its first S units in flight: lane 0 issues bulk copies of
-// the unit's 32 records and 32 norm slots into ring stage i % S, completing
-// on that stage's mbarrier; then it waits for the preparation kernel
-// (griddepcontrol.wait).  Warp w
-// takes the CTA's units w, w + 4, ...  The two tiles of a unit are read
-// before either is computed, so their MMA chains interleave; a tile whose
-// page is bad or that lies past the context computes on stale bytes and
-// stores nothing.
-// Sign term: k-step kk of a QJL word uses bit planes 2 kk and 2 kk + 1 in
-// place (one mask per operand register), weighted 2^(2 kk + 1) after the
-// query side's 2 z / z slots; a Horner step (x 4) between k-steps brings
-// every k-step of a word to weight 2^(2 n - 1) (n k-steps in the word), and
-// words are scaled to the common weight 128.
-template <int BITS, int E, int F>
-__global__ void __maxnreg__(logits_max_regs(BITS, E)) logits_kernel(LogitsParams p) {
-  constexpr bool kInt8 = BITS <= 3;
-  constexpr int KC = kInt8 ? E / 8 : E / 4;   // codebook MMA k-steps
-  constexpr int KQ = F / 8;                   // sign-term MMA k-steps
-  constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
-                   : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
-  constexpr int QW = (F + 31) / 32;           // QJL words per chunk
-  constexpr int W = q0 + QW;
-  constexpr int NB = F > 0 ? 4 : 2;
-  using RS = RingShape<W>;
-  constexpr int S = RS::kStages;
-  constexpr int TILE = RS::kTileCode;
-  constexpr int STAGE = RS::kStageBytes;
-  extern __shared__ __align__(16) uint8_t ring_smem[];
-  __shared__ int64_t page_base[kCtaPages];    // byte offset of this head's block, -1 if bad
-  __shared__ uint64_t ring_bar[kLogitsWarps][4];   // one per ring stage (S <= 4)
+// grid: n_cta CTAs, at least one per line, usually one per SM; a CTA is NC
+// consumer warps (15; 8 for d > 128; 4 when every CTA gets few units) and
+// one producer warp (at most 16 warps: a fifth warp on one of the SM's four
+// schedulers would not get its registers).  The 64-key units of all lines
+// (sequence, KV head, query tile; U units each) are numbered line by line;
+// CTA c owns a contiguous share of them (at most U, so at most two lines)
+// and consumer warp w takes the share's units w, w + NC, ...  Warp w has a
+// ring of S copy slots, each holding one unit (64 records, then their 64
+// norm slots) with a "full" mbarrier (completed by the unit's bulk copies)
+// and an "empty" one (completed when warp w has read the slot).  The
+// producer's lanes put the units in flight in consumption order, in waves
+// of up to 32 units, refilling a slot once it is empty.  A bulk copy stalls the issuing thread while the memory system
+// is saturated, and one thread issues only a few per microsecond, so the
+// copies are spread over the producer's 32 lanes, kept few (one per unit
+// when a 64-token page's head block is the unit: its records and norms are
+// contiguous), and never issued by a consumer warp.
+//
+// Two ways to get the query fragments:
+//  * PREP (d <= 128, one launch per call): the CTA prepares its own queries.
+//    Before its programmatic-dependent-launch wait it only loads the
+//    codebook's [Pi ; S] fragments (constants) into registers -- consumer
+//    warp w holds 16-row tile w; a 16th tile goes to shared memory, for
+//    consumer 0.  After the wait it loads its lines' context lengths,
+//    block-table entries and queries; then the producer starts the stream
+//    while the consumers compute tile w of [Pi q ; S q] for the CTA's 8 query
+//    slots (4 per line) on the tensor cores and quantize it into fragment
+//    bytes in shared memory.
+//  * otherwise (two launches per call): prep_queries_kernel, an ordinary
+//    launch, writes the fragments to the workspace; every earlier kernel on
+//    the stream has finished when it starts, so this kernel may read the
+//    cache before its wait: the producer puts one unit per consumer warp in
+//    flight, the consumers wait and fetch their lines' fragments, and the
+//    producer goes on once they have them (fragment loads issued behind a
+//    full stream of copies would wait for it).
+// Every mbarrier wait is bounded; a CTA where one gives up reports
+// TQ_DEV_ERR_TIMEOUT and lets every copy it issued land before it exits.
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+constexpr int kLogitsPages = 512;    // block-table entries staged per CTA
+constexpr int kLogitsMaxSlots = 64;
+
+__host__ __device__ constexpr int logits_max_consumers(int E) { return E >= 48 ? 8 : 15; }
+// registers per thread: the two-launch form with d <= 128 stays at 112 so
+// that a preparation CTA (128 threads x 64 registers) fits beside its 16
+// warps
+__host__ __device__ constexpr int logits_regs(int E, bool prep) { return prep || E >= 48 ? 128 : 112; }
+
+// A copy slot: one 64-key unit, 64 records (16W bytes each) then 64 norm slots.
+template <int W, int NB>
+struct SlotShape {
+  static constexpr int kRecBytes = 16 * W;
+  static constexpr int kNormOff = 64 * 16 * W;
+  static constexpr int kBytes = (64 * (16 * W + NB) + 15) / 16 * 16;
+};
+
+struct LogitsParams {
+  tq::CacheView cv;
+  int page_shift;            // log2(page_tokens)
+  const int32_t* ctx_len;
+  int n_kv_heads, n_q_heads, G, qtiles;
+  int units;                 // U: 64-key units per line
+  int max_ctx;               // ctx_len values are clamped to [0, max_ctx]
+  int per_cta, extra;        // CTA c owns per_cta units, + 1 when c < extra (lines * U < 2^31)
+  FastDiv div_u, div_qtiles, div_kv;   // / U, / qtiles, / n_kv_heads
+  int nc;                    // consumer warps
+  FastDiv div_nc;
+  int ring_shift;            // S = 1 << ring_shift copy slots per consumer warp
+  int fixed_off;
+  int n_cta;
+  // PREP: queries and the preparation table
+  const void* q;
+  tq_dtype dtype;
+  int d, d16;
+  const uint4* table;        // [Pi ; S] bf16 hi + lo A fragments (tq_codebook::qprep_frag)
+  int prep_tiles;            // 16-row tiles of [Pi ; S]
+  PrepConsts pc;
+  // two launches: the preparation kernel's output
+  const uint2* frag;
+  const uint2* qfrag;
+  const float2* scal;
+  float* out;
+  int64_t out_stride;
+  KeyTables kt;
+};
+
+// The fixed part of a CTA's shared memory (after the slots).
+template <int KC, int KQ>
+struct LogitsFixed {
+  uint64_t full_bar[kLogitsMaxSlots];
+  uint64_t empty_bar[kLogitsMaxSlots];
+  int64_t page_base[kLogitsPages];         // byte offset of the head block, -1 if the page is bad
+  uint2 fr[2][KC * 32];                    // codebook fragments of the two lines
+  uint2 fz[2][(KQ > 0 ? KQ : 1) * 32];     // sign-term fragments
+  float2 scal[8];                          // {c0, c1} of query slot 4 line + q
+  float qn2[8];                            // PREP: ||q||^2 of the 8 query slots
+  uint64_t xtab_bar;                       // PREP: the extra table tile has landed
+  int flags;                               // bit 0: a wait gave up
+  int slot_last[kLogitsMaxSlots];          // last unit issued into each slot
+  uint16_t qs[2][8][128 + 8];              // PREP: bf16 hi / lo of the 8 query slots
+  uint4 xtab[8 * 2 * 32];                  // PREP: A fragments of table tile NC (a 16th tile)
+};
+
+template <int BITS, int E, int F>
+size_t logits_fixed_bytes() {
+  using TS = TileShape<BITS, E, F>;
+  return sizeof(LogitsFixed<TS::KC, TS::KQ>);
+}
+
+// One line (sequence b, KV head h, query tile qt) of a CTA's share: keys
+// [klo, khi) are the share's, keys [klo, k1) are read (k1 = min(khi,
+// context)); its block-table entries are [first, first + npg), staged from
+// entry ebase on.
+struct LineView {
+  int b, h, qt, klo, khi, k1, first, npg, ebase;
+};
+
+template <int BITS, int E, int F, bool PREP>
+__global__ void __maxnreg__(logits_regs(E, PREP)) logits_kernel(LogitsParams p) {
+  using TS = TileShape<BITS, E, F>;
+  constexpr int KC = TS::KC, KQ = TS::KQ, W = TS::W, NB = TS::NB;
+  using SS = SlotShape<W, NB>;
+  constexpr int REC = SS::kRecBytes, NOFF = SS::kNormOff, STAGE = SS::kBytes;
+  static_assert(!PREP || 4 * E <= 128, "the CTAs prepare at most 128 coordinates");
+  extern __shared__ __align__(128) uint8_t smem[];
+  auto& fx = *reinterpret_cast<LogitsFixed<KC, KQ>*>(smem + p.fixed_off);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int NT = blockDim.x;
+  const int NC = p.nc;                       // consumer warps; warp NC is the producer
+  const bool producer = warp == NC;
   const int g = lane >> 2, t = lane & 3;
-  const int gi = blockIdx.y;
-  const int b = gi / p.n_kv_heads, h = gi % p.n_kv_heads;
-  const int qt = blockIdx.z;
-  const int u0 = (int)((int64_t)blockIdx.x * p.units / p.n_chunks);
-  const int u1 = (int)((int64_t)(blockIdx.x + 1) * p.units / p.n_chunks);
-  const int k0 = 32 * u0;
-  const int kend = min(32 * u1, p.max_ctx);
-  const int ps = p.page_shift;
-  const int P = 1 << ps;
-  const int first_page = k0 >> ps;
-  const int n_pgx = k0 < kend ? ((kend - 1) >> ps) - first_page + 1 : 0;   // <= kCtaPages
-  const int ctx = min(p.ctx_len[b], p.max_ctx);
-  const int jt = threadIdx.x;
-  static_assert(kCtaPages <= kLogitsWarps * 32, "one block-table entry per thread");
-  const int64_t pg = jt < n_pgx ? p.cv.block_table[(int64_t)b * p.cv.max_pages + first_page + jt] : 0;
-  if (lane == 0) {
-#pragma unroll
-    for (int s = 0; s < S; ++s) mbar_init(&ring_bar[warp][s], 1);
+  const int c = blockIdx.x;
+  const int i0 = c * p.per_cta + min(c, p.extra);
+  const int n_units = p.per_cta + (c < p.extra ? 1 : 0);
+  const int U = p.units;
+  const int line0 = (int)fdiv((uint32_t)i0, p.div_u);
+  const int n_lines = n_units > 0 ? (int)fdiv((uint32_t)(i0 + n_units - 1), p.div_u) - line0 + 1 : 0;   // 0, 1 or 2
+  const int ua0 = i0 - line0 * U;                                          // first unit within line 0
+  const int split = n_lines > 1 ? (line0 + 1) * U - i0 : n_units;          // units of line 0
+  const int ps = p.page_shift, P = 1 << ps;
+  const int S = 1 << p.ring_shift;
+
+  if (tid < NC * S) {
+    mbar_init(&fx.full_bar[tid], 1);
+    mbar_init(&fx.empty_bar[tid], 1);
+    fx.slot_last[tid] = -1;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const int k1 = min(kend, ctx);     // keys [k0, k1) of this CTA (none when k1 <= k0)
-  const bool has_keys = k0 < k1;
-  bool bad = false;
-  if (jt < n_pgx) {
-    const bool valid = pg >= 0 && pg < p.cv.n_pages;
-    page_base[jt] = valid ? pg * p.cv.page_bytes + (int64_t)h * p.cv.head_block_bytes : -1;
-    // pages past the context are not used: an invalid entry there is no error
-    if (!valid && has_keys && jt <= ((k1 - 1) >> ps) - first_page) {
-      bad = true;
-      report(p.cv.err, TQ_DEV_ERR_PAGE);
+  if (tid == 0) fx.flags = 0;
+  // PREP: the preparation table is a constant of the codebook, loaded
+  // before the wait (consumer warp w: A fragments of 16-row tile w of [Pi ; S])
+  uint4 af[PREP ? 8 : 1][2];
+  if constexpr (PREP) {
+    if (producer && lane == 0 && p.prep_tiles > NC) {
+      // tile NC of the table into shared memory for consumer 0
+      mbar_init(&fx.xtab_bar, 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+      const uint32_t bytes = (uint32_t)p.d16 * 64 * 16;
+      mbar_arrive_tx(&fx.xtab_bar, bytes);
+      bulk_copy_plain(smem_addr(fx.xtab), p.table + (size_t)NC * p.d16 * 64, bytes, &fx.xtab_bar);
     }
+    if (warp < p.prep_tiles && warp < NC) {
+      // volatile loads: issued here, ahead of the wait, not where they are used
+      const uint4* tab = p.table + (size_t)warp * p.d16 * 64 + lane;
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (j < p.d16) {
+          af[j][0] = ldg_early(tab + (2 * j) * 32);
+          af[j][1] = ldg_early(tab + (2 * j + 1) * 32);
+        }
+    }
+    // everything below reads the caller's data, which the previous kernel on
+    // the stream may have written
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
   }
-  // fast path: every used page valid and 32-key units never straddle a page
-  const bool fast = !__syncthreads_or(bad) && P >= 32;   // also publishes the barriers' init
 
-  const int n_units = has_keys ? (k1 - k0 + 31) >> 5 : 0;
-  const int n_my = warp < n_units ? (n_units - warp + kLogitsWarps - 1) / kLogitsWarps : 0;
-  const uint8_t* ring = ring_smem + warp * S * STAGE;
-  const uint32_t ring_s = smem_addr(ring);
-  const int64_t norm_off = (int64_t)P * (16 * W);   // norm slots follow the P records
-  const uint64_t pol = evict_first_policy();   // the cache is streamed once per call
-
-  // lane 0 copies unit i of this warp (32 records + 32 norm slots) into stage
-  // i % S with bulk copies completing on that stage's barrier
-  auto issue = [&](int i) {
-    if (lane != 0) return;
-    uint64_t* bar = &ring_bar[warp][i & (S - 1)];
-    const uint32_t dst = ring_s + (i & (S - 1)) * STAGE;
-    const int ubase = k0 + 32 * (warp + kLogitsWarps * i);
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads of the stage first
-    if (fast) {
-      // one page holds the whole unit (records past the context are read and not used)
-      const int slot = ubase & (P - 1);
-      const uint8_t* hb = p.cv.pages + page_base[(ubase >> ps) - first_page];
-      mbar_arrive_tx(bar, 2 * TILE + 32 * NB);
-      bulk_copy(dst, hb + (int64_t)slot * (16 * W), 2 * TILE, bar, pol);
-      bulk_copy(dst + 2 * TILE, hb + norm_off + slot * NB, 32 * NB, bar, pol);
-      return;
-    }
-    uint32_t bytes = 0;
-    int64_t off[2] = {-1, -1};
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int base = ubase + 16 * hf;
-      if (base < k1) off[hf] = page_base[(base >> ps) - first_page];
-      if (off[hf] >= 0) bytes += TILE + 16 * NB;
-    }
-    mbar_arrive_tx(bar, bytes);        // 0 bytes: the phase completes on the arrival alone
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      if (off[hf] < 0) continue;
-      const int slot = (ubase + 16 * hf) & (P - 1);
-      const uint8_t* hb = p.cv.pages + off[hf];
-      bulk_copy(dst + hf * TILE, hb + (int64_t)slot * (16 * W), TILE, bar, pol);
-      bulk_copy(dst + 2 * TILE + 16 * NB * hf, hb + norm_off + slot * NB, 16 * NB, bar, pol);
-    }
+  auto make_line = [&](int s) {
+    LineView L;
+    const int ln = line0 + s;
+    const int gi = (int)fdiv((uint32_t)ln, p.div_qtiles);
+    L.qt = ln - gi * p.qtiles;
+    L.b = (int)fdiv((uint32_t)gi, p.div_kv);
+    L.h = gi - L.b * p.n_kv_heads;
+    const int ua = s == 0 ? ua0 : 0;
+    const int ub = s == 0 ? ua0 + split : n_units - split;
+    L.klo = 64 * ua;
+    L.khi = min(64 * ub, p.max_ctx);
+    L.first = L.klo >> ps;
+    L.npg = s < n_lines && L.klo < L.khi ? ((L.khi - 1) >> ps) - L.first + 1 : 0;   // L0.npg + L1.npg <= kLogitsPages
+    L.k1 = 0;
+    L.ebase = 0;
+    return L;
   };
-  // the first p.pre_stages units now, the rest of the ring once the query
-  // fragments are in registers (they would queue behind the copies at the SM)
-  int issued = 0;                    // units whose copies were issued
+  LineView L0 = make_line(0), L1 = make_line(1);
+  L1.ebase = L0.npg;
+  const int ctx0 = L0.npg > 0 ? p.ctx_len[L0.b] : 0;   // independent of the block-table loads
+  const int ctx1 = L1.npg > 0 ? p.ctx_len[L1.b] : 0;
+  int64_t pgv[4] = {0, 0, 0, 0};                      // kLogitsPages <= 4 * NT for NT >= 128
 #pragma unroll
-  for (int s = 0; s < S; ++s)
-    if (s < n_my && s < p.pre_stages) issue(issued++);
-
-  const int gq = gi * p.qtiles + qt;
-  // the query fragments and scales come from the preparation kernel
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  uint2 bq[KC];
-  const uint2* fsrc = p.frag + (int64_t)gq * KC * 32 + lane;
-#pragma unroll
-  for (int kk = 0; kk < KC; ++kk) bq[kk] = ld_cg(fsrc + kk * 32);
-  uint2 bz[KQ > 0 ? KQ : 1];
-  float zsumf = 0.0f;
-  if constexpr (KQ > 0) {
-    const uint2* qsrc = p.qfrag + (int64_t)gq * KQ * 32 + lane;
-#pragma unroll
-    for (int kk = 0; kk < KQ; ++kk) bz[kk] = ld_cg(qsrc + kk * 32);
-    // sum_i z_i of query t from its own fragments: weights 1 on the 2 z
-    // slots and 2 on the z slots give 2 sum z in columns (2t, 2t+1)
-    int zs[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int kk = 0; kk < KQ; ++kk) mma_s8s8(zs, 0x01010101u, 0x01010101u, 0x02020202u, 0x02020202u, bz[kk]);
-    zsumf = 0.5f * (float)(256 * zs[0] + zs[1]);
-  }
-  const int qidx = qt * 4 + t;                  // this thread's query within the group
-  const bool qvalid = qidx < p.G;
-  const int hq = h * p.G + (qvalid ? qidx : 0);
-  const float2 sc = ld_cg(p.scal + (int64_t)b * p.n_q_heads + hq);
-  const float c0 = sc.x;
-  const float c1 = F > 0 ? sc.y : 0.0f;
-  float* orow = p.out + ((int64_t)b * p.n_q_heads + hq) * p.out_stride;
-  // logits of rows g (la) and g + 8 (lb) of one tile, for query t
-  auto tile = [&](const uint32_t (&wa)[W], const uint32_t (&wb)[W], uint32_t na, uint32_t nb,
-                  float& la, float& lb) {
-    float cba, cbb;
-    if constexpr (kInt8) {
-      // codebook term: int8 slices of c16 * 2^f against those of (Pi q)
-      int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
-#pragma unroll
-      for (int kk = 0; kk < KC; ++kk) {
-        const uint32_t sa = code_selector<BITS, E>(wa, kk);
-        const uint32_t sb = code_selector<BITS, E>(wb, kk);
-        const uint32_t sa2 = sa >> 16, sb2 = sb >> 16;
-        mma_s8s8(ah, prmt(p.th0, p.th1, sa), prmt(p.th0, p.th1, sb), prmt(p.th0, p.th1, sa2),
-                 prmt(p.th0, p.th1, sb2), bq[kk]);
-        mma_s8s8(al, prmt(p.tl0, p.tl1, sa), prmt(p.tl0, p.tl1, sb), prmt(p.tl0, p.tl1, sa2),
-                 prmt(p.tl0, p.tl1, sb2), bq[kk]);
-      }
-      // columns 2t / 2t+1: high / low slice of query t.  256 hh + hl + lh
-      // stays below 2^31 (|hh| <= 2^22 for d <= 256).
-      cba = fmaf(256.0f, (float)(256 * ah[0] + ah[1] + al[0]), (float)al[1]);
-      cbb = fmaf(256.0f, (float)(256 * ah[2] + ah[3] + al[2]), (float)al[3]);
-    } else {
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int ks = 0; ks < KC; ++ks) {
-        uint32_t a0, a2, a1, a3;
-        decode_nibble_pair(wa, ks, p, a0, a2);
-        decode_nibble_pair(wb, ks, p, a1, a3);
-        mma_f16(acc0, a0, a1, a2, a3, bq[ks]);
-      }
-      // columns 2t (hi) and 2t+1 (lo) belong to query t of this tile
-      cba = acc0[0] + acc0[1];
-      cbb = acc0[2] + acc0[3];
+  for (int k = 0; k < 4; ++k) {
+    const int j = tid + k * NT;
+    if (j < L0.npg + L1.npg) {
+      const LineView& L = j < L0.npg ? L0 : L1;
+      pgv[k] = p.cv.block_table[(int64_t)L.b * p.cv.max_pages + L.first + j - L.ebase];
     }
-    if constexpr (F > 0) {
-      // sign term: in-place bit planes against the int8 slices of 2 z / z
-      int qa[4] = {0, 0, 0, 0};                 // 128 sum beta z (hi, lo columns)
+  }
+  // PREP, warps 0-7: query slot n = warp (line n / 4, query n % 4 of its
+  // tile) as bf16 hi + lo, and ||q||^2
+  if constexpr (PREP) {
+    if (warp < 8) {
+      const LineView& L = warp < 4 ? L0 : L1;
+      const int qi = L.qt * 4 + (warp & 3);
+      const bool valid = (warp >> 2) < n_lines && qi < p.G;
+      float x[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      if (valid) {
+        const int64_t qoff = ((int64_t)L.b * p.n_q_heads + (int64_t)L.h * p.G + qi) * p.d;
 #pragma unroll
-      for (int w = 0; w < QW; ++w) {
-        const int nk = min(4, (F - 32 * w) / 8);   // k-steps of this word (4, or 2 for a half word)
-        int a4[4] = {0, 0, 0, 0};
+        for (int i = 0; i < 4; ++i)
+          if (lane + 32 * i < p.d) x[i] = load_elem(p.q, qoff + lane + 32 * i, p.dtype);
+      }
+      float s2 = 0.0f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          if (k < nk) {
-            if (k > 0) {
+      for (int i = 0; i < 4; ++i) {
+        const int k = lane + 32 * i;
+        if (k < 16 * p.d16) {
+          const uint16_t hb = bf16_bits(x[i]);
+          fx.qs[0][warp][k] = hb;
+          fx.qs[1][warp][k] = bf16_bits(x[i] - __bfloat162float(__ushort_as_bfloat16(hb)));
+        }
+        s2 = fmaf(x[i], x[i], s2);
+      }
 #pragma unroll
-              for (int r = 0; r < 4; ++r) a4[r] *= 4;
+      for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      if (lane == 0) fx.qn2[warp] = s2;
+    }
+  }
+  L0.k1 = min(L0.khi, max(0, min(ctx0, p.max_ctx)));
+  L1.k1 = min(L1.khi, max(0, min(ctx1, p.max_ctx)));
+  bool bad = false;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int j = tid + k * NT;
+    if (j < L0.npg + L1.npg) {
+      const LineView& L = j < L0.npg ? L0 : L1;
+      const int pidx = L.first + j - L.ebase;
+      const bool valid = pgv[k] >= 0 && pgv[k] < p.cv.n_pages;
+      fx.page_base[j] = valid ? pgv[k] * p.cv.page_bytes + (int64_t)L.h * p.cv.head_block_bytes : -1;
+      // pages past the context are not read: an invalid entry there is no error
+      if (!valid && L.k1 > L.klo && pidx <= ((L.k1 - 1) >> ps)) {
+        bad = true;
+        report(p.cv.err, TQ_DEV_ERR_PAGE);
+      }
+    }
+  }
+  // fast path: every used page valid
+  const bool fast = !__syncthreads_or(bad);   // also publishes the barriers' init
+
+  if (producer) {
+    // ---------------------------------------------------------- producer
+    const int64_t norm_off = (int64_t)P * (16 * W);   // norm slots follow the P records
+    const uint64_t pol = evict_first_policy();        // the cache is streamed once per call
+    // the copies of unit i (consumer warp i % NC, its unit i / NC); false
+    // when the wait for the slot gave up
+    auto issue = [&](int i) -> bool {
+      const int j = (int)fdiv((uint32_t)i, p.div_nc), w = i - j * NC;
+      const int slot = w * S + (j & (S - 1));
+      if (j >= S && !mbar_wait_sleep(&fx.empty_bar[slot], (uint32_t)((j >> p.ring_shift) - 1) & 1u)) return false;
+      fx.slot_last[slot] = i;
+      uint64_t* bar = &fx.full_bar[slot];
+      const uint32_t dst = smem_addr(smem) + slot * STAGE;
+      const bool in1 = i >= split;
+      const int pos = 64 * (in1 ? i - split : ua0 + i);
+      const LineView& L = in1 ? L1 : L0;
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // the consumer's reads of the slot first
+      const int eb = L.ebase - L.first;
+      if (fast && P == 64 && pos < L.k1) {
+        // the unit is one page's head block: records and norms in one copy
+        // (records past the context are read and not used)
+        mbar_arrive_tx(bar, 64 * (16 * W + NB));
+        bulk_copy(dst, p.cv.pages + fx.page_base[eb + (pos >> ps)], 64 * (16 * W + NB), bar, pol);
+        return true;
+      }
+      // pieces of min(P, 64) keys (16 on a cache with a bad page) from
+      // their pages: records, then norms
+      const int piece = fast ? min(P, 64) : 16;
+      uint32_t bytes = 0;
+      for (int k = pos; k < pos + 64; k += piece)
+        if (k < L.k1 && fx.page_base[eb + (k >> ps)] >= 0) bytes += piece * (16 * W + NB);
+      mbar_arrive_tx(bar, bytes);          // 0 bytes: the phase completes on the arrival alone
+      for (int k = pos; k < pos + 64; k += piece) {
+        if (k >= L.k1) break;
+        const int64_t off = fx.page_base[eb + (k >> ps)];
+        if (off < 0) continue;
+        const int sl = k & (P - 1);
+        const uint8_t* hb = p.cv.pages + off;
+        bulk_copy(dst + (k - pos) * (16 * W), hb + (int64_t)sl * (16 * W), piece * (16 * W), bar, pol);
+        bulk_copy(dst + NOFF + (k - pos) * NB, hb + norm_off + sl * NB, piece * NB, bar, pol);
+      }
+      return true;
+    };
+    // Units go out in waves of `wave` consecutive units, lane k of a wave
+    // taking unit base + k; a wave holds no two units of one slot and the
+    // waves are ordered, so the uses of a slot are issued in order and a
+    // lane that waits for a slot's release is at most one phase ahead of it
+    // (a parity wait further ahead would return at once).
+    const int wave = min(32, NC * S);
+    bool ok = true;
+    int base = 0;
+    if constexpr (!PREP) {
+      // one unit per consumer warp before the fragments are fetched
+      if (lane < min(n_units, NC)) ok = issue(lane);
+      base = min(n_units, NC);
+      asm volatile("barrier.sync 1, %0;" ::"r"(NT) : "memory");   // the consumers have the fragments
+    }
+    for (; base < n_units; base += wave) {
+      if (lane < wave && base + lane < n_units && ok) ok = issue(base + lane);
+      if (!__all_sync(0xffffffffu, ok)) break;
+    }
+    if (!__all_sync(0xffffffffu, ok) && lane == 0) {
+      atomicOr(&fx.flags, 1);
+      report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------------- consumers
+    if constexpr (PREP) {
+      // tile w of [Pi q ; S q] for the 8 query slots, from the table
+      // fragments, while the first units arrive; consumer 0 also does tile NC
+      // (from the table tile in shared memory) when there are NC + 1 tiles
+      auto prep_tile = [&](int tile, bool from_smem) {
+        const bool two = p.dtype != TQ_BF16;          // bf16 queries are exact in one bf16 term
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (j < p.d16) {
+            const uint4 a0 = from_smem ? fx.xtab[(2 * j) * 32 + lane] : af[j][0];
+            const uint4 a1 = from_smem ? fx.xtab[(2 * j + 1) * 32 + lane] : af[j][1];
+            const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&fx.qs[0][g][16 * j + 2 * t]);
+            const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&fx.qs[0][g][16 * j + 2 * t + 8]);
+            mma_bf16(acc, a0, b0, b1);
+            mma_bf16(acc, a1, b0, b1);
+            if (two) {
+              const uint32_t c0 = *reinterpret_cast<const uint32_t*>(&fx.qs[1][g][16 * j + 2 * t]);
+              const uint32_t c1 = *reinterpret_cast<const uint32_t*>(&fx.qs[1][g][16 * j + 2 * t + 8]);
+              mma_bf16(acc, a0, c0, c1);
+              mma_bf16(acc, a1, c0, c1);
             }
-            const uint32_t m0 = 0x01010101u << (2 * k), m1 = m0 << 1;
-            mma_u8s8(a4, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, bz[4 * w + k]);
           }
         }
-        const int sh = 6 - 2 * (nk - 1);           // weight 2^(2 nk - 1) -> 128
+        // acc: rows g (0, 1) and g + 8 (2, 3) of the tile, query slots 2t (0, 2) and 2t + 1 (1, 3)
 #pragma unroll
-        for (int r = 0; r < 4; ++r) qa[r] += a4[r] << sh;
+        for (int x = 0; x < 4; ++x) {
+          const int n = 2 * t + (x & 1);
+          const int row = 16 * tile + g + 8 * (x >> 1);
+          put_prepared<E, F, TS::kInt8>(acc[x], row, n & 3, sqrtf(fx.qn2[n]), p.pc, fx.fr[n >> 2], fx.fz[n >> 2]);
+        }
+      };
+      if (warp < p.prep_tiles) prep_tile(warp, false);
+      if (warp == 0 && p.prep_tiles > NC) {
+        if (mbar_wait_sleep(&fx.xtab_bar, 0u)) {
+          prep_tile(NC, true);
+        } else if (lane == 0) {
+          atomicOr(&fx.flags, 1);
+          report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+        }
       }
-      // sum_i s_i z_i = sum z - 2 sum beta z
-      const float ta = fmaf(-1.0f / 64.0f, (float)(256 * qa[0] + qa[1]), zsumf);
-      const float tb = fmaf(-1.0f / 64.0f, (float)(256 * qa[2] + qa[3]), zsumf);
-      const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&na));   // ||k||, ||r||
-      const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&nb));
-      la = fa.x * fmaf(c1 * fa.y, ta, c0 * cba);
-      lb = fb.x * fmaf(c1 * fb.y, tb, c0 * cbb);
+      if (tid < 8) fx.scal[tid] = prep_scales<TS::kInt8>(sqrtf(fx.qn2[tid]), p.pc);
+      asm volatile("barrier.sync 2, %0;" ::"r"(NC * 32) : "memory");   // fragments ready (consumers only)
     } else {
-      la = lo_half(na) * (c0 * cba);
-      lb = lo_half(nb) * (c0 * cbb);
+      // the query fragments and scales come from the preparation kernel
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      constexpr int FL = (KC + KQ) * 32;         // fragment words (uint2) per line
+      for (int j = tid; j < n_lines * FL; j += NC * 32) {
+        const int s = j / FL, r = j % FL;
+        const int64_t gq = line0 + s;
+        if (r < KC * 32) fx.fr[s][r] = ld_cg(p.frag + gq * (KC * 32) + r);
+        else if constexpr (KQ > 0) fx.fz[s][r - KC * 32] = ld_cg(p.qfrag + gq * (KQ * 32) + (r - KC * 32));
+      }
+      if (tid < 4 * n_lines) {
+        const LineView& L = tid < 4 ? L0 : L1;
+        const int qi = L.qt * 4 + (tid & 3);
+        fx.scal[tid] = qi < p.G ? ld_cg(p.scal + (int64_t)L.b * p.n_q_heads + (int64_t)L.h * p.G + qi)
+                                : make_float2(0.0f, 0.0f);
+      }
+      asm volatile("barrier.sync 1, %0;" ::"r"(NT) : "memory");   // with the producer
     }
-  };
 
+    const int n_my = warp < n_units ? (int)fdiv((uint32_t)(n_units - warp - 1), p.div_nc) + 1 : 0;   // units of this warp
+    uint64_t* fbars = fx.full_bar + warp * S;
+    uint64_t* ebars = fx.empty_bar + warp * S;
+    const uint8_t* ring = smem + warp * S * STAGE;
+    int cur = -1;
+    QueryFrags<KC, KQ> qf;
+    bool qvalid = false;
+    float* orow = p.out;
+    int k1 = 0, eb = 0;
+    for (int j = 0; j < n_my; ++j) {
+      if (!mbar_wait_sleep(&fbars[j & (S - 1)], (uint32_t)(j >> p.ring_shift) & 1u)) {
+        if (lane == 0) {
+          atomicOr(&fx.flags, 1);
+          report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
+        }
+        break;
+      }
+      const int i = warp + j * NC;
+      const bool in1 = i >= split;
+      const int pos0 = 64 * (in1 ? i - split : ua0 + i);
+      const int s = in1 ? 1 : 0;
+      if (s != cur) {
+        cur = s;
+        const LineView& L = in1 ? L1 : L0;
 #pragma unroll
-  for (int s = 1; s < S; ++s)
-    if (issued == s && s < n_my) issue(issued++);
-  bool timed_out = false;
-  for (int i = 0; i < n_my; ++i) {
-    if (!mbar_wait(&ring_bar[warp][i & (S - 1)], (uint32_t)(i / S) & 1u)) {
-      timed_out = true;
-      break;
-    }
-    const int ubase = k0 + 32 * (warp + kLogitsWarps * i);
-    const uint8_t* stg = ring + (i & (S - 1)) * STAGE;
-    uint32_t wa0[W], wb0[W], wa1[W], wb1[W];
-    lds_chunk<W>(stg + g * (16 * W) + t * (4 * W), wa0);
-    lds_chunk<W>(stg + (g + 8) * (16 * W) + t * (4 * W), wb0);
-    lds_chunk<W>(stg + TILE + g * (16 * W) + t * (4 * W), wa1);
-    lds_chunk<W>(stg + TILE + (g + 8) * (16 * W) + t * (4 * W), wb1);
-    uint32_t na0, nb0, na1, nb1;
-    if constexpr (NB == 4) {
-      const uint32_t* nsl = reinterpret_cast<const uint32_t*>(stg + 2 * TILE);
-      na0 = nsl[g]; nb0 = nsl[g + 8]; na1 = nsl[16 + g]; nb1 = nsl[24 + g];
-    } else {
-      const uint8_t* nsl = stg + 2 * TILE;
-      na0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * g);
-      nb0 = *reinterpret_cast<const unsigned short*>(nsl + 2 * (g + 8));
-      na1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * g);
-      nb1 = *reinterpret_cast<const unsigned short*>(nsl + 32 + 2 * (g + 8));
-    }
-    bool ok0 = true, ok1 = ubase + 16 < k1;
-    if (!fast) {
-      ok0 = page_base[(ubase >> ps) - first_page] >= 0;
-      ok1 = ok1 && page_base[((ubase + 16) >> ps) - first_page] >= 0;
-    }
-    __syncwarp();                    // every read of this stage precedes its reuse
-    if (i + S < n_my) {
-      issue(i + S);
-      issued = i + S + 1;
-    }
-    float la0, lb0, la1, lb1;
-    tile(wa0, wb0, na0, nb0, la0, lb0);
-    tile(wa1, wb1, na1, nb1, la1, lb1);
-    if (qvalid) {
-      const int r = ubase + g;
-      if (fast && ubase + 32 <= k1) {
-        __stcs(orow + r, la0);
-        __stcs(orow + r + 8, lb0);
-        __stcs(orow + r + 16, la1);
-        __stcs(orow + r + 24, lb1);
-      } else {
-        if (ok0 && r < k1) __stcs(orow + r, la0);
-        if (ok0 && r + 8 < k1) __stcs(orow + r + 8, lb0);
-        if (ok1 && r + 16 < k1) __stcs(orow + r + 16, la1);
-        if (ok1 && r + 24 < k1) __stcs(orow + r + 24, lb1);
+        for (int kk = 0; kk < KC; ++kk) qf.bq[kk] = fx.fr[s][kk * 32 + lane];
+#pragma unroll
+        for (int kk = 0; kk < KQ; ++kk) qf.bz[kk] = fx.fz[s][kk * 32 + lane];
+        qf.zsum = query_zsum<KQ>(qf.bz);
+        const float2 sc = fx.scal[4 * s + t];
+        qf.c0 = sc.x;
+        qf.c1 = F > 0 ? sc.y : 0.0f;
+        const int qidx = L.qt * 4 + t;
+        qvalid = qidx < p.G;
+        orow = p.out + ((int64_t)L.b * p.n_q_heads + (int64_t)L.h * p.G + (qvalid ? qidx : 0)) * p.out_stride;
+        k1 = L.k1;
+        eb = L.ebase - L.first;
+      }
+      const uint8_t* stg = ring + (j & (S - 1)) * STAGE;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {          // two 32-key halves of the unit
+        const int pos = pos0 + 32 * hf;
+        const uint8_t* st = stg + hf * 32 * REC;
+        uint32_t wa0[W], wb0[W], wa1[W], wb1[W];
+        lds_chunk<W>(st + g * REC + t * (4 * W), wa0);
+        lds_chunk<W>(st + (g + 8) * REC + t * (4 * W), wb0);
+        lds_chunk<W>(st + (16 + g) * REC + t * (4 * W), wa1);
+        lds_chunk<W>(st + (24 + g) * REC + t * (4 * W), wb1);
+        uint32_t na0, nb0, na1, nb1;
+        unit_norms<NB>(stg + NOFF + hf * 32 * NB, g, na0, nb0, na1, nb1);
+        if (hf == 1) {
+          __syncwarp();                  // every read of this slot precedes its release
+          if (lane == 0) mbar_arrive(&ebars[j & (S - 1)]);
+        }
+        if (pos >= k1) continue;         // past the context: nothing to store
+        bool ok0 = true, ok1 = pos + 16 < k1;
+        if (!fast) {
+          ok0 = fx.page_base[eb + (pos >> ps)] >= 0;
+          ok1 = ok1 && fx.page_base[eb + ((pos + 16) >> ps)] >= 0;
+        }
+        float la0, lb0, la1, lb1;
+        tile_logits<BITS, E, F>(wa0, wb0, na0, nb0, qf, p.kt, la0, lb0);
+        tile_logits<BITS, E, F>(wa1, wb1, na1, nb1, qf, p.kt, la1, lb1);
+        if (qvalid) {
+          const int r = pos + g;
+          if (fast && pos + 32 <= k1) {
+            __stcs(orow + r, la0);
+            __stcs(orow + r + 8, lb0);
+            __stcs(orow + r + 16, la1);
+            __stcs(orow + r + 24, lb1);
+          } else {
+            if (ok0 && r < k1) __stcs(orow + r, la0);
+            if (ok0 && r + 8 < k1) __stcs(orow + r + 8, lb0);
+            if (ok1 && r + 16 < k1) __stcs(orow + r + 16, la1);
+            if (ok1 && r + 24 < k1) __stcs(orow + r + 24, lb1);
+          }
+        }
       }
     }
   }
-  if (timed_out) {
-    // report, then let the copies already issued land (the last unit issued
-    // into each stage; each wait bounded) before the CTA's shared memory is
-    // released
-    if (lane == 0) report(p.cv.err, TQ_DEV_ERR_TIMEOUT);
-    for (int u = max(0, issued - S); u < issued; ++u) mbar_wait(&ring_bar[warp][u & (S - 1)], (uint32_t)(u / S) & 1u);
+  // every thread of the CTA meets here; after a wait that gave up, the
+  // copies already issued land (each wait bounded) before shared memory is
+  // released
+  __syncthreads();
+  if (fx.flags & 1) {
+    for (int k = tid; k < NC * S; k += NT)
+      if (fx.slot_last[k] >= 0)
+        mbar_wait(&fx.full_bar[k], (uint32_t)((int)fdiv((uint32_t)fx.slot_last[k], p.div_nc) >> p.ring_shift) & 1u);
+    if (PREP && tid == 0 && p.prep_tiles > NC) mbar_wait(&fx.xtab_bar, 0u);
   }
 }
 
@@ -677,58 +997,116 @@ static LogitsWs logits_ws_layout(const tq_codebook* cb, int64_t groups, int G, i
   return w;
 }
 
+// One launch when every CTA gets at least this many units.
+constexpr int64_t kPrepMinUnits = 8;
+
 size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
   return logits_ws_layout(cb, groups, G, groups * G).total;
 }
 
+// Shared-memory plan of a logits launch: NW warps x S copy slots (S a power
+// of two, 2 or 4: S = 4 when a warp has more than 2 units and the slots
+// fit), then the fixed part; the two-launch form leaves room for a
+// preparation CTA on the same SM.
+struct LogitsPlan {
+  int nw, ring_shift, fixed_off, smem, smem_max;
+};
+
 template <int BITS, int E, int F>
-static tq_status run_logits(const tqd::LogitsParams& p, const tqd::PrepParams& pp, int parts, int64_t groups,
-                            int qtiles, cudaStream_t st) {
-  constexpr int q0 = BITS == 1 ? (E + 31) / 32 : BITS == 2 ? E / 16
-                   : BITS == 3 ? 3 * (E / 32) + 2 * ((E % 32) / 16) : E / 8;
-  constexpr int W = q0 + (F + 31) / 32;
-  using RS = tqd::RingShape<W>;
-  const int smem = tqd::kLogitsWarps * RS::kStages * RS::kStageBytes;
+static bool logits_plan(int64_t units_per_cta, bool prep, LogitsPlan* pl) {
+  using TS = tqd::TileShape<BITS, E, F>;
+  const int stage = tqd::SlotShape<TS::W, TS::NB>::kBytes;
+  static int optin[64] = {};
+  const int dev = current_device();
+  int smax = dev >= 0 && dev < 64 ? optin[dev] : 0;
+  if (smax == 0) {
+    if (cudaDeviceGetAttribute(&smax, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+    if (dev >= 0 && dev < 64) optin[dev] = smax;
+  }
+  const int budget = prep ? smax : smax - 8 * 1024;
+  const int fixed = (int)((tqd::logits_fixed_bytes<BITS, E, F>() + 15) / 16 * 16);
+  pl->nw = prep ? 15 : units_per_cta >= 16 ? tqd::logits_max_consumers(E) : 4;
+  const int64_t per_warp = (units_per_cta + pl->nw - 1) / pl->nw;
+  int S = per_warp > 2 ? 4 : 2;
+  while (S > 2 && fixed + pl->nw * S * stage > budget) S /= 2;
+  if (fixed + pl->nw * S * stage > budget) return false;
+  pl->ring_shift = S == 4 ? 2 : 1;
+  pl->fixed_off = pl->nw * S * stage;
+  pl->smem = pl->fixed_off + fixed;
+  // the kernel attribute (set once per instance) covers the largest plan
+  const int nw_max = prep ? 15 : tqd::logits_max_consumers(E);
+  pl->smem_max = std::max(pl->smem, fixed + nw_max * 4 * stage <= budget ? fixed + nw_max * 4 * stage
+                                                                         : fixed + nw_max * 2 * stage);
+  return true;
+}
+
+template <int BITS, int E, int F, bool PREP>
+static tq_status launch_logits_kernel(tqd::LogitsParams p, const LogitsPlan& pl, cudaStream_t st) {
   static PerDeviceOnce attr;           // per template instance
   if (const int dev_ = current_device(); attr.need(dev_)) {
-    cudaError_t e = cudaFuncSetAttribute(tqd::logits_kernel<BITS, E, F>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(tqd::logits_kernel<BITS, E, F, PREP>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, pl.smem_max);
     if (e != cudaSuccess) return cuda_fail(e, "tq_logits: smem attribute");
-    // the preparation kernel asks for the logits kernel's shared-memory
-    // split, or its CTAs would keep logits CTAs off their SMs
-    e = cudaFuncSetAttribute(tqd::prep_queries_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return cuda_fail(e, "tq_logits: carveout attribute");
     attr.mark(dev_);
   }
-  tqd::prep_queries_kernel<<<dim3((unsigned)parts, (unsigned)(groups * qtiles)), tqd::kLogitsWarps * 32, 0, st>>>(pp);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
+  p.ring_shift = pl.ring_shift;
+  p.nc = pl.nw;
+  p.div_nc = tqd::make_fastdiv((uint32_t)pl.nw);
+  p.fixed_off = pl.fixed_off;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)p.n_chunks, (unsigned)groups, (unsigned)qtiles);
-  cfg.blockDim = dim3(tqd::kLogitsWarps * 32);
-  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.gridDim = dim3((unsigned)p.n_cta);
+  cfg.blockDim = dim3((pl.nw + 1) * 32);   // consumers + the producer warp
+  cfg.dynamicSmemBytes = (size_t)pl.smem;
   cfg.stream = st;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F>, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::logits_kernel<BITS, E, F, PREP>, p);
   if (e != cudaSuccess) return cuda_fail(e, "tq_logits launch");
   return TQ_OK;
 }
 
+// One launch (the CTAs prepare their queries) when `prep` and d <= 128;
+// otherwise the preparation kernel, then the logits kernel.
+template <int BITS, int E, int F>
+static tq_status run_logits(tqd::LogitsParams p, const tqd::PrepParams& pp, int parts, int64_t tiles,
+                            int64_t units_per_cta, bool prep, cudaStream_t st) {
+  LogitsPlan pl;
+  if constexpr (E <= 32) {
+    if (prep && logits_plan<BITS, E, F>(units_per_cta, true, &pl))
+      return launch_logits_kernel<BITS, E, F, true>(p, pl, st);
+  }
+  if (!logits_plan<BITS, E, F>(units_per_cta, false, &pl))
+    return fail(TQ_EUNSUPPORTED, "tq_logits: shared-memory plan");
+  constexpr bool kInt8 = BITS <= 3;
+  static PerDeviceOnce attr;
+  if (const int dev_ = current_device(); attr.need(dev_)) {
+    // the preparation kernel asks for the logits kernel's shared-memory
+    // split, or its CTAs would keep logits CTAs off their SMs
+    cudaError_t e = cudaFuncSetAttribute(tqd::prep_queries_kernel<E, F, kInt8>,
+                                         cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_logits: carveout attribute");
+    attr.mark(dev_);
+  }
+  tqd::prep_queries_kernel<E, F, kInt8><<<dim3((unsigned)parts, (unsigned)tiles), tqd::kPrepThreads, 0, st>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
+  return launch_logits_kernel<BITS, E, F, false>(p, pl, st);
+}
+
 template <int BITS>
 static tq_status dispatch_logits(const Layout& L, const tqd::LogitsParams& p, const tqd::PrepParams& pp,
-                                 int parts, int64_t groups, int qtiles, cudaStream_t st) {
-  if (L.E == 32 && L.F == 32) return run_logits<BITS, 32, 32>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 32 && L.F == 0) return run_logits<BITS, 32, 0>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 16 && L.F == 16) return run_logits<BITS, 16, 16>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 16 && L.F == 0) return run_logits<BITS, 16, 0>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 64 && L.F == 64) return run_logits<BITS, 64, 64>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 64 && L.F == 0) return run_logits<BITS, 64, 0>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 48 && L.F == 48) return run_logits<BITS, 48, 48>(p, pp, parts, groups, qtiles, st);
-  if (L.E == 48 && L.F == 0) return run_logits<BITS, 48, 0>(p, pp, parts, groups, qtiles, st);
+                                 int parts, int64_t tiles, int64_t upc, bool prep, cudaStream_t st) {
+  if (L.E == 32 && L.F == 32) return run_logits<BITS, 32, 32>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 32 && L.F == 0) return run_logits<BITS, 32, 0>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 16 && L.F == 16) return run_logits<BITS, 16, 16>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 16 && L.F == 0) return run_logits<BITS, 16, 0>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 64 && L.F == 64) return run_logits<BITS, 64, 64>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 64 && L.F == 0) return run_logits<BITS, 64, 0>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 48 && L.F == 48) return run_logits<BITS, 48, 48>(p, pp, parts, tiles, upc, prep, st);
+  if (L.E == 48 && L.F == 0) return run_logits<BITS, 48, 0>(p, pp, parts, tiles, upc, prep, st);
   return fail(TQ_EUNSUPPORTED, "tq_logits: no kernel for this (d, m)");
 }
 
@@ -748,18 +1126,18 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
   uint2* frag = reinterpret_cast<uint2*>(wsb);
   uint2* qfrag = reinterpret_cast<uint2*>(wsb + wl.frag);
   float2* scal = reinterpret_cast<float2*>(wsb + wl.frag + wl.qfrag);
+  int ps = 0;
+  while ((1 << ps) < cv.page_tokens) ++ps;
+  const int64_t units = (max_ctx + 63) / 64;
 
   tqd::PrepParams pp;
   pp.q = q;
   pp.dtype = dt;
   pp.d = L.d;
-  pp.E = L.E;
-  pp.F = L.F;
   pp.n_q_heads = n_q_heads;
   pp.n_kv_heads = cv.n_kv_heads;
   pp.G = G;
   pp.qtiles = qtiles;
-  pp.cb_int8 = L.bits <= 3 ? 1 : 0;
   pp.cb_unscale = std::ldexp(1.0f, -cb->table_exp);
   pp.qjl_scale = (float)cb->qjl_scale;
   // |(S q)_i| <= ||S_i|| ||q||: the float bound is rounded up
@@ -772,57 +1150,69 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
 
   tqd::LogitsParams lp;
   lp.cv = cv;
-  int ps = 0;
-  while ((1 << ps) < cv.page_tokens) ++ps;
   lp.page_shift = ps;
   lp.ctx_len = ctx_len;
   lp.n_kv_heads = cv.n_kv_heads;
   lp.n_q_heads = n_q_heads;
   lp.G = G;
   lp.qtiles = qtiles;
-  // Every CTA slot of the GPU (SMs x resident CTAs) gets one CTA, each an
-  // equal share (to one 32-key unit) of one sequence's keys; more CTAs when a
-  // share would need more than kCtaPages - 2 block-table entries, and then as
-  // many as fill whole waves of the slots (a last, partly filled wave would
-  // run at a fraction of the GPU for as long as a full one).
-  const int64_t units = (max_ctx + 31) / 32;
-  const int64_t tiles = groups * qtiles;
-  const int64_t slots = (int64_t)device_sm_count() * tqd::logits_min_blocks(L.bits, L.E);
-  int64_t n_chunks = std::max<int64_t>(1, slots / tiles);
-  const int64_t max_units_cta = (int64_t)(tqd::kCtaPages - 2) * cv.page_tokens / 32;
-  n_chunks = std::max<int64_t>(n_chunks, (units + max_units_cta - 1) / max_units_cta);
-  n_chunks = std::min<int64_t>(n_chunks, units);
-  const int64_t waves = (n_chunks * tiles + slots - 1) / slots;
-  n_chunks = std::min<int64_t>(std::max<int64_t>(n_chunks, waves * slots / tiles), units);
-  if (n_chunks > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_logits: context too long");
-  lp.n_chunks = (int)n_chunks;
   lp.units = (int)units;
   lp.max_ctx = (int)max_ctx;
+  // CTAs: one per SM, at least one per line (so a CTA spans at most two
+  // lines) and enough that a CTA's block-table entries fit its staging
+  // array; when every CTA would get fewer than 16 units (of 64 keys), four
+  // times as many CTAs of 4 consumer warps (several per SM).
+  const int64_t lines = groups * qtiles;
+  const int64_t items = lines * units;
+  const int64_t max_upc = (int64_t)(tqd::kLogitsPages - 4) * cv.page_tokens / 64;
+  const int64_t n_sm = device_sm_count();
+  int64_t n_cta = std::max(n_sm, lines);
+  if ((items + n_cta - 1) / n_cta < 16) n_cta = std::max(4 * n_sm, lines);
+  n_cta = std::max(n_cta, (items + max_upc - 1) / max_upc);
+  n_cta = std::min(n_cta, items);
+  if (n_cta > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_logits: context too long");
+  const int64_t upc = (items + n_cta - 1) / n_cta;
+  if (items > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_logits: batch * heads * context too large");
+  lp.n_cta = (int)n_cta;
+  lp.per_cta = (int)(items / n_cta);
+  lp.extra = (int)(items % n_cta);
+  lp.div_u = tqd::make_fastdiv((uint32_t)units);
+  lp.div_qtiles = tqd::make_fastdiv((uint32_t)qtiles);
+  lp.div_kv = tqd::make_fastdiv((uint32_t)cv.n_kv_heads);
+  lp.q = q;
+  lp.dtype = dt;
+  lp.d = L.d;
+  lp.d16 = (L.d + 15) / 16;
+  lp.table = cb->qprep_frag;
+  lp.prep_tiles = (L.d_pad + L.m_pad) / 16;
+  lp.pc.cb_unscale = pp.cb_unscale;
+  lp.pc.qjl_scale = pp.qjl_scale;
+  lp.pc.s_rowmax = pp.s_rowmax;
+  // the CTAs prepare their own queries when each gets enough units to
+  // amortize loading the [Pi ; S] table (d <= 128)
+  const bool prep = L.E <= 32 && upc >= kPrepMinUnits;
   lp.frag = frag;
   lp.qfrag = qfrag;
   lp.scal = scal;
   lp.out = out;
   lp.out_stride = out_stride;
-  lp.pre_stages = 1;
-  lp.th0 = cb->int8_hi[0];
-  lp.th1 = cb->int8_hi[1];
-  lp.tl0 = cb->int8_lo[0];
-  lp.tl1 = cb->int8_lo[1];
+  lp.kt.t0 = cb->int8_levels[0];
+  lp.kt.t1 = cb->int8_levels[1];
   const uint16_t* M = cb->mag16;
-  lp.lo0 = lp.lo1 = lp.hi0 = lp.hi1 = 0u;
+  lp.kt.lo0 = lp.kt.lo1 = lp.kt.hi0 = lp.kt.hi1 = 0u;
   if (L.bits == 4) {
     for (int i = 0; i < 4; ++i) {
-      lp.lo0 |= (uint32_t)(M[i] & 0xFF) << (8 * i);
-      lp.lo1 |= (uint32_t)(M[4 + i] & 0xFF) << (8 * i);
-      lp.hi0 |= (uint32_t)(M[i] >> 8) << (8 * i);
-      lp.hi1 |= (uint32_t)(M[4 + i] >> 8) << (8 * i);
+      lp.kt.lo0 |= (uint32_t)(M[i] & 0xFF) << (8 * i);
+      lp.kt.lo1 |= (uint32_t)(M[4 + i] & 0xFF) << (8 * i);
+      lp.kt.hi0 |= (uint32_t)(M[i] >> 8) << (8 * i);
+      lp.kt.hi1 |= (uint32_t)(M[4 + i] >> 8) << (8 * i);
     }
   }
   switch (L.bits) {
-    case 1: return dispatch_logits<1>(L, lp, pp, parts, groups, qtiles, st);
-    case 2: return dispatch_logits<2>(L, lp, pp, parts, groups, qtiles, st);
-    case 3: return dispatch_logits<3>(L, lp, pp, parts, groups, qtiles, st);
-    case 4: return dispatch_logits<4>(L, lp, pp, parts, groups, qtiles, st);
+    case 1: return dispatch_logits<1>(L, lp, pp, parts, lines, upc, prep, st);
+    case 2: return dispatch_logits<2>(L, lp, pp, parts, lines, upc, prep, st);
+    case 3: return dispatch_logits<3>(L, lp, pp, parts, lines, upc, prep, st);
+    case 4: return dispatch_logits<4>(L, lp, pp, parts, lines, upc, prep, st);
   }
   return fail(TQ_EUNSUPPORTED, "tq_logits: bits");
 }

@@ -47,7 +47,7 @@ struct QuantizeTcParams {
   const __nv_bfloat16* pi_bf;    // [2][128][128]: hi, lo of Pi[j][k]
   const __nv_bfloat16* srot_bf;  // [2][128][128]: hi, lo of (S Pi^T)[i][j]
   const float* bound32;          // [2^b - 1]
-  const float* cent32;           // [2^b] float(c16)
+  const float* cent32;           // [2^b] the reconstruction levels
   int64_t n_tiles;
 };
 

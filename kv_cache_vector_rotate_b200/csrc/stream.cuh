@@ -19,6 +19,10 @@ __device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
                : "memory");
 }
+// A plain arrival (no transaction bytes).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
 // One test of the phase of the given parity.
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t done;
@@ -36,6 +40,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitCycles) return false;
   }
 }
+// One test of the phase with a suspend-time hint: the thread may sleep up to
+// `ns` nanoseconds in the test (waking when the phase completes) instead of
+// spinning, so waiting warps leave the issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(done) : "r"(smem_addr(bar)), "r"(parity), "r"(ns) : "memory");
+  return done != 0;
+}
+// mbar_wait with sleeping tests; false after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_sleep(bar, parity, 20000u)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_sleep(bar, parity, 20000u)) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+}
 // Bulk copy (no multicast) of `bytes` global -> shared, completing on `bar`;
 // both addresses 16-byte aligned, bytes a multiple of 16, with an L2
 // eviction-priority policy.
@@ -44,6 +67,17 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
       ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(pol) : "memory");
+}
+// Prefetch of `bytes` global bytes into L2 (no data to the SM); the address
+// 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+// Bulk copy global -> shared with the default L2 policy (data that other
+// CTAs read again, such as constant tables).
+__device__ __forceinline__ void bulk_copy_plain(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_addr(bar)) : "memory");
 }
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t pol;

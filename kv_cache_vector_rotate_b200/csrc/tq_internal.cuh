@@ -73,21 +73,24 @@ struct tq_codebook {
   float* st32;        // [d][m_pad]   S^T, columns >= m zero      (query sketch, coalesced)
   float* srot32;      // [m_pad][d_pad] S Pi^T row-major, zero padded (residual sketch, small appends)
   float* bound32;     // [2^b - 1]    boundaries (fp32)
-  float* cent32;      // [2^b]        float(fp16(c))
+  float* cent32;      // [2^b]        the reconstruction levels (fp32, exact)
   __nv_bfloat16* pi_bf;    // tensor-core operands: [2][d_pad][d_pad] hi, lo of Pi
   __nv_bfloat16* srot_bf;  // [2][m_pad][d_pad] hi, lo of S Pi^T
   // [Pi ; S] (R = d_pad + m_pad rows, d columns padded to d16 = ceil(d/16)
   // blocks of 16) as bf16 hi + lo in mma.m16n8k16 A-fragment order:
   // uint4 [R/16 row tiles][d16][2: hi, lo][32 lanes]
   uint4* qprep_frag;
-  // fp16 bit patterns of the reconstruction magnitudes M[mu] = c16[H + mu]
+  // reconstruction levels (float64 copies of what the kernels use): 8-bit
+  // fixed point levels k_i 2^-table_exp for b <= 3, fp16 levels for b = 4
+  std::vector<double> levels;
+  // fp16 bit patterns of the levels (exact) and of the magnitudes
+  // M[mu] = level[H + mu]
   uint16_t mag16[8];
   uint16_t cent16[16];
-  // b <= 3: c16[i] * 2^table_exp is an integer v_i with |v_i| <= 32639, split
-  // into int8 slices v_i = 256 hi_i + lo_i (hi_i = floor((v_i + 128) / 256));
-  // the slices of levels 0..7 packed as bytes (int8_hi[0] = levels 0..3).
+  // b <= 3: the integers k_i of levels 0..7 as int8 bytes (int8_levels[0] =
+  // levels 0..3)
   int table_exp;
-  uint32_t int8_hi[2], int8_lo[2];
+  uint32_t int8_levels[2];
 };
 
 namespace tq {
@@ -149,6 +152,27 @@ tq_status launch_values(const tq_codebook* cb, const CacheView& cv, const float*
 // ---- device helpers --------------------------------------------------------
 
 namespace tqd {
+
+// Division of 0 <= n < 2^31 by a divisor fixed at launch, without the
+// software division routine: q = (umulhi(n, m) + n) >> s with
+// m = floor(2^32 (2^s - d) / d) + 1, s = ceil(log2 d) (round-up reciprocal;
+// exact for these n), or q = n when d = 1.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  if (d > 1) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) ++l;
+    f.m = (uint32_t)((((uint64_t)1 << 32) * ((1ull << l) - d)) / d + 1);
+    f.s = l;
+  }
+  return f;
+}
+__device__ __forceinline__ uint32_t fdiv(uint32_t n, const FastDiv& f) {
+  return f.d == 1 ? n : (__umulhi(n, f.m) + n) >> f.s;
+}
 
 __device__ __forceinline__ void report(uint32_t* err, uint32_t bits) {
   if (err) atomicOr(err, bits);

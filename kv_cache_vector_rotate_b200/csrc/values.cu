@@ -1,15 +1,15 @@
-// Value path from packed records: v_hat = ||v|| Pi^T c16[idx].
+// Value path from packed records: v_hat = ||v|| Pi^T c[idx] (c: the reconstruction levels).
 //
 // "TurboQuant explained" (a2a-mcp.org), §Stage 1: the MSE stage alone codes
 // the values; reconstruction is the centroid vector rotated back.
 //  * mode A writes v_hat for every token;
 //  * mode B forms o_h = sum_t w_{h,t} v_hat_t for the query heads of a KV head.
 //    The sum is accumulated in the rotated space (acc_h = sum_t w_{h,t}
-//    ||v_t|| c16[idx_t]) and rotated back once per head (o_h = Pi^T acc_h).
+//    ||v_t|| c[idx_t]) and rotated back once per head (o_h = Pi^T acc_h).
 //    Per KV group that is ACC^T = C^T (w ||v||)^T, a contraction over the
 //    tokens, run on the tensor cores: each warp streams 32-token units of
 //    records into a shared-memory ring with bulk copies, each lane decodes
-//    one token's coordinates into fp16 c16 values of a [token][coordinate]
+//    one token's coordinates into fp16 level values of a [token][coordinate]
 //    tile, ldmatrix.trans turns the tile into MMA A fragments (coordinates x
 //    tokens), and the weights times the norms, split into fp16 hi + lo, are
 //    the B columns (4 query heads x 2).  Partial sums of context chunks go to
@@ -48,7 +48,7 @@ __device__ __forceinline__ int unpack_index(const uint32_t* w, int l) {
   return level_index<BITS>(code);
 }
 
-// Stages 16 tokens: cs[tok][j] = ||v|| c16[idx_j] (0 past the context or for
+// Stages 16 tokens: cs[tok][j] = ||v|| c[idx_j] (0 past the context or for
 // an unusable page).  128 threads: 8 threads per token, each decoding every
 // 8th coordinate.
 template <int BITS, int E>
@@ -138,7 +138,7 @@ struct ValuesTcParams {
   float* partial;                  // [n_chunks][groups * qtiles][4][4E]
   const float* pi32;               // [d_pad][d]
   float* out;                      // [batch][n_q_heads][d]
-  uint32_t tlo0, tlo1, thi0, thi1; // low / high bytes of c16 (b <= 3: levels 0..7; b = 4: magnitudes)
+  uint32_t tlo0, tlo1, thi0, thi1; // low / high bytes of the fp16 levels (b <= 3: levels 0..7; b = 4: magnitudes)
 };
 
 template <int W, int E>
@@ -149,7 +149,7 @@ struct ValShape {
   static constexpr int kWarpBytes = kValStages * kStage + kTile + 32 * 16;   // + w ||v|| [32][4] fp32
 };
 
-// fp16 c16 values of the 8 coordinates 8 kk .. 8 kk + 7 of a chunk, as four
+// fp16 level values of the 8 coordinates 8 kk .. 8 kk + 7 of a chunk, as four
 // fp16 pairs (b <= 3: level selector and two byte permutes per 4 values; b =
 // 4: sign-magnitude nibbles).
 template <int BITS, int E>

@@ -25,7 +25,7 @@ EXPORTS = (
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
-    "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook",
+    "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook", "tq_codebook_levels",
 )
 
 
@@ -72,6 +72,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_codebook_build_host": (i32, [ctypes.POINTER(Params), ctypes.POINTER(vp)]),
         "tq_codebook_free": (None, [vp]),
         "tq_codebook_export": (i32, [vp, dp, dp, dp, dp]),
+        "tq_codebook_levels": (i32, [vp, dp, ctypes.POINTER(i32)]),
         "tq_layout": (i32, [vp, i32, i32, ctypes.POINTER(LayoutInfo)]),
         "tq_quantize_append": (i32, [vp, vp, i32, i64, i32, i64, vp, ctypes.POINTER(CacheStruct), vp]),
         "tq_logits_workspace_bytes": (sz, [vp, i64, i32, i32]),
@@ -157,6 +158,15 @@ class Codebook:
             t.ctypes.data_as(dp)))
         return {"pi": pi.reshape(self.d, self.d), "s": s[: self.m * self.d].reshape(self.m, self.d),
                 "centroids": c, "boundaries": t}
+
+    def levels(self):
+        """tq_codebook_levels: (reconstruction levels, scale exponent f or None)."""
+        import numpy as np
+        lev = np.zeros(1 << self.bits)
+        f = ctypes.c_int32(0)
+        _check(load_library().tq_codebook_levels(self.handle, lev.ctypes.data_as(ctypes.POINTER(ctypes.c_double)),
+                                                 ctypes.byref(f)))
+        return lev, (None if f.value == -(1 << 31) else f.value)
 
     def layout(self, page_tokens: int, n_kv_heads: int) -> LayoutInfo:
         info = LayoutInfo()

@@ -248,13 +248,34 @@ def fp16(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64).astype(np.float16)
 
 
+def reconstruction_levels(c: np.ndarray) -> tuple[np.ndarray, int | None]:
+    """The reconstruction levels of a Lloyd-Max codebook.
+
+    READING (TQ §Stage 1 gives the centroids as real numbers, not how they
+    are stored): a codebook of at most 8 levels (b <= 3) keeps its levels in
+    8-bit fixed point on one power-of-two scale -- every centroid rounded
+    (half to even) to an integer multiple of 2^-f, f the largest integer with
+    max|c| 2^f <= 127 -- so that a decoded coordinate is one signed byte; the
+    levels are then exact in fp16 and fp32 too, and the rounding moves each
+    by at most 2^-(f+1) (about 0.1 % more distortion at b = 3, d = 128; pinned
+    in tests/test_oracle_codec.py).  Larger codebooks keep their levels in
+    fp16 (8 bits would merge neighbouring levels).  Returns (levels, f), with
+    f = None for fp16 levels.  The boundaries stay the float64 midpoints of
+    the unrounded centroids."""
+    c = np.asarray(c, dtype=np.float64)
+    if len(c) > 8:
+        return fp16(c).astype(np.float64), None
+    f = int(math.floor(math.log2(127.0 / float(np.max(np.abs(c))))))
+    return np.round(c * 2.0 ** f) / 2.0 ** f, f
+
+
 # ---------------------------------------------------------------------------
 # The codec.  TQ §Stage 1: normalize, rotate, quantize each coordinate.
 # TQ §Stage 2: 1-bit signs of a Gaussian projection of the residual.
 # READINGS:
 #  * the norm ||x|| and the residual norm ||r|| are side values stored as fp16;
-#  * reconstruction uses the fp16-rounded centroids c16 (also in the residual),
-#    the boundaries stay float64;
+#  * reconstruction uses the levels crec = reconstruction_levels(c) (also in
+#    the residual), the boundaries stay float64;
 #  * a tie y == t_i goes to the upper cell; sign(0) = +1;
 #  * the zero vector is quantized as u = 0 (every index is the cell holding 0);
 #  * the QJL sketch keeps one sign per projection row (m bits per key).
@@ -271,8 +292,8 @@ class Codec:
     cb: Codebook
 
     @property
-    def c16(self) -> np.ndarray:
-        return fp16(self.cb.centroids).astype(np.float64)
+    def crec(self) -> np.ndarray:
+        return reconstruction_levels(self.cb.centroids)[0]
 
 
 def make_codec(d: int, bits: int, m: int, seed_pi: int, seed_s: int) -> Codec:
@@ -306,8 +327,8 @@ def quantize_indices(Y: np.ndarray, boundaries: np.ndarray) -> np.ndarray:
 
 def qjl_sketch(codec: Codec, U: np.ndarray, idx: np.ndarray):
     """TQ §Stage 2 for unit rows U coded by idx: (S r, r < 0 bits, fp16 ||r||)
-    with the residual r = u - Pi^T c16[idx] taken in the original space."""
-    R = U - codec.c16[idx] @ codec.Pi
+    with the residual r = u - Pi^T crec[idx] taken in the original space."""
+    R = U - codec.crec[idx] @ codec.Pi
     proj = R @ codec.S.T
     return proj, proj < 0.0, fp16(np.sqrt(np.sum(R * R, axis=1)))
 
@@ -330,13 +351,13 @@ def logits_from_codes(codec: Codec, Qv: np.ndarray, idx: np.ndarray, qneg: np.nd
                       norm16: np.ndarray, rnorm16: np.ndarray) -> np.ndarray:
     """Estimated <q, k> for every (query, key) pair, float64.
 
-    L = ||k|| ( sum_j (Pi q)_j c16[idx_j]
+    L = ||k|| ( sum_j (Pi q)_j crec[idx_j]
                 + sqrt(pi/2)/m ||r|| sum_i (S q)_i sign_i )
     with sign_i = -1 where the stored QJL bit says (S r)_i < 0, else +1.
     """
     Qv = np.asarray(Qv, dtype=np.float64)
     q_rot = Qv @ codec.Pi.T                       # [nq, d]
-    mse = q_rot @ codec.c16[idx].T                # [nq, N]
+    mse = q_rot @ codec.crec[idx].T                # [nq, N]
     out = mse
     if codec.m > 0:
         q_s = Qv @ codec.S.T                      # [nq, m]
@@ -347,8 +368,8 @@ def logits_from_codes(codec: Codec, Qv: np.ndarray, idx: np.ndarray, qneg: np.nd
 
 
 def dequantize(codec: Codec, idx: np.ndarray, norm16: np.ndarray) -> np.ndarray:
-    """v_hat = ||v|| Pi^T c16[idx]  (MSE reconstruction, one row per token)."""
-    return norm16.astype(np.float64)[:, None] * (codec.c16[idx] @ codec.Pi)
+    """v_hat = ||v|| Pi^T crec[idx]  (MSE reconstruction, one row per token)."""
+    return norm16.astype(np.float64)[:, None] * (codec.crec[idx] @ codec.Pi)
 
 
 def weighted_values(codec: Codec, W: np.ndarray, idx: np.ndarray, norm16: np.ndarray) -> np.ndarray:

@@ -78,13 +78,18 @@ def test_host_only_codebook_refuses_kernels():
     assert b"host-only" in lib.tq_last_error()
 
 
-@pytest.mark.parametrize("bits", [1, 2, 3])
-def test_integer_codebook_tables_fit_for_every_supported_d(bits):
-    # The fused-logits kernel for b <= 3 needs every fp16 level times 2^f to be
-    # a 16-bit integer; building the codebook checks it and fails otherwise.
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_reconstruction_levels_match_oracle_for_every_supported_d(bits):
+    # The levels the kernels decode with (8-bit fixed point for b <= 3, fp16
+    # for b = 4), built by the library's host code, equal the oracle's
+    # reconstruction_levels of its own Lloyd-Max centroids, scale included.
     for d in range(8, 257, 8):
         cb = tq.Codebook(d, bits, 0, 3, 4, device=False)
+        lev, f = cb.levels()
+        ref, fr = O.reconstruction_levels(O.lloyd_max(d, bits).centroids)
         cb.close()
+        assert f == fr, d
+        assert np.array_equal(lev, ref), d
 
 
 def test_attend_workspace_is_scores_plus_both_passes():

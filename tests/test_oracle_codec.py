@@ -66,6 +66,32 @@ def test_empirical_mse_matches_codebook_distortion():
     assert abs(err.mean() - d * codec.cb.distortion) < 5 * se
 
 
+@pytest.mark.parametrize("d,b", [(64, 1), (64, 3), (128, 1), (128, 2), (128, 3), (200, 2), (200, 3), (256, 3)])
+def test_reconstruction_levels_eight_bit_fixed_point(d, b):
+    # b <= 3: every level is an integer times 2^-f with |integer| <= 127, f is
+    # the largest such exponent, each level moved by at most 2^-(f+1), the
+    # set stays antisymmetric and ascending, and the distortion of the
+    # rounded levels (exact moments of the Beta law per cell) exceeds the
+    # Lloyd-Max optimum by less than 0.3 %.
+    cb = O.lloyd_max(d, b)
+    lev, f = O.reconstruction_levels(cb.centroids)
+    k = lev * 2.0 ** f
+    assert np.all(k == np.round(k)) and np.max(np.abs(k)) <= 127
+    assert np.max(np.abs(cb.centroids)) * 2.0 ** (f + 1) > 127
+    assert np.max(np.abs(lev - cb.centroids)) <= 2.0 ** -(f + 1)
+    assert np.array_equal(lev, -lev[::-1]) and np.all(np.diff(lev) > 0)
+    e = np.concatenate(([-1.0], cb.boundaries, [1.0]))
+    P, M1, M2 = O.cell_moments(e[:-1], e[1:], d)
+    D_rec = float(np.sum(M2 - 2.0 * lev * M1 + lev * lev * P))
+    assert cb.distortion <= D_rec < cb.distortion * 1.003
+
+
+def test_reconstruction_levels_fp16_beyond_eight_levels():
+    cb = O.lloyd_max(128, 4)
+    lev, f = O.reconstruction_levels(cb.centroids)
+    assert f is None and np.array_equal(lev, O.fp16(cb.centroids).astype(np.float64))
+
+
 def test_three_bit_cosine_similarity_community_figure():
     # TQ §Stage 2 quotes a reconstruction cosine of 0.983+ at 3 bits; the
     # MSE-stage reconstruction alone gives sqrt(1 - d D_3) ~ 0.983.
@@ -98,7 +124,7 @@ def test_qjl_estimator_unbiased_over_seeds_with_closed_form_variance():
         enc = O.encode(codec, k[None, :])
         # use the un-rounded norms so only the sketch is random
         u = k / np.linalg.norm(k)
-        r = u - codec.c16[enc.idx[0]] @ codec.Pi
+        r = u - codec.crec[enc.idx[0]] @ codec.Pi
         L = O.logits_from_codes(codec, q[None, :], enc.idx, enc.qneg,
                                 np.array([np.linalg.norm(k)]), np.array([np.linalg.norm(r)]))
         est.append(L[0, 0])
@@ -123,7 +149,7 @@ def test_unbiased_when_rotation_also_varies():
         codec = O.make_codec(d, b, m, 7000 + seed, 9000 + seed)
         enc = O.encode(codec, k[None, :])
         u = k / np.linalg.norm(k)
-        r = u - codec.c16[enc.idx[0]] @ codec.Pi
+        r = u - codec.crec[enc.idx[0]] @ codec.Pi
         L = O.logits_from_codes(codec, q[None, :], enc.idx, enc.qneg,
                                 np.array([np.linalg.norm(k)]), np.array([np.linalg.norm(r)]))
         errs.append(L[0, 0] - q @ k)
@@ -158,7 +184,7 @@ def test_high_bit_width_recovers_exact_logits():
 
 def test_mse_only_logits_equal_inner_product_with_reconstruction():
     # With m = 0 the logit is <q, v_hat>: rotating the query once (Pi q) and
-    # dotting with c16[idx] is the same as dequantizing the key first.
+    # dotting with crec[idx] is the same as dequantizing the key first.
     rng = np.random.default_rng(8)
     codec = O.make_codec(64, 3, 0, 21, 0)
     K = rng.standard_normal((50, 64))
