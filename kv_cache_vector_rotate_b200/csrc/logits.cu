@@ -493,6 +493,11 @@ __device__ __forceinline__ void prep_part(const PrepParams& p, int gq, int r, Pr
 template <int E, int F, bool INT8>
 __global__ void __launch_bounds__(kPrepThreads) prep_queries_kernel(PrepParams p) {
   __shared__ PrepSmem sm;
+  // launched as a programmatic dependent of the previous kernel on the
+  // stream: the queries (and the workspace, which the previous logits call
+  // may still read) are touched only after that kernel has completed, and
+  // the logits kernel is released only then
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   prep_part<E, F, INT8>(p, blockIdx.y, blockIdx.x, sm);
 }
@@ -526,13 +531,16 @@ __global__ void __launch_bounds__(kPrepThreads) prep_queries_kernel(PrepParams p
 //    while the consumers compute tile w of [Pi q ; S q] for the CTA's 8 query
 //    slots (4 per line) on the tensor cores and quantize it into fragment
 //    bytes in shared memory.
-//  * otherwise (two launches per call): prep_queries_kernel, an ordinary
-//    launch, writes the fragments to the workspace; every earlier kernel on
-//    the stream has finished when it starts, so this kernel may read the
-//    cache before its wait: the producer puts one unit per consumer warp in
-//    flight, the consumers wait and fetch their lines' fragments, and the
-//    producer goes on once they have them (fragment loads issued behind a
-//    full stream of copies would wait for it).
+//  * otherwise (two launches per call): prep_queries_kernel writes the
+//    fragments to the workspace.  It is a programmatic dependent of the
+//    previous kernel on the stream but releases this kernel only after its
+//    own wait, so every earlier kernel has finished when this kernel starts
+//    and it may read the cache before its wait: the producer puts one unit
+//    per consumer warp in flight, the consumers wait and fetch their lines'
+//    fragments, and the producer goes on once they have them (fragment
+//    loads issued behind a full stream of copies would wait for it).  On a
+//    short context this form is the faster one: in-CTA preparation loads
+//    the whole [Pi ; S] table into every CTA.
 // Every mbarrier wait is bounded; a CTA where one gives up reports
 // TQ_DEV_ERR_TIMEOUT and lets every copy it issued land before it exits.
 
@@ -867,8 +875,11 @@ __global__ void __maxnreg__(logits_regs(E, PREP)) logits_kernel(LogitsParams p) 
       if (tid < 8) fx.scal[tid] = prep_scales<TS::kInt8>(sqrtf(fx.qn2[tid]), p.pc);
       asm volatile("barrier.sync 2, %0;" ::"r"(NC * 32) : "memory");   // fragments ready (consumers only)
     } else {
-      // the query fragments and scales come from the preparation kernel
+      // the query fragments and scales come from the preparation kernel;
+      // the next call's preparation kernel may be scheduled from here on (it
+      // waits for this grid to complete before it touches anything)
       asm volatile("griddepcontrol.wait;" ::: "memory");
+      asm volatile("griddepcontrol.launch_dependents;");
       constexpr int FL = (KC + KQ) * 32;         // fragment words (uint2) per line
       for (int j = tid; j < n_lines * FL; j += NC * 32) {
         const int s = j / FL, r = j % FL;
@@ -998,7 +1009,7 @@ static LogitsWs logits_ws_layout(const tq_codebook* cb, int64_t groups, int G, i
 }
 
 // One launch when every CTA gets at least this many units.
-constexpr int64_t kPrepMinUnits = 8;
+constexpr int64_t kPrepMinUnits = 64;
 
 size_t logits_workspace(const tq_codebook* cb, int64_t groups, int G) {
   return logits_ws_layout(cb, groups, G, groups * G).total;
@@ -1090,8 +1101,16 @@ static tq_status run_logits(tqd::LogitsParams p, const tqd::PrepParams& pp, int 
     if (e != cudaSuccess) return cuda_fail(e, "tq_logits: carveout attribute");
     attr.mark(dev_);
   }
-  tqd::prep_queries_kernel<E, F, kInt8><<<dim3((unsigned)parts, (unsigned)tiles), tqd::kPrepThreads, 0, st>>>(pp);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)parts, (unsigned)tiles);
+  cfg.blockDim = dim3(tqd::kPrepThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::prep_queries_kernel<E, F, kInt8>, pp);
   if (e != cudaSuccess) return cuda_fail(e, "tq_logits: query preparation launch");
   return launch_logits_kernel<BITS, E, F, false>(p, pl, st);
 }
