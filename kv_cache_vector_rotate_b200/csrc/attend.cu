@@ -2,20 +2,23 @@
 //
 // "TurboQuant explained" (a2a-mcp.org), §How it works: the attention logits
 // are computed from the compressed keys (the fused logit of §Stage 2) and the
-// values are read back from their codes (§Stage 1).  This entry point chains
-// the library's kernels on the caller's stream:
+// values are read back from their codes (§Stage 1).
+//
+// d <= 128 with equal page sizes: the fused split-K pass (attend_fused.cuh:
+// query preparation, one pass over both caches with an online softmax, a
+// finish kernel).  Otherwise this file's composition of the library's
+// kernels on the caller's stream:
 //   1. tq_logits into a scores buffer of the workspace (query preparation +
 //      logits kernel);
 //   2. softmax_rows_kernel: each (sequence, query head) row of the scores
 //      becomes softmax weights over the valid positions, in place;
 //   3. tq_dequant_values mode B with those weights (accumulate in the rotated
 //      space, Pi^T once per query head).
-// The fused form (one split-K pass with an online softmax) is the next step;
-// this composition fixes the semantics and is the baseline it must beat.
 
+#include <algorithm>
 #include <cmath>
 
-#include "tq_internal.cuh"
+#include "attend_fused.cuh"
 
 namespace tqd {
 
@@ -129,6 +132,114 @@ __global__ void __cluster_dims__(kSmaxCluster, 1, 1) __launch_bounds__(kSmaxThre
 
 namespace tq {
 
+// The fused kernels, one translation unit per key width.
+tq_status launch_attend_fused_k1(const tqd::AttendParams& p, int vbits, int E, int F, int lines, cudaStream_t st);
+tq_status launch_attend_fused_k2(const tqd::AttendParams& p, int vbits, int E, int F, int lines, cudaStream_t st);
+tq_status launch_attend_fused_k3(const tqd::AttendParams& p, int vbits, int E, int F, int lines, cudaStream_t st);
+tq_status launch_attend_fused_k4(const tqd::AttendParams& p, int vbits, int E, int F, int lines, cudaStream_t st);
+tqd::KeyTables key_tables(const tq_codebook* cb);
+
+static bool fused_attend_ok(const tq_codebook* kcb, const tq_codebook* vcb, int kpt, int vpt) {
+  const Layout &K = kcb->lay, &V = vcb->lay;
+  return K.E <= 32 && K.E == V.E && (K.F == 0 || K.F == K.E) && kpt == vpt;
+}
+
+// Grid of the fused kernel: one CTA per SM at least, at least one per line,
+// and few enough units per CTA that its block-table entries fit.
+struct AttendGrid {
+  int64_t lines, units, items, n_cta;
+};
+static AttendGrid attend_grid(int64_t batch, int n_kv_heads, int n_q_heads, int64_t max_ctx, int page_tokens) {
+  AttendGrid gr;
+  const int G = n_q_heads / n_kv_heads;
+  gr.lines = batch * n_kv_heads * ((G + 3) / 4);
+  gr.units = (max_ctx + 63) / 64;
+  gr.items = gr.lines * gr.units;
+  const int64_t max_upc = (int64_t)(tqd::kAttPages - 4) * page_tokens / 64;
+  int64_t n = std::max<int64_t>(device_sm_count(), gr.lines);
+  n = std::max(n, (gr.items + max_upc - 1) / max_upc);
+  gr.n_cta = std::max<int64_t>(1, std::min(n, gr.items));
+  return gr;
+}
+
+struct FusedWs {
+  size_t prep, partial, total;
+};
+static FusedWs fused_ws_layout(const tq_codebook* kcb, int64_t batch, int n_kv_heads, int n_q_heads,
+                               int64_t n_cta) {
+  auto al = [](size_t n) { return (n + 255) / 256 * 256; };
+  FusedWs w;
+  w.prep = al(query_prep_workspace(kcb, batch, n_kv_heads, n_q_heads));
+  w.partial = al((size_t)n_cta * 2 * 4 * (4 * kcb->lay.E + 2) * sizeof(float));
+  w.total = w.prep + w.partial;
+  return w;
+}
+
+static tq_status launch_attend_fused(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb,
+                                     const CacheView& vcv, const void* q, tq_dtype dt, int64_t batch,
+                                     int n_q_heads, const int32_t* ctx_len, int64_t max_ctx, float scale,
+                                     float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int nkv = kcv.n_kv_heads;
+  const AttendGrid gr = attend_grid(batch, nkv, n_q_heads, max_ctx, kcv.page_tokens);
+  const FusedWs w = fused_ws_layout(kcb, batch, nkv, n_q_heads, gr.n_cta);
+  // every check before the first launch
+  if (!ws || ws_bytes < w.total) return fail(TQ_EINVAL, "tq_attend: workspace too small");
+  const int G = n_q_heads / nkv;
+  if (batch * nkv > 65535 || gr.lines > 65535 || gr.items > 0x7fffffffLL || gr.lines * 4 > 0x7fffffffLL)
+    return fail(TQ_EINVAL, "tq_attend: batch * heads * context too large");
+  tqd::AttendParams p;
+  p.kcv = kcv;
+  p.vcv = vcv;
+  int ps = 0;
+  while ((1 << ps) < kcv.page_tokens) ++ps;
+  p.page_shift = ps;
+  p.ctx_len = ctx_len;
+  p.n_kv_heads = nkv;
+  p.n_q_heads = n_q_heads;
+  p.G = G;
+  p.qtiles = (G + 3) / 4;
+  p.units = (int)gr.units;
+  p.max_ctx = (int)max_ctx;
+  p.n_cta = (int)gr.n_cta;
+  p.per_cta = (int)(gr.items / gr.n_cta);
+  p.extra = (int)(gr.items % gr.n_cta);
+  p.div_u = tqd::make_fastdiv((uint32_t)gr.units);
+  p.div_qtiles = tqd::make_fastdiv((uint32_t)p.qtiles);
+  p.div_kv = tqd::make_fastdiv((uint32_t)nkv);
+  p.sl2 = scale * 1.4426950408889634f;   // log2(e)
+  p.kt = key_tables(kcb);
+  {
+    const uint16_t* T = vcb->lay.bits == 4 ? vcb->mag16 : vcb->cent16;   // 8 entries
+    p.tlo0 = p.tlo1 = p.thi0 = p.thi1 = 0u;
+    for (int i = 0; i < 4; ++i) {
+      p.tlo0 |= (uint32_t)(T[i] & 0xFF) << (8 * i);
+      p.tlo1 |= (uint32_t)(T[4 + i] & 0xFF) << (8 * i);
+      p.thi0 |= (uint32_t)(T[i] >> 8) << (8 * i);
+      p.thi1 |= (uint32_t)(T[4 + i] >> 8) << (8 * i);
+    }
+  }
+  uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+  p.partial = reinterpret_cast<float*>(base + w.prep);
+  p.pi32 = vcb->pi32;
+  p.out = out;
+  p.d = kcb->lay.d;
+  const int kb = kcb->lay.bits;
+  if (kb < 1 || kb > 4 || vcb->lay.bits < 1 || vcb->lay.bits > 4) return fail(TQ_EUNSUPPORTED, "tq_attend: bits");
+  PreparedQueries pq;
+  tq_status s = launch_query_prep(kcb, q, dt, batch, nkv, n_q_heads, base, &pq, st);
+  if (s != TQ_OK) return s;
+  p.frag = pq.frag;
+  p.qfrag = pq.qfrag;
+  p.scal = pq.scal;
+  const int E = kcb->lay.E, F = kcb->lay.F, vb = vcb->lay.bits, lines = (int)gr.lines;
+  switch (kb) {
+    case 1: return launch_attend_fused_k1(p, vb, E, F, lines, st);
+    case 2: return launch_attend_fused_k2(p, vb, E, F, lines, st);
+    case 3: return launch_attend_fused_k3(p, vb, E, F, lines, st);
+    default: return launch_attend_fused_k4(p, vb, E, F, lines, st);
+  }
+}
+
 struct AttendWs {
   size_t scores, logits, values, total;
 };
@@ -146,23 +257,42 @@ static AttendWs attend_ws_layout(const tq_codebook* kcb, const tq_codebook* vcb,
 
 size_t attend_workspace(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch, int n_kv_heads,
                         int n_q_heads, int64_t max_ctx) {
-  return attend_ws_layout(kcb, vcb, batch, n_kv_heads, n_q_heads, max_ctx).total;
+  // the fused path needs equal page sizes, which only the call knows: the
+  // workspace covers both paths
+  size_t fused = 0;
+  if (kcb->lay.E <= 32 && kcb->lay.E == vcb->lay.E && batch > 0 && max_ctx > 0) {
+    size_t worst = 0;
+    for (int pt = 16; pt <= 1024; pt *= 2) {   // the grid grows as pages shrink
+      const AttendGrid gr = attend_grid(batch, n_kv_heads, n_q_heads, max_ctx, pt);
+      worst = std::max(worst, fused_ws_layout(kcb, batch, n_kv_heads, n_q_heads, gr.n_cta).total);
+    }
+    fused = worst;
+  }
+  return std::max(fused, attend_ws_layout(kcb, vcb, batch, n_kv_heads, n_q_heads, max_ctx).total);
 }
 
-tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,
-                        const void* q, tq_dtype dt, int64_t batch, int n_q_heads, const int32_t* ctx_len,
-                        int64_t max_ctx, float scale, float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+static tq_status launch_attend_composed(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb,
+                                        const CacheView& vcv, const void* q, tq_dtype dt, int64_t batch,
+                                        int n_q_heads, const int32_t* ctx_len, int64_t max_ctx, float scale,
+                                        float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
   const AttendWs w = attend_ws_layout(kcb, vcb, batch, kcv.n_kv_heads, n_q_heads, max_ctx);
   if (!ws || ws_bytes < w.total) return fail(TQ_EINVAL, "tq_attend: workspace too small");
   if (batch == 0) return TQ_OK;
+  // every check before the first launch
+  if (batch * n_q_heads > 0x7fffffffLL / tqd::kSmaxCluster || max_ctx > 0x7fff0000LL)
+    return fail(TQ_EINVAL, "tq_attend: batch * n_q_heads or max_ctx too large");
+  {
+    const int G = n_q_heads / kcv.n_kv_heads;
+    const int64_t groups = batch * kcv.n_kv_heads;
+    if (groups > 65535 || groups * ((G + 3) / 4) > 65535 || groups * ((G + 3) / 4) * 4 > 0x7fffffffLL)
+      return fail(TQ_EINVAL, "tq_attend: batch * n_kv_heads too large");
+  }
   uint8_t* base = reinterpret_cast<uint8_t*>(ws);
   float* scores = reinterpret_cast<float*>(base);
   if (max_ctx > 0) {
     tq_status s = launch_logits(kcb, kcv, q, dt, batch, n_q_heads, ctx_len, max_ctx, scores, max_ctx,
                                 base + w.scores, w.logits, st);
     if (s != TQ_OK) return s;
-    if (batch * n_q_heads > 0x7fffffffLL / tqd::kSmaxCluster || max_ctx > 0x7fff0000LL)
-      return fail(TQ_EINVAL, "tq_attend: batch * n_q_heads or max_ctx too large");
     tqd::softmax_rows_kernel<<<(unsigned)(batch * n_q_heads * tqd::kSmaxCluster), tqd::kSmaxThreads, 0, st>>>(
         scores, ctx_len, n_q_heads, max_ctx, (int)max_ctx, scale);
     cudaError_t e = cudaGetLastError();
@@ -172,6 +302,17 @@ tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_c
   // ctx_len is 0)
   return launch_values(vcb, vcv, scores, max_ctx, batch, n_q_heads, ctx_len, max_ctx, out, TQ_F32,
                        vcb->lay.d, base + w.scores + w.logits, w.values, st);
+}
+
+tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,
+                        const void* q, tq_dtype dt, int64_t batch, int n_q_heads, const int32_t* ctx_len,
+                        int64_t max_ctx, float scale, float* out, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (batch == 0) return TQ_OK;
+  if (max_ctx > 0 && fused_attend_ok(kcb, vcb, kcv.page_tokens, vcv.page_tokens))
+    return launch_attend_fused(kcb, kcv, vcb, vcv, q, dt, batch, n_q_heads, ctx_len, max_ctx, scale, out, ws,
+                               ws_bytes, st);
+  return launch_attend_composed(kcb, kcv, vcb, vcv, q, dt, batch, n_q_heads, ctx_len, max_ctx, scale, out, ws,
+                                ws_bytes, st);
 }
 
 }  // namespace tq

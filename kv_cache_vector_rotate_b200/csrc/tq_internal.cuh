@@ -134,6 +134,17 @@ tq_status launch_logits(const tq_codebook* cb, const CacheView& cv, const void* 
                         float* out, int64_t out_stride, void* ws, size_t ws_bytes,
                         cudaStream_t st);
 
+// The preparation kernel alone (query fragments for d <= 128, as the logits
+// kernel reads them), a programmatic dependent of the previous kernel.
+struct PreparedQueries {
+  const uint2* frag;
+  const uint2* qfrag;
+  const float2* scal;
+};
+size_t query_prep_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, int n_q_heads);
+tq_status launch_query_prep(const tq_codebook* cb, const void* q, tq_dtype dt, int64_t batch, int n_kv_heads,
+                            int n_q_heads, void* ws, PreparedQueries* pq, cudaStream_t st);
+
 size_t attend_workspace(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch, int n_kv_heads,
                         int n_q_heads, int64_t max_ctx);
 tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,

@@ -1,7 +1,7 @@
-"""GPU tests of tq_attend (logits, cluster row softmax, value pass) against the
-oracle's attention, and of what the value pass and tq_attend write for empty
-contexts and read past the context.  Collected after every other test file.
-"""
+"""GPU tests of tq_attend against the oracle's attention: the fused split-K
+path (d <= 128, equal page sizes) and the composed path (logits, cluster row
+softmax, value pass), full decode-step size, bad pages; and what the value
+pass and tq_attend write for empty contexts and read past the context."""
 
 import numpy as np
 import pytest
@@ -9,7 +9,7 @@ import pytest
 from kv_cache_vector_rotate_b200 import synth
 from oracle import tq_oracle as O
 from parity import VALUE_TOL
-from test_gpu_logits_values import _oracle_cache, _q_tensor
+from gpu_cases import _oracle_cache, _q_tensor
 
 pytestmark = pytest.mark.gpu
 
@@ -23,44 +23,130 @@ def tqm():
     return tqmod
 
 
-@pytest.mark.parametrize("kbits,m,vbits,pt", [(3, 128, 3, 32), (2, 128, 4, 32), (4, 0, 2, 32), (3, 128, 3, 16),
-                                              (3, 128, 3, 256)])
-def test_attend_matches_oracle_attention(tqm, kbits, m, vbits, pt):
-    """tq_attend (logits from the key codes, row softmax, values from their
-    codes) against the oracle's softmax attention given the same codes; a
-    sequence with an empty context gives a zero row.  The logit tolerance
-    (1e-3 of ||q|| ||k|| / sqrt(d)) moves the softmax weights by at most about
-    scale x that, so the output is checked to 2e-3 of its row scale."""
-    batch, heads, G, d = 3, 2, 4, 128
-    ctx = [700, 129, 0]
-    rng = np.random.default_rng(34 + kbits + vbits)
+def _attend_case(tqm, d, kbits, m, vbits, kpt, vpt, ctx, heads, G, seed, qdtype="bf16"):
+    """Both caches written by the oracle, tq_attend on the GPU, and the
+    oracle's softmax attention given the same codes.  The logit tolerance
+    (1e-3 of ||q|| ||k|| / sqrt(d)) moves the softmax weights by at most
+    about scale x that, so the output is checked to 2e-3 of its row scale."""
+    batch = len(ctx)
+    rng = np.random.default_rng(seed)
     keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-1, 1, size=(1, heads, 1, d)))
     vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
     kcodec = O.make_codec(d, kbits, m, synth.SEED_PI, synth.SEED_S)
     vcodec = O.make_codec(d, vbits, 0, synth.SEED_PI, synth.SEED_S)
-    kcb, kcache, kencs, _ = _oracle_cache(tqm, kcodec, O.Layout(d, kbits, m, pt, heads), keys, ctx, pt, 35)
-    vcb, vcache, vencs, _ = _oracle_cache(tqm, vcodec, O.Layout(d, vbits, 0, pt, heads), vals, ctx, pt, 36)
-    _, q = synth.to_bf16(rng.standard_normal((batch, heads * G, d)).astype(np.float32))
+    kcb, kcache, kencs, _ = _oracle_cache(tqm, kcodec, O.Layout(d, kbits, m, kpt, heads), keys, ctx, kpt, seed + 1)
+    vcb, vcache, vencs, _ = _oracle_cache(tqm, vcodec, O.Layout(d, vbits, 0, vpt, heads), vals, ctx, vpt, seed + 2)
+    qf = rng.standard_normal((batch, heads * G, d)).astype(np.float32)
+    q = synth.to_bf16(qf)[1] if qdtype == "bf16" else qf.astype(np.float64)
     ctx_t = torch.tensor(ctx, dtype=torch.int32, device="cuda")
     scale = 1.0 / np.sqrt(d)
-    out = tqm.attend(kcb, kcache, vcb, vcache, _q_tensor(q, "bf16"), ctx_t, max(ctx), scale=scale)
+    out = tqm.attend(kcb, kcache, vcb, vcache, _q_tensor(q, qdtype), ctx_t, max(ctx), scale=scale)
     torch.cuda.synchronize()
     O_gpu = out.cpu().numpy()
     for b in range(batch):
         for h in range(heads):
-            Qg = q[b, h * G:(h + 1) * G]
             if ctx[b] == 0:
                 assert not O_gpu[b, h * G:(h + 1) * G].any()
                 continue
-            _, ke = kencs[(b, h)]
-            _, ve = vencs[(b, h)]
-            o = O.attention_from_codes(kcodec, vcodec, Qg, (ke.idx, ke.qneg, ke.norm16, ke.rnorm16),
-                                       (ve.idx, ve.norm16), scale)
-            vh = O.dequantize(vcodec, ve.idx, ve.norm16)
-            row_scale = np.maximum(np.abs(o).max(axis=1), np.linalg.norm(vh, axis=1).mean() / np.sqrt(d))
-            err = np.abs(O_gpu[b, h * G:(h + 1) * G] - o).max(axis=1)
-            assert np.all(err <= 2e-3 * row_scale), (b, h, err / row_scale)
+            _check_attention(kcodec, vcodec, q[b, h * G:(h + 1) * G], kencs[(b, h)][1], vencs[(b, h)][1],
+                             scale, O_gpu[b, h * G:(h + 1) * G], (b, h))
     assert kcache.errors() == 0 and vcache.errors() == 0
+
+
+def _check_attention(kcodec, vcodec, Qg, ke, ve, scale, got, where, keep=None):
+    if keep is not None:
+        ke = O.Encoded(*(None if x is None else np.asarray(x)[keep] for x in
+                         (ke.idx, ke.qneg, ke.norm16, ke.rnorm16, ke.y, ke.proj)))
+        ve = O.Encoded(*(None if x is None else np.asarray(x)[keep] for x in
+                         (ve.idx, ve.qneg, ve.norm16, ve.rnorm16, ve.y, ve.proj)))
+    o = O.attention_from_codes(kcodec, vcodec, Qg, (ke.idx, ke.qneg, ke.norm16, ke.rnorm16),
+                               (ve.idx, ve.norm16), scale)
+    vh = O.dequantize(vcodec, ve.idx, ve.norm16)
+    row_scale = np.maximum(np.abs(o).max(axis=1), np.linalg.norm(vh, axis=1).mean() / np.sqrt(kcodec.d))
+    err = np.abs(got - o).max(axis=1)
+    assert np.all(err <= 2e-3 * row_scale), (where, err / row_scale)
+
+
+# The fused split-K path: d <= 128 and equal page sizes.  Contexts of 700
+# (ragged last unit), 129 (one token past two units) and 0 (a zero row);
+# 16-token pages (units straddle pages), 256-token pages (several units per
+# page); GQA groups of 1, 2, 4 and 8 query heads (two query tiles).
+@pytest.mark.parametrize("d,kbits,m,vbits,pt,G", [
+    (128, 3, 128, 3, 32, 4), (128, 2, 128, 4, 32, 4), (128, 4, 0, 2, 32, 4), (128, 3, 128, 3, 16, 4),
+    (128, 3, 128, 3, 256, 4), (128, 3, 128, 3, 64, 8), (64, 2, 64, 2, 64, 4), (96, 3, 96, 3, 64, 2),
+    (128, 1, 128, 1, 128, 1), (64, 4, 0, 4, 16, 4)])
+def test_attend_matches_oracle_attention(tqm, d, kbits, m, vbits, pt, G):
+    _attend_case(tqm, d, kbits, m, vbits, pt, pt, [700, 129, 0], 2, G, 34 + kbits + vbits + G)
+
+
+# The composed path (logits, row softmax, value pass): d > 128, or key and
+# value caches with different page sizes.
+@pytest.mark.parametrize("d,kpt,vpt", [(200, 64, 64), (256, 32, 32), (128, 32, 64)])
+def test_attend_composed_path_matches_oracle(tqm, d, kpt, vpt):
+    _attend_case(tqm, d, 3, d, 3, kpt, vpt, [700, 129, 0], 2, 4, 60 + d)
+
+
+def test_attend_many_units_per_cta(tqm):
+    """Two sequences x 8 KV heads x 32 query heads at 8192 / 7777 tokens: CTAs
+    with many units, shares that span two lines (the consumer warps split
+    between them), refills of every ring slot."""
+    _attend_case(tqm, 128, 3, 128, 3, 64, 64, [8192, 7777], 8, 4, 61)
+
+
+def test_attend_decode_config_full_size(tqm):
+    """The decode step at full size (batch 1, 8 KV / 32 query heads, d 128,
+    context 32768, keys b = 3 + QJL m = 128, values b = 3) with the bench's
+    inputs, against the oracle on every head."""
+    batch, hkv, hq, ctx, d, pt = 1, 8, 32, 32768, 128, 64
+    data = synth.decode_step(1002, batch, hkv, hq, ctx, d)
+    kcodec = O.make_codec(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    vcodec = O.make_codec(d, 3, 0, synth.SEED_PI, synth.SEED_S)
+    kcb, kcache, kencs, _ = _oracle_cache(tqm, kcodec, O.Layout(d, 3, 128, pt, hkv), data["k"][1], [ctx], pt, 24)
+    vcb, vcache, vencs, _ = _oracle_cache(tqm, vcodec, O.Layout(d, 3, 0, pt, hkv), data["v"][1], [ctx], pt, 25)
+    qbits, q = data["q"]
+    qt = torch.from_numpy(qbits.view(np.int16)).view(torch.bfloat16).cuda()
+    scale = 1.0 / np.sqrt(d)
+    out = tqm.attend(kcb, kcache, vcb, vcache, qt, torch.tensor([ctx], dtype=torch.int32, device="cuda"), ctx,
+                     scale=scale)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    G = hq // hkv
+    for h in range(hkv):
+        _check_attention(kcodec, vcodec, q[0, h * G:(h + 1) * G], kencs[(0, h)][1], vencs[(0, h)][1], scale,
+                         got[0, h * G:(h + 1) * G], h)
+    assert kcache.errors() == 0 and vcache.errors() == 0
+
+
+@pytest.mark.parametrize("which", ["key", "value"])
+def test_attend_bad_page_is_skipped_and_reported(tqm, which):
+    """A block-table entry out of range inside the context: the call
+    completes, the cache's error word has the page bit, and the tokens of
+    that page leave the softmax (the rest match the oracle's attention over
+    the remaining tokens)."""
+    d, pt, heads, G, ctx = 128, 32, 2, 4, [2048]
+    rng = np.random.default_rng(62)
+    keys = rng.standard_normal((1, heads, ctx[0], d))
+    vals = rng.standard_normal((1, heads, ctx[0], d)) * 2.0
+    kcodec = O.make_codec(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    vcodec = O.make_codec(d, 3, 0, synth.SEED_PI, synth.SEED_S)
+    kcb, kcache, kencs, kbt = _oracle_cache(tqm, kcodec, O.Layout(d, 3, 128, pt, heads), keys, ctx, pt, 63)
+    vcb, vcache, vencs, vbt = _oracle_cache(tqm, vcodec, O.Layout(d, 3, 0, pt, heads), vals, ctx, pt, 63)
+    cache = kcache if which == "key" else vcache
+    bad_page = 17
+    cache.block_table[0, bad_page] = 10 ** 6
+    qf = rng.standard_normal((1, heads * G, d)).astype(np.float32)
+    q = synth.to_bf16(qf)[1]
+    scale = 1.0 / np.sqrt(d)
+    out = tqm.attend(kcb, kcache, vcb, vcache, _q_tensor(q, "bf16"), torch.tensor(ctx, dtype=torch.int32,
+                     device="cuda"), ctx[0], scale=scale)
+    torch.cuda.synchronize()
+    assert cache.errors() & tqm.DEV_ERR_PAGE
+    got = out.cpu().numpy()
+    pos = np.arange(ctx[0])
+    keep = (pos // pt) != bad_page
+    for h in range(heads):
+        _check_attention(kcodec, vcodec, q[0, h * G:(h + 1) * G], kencs[(0, h)][1], vencs[(0, h)][1], scale,
+                         got[0, h * G:(h + 1) * G], h, keep=keep)
 
 def test_attend_with_no_context_clears_out(tqm):
     """max_ctx = 0: every context is empty, so tq_attend writes zero rows over
