@@ -239,7 +239,8 @@ tq_status tq_dequant_values(const tq_codebook* cb, const tq_cache* cache,
                             void* out, tq_dtype out_dtype, int64_t out_stride,
                             void* workspace, size_t workspace_bytes, void* stream);
 
-/* Workspace (device bytes) that tq_attend needs for these sizes. */
+/* Workspace (device bytes) that tq_attend needs for these sizes (either of
+ * its two forms; the page sizes, which choose the form, are not arguments). */
 size_t tq_attend_workspace_bytes(const tq_codebook* key_cb, const tq_codebook* value_cb, int64_t batch,
                                  int32_t n_kv_heads, int32_t n_q_heads, int64_t max_ctx);
 
@@ -254,9 +255,13 @@ size_t tq_attend_workspace_bytes(const tq_codebook* key_cb, const tq_codebook* v
  * tq_dequant_values (same d and n_kv_heads; value_cb has m = 0).  q: device
  * [batch, n_q_heads, d] of dtype; out: device fp32 [batch, n_q_heads, d];
  * scale: usually 1/sqrt(d).  workspace: device, at least
- * tq_attend_workspace_bytes(), 256-byte aligned (the scores, then the
- * workspaces of the two passes).  Four kernel launches on the stream: query
- * preparation, logits, row softmax, value accumulation (+ its finish). */
+ * tq_attend_workspace_bytes(), 256-byte aligned.  A token whose key or value
+ * page is out of range is left out of the softmax (and reported in that
+ * cache's error word).  Kernels on the stream: for d <= 128 and caches with
+ * equal page sizes, the fused split-K form (query preparation, one pass over
+ * both caches with an online softmax writing per-CTA partials, a merge that
+ * applies Pi_v^T); otherwise query preparation, logits, row softmax, value
+ * accumulation and its finish. */
 tq_status tq_attend(const tq_codebook* key_cb, const tq_cache* key_cache, const tq_codebook* value_cb,
                     const tq_cache* value_cache, const void* q, tq_dtype dtype, int64_t batch,
                     int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx, float scale, float* out,

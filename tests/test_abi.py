@@ -92,17 +92,26 @@ def test_reconstruction_levels_match_oracle_for_every_supported_d(bits):
         assert np.array_equal(lev, ref), d
 
 
-def test_attend_workspace_is_scores_plus_both_passes():
-    # tq_attend's workspace: fp32 scores [batch, n_q_heads, max_ctx], then the
-    # logits and values workspaces, each rounded up to 256 bytes.
+def test_attend_workspace_covers_both_paths():
+    # tq_attend's workspace covers its two paths (the page sizes, which pick
+    # the path, are not arguments): the composed path's fp32 scores [batch,
+    # n_q_heads, max_ctx] then the logits and values workspaces, and the
+    # fused path's query fragments then fp32 partials [n_cta][2][4][4E + 2],
+    # n_cta = the largest grid over page sizes 16 .. 1024 (CTAs: at least one
+    # per SM -- 148 without a GPU -- and per line, at most 127 units each for
+    # 16-token pages, at most one per unit); each part rounded up to 256 bytes.
     kcb = tq.Codebook(128, 3, 128, 1, 2, device=False)
     vcb = tq.Codebook(128, 3, 0, 3, 4, device=False)
     lib = tq.load_library()
     al = lambda n: (n + 255) // 256 * 256
-    for batch, hkv, hq, ctx in [(1, 8, 32, 32768), (3, 2, 8, 700), (2, 4, 4, 17)]:
-        want = (al(batch * hq * ctx * 4) + al(lib.tq_logits_workspace_bytes(kcb.handle, batch, hkv, hq))
-                + al(lib.tq_values_workspace_bytes(vcb.handle, batch, hkv, hq, ctx)))
-        assert lib.tq_attend_workspace_bytes(kcb.handle, vcb.handle, batch, hkv, hq, ctx) == want
+    for batch, hkv, hq, ctx in [(1, 8, 32, 32768), (3, 2, 8, 700), (2, 4, 4, 17), (1, 1, 4, 10 ** 6)]:
+        composed = (al(batch * hq * ctx * 4) + al(lib.tq_logits_workspace_bytes(kcb.handle, batch, hkv, hq))
+                    + al(lib.tq_values_workspace_bytes(vcb.handle, batch, hkv, hq, ctx)))
+        lines = batch * hkv * ((hq // hkv + 3) // 4)
+        items = lines * ((ctx + 63) // 64)
+        n_cta = max(1, min(max(148, lines, -(-items // 127)), items))
+        fused = al(lib.tq_logits_workspace_bytes(kcb.handle, batch, hkv, hq)) + al(n_cta * 2 * 4 * 130 * 4)
+        assert lib.tq_attend_workspace_bytes(kcb.handle, vcb.handle, batch, hkv, hq, ctx) == max(composed, fused)
     for args in [(1, 8, 30, 64), (1, 0, 8, 64), (-1, 2, 8, 64), (1, 2, 8, -1)]:
         assert lib.tq_attend_workspace_bytes(kcb.handle, vcb.handle, *args) == 0
     assert lib.tq_attend_workspace_bytes(None, vcb.handle, 1, 2, 8, 64) == 0
