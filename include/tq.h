@@ -195,6 +195,34 @@ tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
                     int64_t out_stride, void* workspace, size_t workspace_bytes,
                     void* stream);
 
+/* Workspace (device bytes) that tq_logits_topk needs for these sizes (0 for
+ * bad arguments, k outside [1, 32]). */
+size_t tq_logits_topk_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                      int32_t n_q_heads, int64_t max_ctx, int32_t k);
+
+/* The k best logits per query head (TQ §Benchmarks: nearest-neighbour search
+ * scored from the codes, top-k recall; the estimate is tq_logits'): for query
+ * head hq of sequence b, the k largest L[b, hq, t] over t < ctx_len[b], best
+ * first, equal scores in increasing t:
+ *   top_scores[(b * n_q_heads + hq) * k + j], top_idx[...] = t
+ * (score -inf and index -1 past the ctx_len[b] found).  Meant for many query
+ * heads per KV head (queries are taken 64 at a time): the codes of 128 keys
+ * are decoded once per 64 queries into tensor memory and scored against them
+ * on the tcgen05 tensor cores, and the epilogue keeps each query's best k.
+ * The scores equal tq_logits' estimate up to fp32 rounding (the query enters
+ * as fp16 hi + lo for the codebook term and fp16 for the sketch term); ties
+ * between scores that differ by rounding may rank either way.  q: device
+ * [batch, n_q_heads, d] of dtype; ctx_len: device int32 [batch]; top_scores /
+ * top_idx: device [batch, n_q_heads, k]; k in [1, 32]; pages of at least 16
+ * tokens (TQ_EUNSUPPORTED otherwise).  workspace: device, at least
+ * tq_logits_topk_workspace_bytes(), 256-byte aligned.  Three kernel launches
+ * (query operands, scoring, merge of the CTAs' lists); a bad page is
+ * reported in the cache's error word and its keys are not ranked. */
+tq_status tq_logits_topk(const tq_codebook* cb, const tq_cache* cache, const void* q, tq_dtype dtype,
+                         int64_t batch, int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx, int32_t k,
+                         float* top_scores, int32_t* top_idx, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
 /* tq_logits for callers that cannot allocate device memory where they call
  * it (a serving loop whose memory is an arena carved up at start-up, a host
  * framework or plugin interface that hands an operator no workspace, code

@@ -442,6 +442,50 @@ tq_status tq_logits(const tq_codebook* cb, const tq_cache* cache, const void* q,
                        workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t tq_logits_topk_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
+                                      int32_t n_q_heads, int64_t max_ctx, int32_t k) {
+  if (!cb || batch < 0 || max_ctx < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads ||
+      k < 1 || k > 32)
+    return 0;
+  return search_workspace(cb, batch, n_kv_heads, n_q_heads, max_ctx, k);
+}
+
+tq_status tq_logits_topk(const tq_codebook* cb, const tq_cache* cache, const void* q, tq_dtype dtype,
+                         int64_t batch, int32_t n_q_heads, const int32_t* ctx_len, int64_t max_ctx, int32_t k,
+                         float* top_scores, int32_t* top_idx, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  tq_status s = check_cb(cb);
+  if (s != TQ_OK) return s;
+  CacheView cv;
+  s = make_view(cb, cache, &cv);
+  if (s != TQ_OK) return s;
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_logits_topk: bad dtype");
+  if (batch < 0 || max_ctx < 0 || max_ctx > INT32_MAX) return fail(TQ_EINVAL, "tq_logits_topk: bad size");
+  if (k < 1 || k > 32) return fail(TQ_EINVAL, "tq_logits_topk: k must be in [1, 32]");
+  if (n_q_heads < cv.n_kv_heads || n_q_heads % cv.n_kv_heads)
+    return fail(TQ_EINVAL, "tq_logits_topk: n_q_heads must be a multiple of the cache's n_kv_heads");
+  if (max_ctx > cv.max_pages * cv.page_tokens)
+    return fail(TQ_EINVAL, "tq_logits_topk: max_ctx exceeds the block table");
+  if (cv.page_tokens < 16) return fail(TQ_EUNSUPPORTED, "tq_logits_topk: pages of fewer than 16 tokens");
+  if (batch == 0) return TQ_OK;
+  if (!top_scores || !top_idx) return fail(TQ_EINVAL, "tq_logits_topk: NULL pointer");
+  if (!aligned(top_scores, 4) || !aligned(top_idx, 4)) return fail(TQ_EINVAL, "tq_logits_topk: misaligned pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (max_ctx == 0) {   // nothing to rank: every entry is (-inf, -1)
+    const size_t n = (size_t)batch * n_q_heads * k;
+    std::vector<float> hs(n, -INFINITY);
+    s = cuda_fail(cudaMemsetAsync(top_idx, 0xFF, n * sizeof(int32_t), st), "tq_logits_topk: clearing idx");
+    if (s != TQ_OK) return s;
+    return cuda_fail(cudaMemcpyAsync(top_scores, hs.data(), n * sizeof(float), cudaMemcpyHostToDevice, st),
+                     "tq_logits_topk: clearing scores");
+  }
+  if (!q || !ctx_len || !workspace) return fail(TQ_EINVAL, "tq_logits_topk: NULL pointer");
+  if (!aligned(q, dtype_size(dtype)) || !aligned(workspace, 256) || !aligned(ctx_len, 4))
+    return fail(TQ_EINVAL, "tq_logits_topk: misaligned pointer");
+  return launch_search(cb, cv, q, dtype, batch, n_q_heads, ctx_len, max_ctx, k, top_scores, top_idx, workspace,
+                       workspace_bytes, st);
+}
+
 size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
                                  int32_t n_q_heads, int64_t max_ctx) {
   if (!cb || batch < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)

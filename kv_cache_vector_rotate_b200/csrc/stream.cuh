@@ -58,6 +58,20 @@ __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity, u
       : "=r"(done) : "r"(smem_addr(bar)), "r"(parity), "r"(ns) : "memory");
   return done != 0;
 }
+// mbar_wait for waits that may be long: between tests the warp sleeps
+// (32 ns, doubling to `max_ns`) and leaves the issue slots to working warps;
+// false after kWaitCycles.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, uint32_t max_ns = 256u) {
+  if (mbar_test(bar, parity)) return true;
+  const long long t0 = clock64();
+  uint32_t ns = 32u;
+  while (true) {
+    __nanosleep(ns);
+    if (mbar_test(bar, parity)) return true;
+    if (clock64() - t0 > kWaitCycles) return false;
+    ns = ns < max_ns ? 2u * ns : max_ns;
+  }
+}
 // mbar_wait with sleeping tests; false after kWaitCycles.
 __device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
   if (mbar_try_sleep(bar, parity, 20000u)) return true;

@@ -145,6 +145,12 @@ size_t query_prep_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads
 tq_status launch_query_prep(const tq_codebook* cb, const void* q, tq_dtype dt, int64_t batch, int n_kv_heads,
                             int n_q_heads, void* ws, PreparedQueries* pq, cudaStream_t st);
 
+size_t search_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, int n_q_heads, int64_t max_ctx,
+                        int k);
+tq_status launch_search(const tq_codebook* cb, const CacheView& cv, const void* q, tq_dtype dt, int64_t batch,
+                        int n_q_heads, const int32_t* ctx_len, int64_t max_ctx, int k, float* out_score,
+                        int32_t* out_idx, void* ws, size_t ws_bytes, cudaStream_t st);
+
 size_t attend_workspace(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch, int n_kv_heads,
                         int n_q_heads, int64_t max_ctx);
 tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,

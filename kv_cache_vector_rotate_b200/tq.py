@@ -25,6 +25,7 @@ EXPORTS = (
     "tq_layout", "tq_quantize_append", "tq_logits_workspace_bytes", "tq_logits",
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
+    "tq_logits_topk_workspace_bytes", "tq_logits_topk",
     "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook", "tq_codebook_levels",
 )
 
@@ -82,6 +83,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                     vp, i32, i64, vp, sz, vp]),
         "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
         "tq_logits_noalloc_scratch_bytes": (sz, []),
+        "tq_logits_topk_workspace_bytes": (sz, [vp, i64, i32, i32, i64, i32]),
+        "tq_logits_topk": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, i32, vp, vp, vp, sz,
+                                 vp]),
         "tq_selftest_wait_timeout": (i32, [vp, vp]),
         "tq_attend_workspace_bytes": (sz, [vp, vp, i64, i32, i32, i64]),
         "tq_attend": (i32, [vp, ctypes.POINTER(CacheStruct), vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32,
@@ -233,6 +237,31 @@ def logits(cb: Codebook, cache: PagedCache, q, ctx_len, max_ctx: int, out=None, 
                                      _ptr(ctx_len), max_ctx, _ptr(out), out.stride(1),
                                      _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
+
+
+def logits_topk_workspace_bytes(cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int, max_ctx: int,
+                                k: int) -> int:
+    return int(load_library().tq_logits_topk_workspace_bytes(cb.handle, batch, n_kv_heads, n_q_heads, max_ctx, k))
+
+
+def logits_topk(cb: Codebook, cache: PagedCache, q, ctx_len, max_ctx: int, k: int, scores=None, idx=None,
+                workspace=None, stream=None):
+    """tq_logits_topk: q [batch, n_q_heads, d] -> (scores fp32, idx int32), each [batch, n_q_heads, k]."""
+    import torch
+    assert q.is_cuda and q.is_contiguous() and q.dim() == 3
+    b, hq, d = q.shape
+    if scores is None:
+        scores = torch.empty(b, hq, k, dtype=torch.float32, device=q.device)
+    if idx is None:
+        idx = torch.empty(b, hq, k, dtype=torch.int32, device=q.device)
+    if workspace is None:
+        n = logits_topk_workspace_bytes(cb, b, cache.n_kv_heads, hq, max_ctx, k)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    cs = cache.struct()
+    _check(load_library().tq_logits_topk(cb.handle, ctypes.byref(cs), _ptr(q), _dtype_code(q), b, hq,
+                                          _ptr(ctx_len), max_ctx, k, _ptr(scores), _ptr(idx),
+                                          _ptr(workspace), workspace.numel(), _stream(stream)))
+    return scores, idx
 
 
 def values_workspace_bytes(cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int, max_ctx: int) -> int:
