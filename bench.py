@@ -432,6 +432,50 @@ def vector_search_phase(dev, n: int = 1_000_000, nq: int = 1000, d: int = 200, k
     return out
 
 
+def polar_phase(dev, n: int = 262144, nq: int = 4, d: int = 128, bits: int = 3, m: int = 128, reps: int = 5):
+    """The recursive polar form of stage 1 on the decode step's keys (8 KV heads
+    x 32768 keys = 262144 bf16 vectors of the decode-step law, d = 128, 3-bit
+    angles, QJL m = 128): tq_polar_encode keys/s, and tq_polar_logits for a GQA
+    group of 4 queries against every record.  The logit path is bound by the
+    FMA pipe: 2 (d - 1) + m FMAs per (key, query); the fraction is of the fp32
+    FMA peak of 148 SMs x 128 lanes x 2 flop at the clock sampled during the
+    run (sm_max_mhz when none).  Median of `reps` event-timed calls after a
+    warm-up."""
+    import torch
+
+    from kv_cache_vector_rotate_b200 import synth, tq
+    K, q = synth.decode_keys_device(1002, 1, 8, 32, n // 8, d)
+    X = K.reshape(n, d).contiguous()
+    Q = q[0, :nq].contiguous()
+    pc = tq.PolarCodec(d, bits, m, synth.SEED_PI, synth.SEED_S)
+    rec = tq.polar_encode(pc, X)
+    out = torch.empty(nq, n, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, nq * (d + m) * 4), dtype=torch.uint8, device=dev)
+    tq.polar_logits(pc, rec, Q, out=out, workspace=ws)
+    torch.cuda.synchronize()
+
+    def med(fn):
+        ts = []
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return float(np.median(ts))
+
+    enc_ms = med(lambda: tq.polar_encode(pc, X, records=rec))
+    log_ms = med(lambda: tq.polar_logits(pc, rec, Q, out=out, workspace=ws))
+    fmas = float(n) * nq * (2 * (d - 1) + m)
+    bytes_ = float(n) * pc.record_bytes + nq * n * 4 + nq * d * 2
+    pc.close()
+    return {"workload": f"{n} bf16 keys d={d} (decode-step law), {bits}-bit angles, QJL m={m}; {nq} queries",
+            "record_bytes": pc.record_bytes, "encode_ms": enc_ms, "encode_keys_per_s": n / (enc_ms * 1e-3),
+            "logits_ms": log_ms, "logits_gbs": bytes_ / (log_ms * 1e-3) / 1e9,
+            "logits_fma_tflops": 2.0 * fmas / (log_ms * 1e-3) / 1e12, "fmas_per_key_query": 2 * (d - 1) + m}
+
+
 def profile_phase(args):
     """Sets up one workload and makes three eager calls of one entry point, for
     ncu captures (no timing, no JSON line):
@@ -661,6 +705,8 @@ def run_ours(args):
     vs = None
     if not args.no_search:
         vs = vector_search_phase(dev)
+    # the recursive polar form on the decode step's keys
+    pol = polar_phase(dev)
 
     n = ws
     steps = args.steps
@@ -699,6 +745,12 @@ def run_ours(args):
         line["key_codecs"] = bud
     if vs is not None:
         line["vector_search"] = vs
+    sm_mhz = line.get("clocks", {}).get("sm_mhz") or line.get("clocks", {}).get("sm_max_mhz") or 1965.0
+    pol["fma_peak_tflops"] = 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+    pol["roofline"] = {"bound": "alu", "achieved": pol["logits_fma_tflops"], "peak": pol["fma_peak_tflops"],
+                       "unit": "TFLOP/s", "frac": pol["logits_fma_tflops"] / pol["fma_peak_tflops"],
+                       "peak_source": "fp32 FMA: 148 SMs x 128 lanes x 2 flop x sampled SM clock"}
+    line["polar"] = pol
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     if rank == 0:

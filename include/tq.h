@@ -317,6 +317,53 @@ tq_status tq_selftest_wait_timeout(uint32_t* error_word, void* stream);
 tq_status tq_polar_angle_codebook(int32_t level, int32_t bits, double* centroids, double* boundaries,
                                   double* distortion);
 
+/* ---- the recursive polar form of stage 1 ("TurboQuant explained", §Stage 1,
+ * PolarQuant paragraph; §Stage 2 on top) ------------------------------------
+ * The rotated unit vector u = Pi x / ||x|| is paired recursively into polar
+ * form: level 1 angles atan2(u[2i+1], u[2i]) in [-pi, pi], level l > 1 angles
+ * atan2(rho[2i+1], rho[2i]) in [0, pi/2] of the previous level's radii, d - 1
+ * angles in all (d a power of two).  Each angle is coded with `bits` bits by
+ * the Lloyd-Max quantizer of its level's law (tq_polar_angle_codebook; a tie
+ * goes to the upper cell); ||x|| is kept in fp16.  With m > 0 the residual
+ * r = u - Pi^T u_hat (original space, u_hat the inverse recursion over the
+ * centroids) keeps the m signs of S r and fp16 ||r||.  Pi and S come from the
+ * same seeds and generators as tq_codebook_build's.  The records are a plain
+ * array (no pages):
+ *   words [0, CW): angle codes, CW = ceil((d - 1) bits / 32), angle a (level 1
+ *                  first, then by index) at bits a bits .. of the little-endian
+ *                  word stream;
+ *   words [CW, CW + m/32): sign bits, bit i set where (S r)_i < 0;
+ *   word CW + m/32: fp16 ||x|| (low half), fp16 ||r|| (high half, 0 when m = 0);
+ *   padded to tq_polar_record_bytes() (a multiple of 16). */
+typedef struct tq_polar tq_polar;
+
+/* Builds the polar codec (host float64 tables, device fp32 copies).  d in {64,
+ * 128, 256}, bits in [1, 4], m a multiple of 32 in [0, d] (TQ_EUNSUPPORTED
+ * otherwise); needs a CUDA device.  Free with tq_polar_free. */
+tq_status tq_polar_build(int32_t d, int32_t bits, int32_t m, uint64_t seed_pi, uint64_t seed_s, tq_polar** out);
+void tq_polar_free(tq_polar* p);
+/* Bytes of one record (0 for NULL). */
+int32_t tq_polar_record_bytes(const tq_polar* p);
+
+/* Encodes x (device [n, d] of dtype) into records (device [n] records,
+ * 16-byte aligned).  A norm that overflows fp16 sets TQ_DEV_ERR_RANGE in
+ * *error_word (device uint32, may be NULL).  One kernel launch. */
+tq_status tq_polar_encode(const tq_polar* p, const void* x, tq_dtype dtype, int64_t n, void* records,
+                          uint32_t* error_word, void* stream);
+
+/* Workspace (device bytes) of tq_polar_logits for nq queries. */
+size_t tq_polar_logits_workspace_bytes(const tq_polar* p, int32_t nq);
+
+/* Logits from the polar records without reconstructing the keys:
+ *   out[j * out_stride + t] = ||x_t|| ( <Pi q_j, u_hat_t> + sqrt(pi/2)/m ||r_t|| <S q_j, sign_t> )
+ * for every query j < nq (device [nq, d] of dtype) and record t < n; the first
+ * term folds the rotated query bottom-up through the angle tree (2 (d - 1)
+ * FMAs per key and query).  workspace: device, at least
+ * tq_polar_logits_workspace_bytes(), 16-byte aligned.  Two kernel launches. */
+tq_status tq_polar_logits(const tq_polar* p, const void* records, int64_t n, const void* q, tq_dtype dtype,
+                          int32_t nq, float* out, int64_t out_stride, void* workspace, size_t workspace_bytes,
+                          void* stream);
+
 /* Message for the last failed call on this thread ("" if none). */
 const char* tq_last_error(void);
 

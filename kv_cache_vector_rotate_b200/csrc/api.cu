@@ -486,6 +486,55 @@ tq_status tq_logits_topk(const tq_codebook* cb, const tq_cache* cache, const voi
                        workspace_bytes, st);
 }
 
+tq_status tq_polar_build(int32_t d, int32_t bits, int32_t m, uint64_t seed_pi, uint64_t seed_s, tq_polar** out) {
+  if (!out) return fail(TQ_EINVAL, "tq_polar_build: out is NULL");
+  *out = nullptr;
+  if (d != 64 && d != 128 && d != 256) return fail(TQ_EUNSUPPORTED, "tq_polar_build: d must be 64, 128 or 256");
+  if (bits < 1 || bits > 4) return fail(TQ_EUNSUPPORTED, "tq_polar_build: bits must be in [1, 4]");
+  if (m < 0 || m > d || m % 32) return fail(TQ_EUNSUPPORTED, "tq_polar_build: m must be a multiple of 32 in [0, d]");
+  int n_dev = 0;
+  if (cudaGetDeviceCount(&n_dev) != cudaSuccess || n_dev == 0) {
+    (void)cudaGetLastError();
+    return fail(TQ_ECUDA, "tq_polar_build: no CUDA device");
+  }
+  return polar_build(d, bits, m, seed_pi, seed_s, out);
+}
+
+void tq_polar_free(tq_polar* p) { polar_free(p); }
+
+int32_t tq_polar_record_bytes(const tq_polar* p) { return p ? polar_record_bytes(p) : 0; }
+
+tq_status tq_polar_encode(const tq_polar* p, const void* x, tq_dtype dtype, int64_t n, void* records,
+                          uint32_t* error_word, void* stream) {
+  if (!p) return fail(TQ_EINVAL, "tq_polar_encode: codec is NULL");
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_polar_encode: bad dtype");
+  if (n < 0) return fail(TQ_EINVAL, "tq_polar_encode: n < 0");
+  if (n == 0) return TQ_OK;
+  if (!x || !records) return fail(TQ_EINVAL, "tq_polar_encode: NULL pointer");
+  if (!aligned(x, dtype_size(dtype)) || !aligned(records, 16) || (error_word && !aligned(error_word, 4)))
+    return fail(TQ_EINVAL, "tq_polar_encode: misaligned pointer");
+  return polar_encode(p, x, dtype, n, records, error_word, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tq_polar_logits_workspace_bytes(const tq_polar* p, int32_t nq) {
+  if (!p || nq < 0) return 0;
+  return polar_logits_workspace(p, nq);
+}
+
+tq_status tq_polar_logits(const tq_polar* p, const void* records, int64_t n, const void* q, tq_dtype dtype,
+                          int32_t nq, float* out, int64_t out_stride, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  if (!p) return fail(TQ_EINVAL, "tq_polar_logits: codec is NULL");
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_polar_logits: bad dtype");
+  if (n < 0 || nq < 0 || out_stride < n) return fail(TQ_EINVAL, "tq_polar_logits: bad size");
+  if (n == 0 || nq == 0) return TQ_OK;
+  if (!records || !q || !out || !workspace) return fail(TQ_EINVAL, "tq_polar_logits: NULL pointer");
+  if (!aligned(records, 16) || !aligned(q, dtype_size(dtype)) || !aligned(out, 4) || !aligned(workspace, 16))
+    return fail(TQ_EINVAL, "tq_polar_logits: misaligned pointer");
+  return polar_logits(p, records, n, q, dtype, nq, out, out_stride, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
                                  int32_t n_q_heads, int64_t max_ctx) {
   if (!cb || batch < 0 || n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)

@@ -151,6 +151,15 @@ tq_status launch_search(const tq_codebook* cb, const CacheView& cv, const void* 
                         int n_q_heads, const int32_t* ctx_len, int64_t max_ctx, int k, float* out_score,
                         int32_t* out_idx, void* ws, size_t ws_bytes, cudaStream_t st);
 
+tq_status polar_build(int d, int bits, int m, uint64_t seed_pi, uint64_t seed_s, tq_polar** out);
+void polar_free(tq_polar* P);
+tq_status polar_encode(const tq_polar* P, const void* x, tq_dtype dt, int64_t n, void* rec, uint32_t* err,
+                       cudaStream_t st);
+size_t polar_logits_workspace(const tq_polar* P, int nq);
+tq_status polar_logits(const tq_polar* P, const void* rec, int64_t n, const void* q, tq_dtype dt, int nq, float* out,
+                       int64_t out_stride, void* ws, size_t ws_bytes, cudaStream_t st);
+int polar_record_bytes(const tq_polar* P);
+
 size_t attend_workspace(const tq_codebook* kcb, const tq_codebook* vcb, int64_t batch, int n_kv_heads,
                         int n_q_heads, int64_t max_ctx);
 tq_status launch_attend(const tq_codebook* kcb, const CacheView& kcv, const tq_codebook* vcb, const CacheView& vcv,

@@ -26,6 +26,8 @@ EXPORTS = (
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
     "tq_logits_topk_workspace_bytes", "tq_logits_topk",
+    "tq_polar_build", "tq_polar_free", "tq_polar_record_bytes", "tq_polar_encode",
+    "tq_polar_logits_workspace_bytes", "tq_polar_logits",
     "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook", "tq_codebook_levels",
 )
 
@@ -84,6 +86,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
         "tq_logits_noalloc_scratch_bytes": (sz, []),
         "tq_logits_topk_workspace_bytes": (sz, [vp, i64, i32, i32, i64, i32]),
+        "tq_polar_build": (i32, [i32, i32, i32, ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(vp)]),
+        "tq_polar_free": (None, [vp]),
+        "tq_polar_record_bytes": (i32, [vp]),
+        "tq_polar_encode": (i32, [vp, vp, i32, i64, vp, vp, vp]),
+        "tq_polar_logits_workspace_bytes": (sz, [vp, i32]),
+        "tq_polar_logits": (i32, [vp, vp, i64, vp, i32, i32, vp, i64, vp, sz, vp]),
         "tq_logits_topk": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, i32, vp, vp, vp, sz,
                                  vp]),
         "tq_selftest_wait_timeout": (i32, [vp, vp]),
@@ -262,6 +270,56 @@ def logits_topk(cb: Codebook, cache: PagedCache, q, ctx_len, max_ctx: int, k: in
                                           _ptr(ctx_len), max_ctx, k, _ptr(scores), _ptr(idx),
                                           _ptr(workspace), workspace.numel(), _stream(stream)))
     return scores, idx
+
+
+class PolarCodec:
+    """Handle of tq_polar: the recursive polar form of stage 1 for (d, bits, m)."""
+
+    def __init__(self, d: int, bits: int, m: int, seed_pi: int, seed_s: int):
+        lib = load_library()
+        self.d, self.bits, self.m = d, bits, m
+        h = ctypes.c_void_p()
+        _check(lib.tq_polar_build(d, bits, m, seed_pi, seed_s, ctypes.byref(h)))
+        self.handle = h
+        self.record_bytes = int(lib.tq_polar_record_bytes(h))
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            load_library().tq_polar_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def polar_encode(pc: PolarCodec, x, records=None, error_word=None, stream=None):
+    """tq_polar_encode: x [n, d] -> records uint8 [n, record_bytes]."""
+    import torch
+    assert x.is_cuda and x.is_contiguous() and x.dim() == 2
+    n = x.shape[0]
+    if records is None:
+        records = torch.zeros(n, pc.record_bytes, dtype=torch.uint8, device=x.device)
+    _check(load_library().tq_polar_encode(pc.handle, _ptr(x), _dtype_code(x), n, _ptr(records),
+                                           _ptr(error_word), _stream(stream)))
+    return records
+
+
+def polar_logits(pc: PolarCodec, records, q, out=None, workspace=None, stream=None):
+    """tq_polar_logits: records [n, record_bytes], q [nq, d] -> out fp32 [nq, n]."""
+    import torch
+    assert q.is_cuda and q.is_contiguous() and q.dim() == 2
+    n, nq = records.shape[0], q.shape[0]
+    if out is None:
+        out = torch.empty(nq, n, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(int(load_library().tq_polar_logits_workspace_bytes(pc.handle, nq)), 16),
+                                dtype=torch.uint8, device=q.device)
+    _check(load_library().tq_polar_logits(pc.handle, _ptr(records), n, _ptr(q), _dtype_code(q), nq, _ptr(out),
+                                           out.stride(0), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
 
 
 def values_workspace_bytes(cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int, max_ctx: int) -> int:
