@@ -308,6 +308,11 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f;
+  // query slot t's B values carry 2^vsc (set by the largest p ||v|| seen, kept
+  // below 2^14) so that the fp16 hi + lo split keeps its precision whatever
+  // the scale of the value norms; the accumulators are undone at the end
+  int vsc = 0;
+  bool vhas = false;
   if (!producer) {
     const int s = warp < NC0 ? 0 : 1;
     const LineView& L = s ? L1 : L0;
@@ -375,7 +380,8 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
         const float m_new = fmaxf(m_run, mx);
         const float alpha = m_new == -INFINITY ? 1.0f : exp2f(m_run - m_new);
-        float psum = 0.0f;
+        float psum = 0.0f, pv[4];
+        float pmax = 0.0f;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const float pr = ok[r] ? exp2f(sv[r] - m_new) : 0.0f;
@@ -383,14 +389,31 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
           // p ||v|| of token g + 8 r (the norm of a token that does not count is not read)
           const int tok = 32 * hf + g + 8 * r;
           const float vn = ok[r] ? __half2float(reinterpret_cast<const __half*>(vst + VNOFF)[tok]) : 0.0f;
-          wn[(g + 8 * r) * 4 + t] = pr * vn;
+          pv[r] = pr * vn;
+          pmax = fmaxf(pmax, fabsf(pv[r]));
         }
+        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 4));
+        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 8));
+        pmax = fmaxf(pmax, __shfl_xor_sync(0xffffffffu, pmax, 16));
+        float beta = alpha;                         // accumulator factor: softmax and scale
+        if (pmax > 0.0f) {
+          const int e = (int)((__float_as_uint(pmax) >> 23) & 0xFFu) - 126;   // 2^(e-1) <= pmax < 2^e
+          const int s_new = min(120, 14 - e);
+          if (!vhas || s_new < vsc) {
+            if (vhas) beta *= __int_as_float((max(-126, s_new - vsc) + 127) << 23);
+            vsc = s_new;
+            vhas = true;
+          }
+        }
+        const float up = vhas ? __int_as_float((vsc + 127) << 23) : 0.0f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) wn[(g + 8 * r) * 4 + t] = pv[r] * up;
         l_run = l_run * alpha + psum;
         m_run = m_new;
-        if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+        if (__any_sync(0xffffffffu, beta != 1.0f)) {
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
-            acc[mt][0] *= alpha; acc[mt][1] *= alpha; acc[mt][2] *= alpha; acc[mt][3] *= alpha;
+            acc[mt][0] *= beta; acc[mt][1] *= beta; acc[mt][2] *= beta; acc[mt][3] *= beta;
           }
         }
         // 3. values: two steps of 16 tokens
@@ -457,10 +480,11 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
     lt += __shfl_xor_sync(0xffffffffu, lt, 8);
     lt += __shfl_xor_sync(0xffffffffu, lt, 16);
     float* rw = red + (warp * 4 + t) * RS;
+    const float unsc = vhas ? __int_as_float((127 - vsc) << 23) : 1.0f;   // 2^-vsc
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
-      rw[16 * mt + g] = acc[mt][0] + acc[mt][1];       // hi + lo columns of query slot t
-      rw[16 * mt + g + 8] = acc[mt][2] + acc[mt][3];
+      rw[16 * mt + g] = (acc[mt][0] + acc[mt][1]) * unsc;       // hi + lo columns of query slot t
+      rw[16 * mt + g + 8] = (acc[mt][2] + acc[mt][3]) * unsc;
     }
     if (g == 0) {
       rw[DP] = m_run;

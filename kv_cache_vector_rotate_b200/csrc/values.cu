@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(128) dequant_kernel(ValuesParams p) {
 
 constexpr int kValWarps = 4;       // warps per CTA of the accumulate kernel
 constexpr int kValCtaPages = 64;   // block-table entries staged per CTA
-constexpr int kValStages = 2;      // ring stages per warp
+constexpr int kValStages = 2;      // ring stages per warp (a power of two: slot i & (S - 1), phase i / S)
+static_assert((kValStages & (kValStages - 1)) == 0, "the ring indexes its slots with i & (S - 1)");
 
 struct ValuesTcParams {
   tq::CacheView cv;
@@ -149,6 +150,9 @@ struct ValShape {
   static constexpr int kTile = 32 * 4 * E * 2;         // fp16 [32 tokens][4E coordinates]
   static constexpr int kWarpBytes = kValStages * kStage + kTile + 32 * 16;   // + w ||v|| [32][4] fp32
 };
+
+// 2^s as a float for s in [-126, 127] (built from the exponent field).
+__device__ __forceinline__ float pow2i(int s) { return __int_as_float((s + 127) << 23); }
 
 // Mode B, pass 1.  grid: (n_chunks, batch * n_kv_heads, query tiles of 4);
 // block 128; dynamic smem kValWarps * ValShape::kWarpBytes.
@@ -262,6 +266,12 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
   float acc[MT][4];
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.0f;
+  // per query slot, the power of two 2^sc that the B values carry: set by
+  // the largest |w ||v||| seen so far (below 2^14), so that fp16 hi + lo keep
+  // their 22 bits whatever the scale of the weights and norms; when a unit
+  // needs a smaller one the accumulators are scaled down exactly
+  int sc[4] = {0, 0, 0, 0};
+  bool has[4] = {false, false, false, false};
   bool timed_out = false;
   int issued = min(S, n_my);
   // the weights of unit i (this lane's token, 4 query slots), loaded one unit ahead
@@ -305,7 +315,30 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
         reinterpret_cast<uint4*>(tile + lane * (DP * 2))[piece ^ (lane & 7)] =
             decode8<BITS, E>(rec + c * W, kk, p);
       }
-    wn[lane] = make_float4(wv[0] * nrm, wv[1] * nrm, wv[2] * nrm, wv[3] * nrm);
+    float wq[4] = {wv[0] * nrm, wv[1] * nrm, wv[2] * nrm, wv[3] * nrm};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      // non-negative floats order as their bit patterns; the exponent field
+      // gives 2^(e - 1) <= max < 2^e
+      const uint32_t mx = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(wq[q])));
+      if (mx != 0u) {                               // warp-uniform
+        const int e = (int)((mx >> 23) & 0xFFu) - 126;
+        const int s_new = min(120, 14 - e);
+        if (!has[q] || s_new < sc[q]) {
+          if (has[q] && t == q) {
+            const float f = pow2i(max(-126, s_new - sc[q]));
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              acc[mt][0] *= f; acc[mt][1] *= f; acc[mt][2] *= f; acc[mt][3] *= f;
+            }
+          }
+          sc[q] = s_new;
+          has[q] = true;
+        }
+      }
+      wq[q] *= pow2i(sc[q]);                        // 0 stays 0 while nothing was seen
+    }
+    wn[lane] = make_float4(wq[0], wq[1], wq[2], wq[3]);
     __syncwarp();                                 // the tile, wn, and every read of the stage
     if (i + S < n_my) {
       issue(i + S);
@@ -344,10 +377,14 @@ __global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcPara
   // the warps' sums meet in shared memory (the rings are free now)
   __syncthreads();
   float* red = reinterpret_cast<float*>(vsm);     // [kValWarps][4][DP]
+  float unsc = 1.0f;                               // undo query slot t's scale
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q == t && has[q]) unsc = pow2i(-sc[q]);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    red[(warp * 4 + t) * DP + 16 * mt + g] = acc[mt][0] + acc[mt][1];
-    red[(warp * 4 + t) * DP + 16 * mt + g + 8] = acc[mt][2] + acc[mt][3];
+    red[(warp * 4 + t) * DP + 16 * mt + g] = (acc[mt][0] + acc[mt][1]) * unsc;
+    red[(warp * 4 + t) * DP + 16 * mt + g + 8] = (acc[mt][2] + acc[mt][3]) * unsc;
   }
   __syncthreads();
   const int gq = gi * p.qtiles + qt;
@@ -440,9 +477,12 @@ namespace tq {
 // Mode B chunking: every CTA slot of the GPU (SMs x 4) gets one CTA, each
 // an equal share (to one 32-token unit) of a sequence; more CTAs when a share
 // would need more than kValCtaPages - 2 block-table entries.
-static int64_t values_chunks(int64_t units_gq, int64_t max_ctx, int page_tokens) {
+// CTAs of the accumulate kernel per (group, query tile): one wave of the
+// CTAs that fit per SM (ctas_per_sm, at most 4), more when a CTA's share
+// would not fit its staged block-table entries.
+static int64_t values_chunks(int64_t units_gq, int64_t max_ctx, int page_tokens, int ctas_per_sm) {
   const int64_t units = (max_ctx + 31) / 32;
-  int64_t n = std::max<int64_t>(1, (int64_t)device_sm_count() * 4 / std::max<int64_t>(1, units_gq));
+  int64_t n = std::max<int64_t>(1, (int64_t)device_sm_count() * ctas_per_sm / std::max<int64_t>(1, units_gq));
   const int64_t max_units_cta = (int64_t)(tqd::kValCtaPages - 2) * page_tokens / 32;
   n = std::max<int64_t>(n, (units + max_units_cta - 1) / max_units_cta);
   return std::min<int64_t>(n, units);
@@ -455,8 +495,49 @@ size_t values_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, in
   if (n_kv_heads <= 0 || n_q_heads <= 0 || max_ctx <= 0) return 0;
   const int G = n_q_heads / n_kv_heads;
   const int64_t gq = batch * n_kv_heads * ((G + 3) / 4);
-  const int64_t chunks = values_chunks(gq, max_ctx, 16);
+  const int64_t chunks = values_chunks(gq, max_ctx, 16, 4);   // 4: the most CTAs per SM the grid assumes
   return (size_t)chunks * gq * 4 * cb->lay.d_pad * sizeof(float);
+}
+
+// CTAs of the accumulate kernel that fit per SM (registers, shared memory), at
+// most 4; per device, per instance.  Sets the kernel's shared-memory limit.
+template <int BITS, int E>
+static int values_occupancy_t() {
+  constexpr int W = tqd::ChunkWords<BITS, E, 0>::W;
+  const int smem = tqd::kValWarps * tqd::ValShape<W, E>::kWarpBytes;
+  static int cache[64] = {};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int occ = 0;
+  if (cudaFuncSetAttribute(tqd::values_acc_kernel<BITS, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tqd::values_acc_kernel<BITS, E>, tqd::kValWarps * 32,
+                                                    smem) != cudaSuccess) {
+    (void)cudaGetLastError();
+    occ = 1;
+  }
+  occ = std::max(1, std::min(occ, 4));
+  if (dev >= 0 && dev < 64) cache[dev] = occ;
+  return occ;
+}
+
+template <int BITS>
+static int values_occupancy_b(int E) {
+  switch (E) {
+    case 16: return values_occupancy_t<BITS, 16>();
+    case 32: return values_occupancy_t<BITS, 32>();
+    case 48: return values_occupancy_t<BITS, 48>();
+    default: return values_occupancy_t<BITS, 64>();
+  }
+}
+
+static int values_occupancy(const Layout& L) {
+  switch (L.bits) {
+    case 1: return values_occupancy_b<1>(L.E);
+    case 2: return values_occupancy_b<2>(L.E);
+    case 3: return values_occupancy_b<3>(L.E);
+    default: return values_occupancy_b<4>(L.E);
+  }
 }
 
 template <int BITS, int E>
@@ -542,7 +623,7 @@ tq_status launch_values(const tq_codebook* cb, const CacheView& cv, const float*
   const int64_t gq = batch * cv.n_kv_heads * tp.qtiles;
   if (mode_b && (batch * cv.n_kv_heads > 65535 || tp.qtiles > 65535 || gq * 4 > 0x7fffffffLL))
     return fail(TQ_EINVAL, "tq_dequant_values: batch * n_kv_heads too large");
-  tp.n_chunks = (int)values_chunks(gq, max_ctx, cv.page_tokens);
+  tp.n_chunks = (int)values_chunks(gq, max_ctx, cv.page_tokens, mode_b ? values_occupancy(L) : 4);
   tp.units = (int)((max_ctx + 31) / 32);
   tp.max_ctx = (int)max_ctx;
   tp.d = L.d;

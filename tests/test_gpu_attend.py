@@ -23,7 +23,7 @@ def tqm():
     return tqmod
 
 
-def _attend_case(tqm, d, kbits, m, vbits, kpt, vpt, ctx, heads, G, seed, qdtype="bf16"):
+def _attend_case(tqm, d, kbits, m, vbits, kpt, vpt, ctx, heads, G, seed, qdtype="bf16", vscale=2.0):
     """Both caches written by the oracle, tq_attend on the GPU, and the
     oracle's softmax attention given the same codes.  The logit tolerance
     (1e-3 of ||q|| ||k|| / sqrt(d)) moves the softmax weights by at most
@@ -31,7 +31,7 @@ def _attend_case(tqm, d, kbits, m, vbits, kpt, vpt, ctx, heads, G, seed, qdtype=
     batch = len(ctx)
     rng = np.random.default_rng(seed)
     keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-1, 1, size=(1, heads, 1, d)))
-    vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
+    vals = rng.standard_normal((batch, heads, max(ctx), d)) * vscale
     kcodec = O.make_codec(d, kbits, m, synth.SEED_PI, synth.SEED_S)
     vcodec = O.make_codec(d, vbits, 0, synth.SEED_PI, synth.SEED_S)
     kcb, kcache, kencs, _ = _oracle_cache(tqm, kcodec, O.Layout(d, kbits, m, kpt, heads), keys, ctx, kpt, seed + 1)
@@ -91,6 +91,12 @@ def test_attend_many_units_per_cta(tqm):
     with many units, shares that span two lines (the consumer warps split
     between them), refills of every ring slot."""
     _attend_case(tqm, 128, 3, 128, 3, 64, 64, [8192, 7777], 8, 4, 61)
+
+
+def test_attend_small_value_norms(tqm):
+    """Value norms near 1e-5 over 8192 tokens (p ||v|| far below fp16's normal
+    range): the fused kernel's B operand carries a power-of-two scale."""
+    _attend_case(tqm, 128, 3, 128, 3, 64, 64, [8192, 3000], 2, 4, 64, vscale=1e-5 / np.sqrt(128))
 
 
 def test_attend_decode_config_full_size(tqm):
@@ -207,4 +213,28 @@ def test_values_mode_b_ignores_bytes_past_the_context(tqm):
             o = Wg @ Vh
             scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
             assert np.all(np.abs(B[b, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None])
+    assert cache.errors() == 0
+
+
+def test_values_mode_b_small_norms_long_context(tqm):
+    """Mode B at context 32768 with value norms near 1e-3 and softmax-like
+    weights (w ||v|| near 3e-8, below fp16's normal range): the B operand
+    carries a power-of-two scale, so the sums keep their precision."""
+    d, bits, pt, heads, G, n = 128, 3, 64, 2, 4, 32768
+    rng = np.random.default_rng(90)
+    V = (rng.standard_normal((1, heads, n, d)) * (1e-3 / np.sqrt(d))).astype(np.float32)
+    codec = O.make_codec(d, bits, 0, synth.SEED_PI, synth.SEED_S)
+    cb, cache, encs, _ = _oracle_cache(tqm, codec, O.Layout(d, bits, 0, pt, heads), V.astype(np.float64), [n], pt, 91)
+    W = synth.softmax_like_weights(92, 1, heads * G, n)
+    out = tqm.dequant_values(cb, cache, torch.tensor([n], dtype=torch.int32, device="cuda"), n, 1,
+                             weights=torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    B = out.cpu().numpy()
+    for h in range(heads):
+        _, e = encs[(0, h)]
+        Vh = O.dequantize(codec, e.idx, e.norm16)
+        Wg = W[0, h * G:(h + 1) * G].astype(np.float64)
+        o = Wg @ Vh
+        scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
+        assert np.all(np.abs(B[0, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None]), h
     assert cache.errors() == 0
