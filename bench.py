@@ -168,10 +168,11 @@ def oracle_logits_sample(n_keys: int, seed: int = 1002):
     pages = np.zeros(lay.page_bytes * (n_keys // PT), np.uint8)
     O.write_pages(lay, pages, bt, 0, 0, np.arange(n_keys), enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
     q = data["q"][1][0]
-    t0 = time.perf_counter()
+    c0, t0 = _cpu_seconds(), time.perf_counter()
     idx, qneg, n16, r16 = O.read_pages(lay, pages, bt, 0, 0, np.arange(n_keys))
     O.logits_from_codes(codec, q, idx, qneg, n16, r16)
     dt = time.perf_counter() - t0
+    _CPU_USE.append((_cpu_seconds() - c0, dt))
     nbytes = n_keys * KEY_REC + 4 * n_keys * 4 + 4 * D * 2
     return nbytes, dt
 
@@ -187,10 +188,12 @@ def oracle_quantize_sample(n_keys: int, seed: int = 1004):
     lay = O.Layout(D, BITS, M, PT, 1)
     bt = synth.block_table(seed, 1, n_keys // PT)
     pages = np.zeros(lay.page_bytes * (n_keys // PT), np.uint8)
-    t0 = time.perf_counter()
+    c0, t0 = _cpu_seconds(), time.perf_counter()
     enc = O.encode(codec, x[0, 0].astype(np.float64))
     O.write_pages(lay, pages, bt, 0, 0, np.arange(n_keys), enc.idx, enc.qneg, enc.norm16, enc.rnorm16)
-    return n_keys, time.perf_counter() - t0
+    dt = time.perf_counter() - t0
+    _CPU_USE.append((_cpu_seconds() - c0, dt))
+    return n_keys, dt
 
 
 def _cpu_model() -> str:
@@ -204,6 +207,24 @@ def _cpu_model() -> str:
     return "unknown"
 
 
+# (process CPU seconds, wall seconds) of every timed oracle region
+_CPU_USE: list = []
+
+
+def _cpu_seconds() -> float:
+    import resource
+    r = resource.getrusage(resource.RUSAGE_SELF)
+    return r.ru_utime + r.ru_stime
+
+
+def _threads_used(since: int = 0) -> float:
+    """Threads the oracle actually kept busy in its timed regions: process CPU
+    time over wall time (numpy's BLAS threads included)."""
+    cpu = sum(c for c, _ in _CPU_USE[since:])
+    wall = sum(w for _, w in _CPU_USE[since:])
+    return round(cpu / wall, 1) if wall > 0 else 1.0
+
+
 def _cpu_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -213,6 +234,7 @@ def _cpu_threads() -> int:
 
 
 def cpu_baseline(budget_s: float = 12.0):
+    mark0 = len(_CPU_USE)
     nb, dt = oracle_logits_sample(4096)
     per_key = dt / 4096
     n = int(min(CTX, max(4096, budget_s / max(per_key, 1e-9) / 2)))
@@ -222,15 +244,25 @@ def cpu_baseline(budget_s: float = 12.0):
     for h in range(heads):
         b_, t_ = oracle_logits_sample(n, seed=1002 + h)
         nb, dt = nb + b_, dt + t_
+    threads_logits = _threads_used(mark0)
+    # the append path: the whole online-append workload (16 x 8 x 4096 keys)
+    # when the calibrated estimate fits 1.5 budgets, else the share that does
+    total = APPEND_CFG["batch"] * APPEND_CFG["heads"] * APPEND_CFG["n_new"]
     nk, dq = oracle_quantize_sample(2048)
-    nk = int(min(1 << 16, max(2048, budget_s / 4 / max(dq / nk, 1e-9))))
+    nk = int(min(total, max(2048, 1.5 * budget_s / max(dq / nk, 1e-9))))
+    mark1 = len(_CPU_USE)
     nk, dq = oracle_quantize_sample(nk)
-    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": _cpu_threads(), "kind": "oracle",
+    threads_q = _threads_used(mark1)
+    return {"value": nb / dt / 1e9, "unit": "GB/s", "cores": threads_logits, "kind": "oracle",
+            "cores_measured_as": "process CPU time / wall time over the timed oracle regions",
+            "threads_available": _cpu_threads(),
             "cpu_model": _cpu_model(), "logical_cpus": os.cpu_count(),
             "sample": f"oracle unpack + logits of {heads} KV head(s) x {n} packed 3-bit keys x 4 query heads "
                       f"({'the whole workload' if heads == HKV else 'one KV head of the workload'}), {dt:.1f} s",
-            "keys_quantized": {"value": nk / dq, "unit": "keys/s",
-                               "sample": f"oracle encode + page packing of {nk} bf16 keys, b=3 + QJL m=128, {dq:.1f} s"}}
+            "keys_quantized": {"value": nk / dq, "unit": "keys/s", "cores": threads_q,
+                               "sample": f"oracle encode + page packing of {nk} bf16 keys"
+                                         f"{' (the whole append workload)' if nk == total else ''}, b=3 + QJL m=128, "
+                                         f"{dq:.1f} s"}}
 
 
 def run_reference(args):
@@ -258,7 +290,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "impl": "reference",
         "config": {"workload": WORKLOAD, "sample_keys_per_step": n_keys},
-        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _cpu_threads(), "kind": "oracle",
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": _threads_used(), "kind": "oracle",
                          "sample": f"{n_keys} keys of one KV head x 4 query heads per step"},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -480,8 +512,10 @@ def profile_phase(args):
     """Sets up one workload and makes three eager calls of one entry point, for
     ncu captures (no timing, no JSON line):
       append        tq_quantize_append of the online-append batch (16 x 8 x 4096 bf16 keys)
-      decode        tq_logits and tq_dequant_values of the decode step (batch 1, ctx 32768)
-      long_b{2,3,4} tq_logits of the long-context workload (batch 4, ctx 131072) at b bits"""
+      decode        tq_logits, tq_dequant_values and tq_attend of the decode step (batch 1, ctx 32768)
+      long_b{2,3,4} tq_logits of the long-context workload (batch 4, ctx 131072) at b bits
+      search        tq_logits_topk, 2e5 unit rows d = 200 (b = 2, m = 200), 1000 queries, k = 10
+      polar         tq_polar_encode and tq_polar_logits (4 queries) of 262144 decode-step keys"""
     import torch
 
     from kv_cache_vector_rotate_b200 import synth, tq
@@ -518,6 +552,26 @@ def profile_phase(args):
         for _ in range(3):
             tq.logits(kcb, kc, q, ctx_t, CTX)
             tq.dequant_values(vcb, vc, ctx_t, CTX, B, weights=W)
+            tq.attend(kcb, kc, vcb, vc, q, ctx_t, CTX)
+    elif ph == "search":
+        n, nq, d, pt = 200000, 1000, 200, 64
+        X = torch.from_numpy(synth.anisotropic_unit(2005, n, d)).to(dev)
+        Q = torch.from_numpy(synth.anisotropic_unit(3005, nq, d)).to(dev).view(1, nq, d)
+        cb = tq.Codebook(d, 2, d, synth.SEED_PI, synth.SEED_S)
+        pps = (n + pt - 1) // pt
+        cache = tq.PagedCache.allocate(cb, pps, pt, 1, torch.from_numpy(synth.block_table(2006, 1, pps)), device=dev)
+        tq.quantize_append(cb, X.view(1, 1, n, d), torch.zeros(1, dtype=torch.int32, device=dev), cache)
+        ctx_t = torch.tensor([n], dtype=torch.int32, device=dev)
+        for _ in range(3):
+            tq.logits_topk(cb, cache, Q, ctx_t, n, 10)
+    elif ph == "polar":
+        n, d = 262144, 128
+        K, q = synth.decode_keys_device(1002, 1, 8, 32, n // 8, d)
+        X = K.reshape(n, d).contiguous()
+        pc = tq.PolarCodec(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+        for _ in range(3):
+            rec = tq.polar_encode(pc, X)
+            tq.polar_logits(pc, rec, q[0, :4].contiguous())
     else:
         bits = int(ph[-1])
         batch, hkv, hq, ctx, d, m, pt = 4, 8, 32, 131072, 128, 128, 64
@@ -809,7 +863,7 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the long-context (batch 4, 131072) phase")
     ap.add_argument("--no-search", action="store_true", help="skip the vector-search (10^6 x d 200) phase")
     ap.add_argument("--no-budget", action="store_true", help="skip the key-codec comparison phase")
-    ap.add_argument("--profile-phase", choices=["append", "decode", "long_b2", "long_b3", "long_b4"],
+    ap.add_argument("--profile-phase", choices=["append", "decode", "long_b2", "long_b3", "long_b4", "search", "polar"],
                     help="set up one workload and make three eager calls (for ncu captures)")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
                     help="seconds of oracle work for --impl reference (all timed and warm-up steps)")

@@ -237,7 +237,10 @@ tq_status tq_logits_topk(const tq_codebook* cb, const tq_cache* cache, const voi
  * on the GPU race; order them on one stream (or with events).  Each call
  * rewrites all of the scratch it reads, so nothing needs clearing.  The first
  * call on a device looks up the array's address (cudaGetSymbolAddress, with
- * that device current); make it before any stream capture.  Allocates
+ * that device current) and keeps it for the life of the process, so a device
+ * reset (cudaDeviceReset, or destroying and re-creating the primary context)
+ * while the library is loaded is not supported: the kept address would be
+ * stale.  Make the first call before any stream capture.  Allocates
  * nothing. */
 tq_status tq_logits_noalloc(const tq_codebook* cb, const tq_cache* cache, const void* q,
                             tq_dtype dtype, int64_t batch, int32_t n_q_heads,
@@ -251,8 +254,10 @@ size_t tq_logits_noalloc_scratch_bytes(void);
 size_t tq_values_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
                                  int32_t n_q_heads, int64_t max_ctx);
 
-/* Value path from packed records (MSE reconstruction v_hat = ||v|| Pi^T
- * c[idx], c the reconstruction levels).  Mode A (weights == NULL): out device [batch, n_kv_heads,
+/* Value path from packed records ("TurboQuant explained", §Stage 1: the
+ * values are coded by the MSE stage alone -- no QJL sketch -- and read back
+ * as the rotated-back centroid vector, v_hat = ||v|| Pi^T c[idx], c the
+ * reconstruction levels).  Mode A (weights == NULL): out device [batch, n_kv_heads,
  * out_stride, d] of out_dtype receives v_hat for t < ctx_len[b].  Mode B
  * (weights != NULL, device fp32 [batch, n_q_heads, w_stride]): out device
  * fp32 [batch, n_q_heads, d] receives sum_{t < ctx_len[b]} weights[b,hq,t]
