@@ -83,10 +83,9 @@ struct PolarParams {
 // First angle of level l (level l has d / 2^l angles).
 __host__ __device__ constexpr int level_offset(int d, int l) { return d - (d >> (l - 1)); }
 
-// The b-bit field at bit `bit` of a little-endian word stream.
+// The b-bit field at bit `bit` of a little-endian word stream (one funnel shift).
 __device__ __forceinline__ uint32_t get_field(const uint32_t* w, int bit, int b) {
-  const uint64_t pair = (uint64_t)w[bit >> 5] | ((uint64_t)w[(bit >> 5) + 1] << 32);
-  return (uint32_t)(pair >> (bit & 31)) & ((1u << b) - 1u);
+  return __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & ((1u << b) - 1u);
 }
 
 // ---- encode: one CTA of 256 threads per 8 vectors -----------------------------------
@@ -288,7 +287,10 @@ __global__ void __launch_bounds__(kPolLogThreads) polar_logits_kernel(PolarParam
   extern __shared__ float4 pol_dsm[];
   auto cs = reinterpret_cast<float2(*)[CSR]>(pol_dsm);                     // [KEYS][CSR]
   auto qs = reinterpret_cast<float(*)[2 * D]>(pol_dsm + (KEYS * CSR + 1) / 2);   // [QL][2D]: Pi q, then S q (m <= D)
-  __shared__ uint32_t sgn[KEYS][8];
+  // per query slot and group of 4 sketch rows, the 16 values sum_k +-z_k of
+  // the group's sign patterns (bit k set: -z_k)
+  auto nt = reinterpret_cast<float(*)[D / 4][16]>(pol_dsm + (KEYS * CSR + 1) / 2 + QL * 2 * D / 4);   // [QL][m/4][16]
+  __shared__ uint32_t recs[KEYS * 48];               // the CTA's records (<= 44 words each), copied once
   __shared__ float kn[KEYS], kr[KEYS];
   __shared__ float tb[8][2][16];
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -301,27 +303,26 @@ __global__ void __launch_bounds__(kPolLogThreads) polar_logits_kernel(PolarParam
     tb[l][w][e] = p.tabs[l * 64 + w * 16 + e];
   }
   __syncthreads();
-  // stage the keys: angle tables, sign words, norms
+  // the records, coalesced (consecutive keys are consecutive records)
+  for (int t = tid; t < nk * RW; t += kPolLogThreads) recs[t] = p.crec[k0 * RW + t];
+  __syncthreads();
+  // stage the keys: angle tables, norms
   for (int t = tid; t < KEYS * (D - 1); t += kPolLogThreads) {
     const int kk = t / (D - 1), a = t % (D - 1);
     float2 c = make_float2(0.0f, 0.0f);
     if (kk < nk) {
-      const uint32_t* r = p.crec + (k0 + kk) * RW;
-      int l = 1;
-      while (a >= level_offset(D, l + 1)) ++l;
+      const uint32_t* r = recs + kk * RW;
+      // level l holds the angles a with D / 2^l < D - a <= D / 2^(l - 1)
+      const int l = L + 1 - (32 - __clz(D - a - 1));
       const int idx = (int)get_field(r, a * B, B);
       c = make_float2(tb[l - 1][0][idx], tb[l - 1][1][idx]);
     }
     cs[kk][a] = c;
   }
-  for (int t = tid; t < KEYS * 8; t += kPolLogThreads) {
-    const int kk = t / 8, w = t % 8;
-    sgn[kk][w] = (kk < nk && w < SW) ? p.crec[(k0 + kk) * RW + CW + w] : 0u;
-  }
   if (tid < KEYS) {
     float a = 0.0f, b = 0.0f;
     if (tid < nk) {
-      const uint32_t nw = p.crec[(k0 + tid) * RW + CW + SW];
+      const uint32_t nw = recs[tid * RW + CW + SW];
       a = __half2float(__ushort_as_half((unsigned short)(nw & 0xFFFFu)));
       b = __half2float(__ushort_as_half((unsigned short)(nw >> 16)));
     }
@@ -337,19 +338,23 @@ __global__ void __launch_bounds__(kPolLogThreads) polar_logits_kernel(PolarParam
       qs[s][e] = qb + s < q_end ? p.qrot[(int64_t)(qb + s) * (D + M) + e] : 0.0f;
     }
     __syncthreads();
+    for (int t = tid; t < QL * (M / 4) * 16; t += kPolLogThreads) {
+      const int s = t / ((M / 4) * 16), rem = t % ((M / 4) * 16), g4 = rem / 16, v = rem % 16;
+      const float* z = &qs[s][D + 4 * g4];
+      nt[s][g4][v] = ((v & 1) ? -z[0] : z[0]) + ((v & 2) ? -z[1] : z[1]) + ((v & 4) ? -z[2] : z[2]) +
+                     ((v & 8) ? -z[3] : z[3]);
+    }
+    __syncthreads();
     const int qi = qb + ql;
     if (qi < q_end && kk < nk) {
       float s = polar_fold<D, L, 0>(qs[ql], cs[kk]);
       if (M > 0) {
-        // <S q, sign> with sign_i = -1 where bit i is set
+        // <S q, sign> with sign_i = -1 where bit i is set: one table entry per 4 rows
         float sk = 0.0f;
         for (int w = 0; w < (M >> 5); ++w) {
-          const uint32_t bits = sgn[kk][w];
+          const uint32_t bits = recs[kk * RW + CW + w];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float z = qs[ql][D + 32 * w + i];
-            sk += __uint_as_float(__float_as_uint(z) ^ (((bits >> i) & 1u) << 31));
-          }
+          for (int n4 = 0; n4 < 8; ++n4) sk += nt[ql][8 * w + n4][(bits >> (4 * n4)) & 15u];
         }
         s = fmaf(p.qjl_scale * kr[kk], sk, s);
       }
@@ -490,7 +495,8 @@ static tq_status launch_polar_logits_t(const tqd::PolarParams& p, cudaStream_t s
   cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::polar_prep_kernel<D>, p);
   if (e != cudaSuccess) return cuda_fail(e, "tq_polar_logits: query preparation launch");
   constexpr int QL = tqd::kPolLogThreads / KEYS;
-  const size_t smem = (size_t)((KEYS * (D - 1) + 1) / 2) * 16 + (size_t)QL * 2 * D * sizeof(float);
+  const size_t smem = (size_t)((KEYS * (D - 1) + 1) / 2) * 16 + (size_t)QL * 2 * D * sizeof(float) +
+                      (size_t)QL * (D / 4) * 16 * sizeof(float);
   static PerDeviceOnce attr;
   if (const int dev_ = current_device(); attr.need(dev_)) {
     e = cudaFuncSetAttribute(tqd::polar_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
