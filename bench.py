@@ -636,8 +636,7 @@ def run_ours(args):
     def step(r, ev=None):
         if ev is not None:
             ev[0].record()
-        tq.quantize_append(kcb, knew, last, kc[r])
-        tq.quantize_append(vcb, vnew, last, vc[r])
+        tq.quantize_append_kv(kcb, knew, vcb, vnew, last, kc[r], vc[r])
         if ev is not None:
             ev[1].record()
         tq.logits(kcb, kc[r], q, ctx_t, CTX, out=Lout, workspace=lws)
@@ -666,7 +665,7 @@ def run_ours(args):
     K = args.steps
     parts = {
         "full": lambda r: step(r),
-        "append": lambda r: (tq.quantize_append(kcb, knew, last, kc[r]), tq.quantize_append(vcb, vnew, last, vc[r])),
+        "append": lambda r: tq.quantize_append_kv(kcb, knew, vcb, vnew, last, kc[r], vc[r]),
         "logits": lambda r: tq.logits(kcb, kc[r], q, ctx_t, CTX, out=Lout, workspace=lws),
         "values": lambda r: tq.dequant_values(vcb, vc[r], ctx_t, CTX, B, weights=W, out=Oout, workspace=vws),
         "attend": lambda r: tq.attend(kcb, kc[r], vcb, vc[r], q, ctx_t, CTX, out=Aout, workspace=aws),
@@ -786,7 +785,7 @@ def run_ours(args):
                 "h2d_bytes_per_step": q.numel() * 2 + knew.numel() * 2 + vnew.numel() * 2,
                 "d2h_bytes_per_step": Lout.numel() * 4 + Oout.numel() * 4,
                 "ms_per_step": e2e_ms / steps},
-        "gpu_launches": 6 * steps,
+        "gpu_launches": 5 * steps,      # per step: the K+V append, logits (2), values (2)
         "clocks": clk,
     }
     if attend_error is not None:

@@ -172,6 +172,18 @@ tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtyp
                              const int32_t* start_pos, const tq_cache* cache,
                              void* stream);
 
+/* The keys and the values of one cache update (TQ §How to implement:
+ * quantize on every cache update), equivalent to tq_quantize_append(key_cb,
+ * k, ...) followed by tq_quantize_append(value_cb, v, ...) with the same
+ * dtype, shape and start_pos.  k, v: device [batch, n_kv_heads, n_new, d].
+ * For d = 128 keys with a sketch (m_pad = 128), values without one, and at
+ * most 256 vectors of each (decode steps), both are coded by one kernel
+ * launch (a cluster of 8 CTAs per vector); other shapes take the two calls. */
+tq_status tq_quantize_append_kv(const tq_codebook* key_cb, const void* k, const tq_codebook* value_cb,
+                                const void* v, tq_dtype dtype, int64_t batch, int32_t n_kv_heads, int64_t n_new,
+                                const int32_t* start_pos, const tq_cache* key_cache, const tq_cache* value_cache,
+                                void* stream);
+
 /* Workspace (device bytes) that tq_logits needs for these sizes. */
 size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,
                                  int32_t n_q_heads);

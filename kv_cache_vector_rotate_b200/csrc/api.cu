@@ -33,6 +33,10 @@ tq_status launch_quantize_simt(const tq_codebook* cb, const void* x, tq_dtype dt
 tq_status launch_quantize_small(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
                                 int n_kv_heads, int64_t n_new, const int32_t* start_pos,
                                 const CacheView& cv, cudaStream_t st, bool* handled);
+tq_status launch_quantize_small_kv(const tq_codebook* kcb, const void* k, const tq_codebook* vcb, const void* v,
+                                   tq_dtype dt, int64_t batch, int n_kv_heads, int64_t n_new,
+                                   const int32_t* start_pos, const CacheView& kcv, const CacheView& vcv,
+                                   cudaStream_t st, bool* handled);
 tq_status launch_quantize_tc(const tq_codebook* cb, const void* x, tq_dtype dt, int64_t batch,
                              int n_kv_heads, int64_t n_new, const int32_t* start_pos,
                              const CacheView& cv, cudaStream_t st, bool* handled);
@@ -409,6 +413,38 @@ tq_status tq_quantize_append(const tq_codebook* cb, const void* x, tq_dtype dtyp
   s = launch_quantize_small(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st, &handled);
   if (handled || s != TQ_OK) return s;
   return launch_quantize_simt(cb, x, dtype, batch, n_kv_heads, n_new, start_pos, cv, st);
+}
+
+tq_status tq_quantize_append_kv(const tq_codebook* key_cb, const void* k, const tq_codebook* value_cb,
+                                const void* v, tq_dtype dtype, int64_t batch, int32_t n_kv_heads, int64_t n_new,
+                                const int32_t* start_pos, const tq_cache* key_cache, const tq_cache* value_cache,
+                                void* stream) {
+  tq_status s = check_cb(key_cb);
+  if (s != TQ_OK) return s;
+  s = check_cb(value_cb);
+  if (s != TQ_OK) return s;
+  if (!dtype_ok(dtype)) return fail(TQ_EINVAL, "tq_quantize_append_kv: bad dtype");
+  if (batch < 0 || n_new < 0) return fail(TQ_EINVAL, "tq_quantize_append_kv: negative size");
+  CacheView kv, vv;
+  s = make_view(key_cb, key_cache, &kv);
+  if (s != TQ_OK) return s;
+  s = make_view(value_cb, value_cache, &vv);
+  if (s != TQ_OK) return s;
+  if (n_kv_heads != key_cache->n_kv_heads || n_kv_heads != value_cache->n_kv_heads)
+    return fail(TQ_EINVAL, "tq_quantize_append_kv: n_kv_heads differs from a cache's");
+  if (batch == 0 || n_new == 0) return TQ_OK;
+  if (!k || !v || !start_pos) return fail(TQ_EINVAL, "tq_quantize_append_kv: NULL pointer");
+  if (!aligned(k, dtype_size(dtype)) || !aligned(v, dtype_size(dtype)) || !aligned(start_pos, 4))
+    return fail(TQ_EINVAL, "tq_quantize_append_kv: misaligned pointer");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bool handled = false;
+  s = launch_quantize_small_kv(key_cb, k, value_cb, v, dtype, batch, n_kv_heads, n_new, start_pos, kv, vv, st,
+                               &handled);
+  if (handled || s != TQ_OK) return s;
+  // other shapes: the two appends one after the other
+  s = tq_quantize_append(key_cb, k, dtype, batch, n_kv_heads, n_new, start_pos, key_cache, stream);
+  if (s != TQ_OK) return s;
+  return tq_quantize_append(value_cb, v, dtype, batch, n_kv_heads, n_new, start_pos, value_cache, stream);
 }
 
 size_t tq_logits_workspace_bytes(const tq_codebook* cb, int64_t batch, int32_t n_kv_heads,

@@ -59,12 +59,11 @@ __device__ __forceinline__ void sm_wait_acquire() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// grid: 8 x rows CTAs in clusters of 8 (cluster = vector blockIdx.x / 8),
-// block 128.  Thread (o, q) = (tid / 8, tid % 8) takes rotated coordinate
-// j = 16 c + o and sketch row i = 16 c + o, over columns [16 q, 16 q + 16).
+// One vector (row) by one cluster of 8 CTAs of 128 threads.  Thread (o, q) =
+// (tid / 8, tid % 8) takes rotated coordinate j = 16 c + o and sketch row
+// i = 16 c + o, over columns [16 q, 16 q + 16).
 template <int BITS, int F>
-__global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
-    quantize_small_kernel(QuantizeSmallParams p) {
+__device__ __forceinline__ void quantize_small_row(const QuantizeSmallParams& p, int64_t row) {
   constexpr int E = 32;
   constexpr int K = 1 << BITS;
   using CW = ChunkWords<BITS, E, F>;
@@ -75,7 +74,6 @@ __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
   __shared__ float sb[16], sc[16];
   const int tid = threadIdx.x, o = tid >> 3, q = tid & 7;
   const uint32_t c = sm_cluster_rank();
-  const int64_t row = blockIdx.x / kSmCluster;
   const int j = 16 * (int)c + o;
 
   // every operand load first: x columns, this row of Pi (and of S_rot)
@@ -200,6 +198,23 @@ __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
   }
 }
 
+// grid: 8 x rows CTAs in clusters of 8 (cluster = vector blockIdx.x / 8), block 128.
+template <int BITS, int F>
+__global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
+    quantize_small_kernel(QuantizeSmallParams p) {
+  quantize_small_row<BITS, F>(p, blockIdx.x / kSmCluster);
+}
+
+// Keys (with the sketch) and values (without) of a decode step in one launch:
+// clusters [0, pk.rows) code keys, the next pv.rows clusters code values.
+template <int KB, int VB>
+__global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
+    quantize_small_kv_kernel(QuantizeSmallParams pk, QuantizeSmallParams pv) {
+  const int64_t v = blockIdx.x / kSmCluster;       // cluster-uniform
+  if (v < pk.rows) quantize_small_row<KB, 32>(pk, v);
+  else quantize_small_row<VB, 0>(pv, v - pk.rows);
+}
+
 }  // namespace tqd
 
 namespace tq {
@@ -242,6 +257,47 @@ tq_status launch_quantize_small(const tq_codebook* cb, const void* x, tq_dtype d
   }
   *handled = true;
   return cuda_fail(cudaGetLastError(), "quantize_small launch");
+}
+
+// Keys and values of the same shape in one launch: both codebooks d = 128,
+// keys with m_pad = 128 and values with m = 0, up to kSmMaxRows vectors each.
+// *handled = false when the shapes do not qualify (nothing launched).
+tq_status launch_quantize_small_kv(const tq_codebook* kcb, const void* k, const tq_codebook* vcb, const void* v,
+                                   tq_dtype dt, int64_t batch, int n_kv_heads, int64_t n_new,
+                                   const int32_t* start_pos, const CacheView& kcv, const CacheView& vcv,
+                                   cudaStream_t st, bool* handled) {
+  const Layout &K = kcb->lay, &V = vcb->lay;
+  *handled = false;
+  const int64_t rows = batch * n_kv_heads * n_new;
+  const bool f32_ok = dt != TQ_F32 || ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15u) == 0;
+  if (K.d != 128 || K.d_pad != 128 || K.m_pad != 128 || V.d != 128 || V.d_pad != 128 || V.m_pad != 0 || rows < 1 ||
+      rows > tqd::kSmMaxRows || !f32_ok)
+    return TQ_OK;
+  auto fill = [&](const tq_codebook* cb, const void* x, const CacheView& cv) {
+    tqd::QuantizeSmallParams p;
+    p.x = x;
+    p.dtype = dt;
+    p.rows = rows;
+    p.n_new = n_new;
+    p.n_kv_heads = n_kv_heads;
+    p.start_pos = start_pos;
+    p.cv = cv;
+    p.pi32 = cb->pi32;
+    p.srot32 = cb->srot32;
+    p.bound32 = cb->bound32;
+    p.cent32 = cb->cent32;
+    return p;
+  };
+  const tqd::QuantizeSmallParams pk = fill(kcb, k, kcv), pv = fill(vcb, v, vcv);
+  const dim3 grid((unsigned)(2 * rows * tqd::kSmCluster));
+#define TQ_KV(KB_, VB_) \
+  if (K.bits == KB_ && V.bits == VB_) tqd::quantize_small_kv_kernel<KB_, VB_><<<grid, tqd::kSmThreads, 0, st>>>(pk, pv);
+#define TQ_KV_ROW(KB_) TQ_KV(KB_, 1) else TQ_KV(KB_, 2) else TQ_KV(KB_, 3) else TQ_KV(KB_, 4)
+  TQ_KV_ROW(1) else TQ_KV_ROW(2) else TQ_KV_ROW(3) else TQ_KV_ROW(4) else return TQ_OK;
+#undef TQ_KV_ROW
+#undef TQ_KV
+  *handled = true;
+  return cuda_fail(cudaGetLastError(), "quantize_small_kv launch");
 }
 
 }  // namespace tq

@@ -26,7 +26,7 @@ EXPORTS = (
     "tq_values_workspace_bytes", "tq_dequant_values", "tq_last_error", "tq_layout_version",
     "tq_logits_noalloc", "tq_logits_noalloc_scratch_bytes", "tq_selftest_wait_timeout",
     "tq_logits_topk_workspace_bytes", "tq_logits_topk",
-    "tq_polar_build", "tq_polar_free", "tq_polar_record_bytes", "tq_polar_encode",
+    "tq_quantize_append_kv", "tq_polar_build", "tq_polar_free", "tq_polar_record_bytes", "tq_polar_encode",
     "tq_polar_logits_workspace_bytes", "tq_polar_logits",
     "tq_attend_workspace_bytes", "tq_attend", "tq_polar_angle_codebook", "tq_codebook_levels",
 )
@@ -86,6 +86,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "tq_logits_noalloc": (i32, [vp, ctypes.POINTER(CacheStruct), vp, i32, i64, i32, vp, i64, vp, i64, vp]),
         "tq_logits_noalloc_scratch_bytes": (sz, []),
         "tq_logits_topk_workspace_bytes": (sz, [vp, i64, i32, i32, i64, i32]),
+        "tq_quantize_append_kv": (i32, [vp, vp, vp, vp, i32, i64, i32, i64, vp, ctypes.POINTER(CacheStruct),
+                                        ctypes.POINTER(CacheStruct), vp]),
         "tq_polar_build": (i32, [i32, i32, i32, ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(vp)]),
         "tq_polar_free": (None, [vp]),
         "tq_polar_record_bytes": (i32, [vp]),
@@ -223,6 +225,20 @@ def quantize_append(cb: Codebook, x, start_pos, cache: PagedCache, stream=None) 
     cs = cache.struct()
     _check(load_library().tq_quantize_append(cb.handle, _ptr(x), _dtype_code(x), b, h, n,
                                               _ptr(start_pos), ctypes.byref(cs), _stream(stream)))
+
+
+def quantize_append_kv(key_cb: Codebook, k, value_cb: Codebook, v, start_pos, key_cache: PagedCache,
+                       value_cache: PagedCache, stream=None) -> None:
+    """tq_quantize_append_kv: the keys k and the values v [batch, n_kv_heads, n_new, d]
+    of one cache update, into their two caches."""
+    assert k.is_cuda and k.is_contiguous() and k.dim() == 4 and v.is_cuda and v.is_contiguous()
+    assert k.shape == v.shape and k.dtype == v.dtype
+    b, h, n, d = k.shape
+    assert d == key_cb.d and d == value_cb.d
+    ks, vs = key_cache.struct(), value_cache.struct()
+    _check(load_library().tq_quantize_append_kv(key_cb.handle, _ptr(k), value_cb.handle, _ptr(v), _dtype_code(k),
+                                                 b, h, n, _ptr(start_pos), ctypes.byref(ks), ctypes.byref(vs),
+                                                 _stream(stream)))
 
 
 def logits_workspace_bytes(cb: Codebook, batch: int, n_kv_heads: int, n_q_heads: int) -> int:

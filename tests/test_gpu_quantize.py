@@ -284,3 +284,59 @@ def test_bounded_wait_runs_out_and_reports(tqm):
     got = _read_back(lay, cache, synth.block_table(30, 1, 1), 0, 0, np.arange(64))
     compare_codes(codec, vals[0, 0], O.encode(codec, vals[0, 0]), *got)
     assert cache.errors() == 0
+
+
+@pytest.mark.parametrize("kbits,vbits,dtype,batch,heads,n_new", [
+    (3, 3, "bf16", 1, 8, 1), (4, 2, "f16", 4, 8, 1), (1, 4, "f32", 3, 4, 5), (2, 1, "bf16", 32, 8, 1),
+    (3, 3, "bf16", 2, 8, 64)])
+def test_append_kv_equals_two_appends(tqm, kbits, vbits, dtype, batch, heads, n_new):
+    """tq_quantize_append_kv (keys b + QJL m = 128, values b without a sketch,
+    d = 128) writes the same page bytes as tq_quantize_append of the keys and
+    then of the values: decode steps at ragged mid-page positions (one
+    launch for both), and a 1024-vector append that takes the two calls.
+    The keys of the first case are also checked against the oracle."""
+    d, pt = 128, 16
+    rng = np.random.default_rng(40 + kbits + 4 * vbits + batch)
+    start = rng.integers(0, 200, size=batch).astype(np.int32)
+    pps = (int(start.max()) + n_new + pt - 1) // pt
+    bt = synth.block_table(41 + batch, batch, pps)
+    xs = []
+    for _ in range(2):
+        xf = rng.standard_normal((batch, heads, n_new, d)).astype(np.float32)
+        xf[rng.random(xf.shape) < 0.01] *= 30.0
+        if dtype == "bf16":
+            bits16, vals = synth.to_bf16(xf)
+            xs.append((_dev_tensor(bits16, "bf16"), vals))
+        else:
+            xs.append((_dev_tensor(xf, dtype), xf.astype(np.float16 if dtype == "f16" else np.float32)))
+    (k, kv), (v, _) = xs
+    kcb = tqm.Codebook(d, kbits, 128, synth.SEED_PI, synth.SEED_S)
+    vcb = tqm.Codebook(d, vbits, 0, synth.SEED_PI, synth.SEED_S)
+    sp = torch.from_numpy(start).cuda()
+    caches = [tqm.PagedCache.allocate(cb, batch * pps, pt, heads, torch.from_numpy(bt)) for cb in (kcb, vcb) * 2]
+    tqm.quantize_append_kv(kcb, k, vcb, v, sp, caches[0], caches[1])
+    tqm.quantize_append(kcb, k, sp, caches[2])
+    tqm.quantize_append(vcb, v, sp, caches[3])
+    torch.cuda.synchronize()
+    assert all(c.errors() == 0 for c in caches)
+    assert torch.equal(caches[0].pages, caches[2].pages)
+    assert torch.equal(caches[1].pages, caches[3].pages)
+    if batch == 1 and heads == 8:
+        codec = O.make_codec(d, kbits, 128, synth.SEED_PI, synth.SEED_S)
+        lay = O.Layout(d, kbits, 128, pt, heads)
+        for h in range(heads):
+            got = _read_back(lay, caches[0], bt, 0, h, start[0] + np.arange(n_new))
+            x64 = kv[0, h].astype(np.float64)
+            compare_codes(codec, x64, O.encode(codec, x64), *got)
+
+
+def test_append_kv_rejects_mismatched_heads(tqm):
+    d, pt = 128, 16
+    kcb = tqm.Codebook(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    vcb = tqm.Codebook(d, 3, 0, synth.SEED_PI, synth.SEED_S)
+    bt = torch.zeros(1, 1, dtype=torch.int32)
+    kc = tqm.PagedCache.allocate(kcb, 1, pt, 8, bt)
+    vc = tqm.PagedCache.allocate(vcb, 1, pt, 4, bt)
+    x = torch.zeros(1, 8, 1, d, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(tqm.TqError):
+        tqm.quantize_append_kv(kcb, x, vcb, x, torch.zeros(1, dtype=torch.int32, device="cuda"), kc, vc)
