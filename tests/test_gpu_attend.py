@@ -238,3 +238,39 @@ def test_values_mode_b_small_norms_long_context(tqm):
         scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
         assert np.all(np.abs(B[0, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None]), h
     assert cache.errors() == 0
+
+
+@pytest.mark.parametrize("d,bits,pt,G,batch,heads", [(128, 3, 32, 6, 3, 3), (64, 4, 16, 3, 2, 5),
+                                                     (128, 1, 128, 9, 1, 2)])
+def test_values_mode_b_ragged_groups_bad_page(tqm, d, bits, pt, G, batch, heads):
+    """Mode B on the fused pass (d <= 128): query groups that are not a
+    multiple of 4 (a ragged second query tile), several (sequence, KV head)
+    lines per CTA, contexts 1500 / 0 / 333, and one out-of-range block-table
+    entry inside sequence 0's context: the page is reported and its tokens
+    are left out of the sums."""
+    ctx = [1500, 0, 333][:batch]
+    rng = np.random.default_rng(300 + d + bits + G)
+    vals = rng.standard_normal((batch, heads, max(ctx), d)) * 2.0
+    codec = O.make_codec(d, bits, 0, synth.SEED_PI, synth.SEED_S)
+    cb, cache, encs, bt = _oracle_cache(tqm, codec, O.Layout(d, bits, 0, pt, heads), vals, ctx, pt, 301 + G)
+    bad_page = 3
+    cache.block_table[0, bad_page] = 10 ** 6
+    W = synth.softmax_like_weights(302 + G, batch, heads * G, max(ctx))
+    out = tqm.dequant_values(cb, cache, torch.tensor(ctx, dtype=torch.int32, device="cuda"), max(ctx), batch,
+                             weights=torch.from_numpy(W).cuda())
+    torch.cuda.synchronize()
+    assert cache.errors() & tqm.DEV_ERR_PAGE
+    B = out.cpu().numpy()
+    for b in range(batch):
+        for h in range(heads):
+            if ctx[b] == 0:
+                assert not B[b, h * G:(h + 1) * G].any()
+                continue
+            _, e = encs[(b, h)]
+            Vh = O.dequantize(codec, e.idx, e.norm16)
+            Wg = W[b, h * G:(h + 1) * G, : ctx[b]].astype(np.float64).copy()
+            if b == 0:
+                Wg[:, (np.arange(ctx[b]) // pt) == bad_page] = 0.0
+            o = Wg @ Vh
+            scale = np.maximum(np.abs(o).max(axis=1), (np.abs(Wg) @ np.linalg.norm(Vh, axis=1)) / np.sqrt(d))
+            assert np.all(np.abs(B[b, h * G:(h + 1) * G] - o) <= VALUE_TOL * scale[:, None]), (b, h)
