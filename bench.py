@@ -512,7 +512,8 @@ def profile_phase(args):
     """Sets up one workload and makes three eager calls of one entry point, for
     ncu captures (no timing, no JSON line):
       append        tq_quantize_append of the online-append batch (16 x 8 x 4096 bf16 keys)
-      decode        tq_logits, tq_dequant_values and tq_attend of the decode step (batch 1, ctx 32768)
+      decode        tq_quantize_append_kv, tq_logits, tq_dequant_values and tq_attend of the decode
+                    step (batch 1, ctx 32768)
       long_b{2,3,4} tq_logits of the long-context workload (batch 4, ctx 131072) at b bits
       search        tq_logits_topk, 2e5 unit rows d = 200 (b = 2, m = 200), 1000 queries, k = 10
       polar         tq_polar_encode and tq_polar_logits (4 queries) of 262144 decode-step keys"""
@@ -549,7 +550,11 @@ def profile_phase(args):
         q = as_bf16(data["q"][0])
         W = torch.from_numpy(synth.softmax_like_weights(1004, B, HQ, CTX)).to(dev)
         ctx_t = torch.full((B,), CTX, dtype=torch.int32, device=dev)
+        last = torch.full((B,), CTX - 1, dtype=torch.int32, device=dev)
+        knew = as_bf16(data["k"][0][:, :, -1:, :])
+        vnew = as_bf16(data["v"][0][:, :, -1:, :])
         for _ in range(3):
+            tq.quantize_append_kv(kcb, knew, vcb, vnew, last, kc, vc)
             tq.logits(kcb, kc, q, ctx_t, CTX)
             tq.dequant_values(vcb, vc, ctx_t, CTX, B, weights=W)
             tq.attend(kcb, kc, vcb, vc, q, ctx_t, CTX)
