@@ -23,9 +23,10 @@
 // s_i <- s_2i cos ph_i + s_2i+1 sin ph_i per level; the last s is
 // <q~, u_hat>, and L = ||x|| (s + sqrt(pi/2)/m ||r|| <S q, sign>).  That is
 // 2 (d - 1) FMAs per key and query, so this path is bound by the FMA pipe,
-// not by HBM.  The cos and sin of the centroids come from per-level tables,
-// staged per key in shared memory and shared by the CTA's queries; the fold
-// is a compile-time tree, so its partial sums stay in registers.
+// not by HBM.  The cos and sin of the centroids come from per-level tables
+// in shared memory, indexed by the angle's code read from the key's code
+// words in registers; the fold is a compile-time tree over 4 queries at
+// once, so its partial sums stay in registers.
 
 #include <algorithm>
 #include <cmath>
@@ -54,7 +55,7 @@ namespace tqd {
 constexpr int kPolVec = 8;         // vectors per encode CTA
 constexpr int kPolThreads = 256;
 constexpr int kPolLogThreads = 128;
-constexpr int kPolQPass = 4;       // queries per pass of a logits CTA
+constexpr int kPolQPass = 4;       // queries per pass of a logits thread
 constexpr int kPolQBlock = 64;     // queries per logits CTA
 
 struct PolarParams {
@@ -259,107 +260,116 @@ __global__ void __launch_bounds__(128) polar_prep_kernel(PolarParams p) {
   }
 }
 
-// The fold of the subtree (level LV, index IX): coordinates IX 2^LV .. of
-// q~ against the key's angle tree (cs: cos, sin of every angle's centroid).
-template <int D, int LV, int IX>
-__device__ __forceinline__ float polar_fold(const float* qv, const float2* cs) {
+// The B-bit field at compile-time bit POS of a key's code words (in registers).
+template <int B, int POS, int CW>
+__device__ __forceinline__ uint32_t code_field(const uint32_t (&cw)[CW]) {
+  constexpr int w = POS >> 5, sh = POS & 31;
+  if constexpr (sh + B <= 32 || w + 1 >= CW) return (cw[w] >> sh) & ((1u << B) - 1u);
+  else return __funnelshift_r(cw[w], cw[w + 1], sh) & ((1u << B) - 1u);
+}
+
+__device__ __forceinline__ float4 fold2(float4 a, float4 b, float2 c) {
+  return make_float4(fmaf(a.x, c.x, b.x * c.y), fmaf(a.y, c.x, b.y * c.y), fmaf(a.z, c.x, b.z * c.y),
+                     fmaf(a.w, c.x, b.w * c.y));
+}
+
+// The fold of the subtree (level LV, index IX) for 4 queries at once: their
+// coordinates IX 2^LV .. of q~ (qs: [coordinate] x 4 queries) against the
+// key's angle tree; the angle's index comes from the key's code words at a
+// compile-time bit position, its (cos, sin) from the level's table.
+template <int D, int B, int LV, int IX, int CW>
+__device__ __forceinline__ float4 polar_fold4(const float4* qs, const uint32_t (&cw)[CW], const float2 (*tb)[16]) {
+  const float2 c = tb[LV - 1][code_field<B, (level_offset(D, LV) + IX) * B>(cw)];
   if constexpr (LV == 1) {
-    const float2 c = cs[IX];
-    return fmaf(qv[2 * IX], c.x, qv[2 * IX + 1] * c.y);
+    return fold2(qs[2 * IX], qs[2 * IX + 1], c);
   } else {
-    const float a = polar_fold<D, LV - 1, 2 * IX>(qv, cs);
-    const float b = polar_fold<D, LV - 1, 2 * IX + 1>(qv, cs);
-    const float2 c = cs[level_offset(D, LV) + IX];
-    return fmaf(a, c.x, b * c.y);
+    const float4 a = polar_fold4<D, B, LV - 1, 2 * IX>(qs, cw, tb);
+    const float4 b = polar_fold4<D, B, LV - 1, 2 * IX + 1>(qs, cw, tb);
+    return fold2(a, b, c);
   }
 }
 
-// ---- logits: KEYS keys x 64 queries per CTA of 128 threads ------------------------
-// grid (ceil(n / KEYS), ceil(nq / 64)).  The keys' angle tables (cos, sin of
-// the centroids) are staged once; then passes of 4 queries: thread (key
-// kk = tid % KEYS, query slot tid / KEYS) folds its key against its query.
-template <int D>
-__global__ void __launch_bounds__(kPolLogThreads) polar_logits_kernel(PolarParams p) {
+// ---- logits: one thread per key, 4 queries per pass --------------------------------
+// grid (ceil(n / 128), ceil(nq / 64)), block 128.  Thread k holds key k's code
+// words in registers (loaded once) and folds them against 4 queries at a
+// time; shared memory holds the level tables, the 4 queries' q~ and S q
+// interleaved by query (one 16-byte load gives a coordinate of all 4), and
+// per group of 4 sketch rows the 16 signed sums of its z values.
+template <int D, int B>
+__global__ void __launch_bounds__(kPolLogThreads, D == 256 ? 2 : D == 128 ? 3 : 4) polar_logits_kernel(PolarParams p) {
   constexpr int L = D == 64 ? 6 : D == 128 ? 7 : 8;
-  constexpr int KEYS = D == 256 ? 16 : 32;
-  constexpr int QL = kPolLogThreads / KEYS;          // query slots per pass (4 or 8)
-  constexpr int CSR = D - 1;                         // row stride (float2): an odd count, rows in distinct banks
-  extern __shared__ float4 pol_dsm[];
-  auto cs = reinterpret_cast<float2(*)[CSR]>(pol_dsm);                     // [KEYS][CSR]
-  auto qs = reinterpret_cast<float(*)[2 * D]>(pol_dsm + (KEYS * CSR + 1) / 2);   // [QL][2D]: Pi q, then S q (m <= D)
-  // per query slot and group of 4 sketch rows, the 16 values sum_k +-z_k of
-  // the group's sign patterns (bit k set: -z_k)
-  auto nt = reinterpret_cast<float(*)[D / 4][16]>(pol_dsm + (KEYS * CSR + 1) / 2 + QL * 2 * D / 4);   // [QL][m/4][16]
-  __shared__ uint32_t recs[KEYS * 48];               // the CTA's records (<= 44 words each), copied once
-  __shared__ float kn[KEYS], kr[KEYS];
-  __shared__ float tb[8][2][16];
+  constexpr int CW = ((D - 1) * B + 31) / 32;
+  constexpr int CW4 = (CW + 3) / 4;                 // 16-byte pieces of the code words
+  __shared__ float2 tb[L][16];                      // (cos, sin) of the level's centroids
+  __shared__ float4 qs[D];                          // q~[coordinate], 4 queries
+  __shared__ float4 zs[D];                          // (S q)[row], 4 queries (m <= d)
+  __shared__ float4 nt[D / 4][16];                  // per group of 4 rows: sum_k +-z_k (bit k set: -z_k)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int tid = threadIdx.x;
-  const int64_t k0 = (int64_t)blockIdx.x * KEYS;
-  const int nk = (int)min((int64_t)KEYS, p.n - k0);
-  const int B = p.bits, M = p.m, RW = p.rec_words, CW = p.code_words, SW = p.sign_words;
-  for (int i = tid; i < L * 32; i += kPolLogThreads) {
-    const int l = i / 32, w = (i / 16) % 2, e = i % 16;
-    tb[l][w][e] = p.tabs[l * 64 + w * 16 + e];
+  const int64_t key = (int64_t)blockIdx.x * kPolLogThreads + tid;
+  const bool has = key < p.n;
+  const int M = p.m, RW = p.rec_words, SW = p.sign_words;
+  for (int i = tid; i < L * 16; i += kPolLogThreads) {
+    const int l = i / 16, e = i % 16;
+    tb[l][e] = make_float2(p.tabs[l * 64 + e], p.tabs[l * 64 + 16 + e]);
   }
-  __syncthreads();
-  // the records, coalesced (consecutive keys are consecutive records)
-  for (int t = tid; t < nk * RW; t += kPolLogThreads) recs[t] = p.crec[k0 * RW + t];
-  __syncthreads();
-  // stage the keys: angle tables, norms
-  for (int t = tid; t < KEYS * (D - 1); t += kPolLogThreads) {
-    const int kk = t / (D - 1), a = t % (D - 1);
-    float2 c = make_float2(0.0f, 0.0f);
-    if (kk < nk) {
-      const uint32_t* r = recs + kk * RW;
-      // level l holds the angles a with D / 2^l < D - a <= D / 2^(l - 1)
-      const int l = L + 1 - (32 - __clz(D - a - 1));
-      const int idx = (int)get_field(r, a * B, B);
-      c = make_float2(tb[l - 1][0][idx], tb[l - 1][1][idx]);
-    }
-    cs[kk][a] = c;
-  }
-  if (tid < KEYS) {
-    float a = 0.0f, b = 0.0f;
-    if (tid < nk) {
-      const uint32_t nw = recs[tid * RW + CW + SW];
-      a = __half2float(__ushort_as_half((unsigned short)(nw & 0xFFFFu)));
-      b = __half2float(__ushort_as_half((unsigned short)(nw >> 16)));
-    }
-    kn[tid] = a;
-    kr[tid] = b;
-  }
-  const int kk = tid % KEYS, ql = tid / KEYS;
-  const int q_begin = blockIdx.y * kPolQBlock, q_end = min(p.nq, q_begin + kPolQBlock);
-  for (int qb = q_begin; qb < q_end; qb += QL) {
-    __syncthreads();                                 // tables staged / the previous pass done
-    for (int t = tid; t < QL * (D + M); t += kPolLogThreads) {
-      const int s = t / (D + M), e = t % (D + M);
-      qs[s][e] = qb + s < q_end ? p.qrot[(int64_t)(qb + s) * (D + M) + e] : 0.0f;
-    }
-    __syncthreads();
-    for (int t = tid; t < QL * (M / 4) * 16; t += kPolLogThreads) {
-      const int s = t / ((M / 4) * 16), rem = t % ((M / 4) * 16), g4 = rem / 16, v = rem % 16;
-      const float* z = &qs[s][D + 4 * g4];
-      nt[s][g4][v] = ((v & 1) ? -z[0] : z[0]) + ((v & 2) ? -z[1] : z[1]) + ((v & 4) ? -z[2] : z[2]) +
-                     ((v & 8) ? -z[3] : z[3]);
-    }
-    __syncthreads();
-    const int qi = qb + ql;
-    if (qi < q_end && kk < nk) {
-      float s = polar_fold<D, L, 0>(qs[ql], cs[kk]);
-      if (M > 0) {
-        // <S q, sign> with sign_i = -1 where bit i is set: one table entry per 4 rows
-        float sk = 0.0f;
-        for (int w = 0; w < (M >> 5); ++w) {
-          const uint32_t bits = recs[kk * RW + CW + w];
+  // this key's code words and norms (records are 16-byte multiples)
+  uint32_t cw[4 * CW4];
+  float kn = 0.0f, kr = 0.0f;
+  if (has) {
+    const uint4* r4 = reinterpret_cast<const uint4*>(p.crec + key * RW);
 #pragma unroll
-          for (int n4 = 0; n4 < 8; ++n4) sk += nt[ql][8 * w + n4][(bits >> (4 * n4)) & 15u];
-        }
-        s = fmaf(p.qjl_scale * kr[kk], sk, s);
-      }
-      p.out[(int64_t)qi * p.out_stride + k0 + kk] = kn[kk] * s;
+    for (int i = 0; i < CW4; ++i) {
+      const uint4 v = __ldg(r4 + i);
+      cw[4 * i] = v.x; cw[4 * i + 1] = v.y; cw[4 * i + 2] = v.z; cw[4 * i + 3] = v.w;
     }
+    const uint32_t nw = __ldg(p.crec + key * RW + CW + SW);
+    kn = __half2float(__ushort_as_half((unsigned short)(nw & 0xFFFFu)));
+    kr = __half2float(__ushort_as_half((unsigned short)(nw >> 16)));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4 * CW4; ++i) cw[i] = 0u;
+  }
+  const int q_begin = blockIdx.y * kPolQBlock, q_end = min(p.nq, q_begin + kPolQBlock);
+  for (int qb = q_begin; qb < q_end; qb += kPolQPass) {
+    __syncthreads();                                 // the previous pass is done with qs, zs, nt
+    for (int t = tid; t < kPolQPass * (D + M); t += kPolLogThreads) {
+      const int s = t / (D + M), e = t % (D + M);
+      const float v = qb + s < q_end ? p.qrot[(int64_t)(qb + s) * (D + M) + e] : 0.0f;
+      float* dst = e < D ? reinterpret_cast<float*>(&qs[e]) : reinterpret_cast<float*>(&zs[e - D]);
+      dst[s] = v;
+    }
+    __syncthreads();
+    for (int t = tid; t < (M / 4) * 16; t += kPolLogThreads) {
+      const int g4 = t / 16, v = t % 16;
+      const float4 z0 = zs[4 * g4], z1 = zs[4 * g4 + 1], z2 = zs[4 * g4 + 2], z3 = zs[4 * g4 + 3];
+      auto sum = [&](float a, float b, float c, float d) {
+        return ((v & 1) ? -a : a) + ((v & 2) ? -b : b) + ((v & 4) ? -c : c) + ((v & 8) ? -d : d);
+      };
+      nt[g4][v] = make_float4(sum(z0.x, z1.x, z2.x, z3.x), sum(z0.y, z1.y, z2.y, z3.y),
+                              sum(z0.z, z1.z, z2.z, z3.z), sum(z0.w, z1.w, z2.w, z3.w));
+    }
+    __syncthreads();
+    if (!has) continue;
+    float4 s = polar_fold4<D, B, L, 0>(qs, cw, tb);
+    if (M > 0) {
+      // <S q, sign> with sign_i = -1 where bit i is set: one table entry per 4 rows
+      float4 sk = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int w = 0; w < SW; ++w) {
+        const uint32_t bits = __ldg(p.crec + key * RW + CW + w);
+#pragma unroll
+        for (int n4 = 0; n4 < 8; ++n4) {
+          const float4 e = nt[8 * w + n4][(bits >> (4 * n4)) & 15u];
+          sk.x += e.x; sk.y += e.y; sk.z += e.z; sk.w += e.w;
+        }
+      }
+      const float f = p.qjl_scale * kr;
+      s = make_float4(fmaf(f, sk.x, s.x), fmaf(f, sk.y, s.y), fmaf(f, sk.z, s.z), fmaf(f, sk.w, s.w));
+    }
+    const float o[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+    for (int j = 0; j < kPolQPass; ++j)
+      if (qb + j < q_end) p.out[(int64_t)(qb + j) * p.out_stride + key] = kn * o[j];
   }
 }
 
@@ -480,9 +490,8 @@ size_t polar_logits_workspace(const tq_polar* P, int nq) {
   return (size_t)nq * (P->d + P->m) * sizeof(float);
 }
 
-template <int D>
+template <int D, int B>
 static tq_status launch_polar_logits_t(const tqd::PolarParams& p, cudaStream_t st) {
-  constexpr int KEYS = D == 256 ? 16 : 32;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attrs[0].val.programmaticStreamSerializationAllowed = 1;
@@ -494,28 +503,30 @@ static tq_status launch_polar_logits_t(const tqd::PolarParams& p, cudaStream_t s
   cfg.blockDim = dim3(128);
   cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::polar_prep_kernel<D>, p);
   if (e != cudaSuccess) return cuda_fail(e, "tq_polar_logits: query preparation launch");
-  constexpr int QL = tqd::kPolLogThreads / KEYS;
-  const size_t smem = (size_t)((KEYS * (D - 1) + 1) / 2) * 16 + (size_t)QL * 2 * D * sizeof(float) +
-                      (size_t)QL * (D / 4) * 16 * sizeof(float);
-  static PerDeviceOnce attr;
-  if (const int dev_ = current_device(); attr.need(dev_)) {
-    e = cudaFuncSetAttribute(tqd::polar_logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return cuda_fail(e, "tq_polar_logits: smem attribute");
-    attr.mark(dev_);
-  }
-  cfg.gridDim = dim3((unsigned)((p.n + KEYS - 1) / KEYS), (unsigned)((p.nq + tqd::kPolQBlock - 1) / tqd::kPolQBlock));
+  cfg.gridDim = dim3((unsigned)((p.n + tqd::kPolLogThreads - 1) / tqd::kPolLogThreads),
+                     (unsigned)((p.nq + tqd::kPolQBlock - 1) / tqd::kPolQBlock));
   cfg.blockDim = dim3(tqd::kPolLogThreads);
-  cfg.dynamicSmemBytes = smem;
-  e = cudaLaunchKernelEx(&cfg, tqd::polar_logits_kernel<D>, p);
+  e = cudaLaunchKernelEx(&cfg, tqd::polar_logits_kernel<D, B>, p);
   if (e != cudaSuccess) return cuda_fail(e, "tq_polar_logits launch");
   return TQ_OK;
+}
+
+template <int D>
+static tq_status launch_polar_logits_d(const tqd::PolarParams& p, cudaStream_t st) {
+  switch (p.bits) {
+    case 1: return launch_polar_logits_t<D, 1>(p, st);
+    case 2: return launch_polar_logits_t<D, 2>(p, st);
+    case 3: return launch_polar_logits_t<D, 3>(p, st);
+    case 4: return launch_polar_logits_t<D, 4>(p, st);
+  }
+  return fail(TQ_EUNSUPPORTED, "tq_polar_logits: bits must be 1..4");
 }
 
 tq_status polar_logits(const tq_polar* P, const void* rec, int64_t n, const void* q, tq_dtype dt, int nq, float* out,
                        int64_t out_stride, void* ws, size_t ws_bytes, cudaStream_t st) {
   if (!ws || ws_bytes < polar_logits_workspace(P, nq)) return fail(TQ_EINVAL, "tq_polar_logits: workspace too small");
-  const int keys = P->d == 256 ? 16 : 32;
-  if ((n + keys - 1) / keys > 0x7fffffffLL || (nq + tqd::kPolQBlock - 1) / tqd::kPolQBlock > 65535)
+  if ((n + tqd::kPolLogThreads - 1) / tqd::kPolLogThreads > 0x7fffffffLL ||
+      (nq + tqd::kPolQBlock - 1) / tqd::kPolQBlock > 65535)
     return fail(TQ_EINVAL, "tq_polar_logits: n or nq too large");
   tqd::PolarParams p = polar_params(P);
   p.crec = reinterpret_cast<const uint32_t*>(rec);
@@ -527,9 +538,9 @@ tq_status polar_logits(const tq_polar* P, const void* rec, int64_t n, const void
   p.out = out;
   p.out_stride = out_stride;
   switch (P->d) {
-    case 64: return launch_polar_logits_t<64>(p, st);
-    case 128: return launch_polar_logits_t<128>(p, st);
-    case 256: return launch_polar_logits_t<256>(p, st);
+    case 64: return launch_polar_logits_d<64>(p, st);
+    case 128: return launch_polar_logits_d<128>(p, st);
+    case 256: return launch_polar_logits_d<256>(p, st);
   }
   return fail(TQ_EUNSUPPORTED, "tq_polar_logits: d must be 64, 128 or 256");
 }
