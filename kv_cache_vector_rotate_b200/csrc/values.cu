@@ -121,7 +121,11 @@ __global__ void __launch_bounds__(128) dequant_kernel(ValuesParams p) {
 
 // ---- mode B on the tensor cores ----------------------------------------------------
 
-constexpr int kValWarps = 4;       // warps per CTA of the accumulate kernel
+// Warps per CTA of the accumulate kernel: 16 for d <= 128 (one CTA per SM,
+// so a line has few partials for the finish to sum), 4 above (the tiles of
+// 16 warps would not fit in shared memory; 2-3 CTAs per SM).
+template <int E>
+__host__ __device__ constexpr int val_warps() { return E <= 32 ? 16 : 4; }
 constexpr int kValCtaPages = 64;   // block-table entries staged per CTA
 constexpr int kValStages = 2;      // ring stages per warp (a power of two: slot i & (S - 1), phase i / S)
 static_assert((kValStages & (kValStages - 1)) == 0, "the ring indexes its slots with i & (S - 1)");
@@ -155,10 +159,10 @@ struct ValShape {
 __device__ __forceinline__ float pow2i(int s) { return __int_as_float((s + 127) << 23); }
 
 // Mode B, pass 1.  grid: (n_chunks, batch * n_kv_heads, query tiles of 4);
-// block 128; dynamic smem kValWarps * ValShape::kWarpBytes.
+// block val_warps * 32; dynamic smem val_warps * ValShape::kWarpBytes.
 // CTA x of a (group, query tile) owns the 32-token units [x U / n_chunks,
 // (x + 1) U / n_chunks) (U = ceil(max_ctx / 32)); warp w takes its units w,
-// w + 4, ...; lane 0 bulk-copies a unit (32 records, 32 norms) into ring
+// w + val_warps, ...; lane 0 bulk-copies a unit (32 records, 32 norms) into ring
 // stage i % 2 (mbarrier, bounded wait).  Lane l decodes token l into row l
 // of the warp's fp16 tile (16-byte pieces XOR-swizzled by row: conflict-free
 // stores and ldmatrix reads) and forms w ||v|| for the 4 query slots; then
@@ -169,7 +173,8 @@ __device__ __forceinline__ float pow2i(int s) { return __int_as_float((s + 127) 
 // finite table values, and nothing read from those slots reaches the sums).  The
 // warps' sums meet in shared memory; the CTA writes one partial.
 template <int BITS, int E>
-__global__ void __launch_bounds__(kValWarps * 32) values_acc_kernel(ValuesTcParams p) {
+__global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesTcParams p) {
+  constexpr int kValWarps = val_warps<E>();
   constexpr int W = ChunkWords<BITS, E, 0>::W;
   using VS = ValShape<W, E>;
   constexpr int REC = VS::kRec, STAGE = VS::kStage, S = kValStages;
@@ -504,14 +509,15 @@ size_t values_workspace(const tq_codebook* cb, int64_t batch, int n_kv_heads, in
 template <int BITS, int E>
 static int values_occupancy_t() {
   constexpr int W = tqd::ChunkWords<BITS, E, 0>::W;
-  const int smem = tqd::kValWarps * tqd::ValShape<W, E>::kWarpBytes;
+  constexpr int NW = tqd::val_warps<E>();
+  const int smem = NW * tqd::ValShape<W, E>::kWarpBytes;
   static int cache[64] = {};
   const int dev = current_device();
   if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   int occ = 0;
   if (cudaFuncSetAttribute(tqd::values_acc_kernel<BITS, E>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tqd::values_acc_kernel<BITS, E>, tqd::kValWarps * 32,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, tqd::values_acc_kernel<BITS, E>, NW * 32,
                                                     smem) != cudaSuccess) {
     (void)cudaGetLastError();
     occ = 1;
@@ -550,7 +556,8 @@ static tq_status run_values(tqd::ValuesParams p, const tqd::ValuesTcParams& tp, 
     return TQ_OK;
   }
   constexpr int W = tqd::ChunkWords<BITS, E, 0>::W;
-  const int smem = tqd::kValWarps * tqd::ValShape<W, E>::kWarpBytes;
+  constexpr int NW = tqd::val_warps<E>();
+  const int smem = NW * tqd::ValShape<W, E>::kWarpBytes;
   static PerDeviceOnce attr;           // per template instance
   if (const int dev_ = current_device(); attr.need(dev_)) {
     cudaError_t e = cudaFuncSetAttribute(tqd::values_acc_kernel<BITS, E>,
@@ -559,7 +566,7 @@ static tq_status run_values(tqd::ValuesParams p, const tqd::ValuesTcParams& tp, 
     attr.mark(dev_);
   }
   dim3 grid((unsigned)tp.n_chunks, (unsigned)groups, (unsigned)tp.qtiles);
-  tqd::values_acc_kernel<BITS, E><<<grid, tqd::kValWarps * 32, smem, st>>>(tp);
+  tqd::values_acc_kernel<BITS, E><<<grid, NW * 32, smem, st>>>(tp);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(groups * tp.qtiles * 4));
   cfg.blockDim = dim3((1024 / (4 * E)) * (4 * E));   // whole chunk lanes of 4E coordinates
