@@ -52,7 +52,7 @@ struct tq_polar {
 
 namespace tqd {
 
-constexpr int kPolVec = 8;         // vectors per encode CTA
+constexpr int kPolVec = 32;        // vectors per encode CTA
 constexpr int kPolThreads = 256;
 constexpr int kPolLogThreads = 128;
 constexpr int kPolQPass = 4;       // queries per pass of a logits thread
@@ -89,19 +89,36 @@ __device__ __forceinline__ uint32_t get_field(const uint32_t* w, int bit, int b)
   return __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31) & ((1u << b) - 1u);
 }
 
-// ---- encode: one CTA of 256 threads per 8 vectors -----------------------------------
+// ---- encode: one CTA of 256 threads per 32 vectors ----------------------------------
+// Shared memory (dynamic): the vectors' working rows, then indices and words.
+template <int D>
+struct PolarEncSmem {
+  float us[kPolVec][D];          // u = x / ||x|| (original space)
+  float ys[kPolVec][D];          // Pi u, then the radii of the level being done
+  float rs[kPolVec][D];          // radii of the next level; u_hat; then r
+  float rt[kPolVec][D / 2];      // ping-pong buffer of the inverse recursion
+  uint32_t cw[kPolVec][33];      // code words (<= 32) + 1 spare
+  uint32_t sw[kPolVec][8];       // sign words (m <= 256)
+  float nrm[kPolVec], rnrm[kPolVec];
+  float tb[8][4][16];
+  uint8_t ix[kPolVec][D];        // angle indices
+};
+
 template <int D>
 __global__ void __launch_bounds__(kPolThreads) polar_encode_kernel(PolarParams p) {
   constexpr int L = D == 64 ? 6 : D == 128 ? 7 : 8;
-  __shared__ float us[kPolVec][D];          // u = x / ||x|| (original space)
-  __shared__ float ys[kPolVec][D];          // Pi u, then the radii of the level being done
-  __shared__ float rs[kPolVec][D];          // radii of the next level; u_hat; then r
-  __shared__ float rt[kPolVec][D / 2];      // ping-pong buffer of the inverse recursion
-  __shared__ uint8_t ix[kPolVec][D];        // angle indices
-  __shared__ uint32_t cw[kPolVec][33];      // code words (<= 32) + 1 spare
-  __shared__ uint32_t sw[kPolVec][8];       // sign words (m <= 256)
-  __shared__ float nrm[kPolVec], rnrm[kPolVec];
-  __shared__ float tb[8][4][16];
+  extern __shared__ __align__(16) uint8_t pol_enc_smem[];
+  auto& sm = *reinterpret_cast<PolarEncSmem<D>*>(pol_enc_smem);
+  auto& us = sm.us;
+  auto& ys = sm.ys;
+  auto& rs = sm.rs;
+  auto& rt = sm.rt;
+  auto& ix = sm.ix;
+  auto& cw = sm.cw;
+  auto& sw = sm.sw;
+  auto& nrm = sm.nrm;
+  auto& rnrm = sm.rnrm;
+  auto& tb = sm.tb;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t v0 = (int64_t)blockIdx.x * kPolVec;
   const int nv = (int)min((int64_t)kPolVec, p.n - v0);
@@ -115,12 +132,12 @@ __global__ void __launch_bounds__(kPolThreads) polar_encode_kernel(PolarParams p
   }
   __syncthreads();
   // ||x|| (warp v)
-  if (warp < kPolVec) {
+  for (int v = warp; v < kPolVec; v += kPolThreads / 32) {
     float s2 = 0.0f;
-    for (int k = lane; k < D; k += 32) s2 = fmaf(us[warp][k], us[warp][k], s2);
+    for (int k = lane; k < D; k += 32) s2 = fmaf(us[v][k], us[v][k], s2);
 #pragma unroll
     for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-    if (lane == 0) nrm[warp] = sqrtf(s2);
+    if (lane == 0) nrm[v] = sqrtf(s2);
   }
   __syncthreads();
   for (int i = tid; i < kPolVec * D; i += kPolThreads) {
@@ -136,10 +153,18 @@ __global__ void __launch_bounds__(kPolThreads) polar_encode_kernel(PolarParams p
     float acc[VPT];
 #pragma unroll
     for (int a = 0; a < VPT; ++a) acc[a] = 0.0f;
-    for (int k = 0; k < D; ++k) {
-      const float pk = __ldg(p.pit32 + (size_t)k * D + j);   // Pi[j][k]
+    for (int k = 0; k < D; k += 4) {          // 4 coordinates per 16-byte shared load
+      float pk[4];
 #pragma unroll
-      for (int a = 0; a < VPT; ++a) acc[a] = fmaf(pk, us[g + VG * a][k], acc[a]);
+      for (int e = 0; e < 4; ++e) pk[e] = __ldg(p.pit32 + (size_t)(k + e) * D + j);   // Pi[j][k + e]
+#pragma unroll
+      for (int a = 0; a < VPT; ++a) {
+        const float4 u4 = *reinterpret_cast<const float4*>(&us[g + VG * a][k]);
+        acc[a] = fmaf(pk[0], u4.x, acc[a]);
+        acc[a] = fmaf(pk[1], u4.y, acc[a]);
+        acc[a] = fmaf(pk[2], u4.z, acc[a]);
+        acc[a] = fmaf(pk[3], u4.w, acc[a]);
+      }
     }
 #pragma unroll
     for (int a = 0; a < VPT; ++a) ys[g + VG * a][j] = acc[a];
@@ -195,28 +220,56 @@ __global__ void __launch_bounds__(kPolThreads) polar_encode_kernel(PolarParams p
       float acc[VPT];
 #pragma unroll
       for (int a = 0; a < VPT; ++a) acc[a] = 0.0f;
-      for (int j = 0; j < D; ++j) {
-        const float pjk = __ldg(p.pi32 + (size_t)j * D + k);   // Pi[j][k]
+      for (int j = 0; j < D; j += 4) {
+        float pjk[4];
 #pragma unroll
-        for (int a = 0; a < VPT; ++a) acc[a] = fmaf(pjk, rs[g + VG * a][j], acc[a]);
+        for (int e = 0; e < 4; ++e) pjk[e] = __ldg(p.pi32 + (size_t)(j + e) * D + k);   // Pi[j + e][k]
+#pragma unroll
+        for (int a = 0; a < VPT; ++a) {
+          const float4 r4 = *reinterpret_cast<const float4*>(&rs[g + VG * a][j]);
+          acc[a] = fmaf(pjk[0], r4.x, acc[a]);
+          acc[a] = fmaf(pjk[1], r4.y, acc[a]);
+          acc[a] = fmaf(pjk[2], r4.z, acc[a]);
+          acc[a] = fmaf(pjk[3], r4.w, acc[a]);
+        }
       }
 #pragma unroll
       for (int a = 0; a < VPT; ++a) ys[g + VG * a][k] = us[g + VG * a][k] - acc[a];
     }
     __syncthreads();
-    if (warp < kPolVec) {
+    for (int v = warp; v < kPolVec; v += kPolThreads / 32) {
       float s2 = 0.0f;
-      for (int k = lane; k < D; k += 32) s2 = fmaf(ys[warp][k], ys[warp][k], s2);
+      for (int k = lane; k < D; k += 32) s2 = fmaf(ys[v][k], ys[v][k], s2);
 #pragma unroll
       for (int o = 16; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-      if (lane == 0) rnrm[warp] = sqrtf(s2);
+      if (lane == 0) rnrm[v] = sqrtf(s2);
     }
-    // the signs of S r: thread (i, vector)
-    for (int t = tid; t < kPolVec * M; t += kPolThreads) {
-      const int v = t / M, i = t % M;
-      float pr = 0.0f;
-      for (int k = 0; k < D; ++k) pr = fmaf(__ldg(p.st32 + (size_t)k * M + i), ys[v][k], pr);
-      if (pr < 0.0f) atomicOr(&sw[v][i >> 5], 1u << (i & 31));
+    // the signs of S r: thread (row i, 8 vectors), each S^T entry loaded once
+    // per 8 vectors; a warp's 32 consecutive rows make one sign word (ballot)
+    constexpr int VB8 = kPolVec / 8;
+    for (int t = tid; t < M * VB8; t += kPolThreads) {
+      const int i = t % M, v8 = 8 * (t / M);
+      float pr[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) pr[a] = 0.0f;
+      for (int k = 0; k < D; k += 4) {
+        float sk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sk[e] = __ldg(p.st32 + (size_t)(k + e) * M + i);
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const float4 y4 = *reinterpret_cast<const float4*>(&ys[v8 + a][k]);
+          pr[a] = fmaf(sk[0], y4.x, pr[a]);
+          pr[a] = fmaf(sk[1], y4.y, pr[a]);
+          pr[a] = fmaf(sk[2], y4.z, pr[a]);
+          pr[a] = fmaf(sk[3], y4.w, pr[a]);
+        }
+      }
+#pragma unroll
+      for (int a = 0; a < 8; ++a) {
+        const uint32_t word = __ballot_sync(0xffffffffu, pr[a] < 0.0f);
+        if ((i & 31) == 0) sw[v8 + a][i >> 5] = word;
+      }
     }
   }
   __syncthreads();
@@ -467,6 +520,20 @@ static tqd::PolarParams polar_params(const tq_polar* P) {
   return p;
 }
 
+template <int D>
+static tq_status launch_polar_encode_t(const tqd::PolarParams& p, int64_t grid, cudaStream_t st) {
+  constexpr size_t smem = sizeof(tqd::PolarEncSmem<D>);
+  static PerDeviceOnce attr;
+  if (const int dev_ = current_device(); attr.need(dev_)) {
+    cudaError_t e = cudaFuncSetAttribute(tqd::polar_encode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_polar_encode: smem attribute");
+    attr.mark(dev_);
+  }
+  tqd::polar_encode_kernel<D><<<(unsigned)grid, tqd::kPolThreads, smem, st>>>(p);
+  return cuda_fail(cudaGetLastError(), "tq_polar_encode launch");
+}
+
 tq_status polar_encode(const tq_polar* P, const void* x, tq_dtype dt, int64_t n, void* rec, uint32_t* err,
                        cudaStream_t st) {
   tqd::PolarParams p = polar_params(P);
@@ -478,12 +545,11 @@ tq_status polar_encode(const tq_polar* P, const void* x, tq_dtype dt, int64_t n,
   const int64_t grid = (n + tqd::kPolVec - 1) / tqd::kPolVec;
   if (grid > 0x7fffffffLL) return fail(TQ_EINVAL, "tq_polar_encode: n too large");
   switch (P->d) {
-    case 64: tqd::polar_encode_kernel<64><<<(unsigned)grid, tqd::kPolThreads, 0, st>>>(p); break;
-    case 128: tqd::polar_encode_kernel<128><<<(unsigned)grid, tqd::kPolThreads, 0, st>>>(p); break;
-    case 256: tqd::polar_encode_kernel<256><<<(unsigned)grid, tqd::kPolThreads, 0, st>>>(p); break;
-    default: return fail(TQ_EUNSUPPORTED, "tq_polar_encode: d must be 64, 128 or 256");
+    case 64: return launch_polar_encode_t<64>(p, grid, st);
+    case 128: return launch_polar_encode_t<128>(p, grid, st);
+    case 256: return launch_polar_encode_t<256>(p, grid, st);
   }
-  return cuda_fail(cudaGetLastError(), "tq_polar_encode launch");
+  return fail(TQ_EUNSUPPORTED, "tq_polar_encode: d must be 64, 128 or 256");
 }
 
 size_t polar_logits_workspace(const tq_polar* P, int nq) {
