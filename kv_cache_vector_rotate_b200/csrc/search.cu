@@ -28,10 +28,11 @@
 // half full, which raises the threshold.  A last kernel merges the CTAs'
 // lists.
 //
-// Warp roles (10 warps): 0-3 decode (thread = key row), 4-7 epilogue (thread
-// = key row, the tensor-memory lanes of warp w % 4), 8 copies the records of
-// 128-key tiles into a ring (bulk copies, no multicast), 9 issues the MMAs
-// and owns the tensor memory.  Every wait is bounded; a CTA where one gives
+// Warp roles (14 warps): 0-3 decode (thread = key row), 4-11 epilogue
+// (thread = key row, the tensor-memory lanes of warp w % 4; warps 4-7 take
+// the tile's queries 0-31, warps 8-11 queries 32-63), 12 copies the records
+// of 128-key tiles into a ring (bulk copies, no multicast), 13 issues the
+// MMAs and owns the tensor memory.  Every wait is bounded; a CTA where one gives
 // up reports TQ_DEV_ERR_TIMEOUT, lets its copies and MMAs finish, frees its
 // tensor memory and returns.
 
@@ -50,7 +51,8 @@ constexpr int kSrMaxK = 32;        // largest k
 constexpr int kSrBuf = 64;         // candidate buffer per query (sorted and cut to k when half full)
 constexpr int kSrRing = 2;         // record-ring slots
 constexpr int kSrAbuf = 4;         // A chunk buffers in tensor memory
-constexpr int kSrThreads = 320;
+constexpr int kSrThreads = 448;    // 4 decoders, 8 epilogue, producer, MMA issuer
+constexpr int kSrProducer = 12, kSrIssuer = 13;   // warp indices
 constexpr float kSrNone = -INFINITY;
 constexpr int kSrNoIdx = 0x7fffffff;
 
@@ -286,7 +288,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&st.d_full[s], 1);
-      mbar_init(&st.d_empty[s], 4);
+      mbar_init(&st.d_empty[s], 8);
     }
     mbar_init(&st.b_ready, 1);
     mbar_init(&st.mma_done, 1);
@@ -295,7 +297,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     st.ovf = 0;
     st.efail = 0;
   }
-  if (warp == 9) {
+  if (warp == kSrIssuer) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_addr(&st.tmem_base)), "r"(512) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
   auto item_line = [&](int t) { return (int)((i0 + t) / RT); };
   auto item_rt = [&](int t) { return (int)((i0 + t) % RT); };
 
-  if (warp == 8) {
+  if (warp == kSrProducer) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       const uint64_t pol = evict_first_policy();
@@ -392,7 +394,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
       for (int t = max(0, issued - kSrRing); t < issued; ++t)
         mbar_wait(&st.rec_full[t % kSrRing], (uint32_t)(t / kSrRing) & 1u);
     }
-  } else if (warp == 9) {
+  } else if (warp == kSrIssuer) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t id_cb = sr_idesc(2 * kSrQ), id_s = sr_idesc(kSrQ);
@@ -520,18 +522,22 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int r = tid - 128;
-    const int ew = warp - 4;                        // epilogue warp = tensor-memory quadrant
-    const uint32_t lane_base = (uint32_t)(32 * ew) << 16;
-    auto ebar = [&]() { asm volatile("barrier.sync 1, 128;" ::: "memory"); };
+    // epilogue warp ew (0-7): tensor-memory quadrant ew % 4 (its rows r),
+    // queries 32 (ew / 4) .. + 31 of the tile (column groups G0, G0 + 1)
+    const int er = tid - 128;                       // 0 .. 255
+    const int ew = warp - 4;
+    const int r = er & 127;
+    const int G0 = 2 * (ew >> 2);
+    const uint32_t lane_base = (uint32_t)(32 * (ew & 3)) << 16;
+    auto ebar = [&]() { asm volatile("barrier.sync 1, 256;" ::: "memory"); };
     int cur_line = line0;
     // a line's query scales, and empty thresholds
     // (query slots past G never take a candidate: their threshold is +inf)
     auto load_scales = [&](int ln) {
-      if (r < kSrQ) {
-        const float2 sc = p.scal[(int64_t)ln * kSrQ + r];
-        const bool real = (ln % p.qtiles) * kSrQ + r < p.G;
-        st.qp[r] = make_float4(sc.x, sc.y, real ? kSrNone : INFINITY, __int_as_float(kSrNoIdx));
+      if (er < kSrQ) {
+        const float2 sc = p.scal[(int64_t)ln * kSrQ + er];
+        const bool real = (ln % p.qtiles) * kSrQ + er < p.G;
+        st.qp[er] = make_float4(sc.x, sc.y, real ? kSrNone : INFINITY, __int_as_float(kSrNoIdx));
       }
       ebar();
     };
@@ -587,18 +593,18 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     };
     // the lists of the finished line go to the partials; the buffers restart
     auto flush = [&](int seg) {
-      for (int qi = 0; qi < 16; ++qi) {
-        const int q = 16 * ew + qi;
+      for (int qi = 0; qi < 8; ++qi) {
+        const int q = 8 * ew + qi;
         if (st.cnt[q] > 0) cut(q);
       }
       ebar();
-      for (int x = r; x < kSrQ * K; x += 128) {
+      for (int x = er; x < kSrQ * K; x += 256) {
         const int q = x / K, kk = x % K;
         const SrEntry e = kk < st.cnt[q] ? st.buf[q][kk] : SrEntry{kSrNone, kSrNoIdx};
         p.part[(((int64_t)c * 2 + seg) * kSrQ + q) * K + kk] = make_float2(e.s, __int_as_float(e.i));
       }
       ebar();
-      if (r < kSrQ) st.cnt[r] = 0;
+      if (er < kSrQ) st.cnt[er] = 0;
       ebar();
     };
     for (int t = 0; t < n_my; ++t) {
@@ -615,30 +621,30 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
       const bool stop = st.efail != 0;
       ebar();
       if (stop) {
-        if (r == 0) fail_now();
+        if (er == 0) fail_now();
         break;
       }
       sr_fence_after();
       const float2 rs = st.rowscale[t & 3][r];
       const int pos = item_rt(t) * kSrRows + r;
       const uint32_t dcb = tmem + lane_base + db * kColD, ds = dcb + 2 * kSrQ;
-      uint32_t consider[2] = {0xffffffffu, 0xffffffffu};   // queries this row still competes for
-      if (rs.x == kSrNone) consider[0] = consider[1] = 0u;
+      uint32_t consider = rs.x == kSrNone ? 0u : 0xffffffffu;   // this warp's queries the row still competes for
       for (int round = 0; round < 64; ++round) {
         // 1. scores of this row for 16 queries at a time (their constants
         //    loaded first); those that reach the query's threshold are
-        //    appended to its buffer, one shared-memory atomic per query and warp
+        //    appended to its buffer, one shared-memory atomic per hit
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const uint32_t want = (consider[g >> 1] >> (16 * (g & 1))) & 0xFFFFu;
+        for (int g = 0; g < 2; ++g) {
+          const int G = G0 + g;                      // column group: queries 16 G .. 16 G + 15
+          const uint32_t want = (consider >> (16 * g)) & 0xFFFFu;
           if (!__any_sync(0xffffffffu, want != 0u)) continue;   // warp-uniform
           float vh[16], vl[16], vs[16];
-          sr_ld16(dcb + 16 * g, vh);
-          sr_ld16(dcb + kSrQ + 16 * g, vl);
-          if constexpr (F > 0) sr_ld16(ds + 16 * g, vs);
+          sr_ld16(dcb + 16 * G, vh);
+          sr_ld16(dcb + kSrQ + 16 * G, vl);
+          if constexpr (F > 0) sr_ld16(ds + 16 * G, vs);
           float4 qv[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) qv[x] = st.qp[16 * g + x];   // broadcast loads
+          for (int x = 0; x < 16; ++x) qv[x] = st.qp[16 * G + x];   // broadcast loads
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
           uint32_t hit = 0u;
 #pragma unroll
@@ -653,41 +659,36 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
           }
           hit &= want;
           uint32_t keep = 0u;                        // hits that did not fit (retried after the cut)
-          uint32_t any = __reduce_or_sync(0xffffffffu, hit);
-          while (any) {                              // warp-uniform loop over the queries hit
-            const int x = __ffs(any) - 1;
-            any &= any - 1;
-            const int q = 16 * g + x;
-            const bool mine = (hit >> x) & 1u;
-            const uint32_t m = __ballot_sync(0xffffffffu, mine);
-            int base = 0;
-            if (lane == __ffs(m) - 1) base = atomicAdd(&st.cnt[q], __popc(m));
-            base = __shfl_sync(0xffffffffu, base, __ffs(m) - 1);
-            if (mine) {
-              const int slot = base + __popc(m & ((1u << lane) - 1u));
-              float sv = 0.0f;
+          // each lane appends its own hits, one shared-memory atomic per hit:
+          // the lanes' atomics go out together, so a warp waits for about as
+          // many round trips as its busiest lane has hits (usually 0 or 1)
+          for (uint32_t h = hit; h != 0u; h &= h - 1u) {
+            const int x = __ffs(h) - 1;
+            const int q = 16 * G + x;
+            const int slot = atomicAdd(&st.cnt[q], 1);
+            float sv = 0.0f;
 #pragma unroll
-              for (int y = 0; y < 16; ++y)
-                if (y == x) sv = vh[y];
-              if (slot < kSrBuf) st.buf[q][slot] = {sv, pos};
-              else keep |= 1u << x;
-            }
+            for (int y = 0; y < 16; ++y)
+              if (y == x) sv = vh[y];
+            if (slot < kSrBuf) st.buf[q][slot] = {sv, pos};
+            else keep |= 1u << x;
           }
+          __syncwarp();
           if (keep) st.ovf = 1;
-          const uint32_t sh = 16 * (g & 1);
-          consider[g >> 1] = (consider[g >> 1] & ~(0xFFFFu << sh)) | (keep << sh);
+          const uint32_t sh = 16 * g;
+          consider = (consider & ~(0xFFFFu << sh)) | (keep << sh);
         }
         ebar();
         // 2. buffers half full (or full) are cut to the k best
-        for (int qi = 0; qi < 16; ++qi) {
-          const int q = 16 * ew + qi;
+        for (int qi = 0; qi < 8; ++qi) {
+          const int q = 8 * ew + qi;
           if (st.cnt[q] >= kSrBuf / 2) cut(q);
         }
         ebar();
         const int again = st.ovf;
         ebar();
         if (!again) break;
-        if (r == 0) st.ovf = 0;
+        if (er == 0) st.ovf = 0;
         ebar();
       }
       sr_fence_before();
@@ -701,7 +702,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
   sr_fence_before();
   __syncthreads();
   sr_fence_after();
-  if (warp == 9)
+  if (warp == kSrIssuer)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512) : "memory");
 }
 
