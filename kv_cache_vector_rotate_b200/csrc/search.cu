@@ -28,11 +28,12 @@
 // half full, which raises the threshold.  A last kernel merges the CTAs'
 // lists.
 //
-// Warp roles (14 warps): 0-3 decode (thread = key row), 4-11 epilogue
-// (thread = key row, the tensor-memory lanes of warp w % 4; warps 4-7 take
-// the tile's queries 0-31, warps 8-11 queries 32-63), 12 copies the records
-// of 128-key tiles into a ring (bulk copies, no multicast), 13 issues the
-// MMAs and owns the tensor memory.  Every wait is bounded; a CTA where one gives
+// Warp roles (18 warps): 0-7 decode (thread = key row, the tensor-memory
+// lanes of warp w % 4; warps 0-3 the even A chunks of a tile, 4-7 the odd
+// ones), 8-15 epilogue (thread = key row, lanes of warp w % 4; warps 8-11
+// take the tile's queries 0-31, warps 12-15 queries 32-63), 16 copies the
+// records of 128-key tiles into a ring (bulk copies, no multicast), 17
+// issues the MMAs and owns the tensor memory.  Every wait is bounded; a CTA where one gives
 // up reports TQ_DEV_ERR_TIMEOUT, lets its copies and MMAs finish, frees its
 // tensor memory and returns.
 
@@ -51,8 +52,10 @@ constexpr int kSrMaxK = 32;        // largest k
 constexpr int kSrBuf = 64;         // candidate buffer per query (sorted and cut to k when half full)
 constexpr int kSrRing = 2;         // record-ring slots
 constexpr int kSrAbuf = 4;         // A chunk buffers in tensor memory
-constexpr int kSrThreads = 448;    // 4 decoders, 8 epilogue, producer, MMA issuer
-constexpr int kSrProducer = 12, kSrIssuer = 13;   // warp indices
+constexpr int kSrThreads = 576;    // 8 decoders, 8 epilogue, producer, MMA issuer
+constexpr int kSrDecoders = 8;     // warps 0-7: two per tensor-memory quadrant (even / odd chunks)
+constexpr int kSrEpi0 = 8;         // warps 8-15: epilogue
+constexpr int kSrProducer = 16, kSrIssuer = 17;   // warp indices
 constexpr float kSrNone = -INFINITY;
 constexpr int kSrNoIdx = 0x7fffffff;
 
@@ -163,6 +166,12 @@ __device__ __forceinline__ void sr_st8(uint32_t taddr, const uint32_t* v) {
                : "memory");
 }
 // 16 consecutive 32-bit columns of this thread's lane (the caller waits).
+__device__ __forceinline__ void sr_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t* u = reinterpret_cast<uint32_t*>(v);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7])
+               : "r"(taddr) : "memory");
+}
 __device__ __forceinline__ void sr_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t* u = reinterpret_cast<uint32_t*>(v);
   asm volatile(
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
   if (tid == 0) {
     for (int s = 0; s < kSrRing; ++s) {
       mbar_init(&st.rec_full[s], 1);
-      mbar_init(&st.rec_empty[s], 4);
+      mbar_init(&st.rec_empty[s], kSrDecoders);
     }
     for (int s = 0; s < kSrAbuf; ++s) {
       mbar_init(&st.a_full[s], 4);
@@ -444,11 +453,11 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
       sr_commit(&st.mma_done);
       mbar_wait(&st.mma_done, (uint32_t)md_phase & 1u);
     }
-  } else if (warp < 4) {
+  } else if (warp < kSrDecoders) {
     // ------------------------------------------------------------ decoders
-    const int r = tid;                              // key row of the tile = tensor-memory lane
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    int a_cnt = 0;
+    const int r = tid & 127;                        // key row of the tile = tensor-memory lane
+    const int parity = warp >> 2;                   // this warp's chunks: parity, parity + 2, ...
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     for (int t = 0; t < n_my; ++t) {
       const int slot = t % kSrRing;
       // warp-uniform exits: the tensor-memory stores below are warp-wide
@@ -472,9 +481,10 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
           rs = make_float2(__half2float(*reinterpret_cast<const __half*>(hb + 64 * REC + (r & 63) * 2)), 0.0f);
         }
       }
-      st.rowscale[t & 3][r] = rs;
+      if (parity == 0) st.rowscale[t & 3][r] = rs;
       bool ok = true;
-      for (int ch = 0; ch < NCH; ++ch, ++a_cnt) {
+      for (int ch = parity; ch < NCH; ch += 2) {
+        const int a_cnt = t * NCH + ch;             // the chunk's place in the A-buffer sequence
         const int ab = a_cnt % kSrAbuf;
         if (a_cnt >= kSrAbuf &&
             !__all_sync(0xffffffffu, mbar_wait_backoff(&st.a_empty[ab], (uint32_t)((a_cnt / kSrAbuf) - 1) & 1u, 128u))) {
@@ -523,11 +533,11 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
   } else {
     // ------------------------------------------------------------ epilogue
     // epilogue warp ew (0-7): tensor-memory quadrant ew % 4 (its rows r),
-    // queries 32 (ew / 4) .. + 31 of the tile (column groups G0, G0 + 1)
-    const int er = tid - 128;                       // 0 .. 255
-    const int ew = warp - 4;
+    // queries 32 (ew / 4) .. + 31 of the tile (8-query column groups G0 .. G0 + 3)
+    const int er = tid - 32 * kSrEpi0;              // 0 .. 255
+    const int ew = warp - kSrEpi0;
     const int r = er & 127;
-    const int G0 = 2 * (ew >> 2);
+    const int G0 = 4 * (ew >> 2);
     const uint32_t lane_base = (uint32_t)(32 * (ew & 3)) << 16;
     auto ebar = [&]() { asm volatile("barrier.sync 1, 256;" ::: "memory"); };
     int cur_line = line0;
@@ -630,25 +640,25 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
       const uint32_t dcb = tmem + lane_base + db * kColD, ds = dcb + 2 * kSrQ;
       uint32_t consider = rs.x == kSrNone ? 0u : 0xffffffffu;   // this warp's queries the row still competes for
       for (int round = 0; round < 64; ++round) {
-        // 1. scores of this row for 16 queries at a time (their constants
+        // 1. scores of this row for 8 queries at a time (their constants
         //    loaded first); those that reach the query's threshold are
         //    appended to its buffer, one shared-memory atomic per hit
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const int G = G0 + g;                      // column group: queries 16 G .. 16 G + 15
-          const uint32_t want = (consider >> (16 * g)) & 0xFFFFu;
+        for (int g = 0; g < 4; ++g) {
+          const int G = G0 + g;                      // column group: queries 8 G .. 8 G + 7
+          const uint32_t want = (consider >> (8 * g)) & 0xFFu;
           if (!__any_sync(0xffffffffu, want != 0u)) continue;   // warp-uniform
-          float vh[16], vl[16], vs[16];
-          sr_ld16(dcb + 16 * G, vh);
-          sr_ld16(dcb + kSrQ + 16 * G, vl);
-          if constexpr (F > 0) sr_ld16(ds + 16 * G, vs);
-          float4 qv[16];
+          float vh[8], vl[8], vs[8];
+          sr_ld8(dcb + 8 * G, vh);
+          sr_ld8(dcb + kSrQ + 8 * G, vl);
+          if constexpr (F > 0) sr_ld8(ds + 8 * G, vs);
+          float4 qv[8];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) qv[x] = st.qp[16 * G + x];   // broadcast loads
+          for (int x = 0; x < 8; ++x) qv[x] = st.qp[8 * G + x];   // broadcast loads
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
           uint32_t hit = 0u;
 #pragma unroll
-          for (int x = 0; x < 16; ++x) {
+          for (int x = 0; x < 8; ++x) {
             float sv = qv[x].x * (vh[x] + vl[x]);
             if constexpr (F > 0) sv = fmaf(qv[x].y * rs.y, vs[x], rs.x * sv);
             else sv = rs.x * sv;
@@ -664,19 +674,19 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
           // many round trips as its busiest lane has hits (usually 0 or 1)
           for (uint32_t h = hit; h != 0u; h &= h - 1u) {
             const int x = __ffs(h) - 1;
-            const int q = 16 * G + x;
+            const int q = 8 * G + x;
             const int slot = atomicAdd(&st.cnt[q], 1);
             float sv = 0.0f;
 #pragma unroll
-            for (int y = 0; y < 16; ++y)
+            for (int y = 0; y < 8; ++y)
               if (y == x) sv = vh[y];
             if (slot < kSrBuf) st.buf[q][slot] = {sv, pos};
             else keep |= 1u << x;
           }
           __syncwarp();
           if (keep) st.ovf = 1;
-          const uint32_t sh = 16 * g;
-          consider = (consider & ~(0xFFFFu << sh)) | (keep << sh);
+          const uint32_t sh = 8 * g;
+          consider = (consider & ~(0xFFu << sh)) | (keep << sh);
         }
         ebar();
         // 2. buffers half full (or full) are cut to the k best
