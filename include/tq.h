@@ -252,8 +252,7 @@ tq_status tq_logits_topk(const tq_codebook* cb, const tq_cache* cache, const voi
  * that device current) and keeps it for the life of the process, so a device
  * reset (cudaDeviceReset, or destroying and re-creating the primary context)
  * while the library is loaded is not supported: the kept address would be
- * stale.  Make the first call before any stream capture.  Allocates
- * nothing. */
+ * stale.  Allocates nothing. */
 tq_status tq_logits_noalloc(const tq_codebook* cb, const tq_cache* cache, const void* q,
                             tq_dtype dtype, int64_t batch, int32_t n_q_heads,
                             const int32_t* ctx_len, int64_t max_ctx, float* out,
