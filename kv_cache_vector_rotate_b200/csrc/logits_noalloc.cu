@@ -19,8 +19,7 @@
 //  * nothing in the array needs clearing: each call overwrites all of the
 //    scratch it reads;
 //  * the first call on a device looks up the array's device address with
-//    cudaGetSymbolAddress (with that device current); make that first call
-//    before any stream capture.
+//    cudaGetSymbolAddress (with that device current) and keeps it.
 // Nothing here allocates: no cudaMalloc, cudaFree or allocating library call.
 
 #include <mutex>
