@@ -107,3 +107,37 @@ def test_bad_page_is_skipped_and_reported(tqm):
         Lo = O.logits_from_codes(codec, Qg, enc.idx[keep], enc.qneg[keep], enc.norm16[keep], enc.rnorm16[keep])
         err = logit_error(L[b, h * G:(h + 1) * G][:, keep], Lo, np.linalg.norm(Qg, axis=1), enc.norm16[keep], d)
         assert err <= LOGIT_TOL, err
+
+
+def test_wide_ctas_ragged_groups_lines_bad_page(tqm):
+    """About 34 units per CTA (15 consumer warps, two-launch form): 2
+    sequences x 4 KV heads x 6 query heads (a ragged second query tile),
+    contexts 20000 and 13000 (the second sequence's lines end early), CTA
+    shares that straddle lines, and one out-of-range block-table entry."""
+    batch, heads, G, pt, d = 2, 4, 6, 64, 128
+    ctx = [20000, 13000]
+    rng = np.random.default_rng(74)
+    keys = rng.standard_normal((batch, heads, max(ctx), d)) * np.exp(rng.uniform(-1, 1, size=(1, heads, 1, d)))
+    codec = O.make_codec(d, 3, 128, synth.SEED_PI, synth.SEED_S)
+    lay = O.Layout(d, 3, 128, pt, heads)
+    cb, cache, encs, bt = _oracle_cache(tqm, codec, lay, keys, ctx, pt, 75)
+    bad_page = 40
+    bt_bad = bt.copy()
+    bt_bad[1, bad_page] = 10 ** 6
+    cache.block_table.copy_(torch.from_numpy(bt_bad))
+    q = _queries(rng, batch, heads * G, d, "bf16")
+    out = torch.full((batch, heads * G, max(ctx)), float("nan"), device="cuda")
+    tqm.logits(cb, cache, _q_tensor(q, "bf16"), torch.tensor(ctx, dtype=torch.int32, device="cuda"), max(ctx),
+               out=out)
+    torch.cuda.synchronize()
+    assert cache.errors() & tqm.DEV_ERR_PAGE
+    L = out.cpu().numpy()
+    lo, hi = bad_page * pt, (bad_page + 1) * pt
+    assert np.all(np.isnan(L[1, :, lo:hi]))
+    assert np.all(np.isnan(L[1, :, ctx[1]:]))
+    for (b, h), (pos, enc) in encs.items():
+        keep = np.arange(ctx[b]) if b == 0 else np.r_[0:lo, hi:ctx[b]]
+        Qg = q[b, h * G:(h + 1) * G]
+        Lo = O.logits_from_codes(codec, Qg, enc.idx[keep], enc.qneg[keep], enc.norm16[keep], enc.rnorm16[keep])
+        err = logit_error(L[b, h * G:(h + 1) * G][:, keep], Lo, np.linalg.norm(Qg, axis=1), enc.norm16[keep], d)
+        assert err <= LOGIT_TOL, (b, h, err)
