@@ -330,6 +330,31 @@ def test_append_kv_equals_two_appends(tqm, kbits, vbits, dtype, batch, heads, n_
             compare_codes(codec, x64, O.encode(codec, x64), *got)
 
 
+@pytest.mark.parametrize("km,vm,d", [(0, 0, 128), (128, 128, 128), (64, 0, 64)])
+def test_append_kv_other_codebooks_take_two_appends(tqm, km, vm, d):
+    """Codebooks the one-launch form does not take (keys without a sketch,
+    values with one, d = 64): tq_quantize_append_kv writes what the two
+    single-cache appends write."""
+    pt, batch, heads = 16, 2, 4
+    rng = np.random.default_rng(60 + km + vm + d)
+    start = rng.integers(0, 60, size=batch).astype(np.int32)
+    pps = (int(start.max()) + 1 + pt - 1) // pt
+    bt = synth.block_table(61, batch, pps)
+    k = _dev_tensor(synth.to_bf16(rng.standard_normal((batch, heads, 1, d)).astype(np.float32))[0], "bf16")
+    v = _dev_tensor(synth.to_bf16(rng.standard_normal((batch, heads, 1, d)).astype(np.float32))[0], "bf16")
+    kcb = tqm.Codebook(d, 3, km, synth.SEED_PI, synth.SEED_S)
+    vcb = tqm.Codebook(d, 2, vm, synth.SEED_PI, synth.SEED_S)
+    sp = torch.from_numpy(start).cuda()
+    caches = [tqm.PagedCache.allocate(cb, batch * pps, pt, heads, torch.from_numpy(bt)) for cb in (kcb, vcb) * 2]
+    tqm.quantize_append_kv(kcb, k, vcb, v, sp, caches[0], caches[1])
+    tqm.quantize_append(kcb, k, sp, caches[2])
+    tqm.quantize_append(vcb, v, sp, caches[3])
+    torch.cuda.synchronize()
+    assert all(c.errors() == 0 for c in caches)
+    assert torch.equal(caches[0].pages, caches[2].pages)
+    assert torch.equal(caches[1].pages, caches[3].pages)
+
+
 def test_append_kv_rejects_mismatched_heads(tqm):
     d, pt = 128, 16
     kcb = tqm.Codebook(d, 3, 128, synth.SEED_PI, synth.SEED_S)
