@@ -202,6 +202,9 @@ __device__ __forceinline__ void quantize_small_row(const QuantizeSmallParams& p,
 template <int BITS, int F>
 __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
     quantize_small_kernel(QuantizeSmallParams p) {
+  // a programmatic dependent of the previous kernel: nothing is read before it finishes
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");
   quantize_small_row<BITS, F>(p, blockIdx.x / kSmCluster);
 }
 
@@ -210,6 +213,8 @@ __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
 template <int KB, int VB>
 __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
     quantize_small_kv_kernel(QuantizeSmallParams pk, QuantizeSmallParams pv) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // as quantize_small_kernel
+  asm volatile("griddepcontrol.launch_dependents;");
   const int64_t v = blockIdx.x / kSmCluster;       // cluster-uniform
   if (v < pk.rows) quantize_small_row<KB, 32>(pk, v);
   else quantize_small_row<VB, 0>(pv, v - pk.rows);
@@ -218,6 +223,22 @@ __global__ void __cluster_dims__(kSmCluster, 1, 1) __launch_bounds__(kSmThreads)
 }  // namespace tqd
 
 namespace tq {
+
+// A launch on `st` that may start while the previous kernel finishes (the
+// kernels wait for it before touching memory).
+template <class... KArgs, class... Args>
+static void launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  (void)cudaLaunchKernelEx(&cfg, kern, args...);   // errors are read by the caller (cudaGetLastError)
+}
 
 // head_dim 128 (d_pad 128, m 0 or m_pad 128), up to kSmMaxRows vectors, rows
 // of f32 16-byte aligned; everything else goes to the other kernels.
@@ -245,14 +266,22 @@ tq_status launch_quantize_small(const tq_codebook* cb, const void* x, tq_dtype d
   const dim3 grid((unsigned)(rows * tqd::kSmCluster));
   const bool q = L.m_pad == 128;
   switch (L.bits) {
-    case 1: q ? tqd::quantize_small_kernel<1, 32><<<grid, tqd::kSmThreads, 0, st>>>(p)
-              : tqd::quantize_small_kernel<1, 0><<<grid, tqd::kSmThreads, 0, st>>>(p); break;
-    case 2: q ? tqd::quantize_small_kernel<2, 32><<<grid, tqd::kSmThreads, 0, st>>>(p)
-              : tqd::quantize_small_kernel<2, 0><<<grid, tqd::kSmThreads, 0, st>>>(p); break;
-    case 3: q ? tqd::quantize_small_kernel<3, 32><<<grid, tqd::kSmThreads, 0, st>>>(p)
-              : tqd::quantize_small_kernel<3, 0><<<grid, tqd::kSmThreads, 0, st>>>(p); break;
-    case 4: q ? tqd::quantize_small_kernel<4, 32><<<grid, tqd::kSmThreads, 0, st>>>(p)
-              : tqd::quantize_small_kernel<4, 0><<<grid, tqd::kSmThreads, 0, st>>>(p); break;
+    case 1:
+      if (q) launch_dependent(tqd::quantize_small_kernel<1, 32>, grid, dim3(tqd::kSmThreads), st, p);
+      else launch_dependent(tqd::quantize_small_kernel<1, 0>, grid, dim3(tqd::kSmThreads), st, p);
+      break;
+    case 2:
+      if (q) launch_dependent(tqd::quantize_small_kernel<2, 32>, grid, dim3(tqd::kSmThreads), st, p);
+      else launch_dependent(tqd::quantize_small_kernel<2, 0>, grid, dim3(tqd::kSmThreads), st, p);
+      break;
+    case 3:
+      if (q) launch_dependent(tqd::quantize_small_kernel<3, 32>, grid, dim3(tqd::kSmThreads), st, p);
+      else launch_dependent(tqd::quantize_small_kernel<3, 0>, grid, dim3(tqd::kSmThreads), st, p);
+      break;
+    case 4:
+      if (q) launch_dependent(tqd::quantize_small_kernel<4, 32>, grid, dim3(tqd::kSmThreads), st, p);
+      else launch_dependent(tqd::quantize_small_kernel<4, 0>, grid, dim3(tqd::kSmThreads), st, p);
+      break;
     default: return TQ_OK;
   }
   *handled = true;
@@ -291,7 +320,8 @@ tq_status launch_quantize_small_kv(const tq_codebook* kcb, const void* k, const 
   const tqd::QuantizeSmallParams pk = fill(kcb, k, kcv), pv = fill(vcb, v, vcv);
   const dim3 grid((unsigned)(2 * rows * tqd::kSmCluster));
 #define TQ_KV(KB_, VB_) \
-  if (K.bits == KB_ && V.bits == VB_) tqd::quantize_small_kv_kernel<KB_, VB_><<<grid, tqd::kSmThreads, 0, st>>>(pk, pv);
+  if (K.bits == KB_ && V.bits == VB_) \
+    launch_dependent(tqd::quantize_small_kv_kernel<KB_, VB_>, grid, dim3(tqd::kSmThreads), st, pk, pv);
 #define TQ_KV_ROW(KB_) TQ_KV(KB_, 1) else TQ_KV(KB_, 2) else TQ_KV(KB_, 3) else TQ_KV(KB_, 4)
   TQ_KV_ROW(1) else TQ_KV_ROW(2) else TQ_KV_ROW(3) else TQ_KV_ROW(4) else return TQ_OK;
 #undef TQ_KV_ROW

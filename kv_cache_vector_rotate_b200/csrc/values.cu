@@ -184,7 +184,10 @@ __global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesT
   __shared__ int64_t page_base[kValCtaPages];
   __shared__ uint64_t bars[kValWarps][S];
 
-  // the finish kernel may start now: it prefetches Pi and then waits for this grid
+  // a programmatic dependent of the previous kernel (nothing is read before it
+  // finishes); the finish kernel may start now: it prefetches Pi and then
+  // waits for this grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -430,6 +433,7 @@ __global__ void __launch_bounds__(1024) values_finish_kernel(ValuesTcParams p) {
     }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;");   // the next kernel may be scheduled (it waits for this one)
   if (hql >= p.G) return;
   const int nq = gridDim.x;                       // groups * qtiles * 4
   const float* src = p.partial + ((int64_t)gq * 4 + q) * DP + k;
@@ -566,15 +570,23 @@ static tq_status run_values(tqd::ValuesParams p, const tqd::ValuesTcParams& tp, 
     attr.mark(dev_);
   }
   dim3 grid((unsigned)tp.n_chunks, (unsigned)groups, (unsigned)tp.qtiles);
-  tqd::values_acc_kernel<BITS, E><<<grid, NW * 32, smem, st>>>(tp);
   cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(NW * 32);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t ea = cudaLaunchKernelEx(&cfg, tqd::values_acc_kernel<BITS, E>, tp);
+  if (ea != cudaSuccess) return cuda_fail(ea, "values: accumulate launch");
+  cfg = {};
   cfg.gridDim = dim3((unsigned)(groups * tp.qtiles * 4));
   cfg.blockDim = dim3((1024 / (4 * E)) * (4 * E));   // whole chunk lanes of 4E coordinates
   cfg.dynamicSmemBytes = 0;
   cfg.stream = st;
-  cudaLaunchAttribute attrs[1];
-  attrs[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attrs[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, tqd::values_finish_kernel<E>, tp);
