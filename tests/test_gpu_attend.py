@@ -86,6 +86,14 @@ def test_attend_composed_path_matches_oracle(tqm, d, kpt, vpt):
     _attend_case(tqm, d, 3, d, 3, kpt, vpt, [700, 129, 0], 2, 4, 60 + d)
 
 
+@pytest.mark.parametrize("G,kbits,vbits", [(6, 3, 2), (3, 2, 4), (12, 4, 3)])
+def test_attend_ragged_query_tiles(tqm, G, kbits, vbits):
+    """GQA groups that are not a multiple of 4 (the last query tile of a line
+    is ragged) on the fused path, at 4000 / 2500 tokens, mixed key and value
+    widths."""
+    _attend_case(tqm, 128, kbits, 128, vbits, 64, 64, [4000, 2500], 2, G, 70 + G)
+
+
 def test_attend_many_units_per_cta(tqm):
     """Two sequences x 8 KV heads x 32 query heads at 8192 / 7777 tokens: CTAs
     with many units, shares that span two lines (the consumer warps split
