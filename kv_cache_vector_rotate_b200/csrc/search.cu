@@ -120,8 +120,7 @@ struct SrState {
   uint64_t b_ready, mma_done;
   uint32_t tmem_base;
   int fail;
-  int ovf;
-  int efail;
+
   SrMeta meta[kSrRing];
   float2 rowscale[4][kSrRows];              // ||k||, ||k|| ||r|| (x = -inf: the key does not count)
   int cnt[kSrQ];
@@ -303,8 +302,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     mbar_init(&st.mma_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     st.fail = 0;
-    st.ovf = 0;
-    st.efail = 0;
+
   }
   if (warp == kSrIssuer) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -540,6 +538,15 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
     const int G0 = 4 * (ew >> 2);
     const uint32_t lane_base = (uint32_t)(32 * (ew & 3)) << 16;
     auto ebar = [&]() { asm volatile("barrier.sync 1, 256;" ::: "memory"); };
+    // the same barrier, returning whether any epilogue thread passed `v`
+    auto ebar_or = [&](bool v) -> bool {
+      uint32_t any;
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.or.pred q, 1, 256, p;\n"
+          " selp.u32 %0, 1, 0, q;\n}"
+          : "=r"(any) : "r"(v ? 1u : 0u) : "memory");
+      return any != 0u;
+    };
     int cur_line = line0;
     // a line's query scales, and empty thresholds
     // (query slots past G never take a candidate: their threshold is +inf)
@@ -625,12 +632,10 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
         load_scales(ln);
       }
       const int db = t & 1;
-      // the epilogue warps leave together (named barriers follow)
-      if (!mbar_wait_backoff(&st.d_full[db], (uint32_t)(t >> 1) & 1u, 128u)) st.efail = 1;
-      ebar();
-      const bool stop = st.efail != 0;
-      ebar();
-      if (stop) {
+      // the epilogue warps leave together (named barriers follow): one
+      // barrier that also tells every warp whether any wait gave up
+      const bool got = mbar_wait_backoff(&st.d_full[db], (uint32_t)(t >> 1) & 1u, 128u);
+      if (ebar_or(!got)) {
         if (er == 0) fail_now();
         break;
       }
@@ -640,6 +645,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
       const uint32_t dcb = tmem + lane_base + db * kColD, ds = dcb + 2 * kSrQ;
       uint32_t consider = rs.x == kSrNone ? 0u : 0xffffffffu;   // this warp's queries the row still competes for
       for (int round = 0; round < 64; ++round) {
+        bool ovf = false;                            // a hit of this thread did not fit its buffer
         // 1. scores of this row for 8 queries at a time (their constants
         //    loaded first); those that reach the query's threshold are
         //    appended to its buffer, one shared-memory atomic per hit
@@ -684,7 +690,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
             else keep |= 1u << x;
           }
           __syncwarp();
-          if (keep) st.ovf = 1;
+          if (keep) ovf = true;
           const uint32_t sh = 8 * g;
           consider = (consider & ~(0xFFu << sh)) | (keep << sh);
         }
@@ -694,12 +700,8 @@ __global__ void __launch_bounds__(kSrThreads, 1) search_kernel(SearchParams p) {
           const int q = 8 * ew + qi;
           if (st.cnt[q] >= kSrBuf / 2) cut(q);
         }
-        ebar();
-        const int again = st.ovf;
-        ebar();
-        if (!again) break;
-        if (er == 0) st.ovf = 0;
-        ebar();
+        // every cut is done; another round only if some hit did not fit
+        if (!ebar_or(ovf)) break;
       }
       sr_fence_before();
       __syncwarp();
