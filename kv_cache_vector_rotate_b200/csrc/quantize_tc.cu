@@ -338,12 +338,11 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
     for (int e = 0; e < 32; ++e) n2 = fmaf(y[e], y[e], n2);
     st.part_x[ch][r] = n2;
     tc_fence_before();
-    if (__syncthreads_or(!ok)) {
-      aborted = true;
-      break;
-    }
+    // the four warps of this row group (warps w % 4 equal) exchange their
+    // partial norms; a failed wait is agreed on at the CTA barrier below
+    asm volatile("barrier.sync %0, 128;" ::"r"(1 + (warp & 3)) : "memory");
     tc_fence_after();
-    if (tid == kIssueY && k + 1 < n_my) issue_x(k + 1);   // X(k) was read by Y(k)
+    if (ok && tid == kIssueY && k + 1 < n_my) issue_x(k + 1);   // X(k) was read by Y(k) (this thread saw it)
     const float nrm = sqrtf((st.part_x[0][r] + st.part_x[1][r]) + (st.part_x[2][r] + st.part_x[3][r]));
     const float inv = nrm > 0.0f ? 1.0f / nrm : 0.0f;
 
@@ -392,7 +391,7 @@ __global__ void __launch_bounds__(kQtcThreads, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // R, visible to the MMAs
     }
     tc_fence_before();
-    if (__syncthreads_or(!ok2)) {                // R complete; every read of Y(k) done
+    if (__syncthreads_or(!ok || !ok2)) {         // R complete; every read of Y(k) done
       aborted = true;
       break;
     }
