@@ -173,11 +173,16 @@ __device__ __forceinline__ float query_zsum(const uint2 (&bz)[KQ > 0 ? KQ : 1]) 
 // Logits of rows g (la) and g + 8 (lb) of one 16-key tile for this thread's
 // query t.  wa / wb: the W words of chunk t of the two keys; na / nb: their
 // norm slots (fp16 ||k||, then fp16 ||r|| when F > 0).
-// Sign term: k-step kk of a QJL word uses bit planes 2 kk and 2 kk + 1 in
-// place (one mask per operand register), weighted 2^(2 kk + 1) after the
-// query side's 2 z / z slots; a Horner step (x 4) between k-steps brings
-// every k-step of a word to weight 2^(2 n - 1) (n k-steps in the word), and
-// words are scaled to the common weight 128.
+// Sign term: k-step kk of a QJL word uses bit planes 2 kk and 2 kk + 1
+// against the query side's 2 z / z slots, every k-step and word brought to
+// the common weight 128, in one of two forms that give the same sums:
+//  * b != 2: the word shifted left by 6 - 2 kk puts the two planes at bits 6
+//    and 7 of each byte (weight 128 at once), so the k-steps accumulate on one
+//    MMA accumulator with nothing between them;
+//  * b = 2: the planes are masked in place (weight 2^(2 kk + 1)) and a Horner
+//    step (x 4) between k-steps brings a word to weight 2^(2 n - 1) (n
+//    k-steps), then the word is scaled to 128.
+// The first form measured faster at b = 1, 3 and 4, the second at b = 2.
 template <int BITS, int E, int F>
 __device__ __forceinline__ void tile_logits(const uint32_t* wa, const uint32_t* wb, uint32_t na, uint32_t nb,
                                             const QueryFrags<TileShape<BITS, E, F>::KC, TileShape<BITS, E, F>::KQ>& qf,
@@ -214,26 +219,37 @@ __device__ __forceinline__ void tile_logits(const uint32_t* wa, const uint32_t* 
     cbb = acc0[2] + acc0[3];
   }
   if constexpr (F > 0) {
-    // sign term: in-place bit planes against the int8 slices of 2 z / z
+    // sign term: bit planes against the int8 slices of 2 z / z
     int qa[4] = {0, 0, 0, 0};                 // 128 sum beta z (hi, lo columns)
 #pragma unroll
     for (int w = 0; w < QW; ++w) {
       const int nk = min(4, (F - 32 * w) / 8);   // k-steps of this word (4, or 2 for a half word)
-      int a4[4] = {0, 0, 0, 0};
+      if constexpr (BITS != 2) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        if (k < nk) {
-          if (k > 0) {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) a4[r] *= 4;
+        for (int k = 0; k < 4; ++k) {
+          if (k < nk) {
+            const uint32_t xa = wa[q0 + w] << (6 - 2 * k), xb = wb[q0 + w] << (6 - 2 * k);
+            mma_u8s8(qa, xa & 0x40404040u, xb & 0x40404040u, xa & 0x80808080u, xb & 0x80808080u,
+                     qf.bz[4 * w + k]);
           }
-          const uint32_t m0 = 0x01010101u << (2 * k), m1 = m0 << 1;
-          mma_u8s8(a4, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, qf.bz[4 * w + k]);
         }
-      }
-      const int sh = 6 - 2 * (nk - 1);           // weight 2^(2 nk - 1) -> 128
+      } else {
+        int a4[4] = {0, 0, 0, 0};
 #pragma unroll
-      for (int r = 0; r < 4; ++r) qa[r] += a4[r] << sh;
+        for (int k = 0; k < 4; ++k) {
+          if (k < nk) {
+            if (k > 0) {
+#pragma unroll
+              for (int r = 0; r < 4; ++r) a4[r] *= 4;
+            }
+            const uint32_t m0 = 0x01010101u << (2 * k), m1 = m0 << 1;
+            mma_u8s8(a4, wa[q0 + w] & m0, wb[q0 + w] & m0, wa[q0 + w] & m1, wb[q0 + w] & m1, qf.bz[4 * w + k]);
+          }
+        }
+        const int sh = 6 - 2 * (nk - 1);         // weight 2^(2 nk - 1) -> 128
+#pragma unroll
+        for (int r = 0; r < 4; ++r) qa[r] += a4[r] << sh;
+      }
     }
     // sum_i s_i z_i = sum z - 2 sum beta z
     const float ta = fmaf(-1.0f / 64.0f, (float)(256 * qa[0] + qa[1]), qf.zsum);
