@@ -52,8 +52,8 @@ APPEND_CFG = dict(batch=16, heads=8, n_new=4096)
 # DRAM bytes (read + write) of one tq_logits call of this workload from an ncu
 # capture of the current kernel (dram__bytes_read.sum + dram__bytes_write.sum,
 # python bench.py --profile-phase decode).
-LOGITS_DRAM_BYTES = 17877504 + 156928
-LOGITS_DRAM_SOURCE = ("ncu --set full, python bench.py --profile-phase decode: logits_kernel 17,877,504 B read, "
+LOGITS_DRAM_BYTES = 17876736 + 156928
+LOGITS_DRAM_SOURCE = ("ncu --set full, python bench.py --profile-phase decode: logits_kernel 17,876,736 B read, "
                       "0 written; prep_queries_kernel 156,928 B read (profiles/logits_kernel_decode_b1_h8x32_ctx32768.md)")
 WORKLOAD = "decode step: batch 1, 8 KV / 32 query heads, head_dim 128, context 32768, keys b=3 + QJL m=128, values b=3"
 

@@ -71,6 +71,13 @@ struct AttendParams {
   int d;
 };
 
+// 16-byte piece slot of coordinates 8 piece .. 8 piece + 7 in row `row` of a
+// value tile.  XOR with the row (mod 8) spreads the 8 rows that one
+// ldmatrix reads over the 8 16-byte bank groups; pieces 8..15 are also XORed
+// with 4, because the two lanes that decode one token write pieces 8 apart
+// at once (both halves of a row then land in different bank groups).
+__device__ __forceinline__ int tile_swz(int row, int piece) { return piece ^ (row & 7) ^ ((piece >> 1) & 4); }
+
 // Shared memory: the consumer warps' rings (S slots each), then their tiles,
 // then this fixed part.
 template <int KC, int KQ>
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
 #pragma unroll
               for (int kk = 0; kk < E / 8; ++kk) {
                 const int piece = ch * (E / 8) + kk;
-                tile4[tk * PW + (piece ^ (tk & 7))] = decode8<VB, E>(cw, kk, p);
+                tile4[tk * PW + tile_swz(tk, piece)] = decode8<VB, E>(cw, kk, p);
               }
             }
           }
@@ -450,7 +457,7 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
           for (int mt = 0; mt < MT; ++mt) {
             const int piece = 2 * mt + (mi & 1);
             uint32_t a0, a1, a2, a3;
-            ldsm_x4_trans(smem_addr(tile + row * (DP * 2) + 16 * (piece ^ rr)), a0, a1, a2, a3);
+            ldsm_x4_trans(smem_addr(tile + row * (DP * 2) + 16 * tile_swz(row, piece)), a0, a1, a2, a3);
             mma_f16(acc[mt], a0, a1, a2, a3, make_uint2(bw[0], bw[1]));
           }
           __syncwarp();                          // the tile is rewritten next
