@@ -478,15 +478,17 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
     __syncthreads();
   }
   // the warps' (m, l, acc) per query slot meet in shared memory (the rings
-  // are free now): red[w][q][0, DP) acc, [DP] m, [DP + 1] l
+  // are free now): red[w][q][0, DP) acc, [DP] m, [DP + 1] l, rows of RSS
+  // floats (padded so that the 4 query slots' lanes of a store fall in
+  // different banks); the partials in global memory have rows of RS floats
   float* red = reinterpret_cast<float*>(smem);
-  constexpr int RS = DP + 2;
+  constexpr int RS = DP + 2, RSS = DP + 8;
   if (!producer) {
     float lt = l_run;
     lt += __shfl_xor_sync(0xffffffffu, lt, 4);
     lt += __shfl_xor_sync(0xffffffffu, lt, 8);
     lt += __shfl_xor_sync(0xffffffffu, lt, 16);
-    float* rw = red + (warp * 4 + t) * RS;
+    float* rw = red + (warp * 4 + t) * RSS;
     const float unsc = vhas ? __int_as_float((127 - vsc) << 23) : 1.0f;   // 2^-vsc
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
@@ -505,14 +507,14 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
     for (int x = tid; x < 4 * RS; x += NT) {
       const int q = x / RS, k = x - q * RS;
       float M = -INFINITY;
-      for (int w = wa; w < wb; ++w) M = fmaxf(M, red[(w * 4 + q) * RS + DP]);
+      for (int w = wa; w < wb; ++w) M = fmaxf(M, red[(w * 4 + q) * RSS + DP]);
       float v = M;
       if (k != DP) {
         v = 0.0f;
         if (M != -INFINITY)
           for (int w = wa; w < wb; ++w) {
-            const float mw = red[(w * 4 + q) * RS + DP];
-            if (mw != -INFINITY) v += red[(w * 4 + q) * RS + k] * exp2f(mw - M);
+            const float mw = red[(w * 4 + q) * RSS + DP];
+            if (mw != -INFINITY) v += red[(w * 4 + q) * RSS + k] * exp2f(mw - M);
           }
       }
       dst[x] = v;
@@ -639,8 +641,8 @@ bool attend_plan(AttendPlan* pl) {
     const int nc = std::min(tqd::kAttMaxWarps, (smax - fixed - 128) / per_warp);
     if (nc >= 3) {
       const int ring = nc * per_warp;
-      // the end-of-kernel merge area (nc x 4 x (4E + 2) floats) reuses the rings
-      if (nc * 4 * (4 * E + 2) * 4 > ring) continue;
+      // the end-of-kernel merge area (nc x 4 x (4E + 8) floats) reuses the rings
+      if (nc * 4 * (4 * E + 8) * 4 > ring) continue;
       pl->nc = nc;
       pl->ring_shift = rs;
       pl->fixed_off = (ring + 127) / 128 * 128;

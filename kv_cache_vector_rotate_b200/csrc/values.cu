@@ -384,15 +384,19 @@ __global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesT
   }
   // the warps' sums meet in shared memory (the rings are free now)
   __syncthreads();
-  float* red = reinterpret_cast<float*>(vsm);     // [kValWarps][4][DP]
+  // [kValWarps][4][RSV]: rows padded by 8 floats, so that the 4 query slots'
+  // lanes (t) of one store fall in different banks
+  constexpr int RSV = DP + 8;
+  static_assert(kValWarps * 4 * RSV * 4 <= kValWarps * VS::kWarpBytes, "the merge rows fit the rings");
+  float* red = reinterpret_cast<float*>(vsm);
   float unsc = 1.0f;                               // undo query slot t's scale
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     if (q == t && has[q]) unsc = pow2i(-sc[q]);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    red[(warp * 4 + t) * DP + 16 * mt + g] = (acc[mt][0] + acc[mt][1]) * unsc;
-    red[(warp * 4 + t) * DP + 16 * mt + g + 8] = (acc[mt][2] + acc[mt][3]) * unsc;
+    red[(warp * 4 + t) * RSV + 16 * mt + g] = (acc[mt][0] + acc[mt][1]) * unsc;
+    red[(warp * 4 + t) * RSV + 16 * mt + g + 8] = (acc[mt][2] + acc[mt][3]) * unsc;
   }
   __syncthreads();
   const int gq = gi * p.qtiles + qt;
@@ -400,7 +404,7 @@ __global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesT
   for (int i = threadIdx.x; i < 4 * DP; i += kValWarps * 32) {
     float s = 0.0f;
 #pragma unroll
-    for (int w2 = 0; w2 < kValWarps; ++w2) s += red[w2 * 4 * DP + i];
+    for (int w2 = 0; w2 < kValWarps; ++w2) s += red[(w2 * 4 + i / DP) * RSV + i % DP];
     dst[i] = s;
   }
 }
