@@ -78,6 +78,29 @@ struct AttendParams {
 // at once (both halves of a row then land in different bank groups).
 __device__ __forceinline__ int tile_swz(int row, int piece) { return piece ^ (row & 7) ^ ((piece >> 1) & 4); }
 
+// N words (N even) from shared memory at a multiple of 8 bytes, in 8-byte
+// loads, or 16-byte ones when N is a multiple of 4 and A16 says the address
+// is a multiple of 16.  The two chunks that a lane decodes (8 VW bytes at
+// token x 16 VW + half x 8 VW) load this way without bank conflicts at
+// VW = 1, 2, 3 (chunk by chunk, two lanes shared each bank).
+template <int N, bool A16>
+__device__ __forceinline__ void lds_pairs(const uint8_t* src, uint32_t (&w)[N]) {
+  static_assert(N % 2 == 0, "pairs of words");
+  if constexpr (A16 && N % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < N / 4; ++i) {
+      const uint4 v = reinterpret_cast<const uint4*>(src)[i];
+      w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < N / 2; ++i) {
+      const uint2 v = reinterpret_cast<const uint2*>(src)[i];
+      w[2 * i] = v.x; w[2 * i + 1] = v.y;
+    }
+  }
+}
+
 // Shared memory: the consumer warps' rings (S slots each), then their tiles,
 // then this fixed part.
 template <int KC, int KQ>
@@ -428,11 +451,12 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
         for (int ks = 0; ks < 2; ++ks) {
           {
             const uint8_t* rec = vst + (32 * hf + 16 * ks + tk) * VREC;
+            uint32_t cw2[2 * VW];                // chunks 2 hh and 2 hh + 1: contiguous
+            lds_pairs<2 * VW, VW % 2 == 0>(rec + hh * (8 * VW), cw2);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
               const int ch = 2 * hh + cc;
-              uint32_t cw[VW];
-              lds_chunk<VW>(rec + ch * (4 * VW), cw);
+              const uint32_t* cw = cw2 + cc * VW;
 #pragma unroll
               for (int kk = 0; kk < E / 8; ++kk) {
                 const int piece = ch * (E / 8) + kk;
