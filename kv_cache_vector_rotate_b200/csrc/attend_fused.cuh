@@ -128,7 +128,7 @@ struct AttShape {
   static constexpr int kValBytes = (64 * (kValRec + 2) + 15) / 16 * 16;
   static constexpr int kSlot = kKeyBytes + kValBytes;
   static constexpr int kTile = 16 * 4 * E * 2;   // fp16 [16 tokens][4E coordinates]
-  static constexpr int kWn = 32 * 4 * 4;         // p ||v|| fp32 [32 tokens][4 slots]
+  static constexpr int kWn = 8 * kBRow * 2;      // p ||v|| as fp16 hi + lo B rows [8][kBRow]
   static constexpr int kWarpTile = kTile + kWn;
 };
 
@@ -361,7 +361,8 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
     uint64_t* ebars = fx.empty_bar + warp * S;
     const uint8_t* ring = smem + warp * S * SH::kSlot;
     uint8_t* tile = smem + NC * S * SH::kSlot + warp * SH::kWarpTile;
-    float* wn = reinterpret_cast<float*>(tile + SH::kTile);
+    unsigned short* wh = reinterpret_cast<unsigned short*>(tile + SH::kTile);
+    const uint32_t* whw = reinterpret_cast<const uint32_t*>(wh);
     uint4* tile4 = reinterpret_cast<uint4*>(tile);
     const int tk = lane >> 1, hh = lane & 1;   // decoding: token tk of a 16-token step, coordinates half hh
     for (int j = 0; j < n_my; ++j) {
@@ -437,7 +438,14 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
         }
         const float up = vhas ? __int_as_float((vsc + 127) << 23) : 0.0f;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) wn[(g + 8 * r) * 4 + t] = pv[r] * up;
+        for (int r = 0; r < 4; ++r) {
+          // token g + 8 r, query slot t: fp16 hi + lo, once per token and slot
+          const float x = pv[r] * up;
+          const __half hi = __float2half_rn(x);
+          const __half lo = __float2half_rn(x - __half2float(hi));
+          wh[(2 * t) * kBRow + g + 8 * r] = __half_as_ushort(hi);
+          wh[(2 * t + 1) * kBRow + g + 8 * r] = __half_as_ushort(lo);
+        }
         l_run = l_run * alpha + psum;
         m_run = m_new;
         if (__any_sync(0xffffffffu, beta != 1.0f)) {
@@ -469,11 +477,7 @@ __global__ void __launch_bounds__((kAttMaxWarps + 1) * 32, 1) attend_kernel(Atte
 #pragma unroll
           for (int r = 0; r < 2; ++r) {
             const int tt = 16 * ks + 2 * t + 8 * r;
-            const float x0 = wn[tt * 4 + (g >> 1)], x1 = wn[(tt + 1) * 4 + (g >> 1)];
-            const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-            const __half v0 = (g & 1) ? __float2half_rn(x0 - __half2float(h0)) : h0;
-            const __half v1 = (g & 1) ? __float2half_rn(x1 - __half2float(h1)) : h1;
-            bw[r] = (uint32_t)__half_as_ushort(v0) | ((uint32_t)__half_as_ushort(v1) << 16);
+            bw[r] = whw[(g * kBRow + tt) / 2];   // B column g: tokens tt, tt + 1
           }
           const int mi = lane >> 3, rr = lane & 7;
           const int row = 8 * (mi >> 1) + rr;

@@ -7,6 +7,13 @@
 
 namespace tqd {
 
+// The MMA B operands of 32 tokens (the weights times the norms, scaled by
+// 2^sc and split into fp16 hi + lo): row c = 2 q + (0: hi, 1: lo) for query
+// slot q, one fp16 column per token, rows kBRow halves apart.  A fragment
+// load reads word (c kBRow + tk) / 2 for c = g, tk = 2 t + const: rows of 20
+// words put the 8 rows in different banks.
+constexpr int kBRow = 40;
+
 // fp16 level values of the 8 coordinates 8 kk .. 8 kk + 7 of a chunk, as four
 // fp16 pairs (b <= 3: level selector and two byte permutes per 4 values; b =
 // 4: sign-magnitude nibbles).  Tables: any struct with the byte-permute words

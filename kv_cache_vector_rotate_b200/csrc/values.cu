@@ -152,7 +152,7 @@ struct ValShape {
   static constexpr int kRec = 16 * W;                  // bytes per record
   static constexpr int kStage = 32 * kRec + 64;        // 32 records + 32 fp16 norms
   static constexpr int kTile = 32 * 4 * E * 2;         // fp16 [32 tokens][4E coordinates]
-  static constexpr int kWarpBytes = kValStages * kStage + kTile + 32 * 16;   // + w ||v|| [32][4] fp32
+  static constexpr int kWarpBytes = kValStages * kStage + kTile + 8 * kBRow * 2;   // + the B rows
 };
 
 // 2^s as a float for s in [-126, 127] (built from the exponent field).
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesT
   uint8_t* wbase = vsm + warp * VS::kWarpBytes;
   const uint32_t ring_s = smem_addr(wbase);
   uint8_t* tile = wbase + S * STAGE;
-  float4* wn = reinterpret_cast<float4*>(tile + VS::kTile);
+  unsigned short* wh = reinterpret_cast<unsigned short*>(tile + VS::kTile);   // [8][kBRow] fp16 B rows
   const int64_t norm_off = (int64_t)P * REC;
   const uint64_t pol = evict_first_policy();
 
@@ -346,25 +346,30 @@ __global__ void __launch_bounds__(val_warps<E>() * 32) values_acc_kernel(ValuesT
       }
       wq[q] *= pow2i(sc[q]);                        // 0 stays 0 while nothing was seen
     }
-    wn[lane] = make_float4(wq[0], wq[1], wq[2], wq[3]);
-    __syncwarp();                                 // the tile, wn, and every read of the stage
+    // token `lane`'s B values: w ||v|| 2^sc split into fp16 hi + lo, once per
+    // token and query slot
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half hi = __float2half_rn(wq[q]);
+      const __half lo = __float2half_rn(wq[q] - __half2float(hi));
+      wh[(2 * q) * kBRow + lane] = __half_as_ushort(hi);
+      wh[(2 * q + 1) * kBRow + lane] = __half_as_ushort(lo);
+    }
+    __syncwarp();                                 // the tile, the B rows, and every read of the stage
     if (i + S < n_my) {
       issue(i + S);
       issued = i + S + 1;
     }
-    // 2 k-steps of 16 tokens: B column g = slice g & 1 of query slot g >> 1
-    const float* wnf = reinterpret_cast<const float*>(wn);
+    // 2 k-steps of 16 tokens: B column g = row g (slice g & 1 of query slot
+    // g >> 1), tokens tk and tk + 1 in one word
+    const uint32_t* whw = reinterpret_cast<const uint32_t*>(wh);
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       uint32_t bw[2];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int tk = 16 * j + 2 * t + 8 * r;
-        const float x0 = wnf[tk * 4 + (g >> 1)], x1 = wnf[(tk + 1) * 4 + (g >> 1)];
-        const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-        const __half v0 = (g & 1) ? __float2half_rn(x0 - __half2float(h0)) : h0;
-        const __half v1 = (g & 1) ? __float2half_rn(x1 - __half2float(h1)) : h1;
-        bw[r] = (uint32_t)__half_as_ushort(v0) | ((uint32_t)__half_as_ushort(v1) << 16);
+        bw[r] = whw[(g * kBRow + tk) / 2];
       }
       const int mi = lane >> 3, rr = lane & 7;
       const int row = 16 * j + 8 * (mi >> 1) + rr;
